@@ -1,0 +1,227 @@
+"""Host oracle for group-wise affine quantization and quantized products.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline leg call it; the CUDA library never does. The arithmetic
+lives in ``oracle.cpp`` (plain C++, fp32 quantizer, fp64 products); this module
+only marshals CPU torch tensors through ctypes.
+
+Parity status: every function is pinned by tests/test_oracle_pins.py against
+closed forms, hand-built integer groups and brute force (no function here is
+"parity unpinned").
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+_LOCK = threading.Lock()
+_LIB = None
+
+F32, BF16 = 0, 1
+_DT = {torch.float32: F32, torch.bfloat16: BF16}
+_TORCH = {F32: torch.float32, BF16: torch.bfloat16}
+
+_p = C.c_void_p
+_i64 = C.c_int64
+_i = C.c_int
+
+
+def load(path: str | None = None):
+    """Load liboracle.so, compiling it first if it is missing or older than its source."""
+    global _LIB
+    with _LOCK:
+        if path is not None:
+            return _bind(C.CDLL(path))
+        if _LIB is None:
+            if _build.stale():
+                _build.build()
+            _LIB = _bind(C.CDLL(_build.LIB))
+        return _LIB
+
+
+def _bind(lib):
+    lib.orc_threads.restype = _i
+    lib.orc_set_threads.argtypes = [_i]
+    lib.orc_cast_bf16.argtypes = [_p, _p, _i64]
+    lib.orc_quantize_affine.argtypes = [_p, _i, _i64, _i64, _i, _i, _p, _p, _p]
+    lib.orc_quantize_affine.restype = _i
+    lib.orc_dequantize.argtypes = [_p, _p, _p, _i, _i64, _i64, _i, _i, _p]
+    lib.orc_dequantize.restype = _i
+    lib.orc_qmm.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i, _p, _p]
+    lib.orc_qmm.restype = _i
+    lib.orc_qmm_sampled.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i,
+                                    _i64, _p, _p, _p, _p]
+    lib.orc_qmm_sampled.restype = _i
+    lib.orc_gather_qmm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _p,
+                                   _i, _i, _i, _i, _p, _p]
+    lib.orc_gather_qmm.restype = _i
+    lib.orc_gather_qmm_sampled.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p,
+                                           _p, _p, _i, _i, _i, _i, _i64, _p, _p, _p, _p]
+    lib.orc_gather_qmm_sampled.restype = _i
+    return lib
+
+
+def _cpu(t: torch.Tensor) -> torch.Tensor:
+    assert t.device.type == "cpu", "the oracle reads host tensors only"
+    return t.contiguous()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments")
+
+
+def threads() -> int:
+    return load().orc_threads()
+
+
+def set_threads(n: int):
+    load().orc_set_threads(n)
+
+
+def cast_bf16(x: torch.Tensor, lib=None) -> torch.Tensor:
+    """fp32 -> bf16 by the oracle's own round-to-nearest-even on the bits."""
+    lib = lib or load()
+    x = _cpu(x.to(torch.float32))
+    out = torch.empty(x.shape, dtype=torch.int16)
+    lib.orc_cast_bf16(x.data_ptr(), out.data_ptr(), x.numel())
+    return out.view(torch.bfloat16)
+
+
+def quantize_affine(w: torch.Tensor, group_size: int, bits: int, lib=None):
+    """Affine quantization of w [..., rows, cols] along cols.
+
+    Returns (codes uint32-as-int32 [..., rows, cols*bits/32], scales, biases
+    [..., rows, cols/group_size] in w's dtype)."""
+    lib = lib or load()
+    w = _cpu(w)
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    codes = torch.zeros(*w.shape[:-1], cols * bits // 32, dtype=torch.int32)
+    scales = torch.empty(*w.shape[:-1], cols // group_size, dtype=w.dtype)
+    biases = torch.empty_like(scales)
+    rc = lib.orc_quantize_affine(w.data_ptr(), _DT[w.dtype], rows, cols, group_size, bits,
+                                 codes.data_ptr(), scales.data_ptr(), biases.data_ptr())
+    _check(rc, "quantize_affine")
+    return codes, scales, biases
+
+
+def dequantize(codes, scales, biases, group_size: int, bits: int, lib=None) -> torch.Tensor:
+    """fp64 w_hat = scale * code + bias, shape [..., rows, cols]."""
+    lib = lib or load()
+    codes, scales, biases = _cpu(codes), _cpu(scales), _cpu(biases)
+    cols = codes.shape[-1] * 32 // bits
+    rows = codes.numel() // codes.shape[-1]
+    out = torch.empty(*codes.shape[:-1], cols, dtype=torch.float64)
+    rc = lib.orc_dequantize(codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                            _DT[scales.dtype], rows, cols, group_size, bits, out.data_ptr())
+    _check(rc, "dequantize")
+    return out
+
+
+def qmm(x, codes, scales, biases, group_size: int, bits: int, transpose: bool = True, lib=None):
+    """fp64 (y, a) for x [M, K]; weights [N, K] (transpose) or [K, N].
+
+    a = sum_k |x * w_hat| per output, the scale of the tolerance."""
+    lib = lib or load()
+    x, codes, scales, biases = _cpu(x), _cpu(codes), _cpu(scales), _cpu(biases)
+    M, K = x.shape
+    if transpose:
+        N = codes.shape[0]
+    else:
+        N = codes.shape[1] * 32 // bits
+    y = torch.empty(M, N, dtype=torch.float64)
+    a = torch.empty(M, N, dtype=torch.float64)
+    rc = lib.orc_qmm(x.data_ptr(), _DT[x.dtype], M, K, N, codes.data_ptr(), scales.data_ptr(),
+                     biases.data_ptr(), _DT[scales.dtype], group_size, bits, int(transpose),
+                     y.data_ptr(), a.data_ptr())
+    _check(rc, "qmm")
+    return y, a
+
+
+def qmm_sampled(x, codes, scales, biases, group_size, bits, transpose, m_idx, n_idx, lib=None):
+    """(y, a) at the positions (m_idx[s], n_idx[s]) only."""
+    lib = lib or load()
+    x, codes, scales, biases = _cpu(x), _cpu(codes), _cpu(scales), _cpu(biases)
+    M, K = x.shape
+    N = codes.shape[0] if transpose else codes.shape[1] * 32 // bits
+    m_idx = _cpu(torch.as_tensor(m_idx, dtype=torch.int64))
+    n_idx = _cpu(torch.as_tensor(n_idx, dtype=torch.int64))
+    S = m_idx.numel()
+    y = torch.empty(S, dtype=torch.float64)
+    a = torch.empty(S, dtype=torch.float64)
+    rc = lib.orc_qmm_sampled(x.data_ptr(), _DT[x.dtype], M, K, N, codes.data_ptr(),
+                             scales.data_ptr(), biases.data_ptr(), _DT[scales.dtype], group_size,
+                             bits, int(transpose), S, m_idx.data_ptr(), n_idx.data_ptr(),
+                             y.data_ptr(), a.data_ptr())
+    _check(rc, "qmm_sampled")
+    return y, a
+
+
+def _u32(t):
+    if t is None:
+        return None
+    return _cpu(torch.as_tensor(t).to(torch.int64).to(torch.int32))
+
+
+def gather_qmm(x, codes, scales, biases, lhs, rhs, group_size, bits, transpose=True, lib=None):
+    """fp64 (y, a) [R, N]: row r = x[lhs[r]] times expert rhs[r] (lhs None: identity)."""
+    lib = lib or load()
+    x, codes, scales, biases = _cpu(x), _cpu(codes), _cpu(scales), _cpu(biases)
+    x2 = x.reshape(-1, x.shape[-1])
+    x_rows, K = x2.shape
+    E = codes.shape[0]
+    N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    lhs_t, rhs_t = _u32(lhs), _u32(rhs)
+    R = rhs_t.numel()
+    y = torch.empty(R, N, dtype=torch.float64)
+    a = torch.empty(R, N, dtype=torch.float64)
+    rc = lib.orc_gather_qmm(x2.data_ptr(), _DT[x.dtype], x_rows, K,
+                            None if lhs_t is None else lhs_t.data_ptr(), rhs_t.data_ptr(), R, E, N,
+                            codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                            _DT[scales.dtype], group_size, bits, int(transpose), y.data_ptr(),
+                            a.data_ptr())
+    _check(rc, "gather_qmm")
+    return y, a
+
+
+def gather_qmm_sampled(x, codes, scales, biases, lhs, rhs, group_size, bits, transpose,
+                       r_idx, n_idx, lib=None):
+    lib = lib or load()
+    x, codes, scales, biases = _cpu(x), _cpu(codes), _cpu(scales), _cpu(biases)
+    x2 = x.reshape(-1, x.shape[-1])
+    x_rows, K = x2.shape
+    E = codes.shape[0]
+    N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    lhs_t, rhs_t = _u32(lhs), _u32(rhs)
+    R = rhs_t.numel()
+    r_idx = _cpu(torch.as_tensor(r_idx, dtype=torch.int64))
+    n_idx = _cpu(torch.as_tensor(n_idx, dtype=torch.int64))
+    S = r_idx.numel()
+    y = torch.empty(S, dtype=torch.float64)
+    a = torch.empty(S, dtype=torch.float64)
+    rc = lib.orc_gather_qmm_sampled(x2.data_ptr(), _DT[x.dtype], x_rows, K,
+                                    None if lhs_t is None else lhs_t.data_ptr(),
+                                    rhs_t.data_ptr(), R, E, N, codes.data_ptr(),
+                                    scales.data_ptr(), biases.data_ptr(), _DT[scales.dtype],
+                                    group_size, bits, int(transpose), S, r_idx.data_ptr(),
+                                    n_idx.data_ptr(), y.data_ptr(), a.data_ptr())
+    _check(rc, "gather_qmm_sampled")
+    return y, a
+
+
+# Acceptance bounds (spec tolerance): |y - y_ref| <= rel * a + 1e-5 with
+# rel = 4e-3 for bf16 activations and 1e-5 for fp32.
+TOL_REL = {torch.bfloat16: 4e-3, torch.float32: 1e-5}
+TOL_ABS = 1e-5
+
+
+def within_tolerance(y, y_ref, a, dtype) -> torch.Tensor:
+    """Element-wise acceptance mask of the product tolerance."""
+    err = (y.to(torch.float64) - y_ref).abs()
+    return err <= TOL_REL[dtype] * a + TOL_ABS

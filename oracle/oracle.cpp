@@ -1,0 +1,314 @@
+// Host oracle for group-wise affine quantization and the quantized products.
+//
+// TEST INFRASTRUCTURE ONLY. This file is the slow, plain CPU statement of what
+// the CUDA library computes. Only the tests, the smoke check and the bench's
+// CPU-baseline leg load it. It shares no code, header, table or helper with the
+// CUDA library, and the CUDA library never calls it.
+//
+// Sources (nuvec documentation pages):
+//   [Q-Affine]   "Docs / Quantization", section "Affine": groups of group_size
+//                values along each row, one scale and one bias per group,
+//                bits-wide integer codes packed into uint32 words,
+//                w ~= scale * code + bias; 4-bit/g64 is about 4.5 bits/weight.
+//   [Q-Example]  same section, the example: quantize W [out, in], then
+//                quantized_matmul(q, transpose=true) is x . w^T.
+//   [Q-Products] "Docs / Quantization", section "Products on the GPU".
+//   [Q-MoE]      "Docs / Quantization", section "Mixture of experts":
+//                gather_qmm multiplies each row by the expert chosen for it.
+//   [Crate-Quantized] nuvec crate docs, "Structs": Quantized holds uint32
+//                codes, one scale per group in the weights' dtype, biases.
+//
+// What the pages leave open, and the reading taken here (all listed in the
+// design notes):
+//   * quantizer arithmetic: scale = (max - min) / (2^bits - 1), bias = min,
+//     code = clamp(round((w - bias) / scale), 0, 2^bits - 1), every step an
+//     IEEE fp32 operation (subtract, divide) rounded to nearest-even;
+//   * round() is round-half-to-even (the IEEE default mode);
+//   * the codes use the unrounded fp32 scale and bias; the stored scale and
+//     bias are then cast to the weights' dtype (bf16: round-to-nearest-even);
+//   * a constant group (scale == 0) gets code 0 everywhere;
+//   * code j of a uint32 word sits at bits [j*bits, (j+1)*bits);
+//   * the product's reference value is the fp64 dot of x with the dequantized
+//     weights (stored scale and bias), summed in k order.
+//
+// Pins: every function here is checked in tests/test_oracle_pins.py against
+// closed forms and brute force (hand-built integer groups, pack words written
+// out from the bit definition, exact integer products, the round-trip bound).
+//
+// Build: g++ -O2 -ffp-contract=off -fopenmp -fPIC -shared (no fast-math): fp32
+// arithmetic on x86-64 is SSE, so each float operation rounds once, as IEEE
+// specifies. Output elements are computed independently and each sum runs in
+// k order, so results do not depend on the thread count.
+
+#include <cstdint>
+#include <cstring>
+#include <cmath>
+#include <cfenv>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+enum { DT_F32 = 0, DT_BF16 = 1 };
+
+// ---- storage dtypes ------------------------------------------------------
+
+// bf16 is the upper half of an fp32 bit pattern: widening is exact.
+double load_value(const void* base, int dtype, int64_t i) {
+    if (dtype == DT_F32) return (double)((const float*)base)[i];
+    uint32_t bits = (uint32_t)((const uint16_t*)base)[i] << 16;
+    float f;
+    std::memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+float load_f32(const void* base, int dtype, int64_t i) {
+    return (float)load_value(base, dtype, i);
+}
+
+// Narrow fp32 to bf16 by rounding the fp32 bit pattern to nearest, ties to
+// even, at bit 16 (plain integer rounding on the bits; finite inputs).
+uint16_t f32_to_bf16(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    uint32_t keep = u >> 16;
+    uint32_t rest = u & 0xFFFFu;
+    if (rest > 0x8000u || (rest == 0x8000u && (keep & 1u))) keep += 1;
+    return (uint16_t)keep;
+}
+
+void store_value(void* base, int dtype, int64_t i, float v) {
+    if (dtype == DT_F32) ((float*)base)[i] = v;
+    else ((uint16_t*)base)[i] = f32_to_bf16(v);
+}
+
+// ---- packing [Q-Affine]: code j of a word at bits [j*bits, (j+1)*bits) ----
+
+int64_t words_per_row(int64_t cols, int bits) { return cols * bits / 32; }
+
+uint32_t code_at(const uint32_t* codes, int64_t row, int64_t col, int64_t cols, int bits) {
+    const int per_word = 32 / bits;
+    uint32_t word = codes[row * words_per_row(cols, bits) + col / per_word];
+    int j = (int)(col % per_word);
+    return (word >> (j * bits)) & ((1u << bits) - 1u);
+}
+
+// ---- dequantize [Q-Affine]: w_hat = scale * code + bias, in fp64 ----------
+
+double dequant_at(const uint32_t* codes, const void* scales, const void* biases, int sdtype,
+                  int64_t row, int64_t col, int64_t cols, int gs, int bits) {
+    int64_t g = row * (cols / gs) + col / gs;
+    double s = load_value(scales, sdtype, g);
+    double b = load_value(biases, sdtype, g);
+    return s * (double)code_at(codes, row, col, cols, bits) + b;
+}
+
+bool valid_quant(int64_t cols, int gs, int bits) {
+    if (gs != 32 && gs != 64 && gs != 128) return false;
+    if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return false;
+    return cols > 0 && cols % gs == 0;
+}
+
+// One output element of a product: sum_k x[k] * w_hat(k), sequential in k.
+// transpose = 1: the weights are stored [N, K] (row n holds output n).
+// transpose = 0: the weights are stored [K, N] (row k), grouped along N.
+void dot_one(const void* x_row, int xdtype, int64_t K, int64_t N, int64_t n,
+             const uint32_t* codes, const void* scales, const void* biases, int sdtype,
+             int gs, int bits, int transpose, double* y, double* a) {
+    double acc = 0.0, mag = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double xv = load_value(x_row, xdtype, k);
+        double wv = transpose ? dequant_at(codes, scales, biases, sdtype, n, k, K, gs, bits)
+                              : dequant_at(codes, scales, biases, sdtype, k, n, N, gs, bits);
+        double p = xv * wv;
+        acc += p;
+        mag += std::fabs(p);
+    }
+    *y = acc;
+    *a = mag;
+}
+
+const void* row_ptr(const void* base, int dtype, int64_t row, int64_t len) {
+    size_t esz = dtype == DT_F32 ? 4 : 2;
+    return (const char*)base + (size_t)row * (size_t)len * esz;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orc_threads() {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+// fp32 -> bf16 bit patterns, round to nearest even.
+void orc_cast_bf16(const float* in, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16(in[i]);
+}
+
+// Affine quantizer [Q-Affine, Q-Example, Crate-Quantized].
+// w [rows, cols] in `dtype` (0 = fp32, 1 = bf16), grouped along cols.
+// Writes codes [rows, cols*bits/32] uint32 and scales/biases
+// [rows, cols/group_size] in `dtype`. Returns 0, or -1 on bad arguments.
+int orc_quantize_affine(const void* w, int dtype, int64_t rows, int64_t cols, int gs,
+                        int bits, uint32_t* codes, void* scales, void* biases) {
+    if (!valid_quant(cols, gs, bits) || rows < 0) return -1;
+    if (std::fegetround() != FE_TONEAREST) return -1;
+    const int64_t groups = cols / gs;
+    const int per_word = 32 / bits;
+    const float levels = (float)((1u << bits) - 1u);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const int64_t c0 = g * gs;
+            // Step 1: the group's minimum and maximum.
+            float mn = load_f32(w, dtype, r * cols + c0), mx = mn;
+            for (int i = 1; i < gs; ++i) {
+                float v = load_f32(w, dtype, r * cols + c0 + i);
+                if (v < mn) mn = v;
+                if (v > mx) mx = v;
+            }
+            // Step 2: scale spreads the range over the 2^bits - 1 steps; bias = min.
+            float range = mx - mn;
+            float scale = range / levels;
+            float bias = mn;
+            // Step 3: one code per value, round-half-even, clamped.
+            for (int i = 0; i < gs; ++i) {
+                uint32_t q = 0;
+                if (scale != 0.0f) {
+                    float v = load_f32(w, dtype, r * cols + c0 + i);
+                    float t = (v - bias) / scale;
+                    float rq = std::nearbyint(t);
+                    if (rq < 0.0f) rq = 0.0f;
+                    if (rq > levels) rq = levels;
+                    q = (uint32_t)rq;
+                }
+                // Step 4: pack code (c0 + i) into its word.
+                int64_t col = c0 + i;
+                int64_t wi = r * words_per_row(cols, bits) + col / per_word;
+                int j = (int)(col % per_word);
+                if (j == 0) codes[wi] = 0u;
+                codes[wi] |= q << (j * bits);
+            }
+            // Step 5: store scale and bias in the weights' dtype.
+            store_value(scales, dtype, r * groups + g, scale);
+            store_value(biases, dtype, r * groups + g, bias);
+        }
+    }
+    return 0;
+}
+
+// Dequantize to fp64: out[r, c] = scale * code + bias [Q-Affine].
+int orc_dequantize(const uint32_t* codes, const void* scales, const void* biases, int sdtype,
+                   int64_t rows, int64_t cols, int gs, int bits, double* out) {
+    if (!valid_quant(cols, gs, bits)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = dequant_at(codes, scales, biases, sdtype, r, c, cols, gs, bits);
+    return 0;
+}
+
+// Quantized product [Q-Example, Q-Products]: y[m, n] = sum_k x[m, k] * w_hat(n, k)
+// with transpose = 1 (weights [N, K]); transpose = 0 uses weights [K, N].
+// Also returns a[m, n] = sum_k |x[m, k] * w_hat|, the scale of the tolerance.
+int orc_qmm(const void* x, int xdtype, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+            const void* scales, const void* biases, int sdtype, int gs, int bits, int transpose,
+            double* y, double* a) {
+    if (!valid_quant(transpose ? K : N, gs, bits)) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            dot_one(row_ptr(x, xdtype, m, K), xdtype, K, N, n, codes, scales, biases, sdtype,
+                    gs, bits, transpose, &y[m * N + n], &a[m * N + n]);
+    return 0;
+}
+
+// The same product at S chosen output positions (m_idx[s], n_idx[s]) only.
+int orc_qmm_sampled(const void* x, int xdtype, int64_t M, int64_t K, int64_t N,
+                    const uint32_t* codes, const void* scales, const void* biases, int sdtype,
+                    int gs, int bits, int transpose, int64_t S, const int64_t* m_idx,
+                    const int64_t* n_idx, double* y, double* a) {
+    if (!valid_quant(transpose ? K : N, gs, bits)) return -1;
+    for (int64_t s = 0; s < S; ++s)
+        if (m_idx[s] < 0 || m_idx[s] >= M || n_idx[s] < 0 || n_idx[s] >= N) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < S; ++s)
+        dot_one(row_ptr(x, xdtype, m_idx[s], K), xdtype, K, N, n_idx[s], codes, scales, biases,
+                sdtype, gs, bits, transpose, &y[s], &a[s]);
+    return 0;
+}
+
+// Mixture-of-experts product [Q-MoE]: for each pair r, output row r is
+// x[lhs[r]] times expert rhs[r]'s weights (experts stored [E, N, K] with
+// transpose = 1, or [E, K, N] with transpose = 0). lhs may be null (identity).
+// Returns -1 if an index is out of range.
+int orc_gather_qmm(const void* x, int xdtype, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                   const uint32_t* rhs, int64_t R, int64_t E, int64_t N, const uint32_t* codes,
+                   const void* scales, const void* biases, int sdtype, int gs, int bits,
+                   int transpose, double* y, double* a) {
+    if (!valid_quant(transpose ? K : N, gs, bits)) return -1;
+    for (int64_t r = 0; r < R; ++r) {
+        int64_t t = lhs ? (int64_t)lhs[r] : r;
+        if (t >= x_rows || (int64_t)rhs[r] >= E) return -1;
+    }
+    const int64_t words_e = N * K * bits / 32;
+    const int64_t groups_e = N * K / gs;
+    const size_t sz = sdtype == DT_F32 ? 4 : 2;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t t = lhs ? (int64_t)lhs[r] : r;
+            int64_t e = (int64_t)rhs[r];
+            dot_one(row_ptr(x, xdtype, t, K), xdtype, K, N, n, codes + e * words_e,
+                    (const char*)scales + (size_t)(e * groups_e) * sz,
+                    (const char*)biases + (size_t)(e * groups_e) * sz, sdtype, gs, bits,
+                    transpose, &y[r * N + n], &a[r * N + n]);
+        }
+    return 0;
+}
+
+// The same gather at S chosen (pair, output) positions.
+int orc_gather_qmm_sampled(const void* x, int xdtype, int64_t x_rows, int64_t K,
+                           const uint32_t* lhs, const uint32_t* rhs, int64_t R, int64_t E,
+                           int64_t N, const uint32_t* codes, const void* scales,
+                           const void* biases, int sdtype, int gs, int bits, int transpose,
+                           int64_t S, const int64_t* r_idx, const int64_t* n_idx, double* y,
+                           double* a) {
+    if (!valid_quant(transpose ? K : N, gs, bits)) return -1;
+    for (int64_t s = 0; s < S; ++s) {
+        int64_t r = r_idx[s];
+        if (r < 0 || r >= R || n_idx[s] < 0 || n_idx[s] >= N) return -1;
+        int64_t t = lhs ? (int64_t)lhs[r] : r;
+        if (t >= x_rows || (int64_t)rhs[r] >= E) return -1;
+    }
+    const int64_t words_e = N * K * bits / 32;
+    const int64_t groups_e = N * K / gs;
+    const size_t sz = sdtype == DT_F32 ? 4 : 2;
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < S; ++s) {
+        int64_t r = r_idx[s];
+        int64_t t = lhs ? (int64_t)lhs[r] : r;
+        int64_t e = (int64_t)rhs[r];
+        dot_one(row_ptr(x, xdtype, t, K), xdtype, K, N, n_idx[s], codes + e * words_e,
+                (const char*)scales + (size_t)(e * groups_e) * sz,
+                (const char*)biases + (size_t)(e * groups_e) * sz, sdtype, gs, bits, transpose,
+                &y[s], &a[s]);
+    }
+    return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,355 @@
+"""Pins of the host oracle: facts fixed by the pages and by mathematics, not by
+the oracle itself.
+
+Each ``pin_*`` takes a loaded oracle library (ctypes handle) and raises
+AssertionError when the oracle disagrees with the fact. test_oracle_pins.py runs
+them on the real oracle; test_oracle_mutations.py runs them on copies of the
+oracle with a planted mistake and expects at least one pin to fail each time.
+
+Sources: "Docs / Quantization" (sections "Affine", "Mixture of experts") and
+the nuvec crate docs ("Structs": Quantized).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------------------
+# golden fixture readers
+# ---------------------------------------------------------------------------
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield [p.strip() for p in line.split("|")]
+
+
+def pack_word_cases():
+    for bits, codes, word in _rows("pack_words.txt"):
+        yield int(bits), [int(c) for c in codes.split()], int(word, 16)
+
+
+def handbuilt_cases():
+    for name, bits, gs, vals, scale, bias, codes in _rows("handbuilt_groups.txt"):
+        yield (name, int(bits), int(gs), [float(v) for v in vals.split()], float(scale),
+               float(bias), [int(c) for c in codes.split()])
+
+
+def _cycle(vals, n):
+    return [vals[i % len(vals)] for i in range(n)]
+
+
+def _u32(t):
+    return t.to(torch.int64) & 0xFFFFFFFF
+
+
+def _unpack_div_mod(words: torch.Tensor, bits: int) -> torch.Tensor:
+    """Codes from packed words by integer division and remainder (no shifts, no
+    masks): code j of word w is floor(w / 2^(j*bits)) mod 2^bits."""
+    per = 32 // bits
+    w = _u32(words).tolist()
+    out = []
+    for row in w:
+        r = []
+        for word in row:
+            for j in range(per):
+                r.append((word // (2 ** (j * bits))) % (2 ** bits))
+        out.append(r)
+    return torch.tensor(out, dtype=torch.int64)
+
+
+def _groups_with_extremes(rows, cols, gs, bits, gen):
+    """Integer weights in [0, 2^b-1] where every group along a row holds both 0
+    and 2^b-1, so the quantizer must return scale 1, bias 0 and code = weight."""
+    hi = 2 ** bits - 1
+    w = torch.randint(0, hi + 1, (rows, cols), generator=gen)
+    for g in range(cols // gs):
+        pos = torch.randperm(gs, generator=gen)[:2] + g * gs
+        w[:, pos[0]] = 0
+        w[:, pos[1]] = hi
+    return w
+
+
+# ---------------------------------------------------------------------------
+# pins
+# ---------------------------------------------------------------------------
+def pin_pack_words(lib):
+    """Hand-written words: a group holding the word's codes (plus 0 and the top
+    code, so scale is 1 and bias 0) must pack into exactly that word."""
+    for bits, codes, word in pack_word_cases():
+        gs = 32 if bits >= 2 else 32
+        per = 32 // bits
+        hi = 2 ** bits - 1
+        vals = list(codes) + [0, hi] * ((gs - per) // 2) if per < gs else list(codes)
+        vals = vals[:gs] + [0] * (gs - len(vals))
+        if per == gs:  # the word is the whole group: it must hold 0 and hi itself
+            assert 0 in codes and hi in codes, "fixture needs 0 and the top code"
+        w = torch.tensor([vals], dtype=torch.float32)
+        c, s, b = O.quantize_affine(w, gs, bits, lib=lib)
+        assert float(s[0, 0]) == 1.0 and float(b[0, 0]) == 0.0, (bits, codes)
+        got = int(_u32(c)[0, 0])
+        assert got == word, f"bits={bits} codes={codes}: {got:#010x} != {word:#010x}"
+
+
+def pin_unpack_words(lib):
+    """Dequantizing a hand-written word with scale 1 and bias 0 returns its codes."""
+    for bits, codes, word in pack_word_cases():
+        gs = 32
+        words = torch.zeros(1, gs * bits // 32, dtype=torch.int32)
+        words[0, 0] = word - 2 ** 32 if word >= 2 ** 31 else word
+        ones = torch.ones(1, 1)
+        zeros = torch.zeros(1, 1)
+        wh = O.dequantize(words, ones, zeros, gs, bits, lib=lib)
+        assert wh[0, :len(codes)].tolist() == [float(c) for c in codes], (bits, codes)
+
+
+def pin_handbuilt_groups(lib):
+    """Hand-built groups (golden/handbuilt_groups.txt): exact scale, bias, codes,
+    for fp32 storage, and through bf16 storage where every number is bf16-exact."""
+    for name, bits, gs, vals, scale, bias, codes in handbuilt_cases():
+        for dt in (torch.float32, torch.bfloat16):
+            w = torch.tensor([_cycle(vals, gs), _cycle(vals[::-1], gs)], dtype=torch.float32)
+            assert torch.equal(w.to(dt).to(torch.float32), w), name
+            c, s, b = O.quantize_affine(w.to(dt), gs, bits, lib=lib)
+            got = _unpack_div_mod(c, bits)
+            assert s.to(torch.float32).tolist() == [[scale], [scale]], (name, dt, s)
+            assert b.to(torch.float32).tolist() == [[bias], [bias]], (name, dt, b)
+            assert got[0].tolist() == _cycle(codes, gs), (name, dt)
+            assert got[1].tolist() == _cycle(codes[::-1], gs), (name, dt)
+
+
+def pin_bf16_cast(lib):
+    """The oracle's fp32 -> bf16 rounding equals torch's round-to-nearest-even
+    cast (a library routine), including exact ties."""
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(4096, generator=g) * torch.logspace(-20, 20, 4096)
+    ties = torch.tensor([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2 ** -100 * (1 + 2 ** -8),
+                         3.0, 0.0, -0.0, 65504.0], dtype=torch.float32)
+    x = torch.cat([x, ties])
+    got = O.cast_bf16(x, lib=lib)
+    ref = x.to(torch.bfloat16)
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert float(got[4096]) == 1.0 and float(got[4097]) == 1 + 2 ** -6
+
+
+def pin_stored_scale_is_bf16_rounding(lib):
+    """bf16 weights store scale = bf16(fp32((max-min)/(2^b-1))): range 1 at 4 bits
+    gives 1/15 in fp32, stored rounded to bf16 (the weights' dtype)."""
+    vals = [0.0, 1.0] + [0.5] * 62
+    w = torch.tensor([vals]).to(torch.bfloat16)
+    c, s, b = O.quantize_affine(w, 64, 4, lib=lib)
+    want = (torch.tensor(1.0, dtype=torch.float32) / torch.tensor(15.0)).to(torch.bfloat16)
+    assert s.dtype == torch.bfloat16 and s[0, 0].view(torch.int16) == want.view(torch.int16)
+    assert float(b[0, 0]) == 0.0
+    # the code of 0.5 is rne(0.5 / fp32(1/15)) = rne(7.4999998...) = 7
+    assert _unpack_div_mod(c, 4)[0, 2] == 7
+
+
+def pin_extremes_and_range(lib):
+    """On random data every group's minimum gets code 0, its maximum the top code,
+    and every code lies in [0, 2^b - 1]."""
+    g = torch.Generator().manual_seed(3)
+    for bits in (1, 2, 4, 8):
+        for gs in (32, 64, 128):
+            w = torch.randn(16, 256, generator=g)
+            c, s, b = O.quantize_affine(w, gs, bits, lib=lib)
+            q = _unpack_div_mod(c, bits).reshape(16, 256 // gs, gs)
+            wg = w.reshape(16, 256 // gs, gs)
+            amin = wg.argmin(-1, keepdim=True)
+            amax = wg.argmax(-1, keepdim=True)
+            assert (q.gather(-1, amin) == 0).all(), (bits, gs)
+            assert (q.gather(-1, amax) == 2 ** bits - 1).all(), (bits, gs)
+            assert q.min() >= 0 and q.max() <= 2 ** bits - 1
+            # bias is the group minimum, scale the range over the step count
+            assert torch.equal(b.reshape(16, -1), wg.min(-1).values)
+
+
+def pin_round_trip_bound(lib):
+    """|w_hat - w| <= scale/2 (+ fp32 rounding of the division and, for bf16
+    storage, the cast of scale and bias) on random data at every width."""
+    g = torch.Generator().manual_seed(5)
+    for dt in (torch.float32, torch.bfloat16):
+        for bits in (1, 2, 4, 8):
+            for gs in (32, 64, 128):
+                w = (torch.randn(32, 512, generator=g) * 0.02).to(dt)
+                c, s, b = O.quantize_affine(w, gs, bits, lib=lib)
+                wh = O.dequantize(c, s, b, gs, bits, lib=lib)
+                w64 = w.to(torch.float64).reshape(32, -1, gs)
+                wg = w.to(torch.float32).reshape(32, -1, gs)
+                scale_f = ((wg.max(-1).values - wg.min(-1).values) / (2 ** bits - 1)).to(torch.float64)
+                bound = 0.5 * scale_f * (1 + 2 ** -20) + 2 ** -23 * w64.abs().amax(-1)
+                if dt == torch.bfloat16:
+                    bias_abs = b.to(torch.float64).reshape(32, -1).abs()
+                    bound = bound + 2 ** -8 * (bias_abs + (2 ** bits - 1) * scale_f)
+                err = (wh.reshape(32, -1, gs) - w64).abs().amax(-1)
+                assert (err <= bound).all(), (dt, bits, gs, float((err - bound).max()))
+
+
+def pin_bits_per_weight(lib):
+    """4-bit, groups of 64, 16-bit scale and bias: 4.5 bits per weight; with fp32
+    scale and bias (the tiny workload) 5 bits per weight."""
+    w = torch.randn(8, 1024)
+    for dt, want in ((torch.bfloat16, 4.5), (torch.float32, 5.0)):
+        c, s, b = O.quantize_affine(w.to(dt), 64, 4, lib=lib)
+        total_bits = 8 * (c.numel() * 4 + s.numel() * s.element_size() + b.numel() * b.element_size())
+        assert total_bits / w.numel() == want
+
+
+def pin_integer_products(lib):
+    """Integer-valued groups (scale 1, bias 0) and integer x: the quantized product
+    is an integer matmul, computed exactly by torch int64 matmul; both layouts."""
+    gen = torch.Generator().manual_seed(11)
+    for bits in (1, 2, 4, 8):
+        for gs in (32, 64, 128):
+            N, K, M = 24, 256, 5
+            wi = _groups_with_extremes(N, K, gs, bits, gen)
+            xi = torch.randint(-2, 3, (M, K), generator=gen)
+            for dt in (torch.float32, torch.bfloat16):
+                c, s, b = O.quantize_affine(wi.to(dt), gs, bits, lib=lib)
+                y, a = O.qmm(xi.to(dt), c, s, b, gs, bits, True, lib=lib)
+                exact = xi @ wi.T
+                assert torch.equal(y, exact.to(torch.float64)), (bits, gs, dt)
+                assert torch.equal(a, (xi.abs() @ wi.T).to(torch.float64))
+            # transpose = 0: weights stored [K, N], grouped along N
+            wt = _groups_with_extremes(K, 256, gs, bits, gen)
+            c, s, b = O.quantize_affine(wt.to(torch.float32), gs, bits, lib=lib)
+            y, a = O.qmm(xi.to(torch.float32), c, s, b, gs, bits, False, lib=lib)
+            assert torch.equal(y, (xi @ wt).to(torch.float64)), (bits, gs, "transpose=0")
+
+
+def pin_affine_integer_products(lib):
+    """w = 2*code - 5 per group: scale 2 and bias -5 are exact, so the product
+    must equal x @ (2*c - 5)^T exactly (the bias term and its sign)."""
+    gen = torch.Generator().manual_seed(13)
+    N, K, M, gs, bits = 16, 128, 3, 32, 4
+    ci = _groups_with_extremes(N, K, gs, bits, gen)
+    w = (2 * ci - 5).to(torch.float32)
+    c, s, b = O.quantize_affine(w, gs, bits, lib=lib)
+    assert (s == 2).all() and (b == -5).all()
+    xi = torch.randint(-3, 4, (M, K), generator=gen)
+    y, _ = O.qmm(xi.to(torch.float32), c, s, b, gs, bits, True, lib=lib)
+    assert torch.equal(y, (xi @ (2 * ci - 5).T).to(torch.float64))
+
+
+def pin_brute_force_8x8(lib):
+    """An 8x8 output (M = 8, N = 8, K = 2 groups) on random data against a
+    brute-force sum: codes unpacked by division and remainder, scale and bias
+    read back from storage, products summed exactly (math.fsum)."""
+    g = torch.Generator().manual_seed(17)
+    for dt in (torch.float32, torch.bfloat16):
+        for bits, gs in ((4, 64), (2, 32), (8, 64), (4, 128)):
+            K = 2 * gs
+            w = torch.randn(8, K, generator=g).to(dt)
+            x = torch.randn(8, K, generator=g).to(dt)
+            c, s, b = O.quantize_affine(w, gs, bits, lib=lib)
+            q = _unpack_div_mod(c, bits)
+            sv = s.to(torch.float64).tolist()
+            bv = b.to(torch.float64).tolist()
+            xv = x.to(torch.float64).tolist()
+            y, a = O.qmm(x, c, s, b, gs, bits, True, lib=lib)
+            for m in range(8):
+                for n in range(8):
+                    terms = [xv[m][k] * (sv[n][k // gs] * int(q[n, k]) + bv[n][k // gs])
+                             for k in range(K)]
+                    exact = math.fsum(terms)
+                    mag = math.fsum(abs(t) for t in terms)
+                    assert abs(float(y[m, n]) - exact) <= 1e-13 * mag + 1e-300, (dt, bits, gs, m, n)
+                    assert abs(float(a[m, n]) - mag) <= 1e-13 * mag
+
+
+def pin_scaling_invariant(lib):
+    """y(2^j x) == 2^j y(x) exactly (power-of-two scaling is exact in fp64)."""
+    g = torch.Generator().manual_seed(19)
+    w = torch.randn(32, 256, generator=g)
+    x = torch.randn(3, 256, generator=g)
+    c, s, b = O.quantize_affine(w, 64, 4, lib=lib)
+    y1, _ = O.qmm(x, c, s, b, 64, 4, True, lib=lib)
+    y8, _ = O.qmm(x * 8, c, s, b, 64, 4, True, lib=lib)
+    assert torch.equal(y8, 8 * y1)
+
+
+def pin_transpose_layouts_agree(lib):
+    """The same integer weight matrix stored [N, K] (grouped along K) and stored
+    transposed [K, N] (grouped along N) gives the same product x @ W^T. Values:
+    0 where (n + k) % gs == 0, the top code where it is 1, random elsewhere, so
+    every group of either grouping holds both extremes (scale 1, bias 0)."""
+    gen = torch.Generator().manual_seed(23)
+    gs, bits, n = 32, 4, 96
+    W = torch.randint(0, 16, (n, n), generator=gen)
+    diag = (torch.arange(n)[:, None] + torch.arange(n)[None, :]) % gs
+    W[diag == 0] = 0
+    W[diag == 1] = 15
+    x = torch.randint(-2, 3, (4, n), generator=gen)
+    c1, s1, b1 = O.quantize_affine(W.to(torch.float32), gs, bits, lib=lib)
+    c2, s2, b2 = O.quantize_affine(W.T.contiguous().to(torch.float32), gs, bits, lib=lib)
+    y1, _ = O.qmm(x.float(), c1, s1, b1, gs, bits, True, lib=lib)
+    y2, _ = O.qmm(x.float(), c2, s2, b2, gs, bits, False, lib=lib)
+    assert torch.equal(y1, (x @ W.T).double()) and torch.equal(y2, y1)
+
+
+def pin_gather(lib):
+    """gather_qmm on the page's example shapes (q from [8,128,256], x [4,1,256],
+    experts [0,0,3,5] -> y [4,128]) equals each row times its expert's
+    dequantized weights; lhs selects the x row; out-of-range ids are refused."""
+    g = torch.Generator().manual_seed(29)
+    for dt in (torch.float32, torch.bfloat16):
+        w = torch.randn(8, 128, 256, generator=g).to(dt)
+        x = torch.randn(4, 1, 256, generator=g).to(dt)
+        c, s, b = O.quantize_affine(w, 64, 4, lib=lib)
+        ids = torch.tensor([0, 0, 3, 5])
+        y, a = O.gather_qmm(x, c, s, b, None, ids, 64, 4, True, lib=lib)
+        assert tuple(y.shape) == (4, 128)
+        wh = O.dequantize(c, s, b, 64, 4, lib=lib)  # [8, 128, 256] fp64
+        x2 = x.reshape(4, 256).to(torch.float64)
+        for r in range(4):
+            ref = wh[int(ids[r])] @ x2[r]
+            mag = wh[int(ids[r])].abs() @ x2[r].abs()
+            assert ((y[r] - ref).abs() <= 1e-12 * mag).all(), (dt, r)
+        # lhs picks rows of x; pairs (token, expert)
+        lhs = torch.tensor([3, 1, 1, 0, 2])
+        rhs = torch.tensor([7, 2, 6, 6, 0])
+        y2, _ = O.gather_qmm(x, c, s, b, lhs, rhs, 64, 4, True, lib=lib)
+        for r in range(5):
+            ref = wh[int(rhs[r])] @ x2[int(lhs[r])]
+            assert ((y2[r] - ref).abs() <= 1e-12 * (wh[int(rhs[r])].abs() @ x2[int(lhs[r])].abs())).all()
+        # all rows on expert 5: the gather is a plain quantized product with expert 5
+        y3, _ = O.gather_qmm(x, c, s, b, None, torch.full((4,), 5), 64, 4, True, lib=lib)
+        y4, _ = O.qmm(x.reshape(4, 256), c[5], s[5], b[5], 64, 4, True, lib=lib)
+        assert torch.equal(y3, y4)
+    try:
+        O.gather_qmm(x, c, s, b, None, torch.tensor([0, 8, 1, 1]), 64, 4, True, lib=lib)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("expert id 8 of 8 experts accepted")
+
+
+def pin_sampled_match_full(lib):
+    """The sampled product entry points agree with the full ones."""
+    g = torch.Generator().manual_seed(31)
+    w = torch.randn(40, 256, generator=g).to(torch.bfloat16)
+    x = torch.randn(6, 256, generator=g).to(torch.bfloat16)
+    c, s, b = O.quantize_affine(w, 64, 4, lib=lib)
+    y, a = O.qmm(x, c, s, b, 64, 4, True, lib=lib)
+    mi = torch.tensor([0, 5, 3, 3])
+    ni = torch.tensor([0, 39, 17, 18])
+    ys, as_ = O.qmm_sampled(x, c, s, b, 64, 4, True, mi, ni, lib=lib)
+    assert torch.equal(ys, y[mi, ni]) and torch.equal(as_, a[mi, ni])
+    we = torch.randn(3, 40, 256, generator=g).to(torch.bfloat16)
+    c, s, b = O.quantize_affine(we, 64, 4, lib=lib)
+    lhs, rhs = torch.tensor([0, 1, 5, 5]), torch.tensor([2, 0, 1, 2])
+    y, a = O.gather_qmm(x, c, s, b, lhs, rhs, 64, 4, True, lib=lib)
+    ri, ni = torch.tensor([3, 0, 2]), torch.tensor([1, 39, 20])
+    ys, as_ = O.gather_qmm_sampled(x, c, s, b, lhs, rhs, 64, 4, True, ri, ni, lib=lib)
+    assert torch.equal(ys, y[ri, ni]) and torch.equal(as_, a[ri, ni])
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
