@@ -1,0 +1,156 @@
+/*
+ * nvq.h: C ABI of the group-wise affine quantized products for NVIDIA B200 (sm_100a).
+ *
+ * The format (nuvec documentation, "Docs / Quantization", section "Affine"):
+ * each row of a weight matrix is cut into groups of group_size consecutive
+ * values (32, 64 or 128). Each group has one scale and one bias, and each value
+ * becomes an integer code of `bits` bits packed into uint32 words, so that
+ *     w ~= scale * code + bias.
+ * Code j of a word sits at bits [j*bits, (j+1)*bits). Scales and biases have
+ * the weights' dtype (nuvec crate docs, "Structs": Quantized). This library
+ * supports bits 2, 4 and 8.
+ *
+ * Layouts (all dense, row-major, no padding):
+ *   weights [rows, cols], grouped along cols:
+ *     codes  uint32 [rows, cols * bits / 32]
+ *     scales dtype  [rows, cols / group_size]
+ *     biases dtype  [rows, cols / group_size]
+ *   For products, transpose = 1 means the weights are stored [N, K] (row n holds
+ *   output feature n, grouped along K) and y = x . w^T; transpose = 0 means they
+ *   are stored [K, N], grouped along N, and y = x . w.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer (unless stated otherwise) owned
+ *     by the caller; the library allocates no device memory, keeps no state
+ *     between calls and never synchronises the stream. All work is enqueued on
+ *     `stream` (NULL = the legacy default stream), in call order.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Argument errors are found on the host before anything is launched and
+ *     are returned synchronously: NV_ERR_INVALID_ARG (a shape, pointer or
+ *     alignment is wrong), NV_ERR_UNSUPPORTED (a valid-looking combination this
+ *     library does not implement, e.g. bits = 3), NV_ERR_WORKSPACE (too small).
+ *     A failed launch returns NV_ERR_CUDA. Nothing traps on the device: data
+ *     errors found while running (an expert id out of range) set flag bits that
+ *     nv_gather_qmm_flags reads.
+ *   - Results are deterministic: the same call on the same inputs gives the same
+ *     bits, run to run (nuvec crate docs, section "Determinism").
+ */
+#ifndef NVQ_H
+#define NVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* The same type as cudaStream_t. */
+typedef struct CUstream_st* nv_stream_t;
+
+typedef enum nv_status {
+    NV_OK = 0,
+    NV_ERR_INVALID_ARG = 1,
+    NV_ERR_UNSUPPORTED = 2,
+    NV_ERR_WORKSPACE = 3,
+    NV_ERR_CUDA = 4
+} nv_status;
+
+typedef enum nv_dtype {
+    NV_F32 = 0,  /* IEEE binary32 */
+    NV_BF16 = 1  /* bfloat16 */
+} nv_dtype;
+
+/* Products with at most this many rows give each row the bits of its one-row
+ * product under row_exact (nuvec crate docs: constant ROW_INDEPENDENT_ROWS and
+ * function with_row_exact; "Docs / Quantization", section "Products on the
+ * GPU": "up to 8 rows"). */
+#define NV_ROW_INDEPENDENT_ROWS 8
+
+/* Device anomaly flags written by nv_gather_qmm into its workspace. */
+#define NV_FLAG_EXPERT_OUT_OF_RANGE 0x1u /* an rhs id >= E: that row's output is zero */
+#define NV_FLAG_NOT_SORTED 0x2u          /* sorted = 1 but rhs ids decrease somewhere */
+#define NV_FLAG_TOKEN_OUT_OF_RANGE 0x4u  /* an lhs id >= x_rows: that row's output is zero */
+
+/* Readable text for a status code (static storage, never NULL). */
+const char* nv_status_string(nv_status s);
+
+/*
+ * Affine quantizer ("Docs / Quantization", section "Affine", and its example
+ * w.quantize(Quant::affine(64, 4))).
+ *
+ * w       [rows, cols] in `dt` (NV_F32 or NV_BF16), grouped along cols.
+ * codes   uint32 [rows, cols * bits / 32] (output).
+ * scales, biases  `dt` [rows, cols / group_size] (outputs).
+ * Per group, in IEEE fp32 with round-to-nearest-even at every step:
+ *   scale = (max - min) / (2^bits - 1), bias = min,
+ *   code  = clamp(round_half_even((w - bias) / scale), 0, 2^bits - 1),
+ *   a constant group (scale == 0) gets code 0; scale and bias are stored in
+ *   `dt` (bf16 by round-to-nearest-even). The minimum of a group holding both
+ *   -0 and +0 is -0, the maximum +0. Inputs must be finite.
+ * group_size in {32, 64, 128}; bits in {2, 4, 8}; cols % group_size == 0.
+ * Other bit widths return NV_ERR_UNSUPPORTED.
+ */
+nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t cols,
+                             int group_size, int bits, uint32_t* codes, void* scales,
+                             void* biases, nv_stream_t stream);
+
+/*
+ * Quantized product ("Docs / Quantization", sections "Affine" (example
+ * x.quantized_matmul(&q, true)) and "Products on the GPU").
+ *
+ * x      [M, K] in `dt`; y [M, N] in `dt` (the output follows x's dtype).
+ * transpose = 1: weights stored [N, K] (codes [N, K*bits/32], scales/biases
+ *   [N, K/group_size]), y = x . w^T.  transpose = 0: weights stored [K, N]
+ *   (codes [K, N*bits/32], scales/biases [K, N/group_size]), y = x . w.
+ * Scales and biases have dtype `dt` too: supported pairs are (F32, F32) and
+ * (BF16, BF16). Accumulation is fp32.
+ * row_exact = 1 (M <= NV_ROW_INDEPENDENT_ROWS, else NV_ERR_INVALID_ARG): each
+ *   row's result equals, bit for bit, the same call with that row alone (M = 1).
+ * Routing is a pure function of (M, N, K, dt, group_size, bits, transpose,
+ * row_exact): matrix-vector kernels for M <= 8, tensor-core tiles above.
+ * M == 0 or N == 0 is a no-op returning NV_OK.
+ */
+nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
+                 const uint32_t* codes, const void* scales, const void* biases, int group_size,
+                 int bits, int transpose, int row_exact, void* y, nv_stream_t stream);
+
+/* Bytes of device workspace nv_gather_qmm needs for R pairs and E experts. */
+size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E);
+
+/*
+ * Mixture-of-experts product ("Docs / Quantization", section "Mixture of
+ * experts": gather_qmm multiplies each row by the expert chosen for it without
+ * gathering the weights first).
+ *
+ * x        [x_rows, K] in `dt`.
+ * lhs_idx  uint32 [R] or NULL: pair r reads row lhs_idx[r] of x (NULL: row r).
+ * rhs_idx  uint32 [R]: pair r uses expert rhs_idx[r] in [0, E).
+ * codes/scales/biases: E experts back to back, each laid out as for nv_qmm
+ *   (transpose = 1: [E, N, K]; transpose = 0: [E, K, N]).
+ * y        [R, N] in `dt`: row r is x[lhs[r]] times expert rhs[r], in pair order.
+ * sorted   = 1 is the caller's promise that rhs_idx never decreases (the
+ *   option sorted_indices); a broken promise is flagged (NV_FLAG_NOT_SORTED)
+ *   and the result is still correct.
+ * row_exact = 1: each row gets the bits of its one-row product nv_qmm(M = 1)
+ *   with its expert's weights.
+ * workspace: device memory of at least nv_gather_qmm_workspace_size(R, E)
+ *   bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *   matter. Calls that share a workspace must not overlap on the GPU.
+ */
+nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
+                        const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R, int64_t E,
+                        int64_t N, const uint32_t* codes, const void* scales, const void* biases,
+                        int group_size, int bits, int transpose, int sorted, int row_exact,
+                        void* workspace, size_t workspace_bytes, void* y, nv_stream_t stream);
+
+/* Copy the anomaly flags of the last nv_gather_qmm that used `workspace` into
+ * *host_flags (a HOST pointer). Synchronises `stream`. */
+nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVQ_H */

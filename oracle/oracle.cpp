@@ -27,6 +27,7 @@
 //   * the codes use the unrounded fp32 scale and bias; the stored scale and
 //     bias are then cast to the weights' dtype (bf16: round-to-nearest-even);
 //   * a constant group (scale == 0) gets code 0 everywhere;
+//   * a group holding both -0 and +0 has minimum -0 and maximum +0;
 //   * code j of a uint32 word sits at bits [j*bits, (j+1)*bits);
 //   * the product's reference value is the fp64 dot of x with the dequantized
 //     weights (stored scale and bias), summed in k order.
@@ -176,10 +177,12 @@ int orc_quantize_affine(const void* w, int dtype, int64_t rows, int64_t cols, in
             const int64_t c0 = g * gs;
             // Step 1: the group's minimum and maximum.
             float mn = load_f32(w, dtype, r * cols + c0), mx = mn;
+            // A group holding both zeros has minimum -0 and maximum +0, so the
+            // result does not depend on the order the values are visited in.
             for (int i = 1; i < gs; ++i) {
                 float v = load_f32(w, dtype, r * cols + c0 + i);
-                if (v < mn) mn = v;
-                if (v > mx) mx = v;
+                if (v < mn || (v == mn && std::signbit(v))) mn = v;
+                if (v > mx || (v == mx && !std::signbit(v))) mx = v;
             }
             // Step 2: scale spreads the range over the 2^bits - 1 steps; bias = min.
             float range = mx - mn;

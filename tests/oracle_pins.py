@@ -126,6 +126,21 @@ def pin_handbuilt_groups(lib):
             assert got[1].tolist() == _cycle(codes[::-1], gs), (name, dt)
 
 
+def pin_signed_zero_extremes(lib):
+    """A group whose smallest values are -0 and +0 (in either order) has bias -0;
+    one whose largest are -0 and +0 has its range measured to +0."""
+    for vals in ([0.0, -0.0, 1.0], [-0.0, 0.0, 1.0], [1.0, 0.0, -0.0]):
+        w = torch.tensor([_cycle(vals, 32)], dtype=torch.float32)
+        c, s, b = O.quantize_affine(w, 32, 4, lib=lib)
+        assert b.view(torch.int32)[0, 0] == torch.tensor(-0.0).view(torch.int32), vals
+        assert float(s[0, 0]) == 1.0 / 15.0 or float(s[0, 0]) == float(torch.tensor(1.0) / 15)
+    for vals in ([0.0, -0.0, -1.0], [-0.0, 0.0, -1.0]):
+        w = torch.tensor([_cycle(vals, 32)], dtype=torch.float32)
+        c, s, b = O.quantize_affine(w, 32, 4, lib=lib)
+        assert float(b[0, 0]) == -1.0 and float(s[0, 0]) == float(torch.tensor(1.0) / 15)
+        assert set(_unpack_div_mod(c, 4)[0].tolist()) == {15, 0}
+
+
 def pin_bf16_cast(lib):
     """The oracle's fp32 -> bf16 rounding equals torch's round-to-nearest-even
     cast (a library routine), including exact ties."""

@@ -44,6 +44,8 @@ MUTANTS = [
      "(void)rest;"),
     ("gather wrong expert", "        int64_t e = (int64_t)rhs[r];\n            dot_one",
      "        int64_t e = (int64_t)rhs[R - 1 - r];\n            dot_one"),
+    ("signed zero by order", "if (v < mn || (v == mn && std::signbit(v))) mn = v;",
+     "if (v < mn) mn = v;"),
     ("constant group top code", "uint32_t q = 0;", "uint32_t q = (uint32_t)levels;"),
 ]
 
