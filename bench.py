@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Throughput of the group-wise affine quantized products on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvq|reference]
+
+One step is one pass of the hot path over one batch of the headline workload:
+a 4-bit, group-64 decode product y = x . w^T with x [1, 4096] bf16 and
+W [14336, 4096] (Llama-8B MLP shape), i.e. one nv_qmm call. The JSON line
+reports HBM GB/s of algorithmic bytes (codes + scales + biases + x + y); the
+other workloads (8-bit and transposed decode, few rows, prefill, mixture of
+experts) are measured in the same run and reported under "also".
+
+Timing: W untimed warm-up steps, then K timed steps captured in CUDA graphs and
+bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
+events on the launching stream; max over ranks. The weights rotate over enough
+copies that the set touched between two uses of a copy exceeds the L2 cache.
+Multi-GPU runs are independent replicas (the product does not shard here):
+value = bytes processed by all ranks / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from group_wise_affine_dequant_b200 import workloads as W  # noqa: E402
+
+METRIC = "4-bit g64 qmm: decode HBM GB/s (% of 8 TB/s); prefill TFLOP/s; gather_qmm tok/s"
+HBM_NOMINAL_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def qbytes(N, K, bits, gs, sbytes=2):
+    """Bytes of a quantized [N, K] matrix: codes + scales + biases."""
+    return N * K * bits // 8 + 2 * (N * K // gs) * sbytes
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 6:
+                    try:
+                        rows.append((float(parts[0]), float(parts[1]), parts[2:]))
+                    except ValueError:
+                        pass
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, _, r in rows for n, v in zip(names, r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def timed_graph(fn_step, steps: int, warmup: int, stream, chunk: int = 512):
+    """Warm up, capture the steps in CUDA graphs, time K steps with CUDA events
+    on `stream`. fn_step(i) enqueues step i on the current stream. Returns ms."""
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            fn_step(i)
+    stream.synchronize()
+    graphs = []
+    done = 0
+    while done < steps:
+        n = min(chunk, steps - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(done, done + n):
+                fn_step(i)
+        graphs.append(g)
+        done += n
+    for g in graphs:  # one untimed replay: graph upload
+        g.replay()
+    stream.synchronize()
+    return graphs
+
+
+def replay_timed(graphs, stream, barrier):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for g in graphs:
+            g.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return start.elapsed_time(end)
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "group_wise_affine_dequant_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("src_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- workloads
+class Decode:
+    """x [M, K] . W[N, K]^T (transpose) or x . W[K, N], quantized (bits, gs)."""
+
+    def __init__(self, dev, N=14336, K=4096, M=1, bits=4, gs=64, transpose=True, l2_bytes=None):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        self.N, self.K, self.M, self.bits, self.gs, self.t = N, K, M, bits, gs, transpose
+        shape = (N, K) if transpose else (K, N)
+        w = W.normal(shape, 0.02, 0, "bf16").to(dev)
+        c, s, b = nvq.nv_quantize_affine(w, gs, bits)
+        del w
+        wbytes = qbytes(N, K, bits, gs)
+        l2 = l2_bytes or torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))  # 3x L2 between reuses of a copy
+        self.ws = [(c.clone(), s.clone(), b.clone()) for _ in range(self.copies)]
+        self.x = W.activations(M, K).to(dev)
+        self.y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.bytes = wbytes + 2 * M * (K + N)
+        self.flops = 2 * M * N * K
+
+    def step(self, i):
+        c, s, b = self.ws[i % self.copies]
+        self.nvq.nv_qmm(self.x, c, s, b, self.gs, self.bits, self.t, out=self.y)
+
+
+class DecodeE2E(Decode):
+    """The same product from host buffers: pinned x in, y out, every step."""
+
+    def __init__(self, dev, **kw):
+        super().__init__(dev, **kw)
+        self.xh = self.x.cpu().pin_memory()
+        self.yh = torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
+        self.h2d = self.xh.numel() * 2
+        self.d2h = self.yh.numel() * 2
+
+    def step(self, i):
+        self.x.copy_(self.xh, non_blocking=True)
+        super().step(i)
+        self.yh.copy_(self.y, non_blocking=True)
+
+
+class Gather:
+    """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4."""
+
+    def __init__(self, dev, sorted_pairs: bool):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        m = W.MOE
+        self.E, self.N, self.K, self.T = m["E"], m["N"], m["K"], m["tokens"]
+        w = W.normal((self.E, self.N, self.K), 0.02, 0, "bf16").to(dev)
+        c, s, b = nvq.nv_quantize_affine(w, 64, 4)
+        del w
+        wbytes = qbytes(self.E * self.N, self.K, 4, 64)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))
+        self.ws = [(c.clone(), s.clone(), b.clone()) for _ in range(self.copies)]
+        ids = W.expert_ids(self.T, self.E, m["top_k"], 2)
+        lhs, rhs = W.flatten_pairs(ids)
+        if sorted_pairs:
+            lhs, rhs, _ = W.stable_sort_pairs(lhs, rhs)
+        self.sorted = sorted_pairs
+        self.lhs = lhs.to(torch.int32).to(dev)
+        self.rhs = rhs.to(torch.int32).to(dev)
+        self.R = rhs.numel()
+        self.x = W.normal((self.T, self.K), 1.0, 1, "bf16").to(dev)
+        self.y = torch.empty(self.R, self.N, dtype=torch.bfloat16, device=dev)
+        self.wsp = torch.empty(nvq.nv_gather_qmm_workspace_size(self.R, self.E), dtype=torch.uint8,
+                               device=dev)
+        self.bytes = wbytes + self.T * self.K * 2 + self.R * self.N * 2 + self.R * 8
+
+    def step(self, i):
+        c, s, b = self.ws[i % self.copies]
+        self.nvq.nv_gather_qmm(self.x, c, s, b, self.rhs, self.lhs, 64, 4, True, self.sorted,
+                               False, workspace=self.wsp, out=self.y)
+
+
+# --------------------------------------------------------------------------- arms
+def run_nvq(args):
+    import torch.distributed as dist
+    ws, rank, local = dist_env()
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=torch.device(f"cuda:{local}"),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device(f"cuda:{local}")
+    stream = torch.cuda.Stream(dev)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v: float) -> float:
+        if ws == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk, pk_kind = peaks()
+    K, Wm = args.steps, args.warmup
+
+    # ---- headline: 4-bit g64 decode
+    dec = Decode(dev)
+    graphs = timed_graph(dec.step, K, Wm, stream)
+    with ClockSampler(local) as clk:
+        ms = replay_timed(graphs, stream, barrier)
+        # keep the clock sampler fed for at least ~0.5 s of load
+        t_end = time.time() + max(0.0, 0.6 - ms / 1e3)
+        while time.time() < t_end:
+            replay_timed(graphs, stream, lambda: None)
+    del graphs
+    ms = max_over_ranks(ms)
+    per_step_s = ms / 1e3 / K
+    value = ws * dec.bytes / per_step_s / 1e9
+    achieved = dec.bytes / per_step_s / 1e9  # one launch per step on this rank
+    clocks = clk.summary()
+
+    # ---- end to end through host buffers
+    e2e = DecodeE2E(dev)
+    graphs = timed_graph(e2e.step, K, Wm, stream)
+    ms_e2e = max_over_ranks(replay_timed(graphs, stream, barrier))
+    del graphs
+    e2e_value = ws * e2e.bytes / (ms_e2e / 1e3 / K) / 1e9
+
+    # ---- the other workloads, same rules (fewer steps)
+    also = {}
+    ks = max(3, min(K, 400))
+    for name, mk in (("decode_8bit_gbs", lambda: Decode(dev, bits=8)),
+                     ("decode_transposed_gbs", lambda: Decode(dev, N=14336, K=4096, transpose=False)),
+                     ("decode_transposed_8bit_gbs", lambda: Decode(dev, transpose=False, bits=8)),
+                     ("fewrow_m8_14336x4096_gbs", lambda: Decode(dev, M=8)),
+                     ("fewrow_m8_4096x4096_gbs", lambda: Decode(dev, N=4096, M=8))):
+        wl = mk()
+        g = timed_graph(wl.step, ks, Wm, stream)
+        t = max_over_ranks(replay_timed(g, stream, barrier))
+        also[name] = round(ws * wl.bytes / (t / 1e3 / ks) / 1e9, 1)
+        del g, wl
+    for name, srt in (("gather_sorted", True), ("gather_unsorted", False)):
+        wl = Gather(dev, srt)
+        g = timed_graph(wl.step, ks, Wm, stream)
+        t = max_over_ranks(replay_timed(g, stream, barrier))
+        step_s = t / 1e3 / ks
+        also[name + "_tok_s"] = round(ws * wl.T / step_s, 1)
+        also[name + "_gbs"] = round(ws * wl.bytes / step_s / 1e9, 1)
+        del g, wl
+    also["prefill_tflops"] = None  # tensor-core path not built yet
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": round(ms / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+        "pct_of_8tbs": round(100 * achieved / HBM_NOMINAL_GBS, 2),
+        "config": {"workload": "decode x[1,4096] . W[14336,4096]^T, affine 4-bit g64, bf16",
+                   "M": 1, "N": 14336, "K": 4096, "bits": 4, "group_size": 64,
+                   "bytes_per_step": dec.bytes, "parallelism": f"replicas x{ws}",
+                   "l2": f"weights rotate over {dec.copies} copies (> 3x L2 between reuses)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                     "peak_kind": pk_kind, "unit": "GB/s",
+                     "frac": round(achieved / pk["hbm_gbs"], 4),
+                     "traffic": traffic_for("qmv_decode_b4_g64")},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": e2e.h2d,
+                "d2h_bytes_per_step": e2e.d2h},
+        "gpu_launches": K,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+        "also": also,
+        "cpu_baseline": None,
+    }
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+def cpu_baseline(budget_s: float = 10.0, steps: int | None = None):
+    """The oracle on the host's cores, on the decode workload: whole products
+    (all 14336 outputs) repeated for about budget_s seconds."""
+    import oracle as O
+    w = W.decode_weight()
+    c, s, b = O.quantize_affine(w, 64, 4)
+    x = W.activations(1, 4096)
+    bytes_ = qbytes(14336, 4096, 4, 64) + 2 * (4096 + 14336)
+    t0 = time.perf_counter()
+    O.qmm(x, c, s, b, 64, 4, True)
+    one = time.perf_counter() - t0
+    reps = steps or max(1, int(budget_s / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.qmm(x, c, s, b, 64, 4, True)
+    dt = time.perf_counter() - t0
+    return {"value": round(reps * bytes_ / dt / 1e9, 4), "unit": "GB/s", "cores": O.threads(),
+            "kind": "oracle",
+            "sample": f"{reps} whole decode products x[1,4096] . W[14336,4096]^T (4-bit g64), "
+                      f"fp64 dequantize-then-dot, {dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import oracle as O
+    w = W.decode_weight()
+    c, s, b = O.quantize_affine(w, 64, 4)
+    x = W.activations(1, 4096)
+    N, K = 14336, 4096
+    # each step: a bounded, fixed sample of output rows, so K steps end in minutes
+    t0 = time.perf_counter()
+    O.qmm_sampled(x, c, s, b, 64, 4, True, torch.zeros(1024, dtype=torch.int64),
+                  torch.arange(1024))
+    per_row = (time.perf_counter() - t0) / 1024
+    total_budget = 60.0
+    rows = int(max(64, min(N, total_budget / max(1, args.steps + args.warmup) / max(per_row, 1e-9))))
+    n_idx = torch.arange(rows, dtype=torch.int64)
+    m_idx = torch.zeros(rows, dtype=torch.int64)
+    for _ in range(args.warmup):
+        O.qmm_sampled(x, c, s, b, 64, 4, True, m_idx, n_idx)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.qmm_sampled(x, c, s, b, 64, 4, True, m_idx, n_idx)
+    dt = time.perf_counter() - t0
+    bytes_per_step = rows * (K * 4 // 8 + 2 * 2 * K // 64) + 2 * K + 2 * rows
+    value = args.steps * bytes_per_step / dt / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+        "config": {"workload": "decode x[1,4096] . W[14336,4096]^T, affine 4-bit g64, bf16",
+                   "M": 1, "N": N, "K": K, "bits": 4, "group_size": 64,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": O.threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} of {N} output rows per step (fp64 oracle)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="nvq", choices=["nvq", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_nvq(args)
+
+
+if __name__ == "__main__":
+    main()

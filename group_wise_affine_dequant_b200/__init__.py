@@ -1,6 +1,18 @@
 """Group-wise affine quantized matrix products on B200 (sm_100a).
 
-The compute path is the C-ABI library ``libnvq.so`` (CUDA kernels); the
-Python functions here only marshal torch tensors and streams into it. Import
-``group_wise_affine_dequant_b200.workloads`` for the seeded synthetic inputs.
+The compute path is the C-ABI library ``libnvq.so`` (CUDA kernels, declared in
+include/nvq.h); the functions exported here only marshal torch tensors and
+streams into it. ``group_wise_affine_dequant_b200.workloads`` holds the seeded
+synthetic inputs.
 """
+from .binding import (  # noqa: F401
+    NV_ROW_INDEPENDENT_ROWS,
+    NvqError,
+    lib,
+    nv_gather_qmm,
+    nv_gather_qmm_flags,
+    nv_gather_qmm_workspace_size,
+    nv_qmm,
+    nv_quantize_affine,
+    nv_status_string,
+)

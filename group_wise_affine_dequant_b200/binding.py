@@ -1,0 +1,181 @@
+"""Python binding of libnvq.so (include/nvq.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls. It checks
+nothing the library does not check itself beyond what torch needs (device,
+contiguity, dtype of the output it allocates); every step of the computation
+runs in the CUDA kernels behind the C ABI. There is no CPU fallback: if the
+library is missing or a call fails, an exception says so.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+NV_OK, NV_ERR_INVALID_ARG, NV_ERR_UNSUPPORTED, NV_ERR_WORKSPACE, NV_ERR_CUDA = range(5)
+NV_F32, NV_BF16 = 0, 1
+NV_ROW_INDEPENDENT_ROWS = 8
+NV_FLAG_EXPERT_OUT_OF_RANGE = 0x1
+NV_FLAG_NOT_SORTED = 0x2
+NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
+
+# Every entry point declared in include/nvq.h.
+EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_qmm", "nv_gather_qmm_workspace_size",
+           "nv_gather_qmm", "nv_gather_qmm_flags")
+
+_DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
+_LOCK = threading.Lock()
+_LIB = None
+
+_p, _i64, _i, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_size_t
+
+
+class NvqError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn}: {text}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """The loaded C library (ctypes), built first if it is missing."""
+    global _LIB
+    with _LOCK:
+        if _LIB is None:
+            path = _build.LIB
+            if not os.path.exists(path):
+                _build.build()
+            if not os.path.exists(path):
+                raise RuntimeError(f"libnvq.so missing at {path}; the CUDA library is required")
+            L = C.CDLL(path)
+            L.nv_status_string.argtypes = [_i]
+            L.nv_status_string.restype = C.c_char_p
+            L.nv_quantize_affine.argtypes = [_p, _i, _i64, _i64, _i, _i, _p, _p, _p, _p]
+            L.nv_quantize_affine.restype = _i
+            L.nv_qmm.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i, _p, _p]
+            L.nv_qmm.restype = _i
+            L.nv_gather_qmm_workspace_size.argtypes = [_i64, _i64]
+            L.nv_gather_qmm_workspace_size.restype = _sz
+            L.nv_gather_qmm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _p,
+                                        _i, _i, _i, _i, _i, _p, _sz, _p, _p]
+            L.nv_gather_qmm.restype = _i
+            L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
+            L.nv_gather_qmm_flags.restype = _i
+            _LIB = L
+        return _LIB
+
+
+def nv_status_string(status: int) -> str:
+    return lib().nv_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != NV_OK:
+        raise NvqError(fn, status, nv_status_string(status))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def nv_quantize_affine(w: torch.Tensor, group_size: int = 64, bits: int = 4, stream=None):
+    """Quantize w [..., cols] along its last axis. Returns (codes int32-as-uint32,
+    scales, biases) with scales/biases in w's dtype."""
+    _dev(w, "w")
+    cols = w.shape[-1]
+    rows = w.numel() // cols if cols else 0
+    codes = torch.empty(*w.shape[:-1], cols * bits // 32, dtype=torch.int32, device=w.device)
+    scales = torch.empty(*w.shape[:-1], max(cols // group_size, 0), dtype=w.dtype, device=w.device)
+    biases = torch.empty_like(scales)
+    st = lib().nv_quantize_affine(w.data_ptr(), _DT.get(w.dtype, -1), rows, cols, group_size, bits,
+                                  codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                                  _stream(stream))
+    _check("nv_quantize_affine", st)
+    return codes, scales, biases
+
+
+def nv_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+           group_size: int = 64, bits: int = 4, transpose: bool = True, row_exact: bool = False,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x . w^T (transpose, weights [N, K]) or x . w (weights [K, N]); y in x's dtype."""
+    for t, n in ((x, "x"), (codes, "codes"), (scales, "scales"), (biases, "biases")):
+        _dev(t, n)
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    N = codes.shape[-2] if transpose else codes.shape[-1] * 32 // bits
+    y = out if out is not None else torch.empty(*x.shape[:-1], N, dtype=x.dtype, device=x.device)
+    _dev(y, "out")
+    if scales.dtype != x.dtype:
+        raise NvqError("nv_qmm", NV_ERR_UNSUPPORTED, nv_status_string(NV_ERR_UNSUPPORTED))
+    st = lib().nv_qmm(x.data_ptr(), _DT.get(x.dtype, -1), M, K, N, codes.data_ptr(),
+                      scales.data_ptr(), biases.data_ptr(), group_size, bits, int(transpose),
+                      int(row_exact), y.data_ptr(), _stream(stream))
+    _check("nv_qmm", st)
+    return y
+
+
+def nv_gather_qmm_workspace_size(R: int, E: int) -> int:
+    return int(lib().nv_gather_qmm_workspace_size(R, E))
+
+
+def nv_gather_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                  biases: torch.Tensor, rhs: torch.Tensor, lhs: torch.Tensor | None = None,
+                  group_size: int = 64, bits: int = 4, transpose: bool = True,
+                  sorted: bool = False, row_exact: bool = False,
+                  workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Row r of the result is x[lhs[r]] times expert rhs[r] (lhs None: row r).
+
+    x [x_rows, K] (or [x_rows, 1, K]); codes/scales/biases [E, ...] as for nv_qmm;
+    rhs, lhs int32 (uint32 values) [R]. Returns y [R, N] in x's dtype."""
+    for t, n in ((x, "x"), (codes, "codes"), (scales, "scales"), (biases, "biases"), (rhs, "rhs")):
+        _dev(t, n)
+    if lhs is not None:
+        _dev(lhs, "lhs")
+    K = x.shape[-1]
+    x_rows = x.numel() // K if K else 0
+    E = codes.shape[0]
+    N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    R = rhs.numel()
+    ws_bytes = nv_gather_qmm_workspace_size(R, E)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
+    y = out if out is not None else torch.empty(R, N, dtype=x.dtype, device=x.device)
+    st = lib().nv_gather_qmm(x.data_ptr(), _DT.get(x.dtype, -1), x_rows, K, _ptr(lhs),
+                             rhs.data_ptr(), R, E, N, codes.data_ptr(), scales.data_ptr(),
+                             biases.data_ptr(), group_size, bits, int(transpose), int(sorted),
+                             int(row_exact), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), y.data_ptr(),
+                             _stream(stream))
+    _check("nv_gather_qmm", st)
+    return y
+
+
+def nv_gather_qmm_flags(workspace: torch.Tensor, stream=None) -> int:
+    flags = C.c_uint32(0)
+    st = lib().nv_gather_qmm_flags(workspace.data_ptr(), C.addressof(flags), _stream(stream))
+    _check("nv_gather_qmm_flags", st)
+    return int(flags.value)

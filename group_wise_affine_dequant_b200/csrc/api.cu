@@ -1,0 +1,152 @@
+// The C ABI (include/nvq.h): argument checks on the host, then a pure routing
+// decision (a function of shapes, dtype, group size, bits, layout and
+// row_exact only, nuvec crate docs, "Determinism": "Routing is pure") and the
+// launches. Nothing here allocates device memory or synchronises a stream,
+// except nv_gather_qmm_flags, whose job is to read a result back.
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nv_status check_quant(int gs, int bits) {
+    if (bits == 1 || bits == 3 || bits == 5 || bits == 6) return NV_ERR_UNSUPPORTED;
+    if (bits != 2 && bits != 4 && bits != 8) return NV_ERR_INVALID_ARG;
+    if (gs != 32 && gs != 64 && gs != 128) return NV_ERR_INVALID_ARG;
+    return NV_OK;
+}
+
+bool valid_dtype(nv_dtype dt) { return dt == NV_F32 || dt == NV_BF16; }
+
+nv_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return NV_OK;
+    return NV_ERR_CUDA;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nv_status_string(nv_status s) {
+    switch (s) {
+        case NV_OK: return "NV_OK: success";
+        case NV_ERR_INVALID_ARG: return "NV_ERR_INVALID_ARG: a shape, pointer or alignment is invalid";
+        case NV_ERR_UNSUPPORTED: return "NV_ERR_UNSUPPORTED: valid combination not implemented (bit width or dtype)";
+        case NV_ERR_WORKSPACE: return "NV_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case NV_ERR_CUDA: return "NV_ERR_CUDA: a CUDA launch or call failed";
+    }
+    return "unknown nv_status";
+}
+
+nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t cols,
+                             int group_size, int bits, uint32_t* codes, void* scales,
+                             void* biases, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    nv_status st = check_quant(group_size, bits);
+    if (st != NV_OK) return st;
+    if (rows < 0 || cols <= 0 || cols % group_size != 0) return NV_ERR_INVALID_ARG;
+    if (rows == 0) return NV_OK;
+    if (!w || !codes || !scales || !biases) return NV_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases))
+        return NV_ERR_INVALID_ARG;
+    return from_cuda(nvq::launch_quantize_affine(w, dt, rows, cols, group_size, bits, codes,
+                                                 scales, biases, stream, sm_count()));
+}
+
+nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
+                 const uint32_t* codes, const void* scales, const void* biases, int group_size,
+                 int bits, int transpose, int row_exact, void* y, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    nv_status st = check_quant(group_size, bits);
+    if (st != NV_OK) return st;
+    if (M < 0 || K <= 0 || N < 0) return NV_ERR_INVALID_ARG;
+    if ((transpose ? K : N) % group_size != 0) return NV_ERR_INVALID_ARG;
+    if (row_exact && M > NV_ROW_INDEPENDENT_ROWS) return NV_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return NV_OK;
+    if (!x || !codes || !scales || !biases || !y) return NV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases) ||
+        !aligned16(y))
+        return NV_ERR_INVALID_ARG;
+
+    cudaStream_t s = stream;
+    const int sms = sm_count();
+    if (dt == NV_BF16) {
+        if (transpose) {
+            if (M <= NV_ROW_INDEPENDENT_ROWS && nvq::qmv_supported(bits, group_size))
+                return from_cuda(nvq::launch_qmv(x, M, K, N, codes, scales, biases, group_size,
+                                                 bits, y, s, sms));
+            if (M > NV_ROW_INDEPENDENT_ROWS && nvq::tc_supported(M, K, N, bits, group_size))
+                return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases,
+                                                    group_size, bits, y, s, sms));
+        } else {
+            if (M <= NV_ROW_INDEPENDENT_ROWS && nvq::qmvt_supported_m(bits, group_size, M))
+                return from_cuda(nvq::launch_qmvt(x, M, K, N, codes, scales, biases, group_size,
+                                                  bits, y, s, sms));
+        }
+    }
+    return from_cuda(nvq::launch_qmm_simt(x, dt, M, K, N, codes, scales, biases, group_size, bits,
+                                          transpose, y, s));
+}
+
+size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E) {
+    if (R < 0 || E < 0) return 0;
+    return nvq::gather_workspace_bytes(R, E);
+}
+
+nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
+                        const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R, int64_t E,
+                        int64_t N, const uint32_t* codes, const void* scales, const void* biases,
+                        int group_size, int bits, int transpose, int sorted, int row_exact,
+                        void* workspace, size_t workspace_bytes, void* y, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    nv_status st = check_quant(group_size, bits);
+    if (st != NV_OK) return st;
+    if (x_rows < 0 || K <= 0 || R < 0 || E <= 0 || N < 0) return NV_ERR_INVALID_ARG;
+    if ((transpose ? K : N) % group_size != 0) return NV_ERR_INVALID_ARG;
+    if (R > (int64_t(1) << 31) - 1) return NV_ERR_INVALID_ARG;
+    if (E > nvq::kMaxExperts) return NV_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace)) return NV_ERR_WORKSPACE;
+    if (workspace_bytes < nvq::gather_workspace_bytes(R, E)) return NV_ERR_WORKSPACE;
+    if (R == 0) return NV_OK;
+    if (!x || !rhs_idx || !codes || !scales || !biases || !y) return NV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases) ||
+        !aligned16(y) || !aligned16(rhs_idx) || (lhs_idx && !aligned16(lhs_idx)))
+        return NV_ERR_INVALID_ARG;
+
+    cudaStream_t s = stream;
+    const int sms = sm_count();
+    nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
+    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
+    if (e != cudaSuccess) return NV_ERR_CUDA;
+    if (N == 0) return NV_OK;
+    (void)row_exact;  // every route below gives each pair the bits of its one-row product
+    if (dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size))
+        return from_cuda(nvq::launch_qmv_gather(x, K, N, codes, scales, biases, group_size, bits,
+                                                lhs_idx, ws.perm, ws.problems, ws.num_problems,
+                                                ws.max_problems, E, y, s, sms));
+    return from_cuda(nvq::launch_gather_simt(x, dt, x_rows, K, lhs_idx, rhs_idx, R, E, N, codes,
+                                             scales, biases, group_size, bits, transpose, y, s));
+}
+
+nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream) {
+    if (!workspace || !aligned16(workspace) || !host_flags) return NV_ERR_INVALID_ARG;
+    cudaStream_t s = stream;
+    if (cudaMemcpyAsync(host_flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return NV_ERR_CUDA;
+    return from_cuda(cudaStreamSynchronize(s));
+}
+
+}  // extern "C"

@@ -1,0 +1,462 @@
+// Quantized matrix-vector products for 1 to 8 rows of bf16 activations,
+// weights stored [N, K] ("Docs / Quantization", sections "Affine" and "Products
+// on the GPU": matrix-vector kernels for few rows, reading each weight group
+// once for all rows).
+//
+// Design (sm_100a):
+//  * The weights stream from HBM exactly once per call. Each thread loads
+//    LW consecutive code words of one row with one vector load.
+//  * Codes become bf16 exactly: OR-ing a code (< 128) into the mantissa of 128.0
+//    gives 128 + code, two codes per 32-bit register, one LOP3 each (8-bit codes
+//    go through as their two 4-bit halves, the high half against 16 * x).
+//  * The multiply-adds run on the tensor cores (mma.sync m16n8k16): A = 16 weight
+//    rows x 16 k of codes, B = the activations (one column per activation row,
+//    up to 8), fp32 accumulation. Which physical k feeds which MMA k-slot is
+//    chosen so that each thread's loaded words feed its own A fragments; the
+//    activations are permuted the same way once, in registers.
+//  * Scale and bias are applied per group outside the MMA:
+//        sum_k x_k w_k = s * sum_k x_k (128 + c_k) + (b - 128 s) * sum_k x_k,
+//    so every product x * code is exact and only the group sums round.
+//  * A warp owns a k-slice of 16 MMA k-steps (256 k at 2/4 bits, 128 at 8) and
+//    keeps its activations in registers while it walks the rows of its CTA.
+//    Each CTA owns a contiguous range of rows (N split evenly over the SMs) and
+//    reduces the slices in a fixed order through shared memory.
+//  * Every output (row n, activation row m) is computed by the same sequence
+//    of operations whatever M is, so an M-row call gives each row the bits of
+//    its one-row call (row exactness, nuvec crate docs, "Determinism").
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace nvq {
+namespace {
+
+template <int BITS, int GS>
+struct Shape {
+    static constexpr int PER = 32 / BITS;                // codes per word
+    static constexpr int GW = GS * BITS / 32;            // words per group
+    static constexpr int LW = GW / 4 < 4 ? GW / 4 : 4;   // words per thread per row per chunk
+    static constexpr int MPW = BITS == 2 ? 4 : 2;        // MMAs per word
+    static constexpr int NP = 2 * MPW;                   // bf16x2 registers per unpacked word
+    static constexpr int CW = 4 * LW;                    // words per chunk (one lane quad)
+    static constexpr int CK = CW * PER;                  // k per chunk
+    static constexpr int MMAS = LW * MPW;                // MMAs per chunk
+    static constexpr int KS = 16 / MMAS;                 // chunks per warp slice
+    static constexpr int KSLICE = KS * CK;               // k per warp slice
+    static constexpr int GPS = KSLICE / GS > 0 ? KSLICE / GS : 1;  // groups per slice
+    static constexpr int CPG = GS / CK;                  // chunks per group
+    static constexpr int XMMA = BITS == 8 ? 1 : MPW;     // MMAs per word whose B is x itself
+    // sum_k x (128 + c) = sum x c + OFF sum x; 8-bit codes add 128 twice, once x16.
+    static constexpr float OFF = BITS == 8 ? 2176.0f : 128.0f;
+    static_assert(LW >= 1, "group too small for this kernel");
+    static_assert(CK <= GS && GS % CK == 0, "a chunk lies inside one group");
+};
+
+// Word -> NP bf16x2 registers; MMA u of the word uses p[2u] (k-slots 2t, 2t+1)
+// and p[2u+1] (k-slots 2t+8, 2t+9).
+template <int BITS>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* p) {
+    if constexpr (BITS == 4) {
+        p[0] = codes_to_bf16x2(w, 0x000F000Fu);        // (c0, c4)
+        p[1] = codes_to_bf16x2(w >> 4, 0x000F000Fu);   // (c1, c5)
+        p[2] = codes_to_bf16x2(w >> 8, 0x000F000Fu);   // (c2, c6)
+        p[3] = codes_to_bf16x2(w >> 12, 0x000F000Fu);  // (c3, c7)
+    } else if constexpr (BITS == 8) {
+        p[0] = codes_to_bf16x2(w, 0x000F000Fu);        // low halves of (c0, c2)
+        p[1] = codes_to_bf16x2(w >> 8, 0x000F000Fu);   // low halves of (c1, c3)
+        p[2] = codes_to_bf16x2(w >> 4, 0x000F000Fu);   // high halves of (c0, c2)
+        p[3] = codes_to_bf16x2(w >> 12, 0x000F000Fu);  // high halves of (c1, c3)
+    } else {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) p[s] = codes_to_bf16x2(w >> (2 * s), 0x00030003u);  // (c_s, c_s+8)
+    }
+}
+
+// The activations matching unpack_word: b[u][0..1] for MMA u of a word whose
+// first k is k0. xv holds x[k0 .. k0 + PER) as bf16 pairs.
+template <int BITS>
+__device__ __forceinline__ void x_fragments(const uint32_t* xv, uint32_t (*b)[2]) {
+    if constexpr (BITS == 4) {
+        b[0][0] = pair_lo(xv[0], xv[2]);  // (x0, x4)
+        b[0][1] = pair_hi(xv[0], xv[2]);  // (x1, x5)
+        b[1][0] = pair_lo(xv[1], xv[3]);  // (x2, x6)
+        b[1][1] = pair_hi(xv[1], xv[3]);  // (x3, x7)
+    } else if constexpr (BITS == 8) {
+        b[0][0] = pair_lo(xv[0], xv[1]);  // (x0, x2)
+        b[0][1] = pair_hi(xv[0], xv[1]);  // (x1, x3)
+        const __nv_bfloat162 sixteen = __floats2bfloat162_rn(16.0f, 16.0f);
+        __nv_bfloat162 h0 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&b[0][0]), sixteen);
+        __nv_bfloat162 h1 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&b[0][1]), sixteen);
+        b[1][0] = *reinterpret_cast<uint32_t*>(&h0);
+        b[1][1] = *reinterpret_cast<uint32_t*>(&h1);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            b[u][0] = pair_lo(xv[u], xv[4 + u]);  // (x_2u, x_2u+8)
+            b[u][1] = pair_hi(xv[u], xv[4 + u]);  // (x_2u+1, x_2u+9)
+        }
+    }
+}
+
+template <int LW>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* w) {
+    if constexpr (LW == 1) {
+        w[0] = __ldg(p);
+    } else if constexpr (LW == 2) {
+        uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        w[0] = v.x; w[1] = v.y;
+    } else {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    }
+}
+
+// GPS consecutive bf16 values (a slice's scales or biases for one row), packed
+// two per register.
+template <int GPS>
+__device__ __forceinline__ void load_groups(const uint16_t* p, uint32_t* v) {
+    if constexpr (GPS == 1) {
+        v[0] = __ldg(p);
+    } else if constexpr (GPS == 2) {
+        v[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+    } else if constexpr (GPS == 4) {
+        uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+        v[0] = q.x; v[1] = q.y;
+    } else {
+        uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    }
+}
+
+__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
+    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
+}
+
+struct QmvParams {
+    const uint16_t* x;       // bf16 [x_rows, K]
+    const uint32_t* codes;   // [E][N, K*bits/32]
+    const uint16_t* scales;  // [E][N, K/gs]
+    const uint16_t* biases;
+    uint16_t* y;             // bf16 [*, N]
+    int64_t N, K;
+    int M;                   // rows (plain product)
+    int ctas_per_problem;    // G: CTAs along N
+    int rows_cap;            // max rows of one CTA, multiple of 16
+    // gather only
+    const uint32_t* lhs;     // nullable
+    const uint32_t* perm;
+    const uint32_t* problems;      // [P][4] = (expert, start, count, 0)
+    const uint32_t* num_problems;
+    int64_t E;
+};
+
+constexpr int kMaxWarps = 16;
+
+template <int BITS, int GS, bool GATHER>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams prm) {
+    using S = Shape<BITS, GS>;
+    extern __shared__ float red[];  // [nslices][rows_cap][M] partial sums
+    __shared__ int64_t s_xrow[8];
+    __shared__ int64_t s_yrow[8];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t N = prm.N, K = prm.K;
+    const int64_t wpr = K * BITS / 32;  // code words per row
+    const int64_t gpr = K / GS;         // groups per row
+
+    int M;
+    const uint32_t* codes = prm.codes;
+    const uint16_t* scales = prm.scales;
+    const uint16_t* biases = prm.biases;
+    bool zero_problem = false;
+    if constexpr (GATHER) {
+        const uint32_t p = blockIdx.y;
+        if (p >= __ldg(prm.num_problems)) return;
+        const uint32_t e = __ldg(prm.problems + 4 * p);
+        const uint32_t start = __ldg(prm.problems + 4 * p + 1);
+        M = static_cast<int>(__ldg(prm.problems + 4 * p + 2));
+        zero_problem = e >= prm.E;  // pairs with an invalid id get zeros
+        if (!zero_problem) {
+            codes += static_cast<int64_t>(e) * N * wpr;
+            scales += static_cast<int64_t>(e) * N * gpr;
+            biases += static_cast<int64_t>(e) * N * gpr;
+        }
+        if (threadIdx.x < M) {
+            const uint32_t pair = __ldg(prm.perm + start + threadIdx.x);
+            s_yrow[threadIdx.x] = pair;
+            s_xrow[threadIdx.x] = prm.lhs ? __ldg(prm.lhs + pair) : pair;
+        }
+    } else {
+        M = prm.M;
+        if (threadIdx.x < M) {
+            s_xrow[threadIdx.x] = threadIdx.x;
+            s_yrow[threadIdx.x] = threadIdx.x;
+        }
+    }
+    __syncthreads();
+
+    const int64_t G = prm.ctas_per_problem;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * N / G;
+    const int64_t n1 = static_cast<int64_t>(blockIdx.x + 1) * N / G;
+    const int rows = static_cast<int>(n1 - n0);
+    if (rows <= 0) return;
+
+    if (zero_problem) {
+        for (int i = threadIdx.x; i < rows * M; i += blockDim.x) {
+            const int m = i / rows, r = i % rows;
+            prm.y[s_yrow[m] * N + n0 + r] = 0;
+        }
+        return;
+    }
+
+    const int tiles = (rows + 15) / 16;
+    const int rows_cap = prm.rows_cap;
+    const int nslices = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
+    const uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
+
+    for (int sl = warp; sl < nslices; sl += nwarps) {
+        const int64_t kslice0 = static_cast<int64_t>(sl) * S::KSLICE;
+        // Vector loads of a slice's scales need every row to start on a slice boundary.
+        const bool full_slice = K % S::KSLICE == 0;
+
+        // ---- activations of this slice: B fragments and per-chunk sums ----
+        uint32_t bfr[S::KS][S::MMAS][2];
+        float xs[S::KS][2];
+#pragma unroll
+        for (int q = 0; q < S::KS; ++q) {
+            const int64_t kq = kslice0 + q * S::CK;
+            const bool valid = kq < K && g < M;
+#pragma unroll
+            for (int j = 0; j < S::LW; ++j) {
+                const int64_t k0 = kq + (t * S::LW + j) * S::PER;
+                uint32_t xv[S::PER / 2];
+                if (valid) {
+                    const uint16_t* xp = prm.x + s_xrow[g] * K + k0;
+                    if constexpr (S::PER == 4) {
+                        uint2 v = __ldg(reinterpret_cast<const uint2*>(xp));
+                        xv[0] = v.x; xv[1] = v.y;
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < S::PER / 8; ++h) {
+                            uint4 v = __ldg(reinterpret_cast<const uint4*>(xp) + h);
+                            xv[4 * h] = v.x; xv[4 * h + 1] = v.y;
+                            xv[4 * h + 2] = v.z; xv[4 * h + 3] = v.w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < S::PER / 2; ++h) xv[h] = 0u;
+                }
+                x_fragments<BITS>(xv, &bfr[q][j * S::MPW]);
+            }
+            // sum of this chunk's activations, per activation row: an MMA with A = 1.
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < S::LW; ++j)
+#pragma unroll
+                for (int u = 0; u < S::XMMA; ++u)
+                    mma_bf16_16816(d, kOnes, kOnes, kOnes, kOnes, bfr[q][j * S::MPW + u][0],
+                                   bfr[q][j * S::MPW + u][1]);
+            xs[q][0] = d[0];
+            xs[q][1] = d[1];
+        }
+
+        // ---- walk the CTA's rows, 16 per tile ----
+        for (int tile = 0; tile < tiles; ++tile) {
+            const int64_t ra = n0 + tile * 16 + g;
+            const int64_t rb = ra + 8;
+            const bool va = ra < n1, vb = rb < n1;
+            uint32_t wa[S::KS][S::LW], wb[S::KS][S::LW];
+            uint32_t sa[(S::GPS + 1) / 2], sb[(S::GPS + 1) / 2];
+            uint32_t ba[(S::GPS + 1) / 2], bb[(S::GPS + 1) / 2];
+#pragma unroll
+            for (int q = 0; q < S::KS; ++q) {
+                const int64_t kq = kslice0 + q * S::CK;
+                const int64_t woff = kq / S::PER + t * S::LW;
+                const bool vq = kq < K;
+                if (va && vq) load_words<S::LW>(codes + ra * wpr + woff, wa[q]);
+                else for (int j = 0; j < S::LW; ++j) wa[q][j] = 0u;
+                if (vb && vq) load_words<S::LW>(codes + rb * wpr + woff, wb[q]);
+                else for (int j = 0; j < S::LW; ++j) wb[q][j] = 0u;
+            }
+            const int64_t g0 = kslice0 / GS;
+            if (full_slice) {
+                if (va) { load_groups<S::GPS>(scales + ra * gpr + g0, sa); load_groups<S::GPS>(biases + ra * gpr + g0, ba); }
+                if (vb) { load_groups<S::GPS>(scales + rb * gpr + g0, sb); load_groups<S::GPS>(biases + rb * gpr + g0, bb); }
+            } else {
+#pragma unroll
+                for (int i = 0; i < (S::GPS + 1) / 2; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
+#pragma unroll
+                for (int i = 0; i < S::GPS; ++i) {
+                    if ((g0 + i) * GS < K) {
+                        const int sh = (i & 1) * 16;
+                        if (va) { sa[i >> 1] |= uint32_t(__ldg(scales + ra * gpr + g0 + i)) << sh;
+                                  ba[i >> 1] |= uint32_t(__ldg(biases + ra * gpr + g0 + i)) << sh; }
+                        if (vb) { sb[i >> 1] |= uint32_t(__ldg(scales + rb * gpr + g0 + i)) << sh;
+                                  bb[i >> 1] |= uint32_t(__ldg(biases + rb * gpr + g0 + i)) << sh; }
+                    }
+                }
+            }
+
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < S::KS; ++q) {
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < S::LW; ++j) {
+                    uint32_t pa[S::NP], pb[S::NP];
+                    unpack_word<BITS>(wa[q][j], pa);
+                    unpack_word<BITS>(wb[q][j], pb);
+#pragma unroll
+                    for (int u = 0; u < S::MPW; ++u)
+                        mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
+                                       bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
+                }
+                const int gi = q / S::CPG;
+                const float s_a = group_value(sa, gi), s_b = group_value(sb, gi);
+                const float b_a = fmaf(-S::OFF, s_a, group_value(ba, gi));
+                const float b_b = fmaf(-S::OFF, s_b, group_value(bb, gi));
+                acc[0] = fmaf(b_a, xs[q][0], fmaf(s_a, d[0], acc[0]));
+                acc[1] = fmaf(b_a, xs[q][1], fmaf(s_a, d[1], acc[1]));
+                acc[2] = fmaf(b_b, xs[q][0], fmaf(s_b, d[2], acc[2]));
+                acc[3] = fmaf(b_b, xs[q][1], fmaf(s_b, d[3], acc[3]));
+            }
+            const int r0 = tile * 16 + g;
+            float* base = red + static_cast<int64_t>(sl) * rows_cap * M;
+            const int m0 = 2 * t, m1 = 2 * t + 1;
+            if (m0 < M) { base[r0 * M + m0] = acc[0]; base[(r0 + 8) * M + m0] = acc[2]; }
+            if (m1 < M) { base[r0 * M + m1] = acc[1]; base[(r0 + 8) * M + m1] = acc[3]; }
+        }
+    }
+    __syncthreads();
+
+    // ---- fixed-order reduction over the slices ----
+    for (int i = threadIdx.x; i < rows * M; i += blockDim.x) {
+        const int m = i / rows, r = i % rows;
+        float v = red[static_cast<int64_t>(r) * M + m];
+        for (int sl = 1; sl < nslices; ++sl) v += red[(static_cast<int64_t>(sl) * rows_cap + r) * M + m];
+        prm.y[s_yrow[m] * N + n0 + r] = f32_to_bf16_bits(v);
+    }
+}
+
+template <bool GATHER>
+using KernelPtr = void (*)(const QmvParams);
+
+template <bool GATHER>
+KernelPtr<GATHER> pick(int bits, int gs) {
+    if (bits == 4 && gs == 32) return qmv_kernel<4, 32, GATHER>;
+    if (bits == 4 && gs == 64) return qmv_kernel<4, 64, GATHER>;
+    if (bits == 4 && gs == 128) return qmv_kernel<4, 128, GATHER>;
+    if (bits == 8 && gs == 32) return qmv_kernel<8, 32, GATHER>;
+    if (bits == 8 && gs == 64) return qmv_kernel<8, 64, GATHER>;
+    if (bits == 8 && gs == 128) return qmv_kernel<8, 128, GATHER>;
+    if (bits == 2 && gs == 64) return qmv_kernel<2, 64, GATHER>;
+    if (bits == 2 && gs == 128) return qmv_kernel<2, 128, GATHER>;
+    return nullptr;
+}
+
+int kslice_of(int bits) { return bits == 8 ? 128 : 256; }
+
+// Split N over CTAs: every SM busy, at most 128 rows a CTA, and the slice
+// partials (nslices x rows x M fp32) inside shared memory.
+struct Plan {
+    int ctas, rows_cap, warps;
+    size_t smem;
+};
+
+Plan plan(int64_t N, int64_t K, int M, int bits, int num_sms, bool gather) {
+    const int64_t nslices = (K + kslice_of(bits) - 1) / kslice_of(bits);
+    const size_t smem_cap = 200 * 1024;
+    // A gather launches one set of CTAs per (expert, <= 8 pairs) problem, so
+    // its CTAs take up to 128 rows each instead of spreading one matrix over
+    // every SM.
+    int64_t ctas = gather ? (N + 127) / 128
+                          : std::max<int64_t>(std::min<int64_t>(num_sms, (N + 15) / 16),
+                                              (N + 127) / 128);
+    for (;;) {
+        const int64_t rows = (N + ctas - 1) / ctas;
+        const int64_t cap = (rows + 15) / 16 * 16;
+        const size_t smem = static_cast<size_t>(nslices * cap * M) * sizeof(float);
+        if (smem <= smem_cap || cap <= 16) {
+            Plan p;
+            p.ctas = static_cast<int>(ctas);
+            p.rows_cap = static_cast<int>(cap);
+            p.warps = static_cast<int>(std::min<int64_t>(kMaxWarps, nslices));
+            p.smem = smem;
+            return p;
+        }
+        ctas = ctas * 2;
+    }
+}
+
+template <bool GATHER>
+cudaError_t launch(KernelPtr<GATHER> k, const Plan& p, dim3 grid, const QmvParams& prm,
+                   cudaStream_t stream) {
+    if (p.smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(p.smem));
+        if (e != cudaSuccess) return e;
+    }
+    k<<<grid, p.warps * 32, p.smem, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool qmv_supported(int bits, int gs) { return pick<false>(bits, gs) != nullptr; }
+
+cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+                       const void* scales, const void* biases, int gs, int bits, void* y,
+                       cudaStream_t stream, int num_sms) {
+    auto k = pick<false>(bits, gs);
+    if (!k) return cudaErrorInvalidValue;
+    Plan p = plan(N, K, static_cast<int>(M), bits, num_sms, false);
+    QmvParams prm{};
+    prm.x = static_cast<const uint16_t*>(x);
+    prm.codes = codes;
+    prm.scales = static_cast<const uint16_t*>(scales);
+    prm.biases = static_cast<const uint16_t*>(biases);
+    prm.y = static_cast<uint16_t*>(y);
+    prm.N = N;
+    prm.K = K;
+    prm.M = static_cast<int>(M);
+    prm.ctas_per_problem = p.ctas;
+    prm.rows_cap = p.rows_cap;
+    return launch<false>(k, p, dim3(p.ctas, 1, 1), prm, stream);
+}
+
+cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_t* codes,
+                              const void* scales, const void* biases, int gs, int bits,
+                              const uint32_t* lhs, const uint32_t* perm,
+                              const uint32_t* problems, const uint32_t* num_problems,
+                              int64_t max_problems, int64_t E, void* y, cudaStream_t stream,
+                              int num_sms) {
+    auto k = pick<true>(bits, gs);
+    if (!k) return cudaErrorInvalidValue;
+    if (max_problems <= 0) return cudaSuccess;
+    // Every problem covers all N rows of one expert for <= 8 pairs.
+    Plan p = plan(N, K, 8, bits, num_sms, true);
+    QmvParams prm{};
+    prm.x = static_cast<const uint16_t*>(x);
+    prm.codes = codes;
+    prm.scales = static_cast<const uint16_t*>(scales);
+    prm.biases = static_cast<const uint16_t*>(biases);
+    prm.y = static_cast<uint16_t*>(y);
+    prm.N = N;
+    prm.K = K;
+    prm.M = 8;
+    prm.ctas_per_problem = p.ctas;
+    prm.rows_cap = p.rows_cap;
+    prm.lhs = lhs;
+    prm.perm = perm;
+    prm.problems = problems;
+    prm.num_problems = num_problems;
+    prm.E = E;
+    return launch<true>(k, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), prm, stream);
+}
+
+}  // namespace nvq

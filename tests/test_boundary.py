@@ -1,0 +1,124 @@
+"""The C-ABI library on the host: it loads, exports every entry point the
+header declares, and turns every invalid argument into its status code before
+launching anything (CPU only; no compute call is made without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import group_wise_affine_dequant_b200 as nvq
+from group_wise_affine_dequant_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvq.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nv_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_entry_points() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = nvq.lib()
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for s in range(5):
+        txt = nvq.nv_status_string(s)
+        assert txt.startswith(("NV_OK", "NV_ERR")), txt
+    assert "unknown" in nvq.nv_status_string(99)
+
+
+def _qmm(**kw):
+    a = dict(x=16, dt=1, M=1, K=64, N=16, codes=16, scales=16, biases=16, gs=64, bits=4,
+             transpose=1, row_exact=0, y=16, stream=None)
+    a.update(kw)
+    return nvq.lib().nv_qmm(a["x"], a["dt"], a["M"], a["K"], a["N"], a["codes"], a["scales"],
+                            a["biases"], a["gs"], a["bits"], a["transpose"], a["row_exact"], a["y"],
+                            a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=3), B.NV_ERR_UNSUPPORTED),
+    (dict(bits=5), B.NV_ERR_UNSUPPORTED),
+    (dict(bits=6), B.NV_ERR_UNSUPPORTED),
+    (dict(bits=1), B.NV_ERR_UNSUPPORTED),
+    (dict(bits=7), B.NV_ERR_INVALID_ARG),
+    (dict(gs=16), B.NV_ERR_INVALID_ARG),
+    (dict(gs=96), B.NV_ERR_INVALID_ARG),
+    (dict(dt=7), B.NV_ERR_UNSUPPORTED),
+    (dict(M=-1), B.NV_ERR_INVALID_ARG),
+    (dict(K=0), B.NV_ERR_INVALID_ARG),
+    (dict(K=96), B.NV_ERR_INVALID_ARG),            # K not a multiple of the group size
+    (dict(transpose=0, N=48), B.NV_ERR_INVALID_ARG),  # transpose=0 groups along N
+    (dict(row_exact=1, M=9), B.NV_ERR_INVALID_ARG),
+    (dict(x=0), B.NV_ERR_INVALID_ARG),
+    (dict(y=0), B.NV_ERR_INVALID_ARG),
+    (dict(codes=8), B.NV_ERR_INVALID_ARG),         # misaligned
+    (dict(scales=18), B.NV_ERR_INVALID_ARG),
+    (dict(M=0), B.NV_OK),                          # empty: nothing to launch
+    (dict(N=0), B.NV_OK),
+])
+def test_qmm_argument_errors(kw, status):
+    assert _qmm(**kw) == status
+
+
+def test_quantize_argument_errors():
+    q = nvq.lib().nv_quantize_affine
+    assert q(16, 1, 4, 64, 64, 3, 16, 16, 16, None) == B.NV_ERR_UNSUPPORTED
+    assert q(16, 1, 4, 96, 64, 4, 16, 16, 16, None) == B.NV_ERR_INVALID_ARG
+    assert q(16, 1, -1, 64, 64, 4, 16, 16, 16, None) == B.NV_ERR_INVALID_ARG
+    assert q(16, 1, 4, 64, 64, 4, 0, 16, 16, None) == B.NV_ERR_INVALID_ARG
+    assert q(24, 1, 4, 64, 64, 4, 16, 16, 16, None) == B.NV_ERR_INVALID_ARG
+    assert q(16, 1, 0, 64, 64, 4, 16, 16, 16, None) == B.NV_OK
+
+
+def test_gather_argument_errors():
+    L = nvq.lib()
+    R, E = 2048, 64
+    need = L.nv_gather_qmm_workspace_size(R, E)
+    assert need >= 4 * R
+
+    def call(ws=16, ws_bytes=need, **kw):
+        a = dict(x=16, dt=1, x_rows=512, K=2048, lhs=16, rhs=16, R=R, E=E, N=1536, codes=16,
+                 scales=16, biases=16, gs=64, bits=4, transpose=1, sorted=0, row_exact=0, y=16)
+        a.update(kw)
+        return L.nv_gather_qmm(a["x"], a["dt"], a["x_rows"], a["K"], a["lhs"], a["rhs"], a["R"],
+                               a["E"], a["N"], a["codes"], a["scales"], a["biases"], a["gs"],
+                               a["bits"], a["transpose"], a["sorted"], a["row_exact"], ws,
+                               ws_bytes, a["y"], None)
+
+    assert call(ws_bytes=need - 1) == B.NV_ERR_WORKSPACE
+    assert call(ws=0) == B.NV_ERR_WORKSPACE
+    assert call(ws=8) == B.NV_ERR_WORKSPACE
+    assert call(bits=5) == B.NV_ERR_UNSUPPORTED
+    assert call(E=0) == B.NV_ERR_INVALID_ARG
+    assert call(E=5000, ws_bytes=L.nv_gather_qmm_workspace_size(R, 5000)) == B.NV_ERR_UNSUPPORTED
+    assert call(K=100) == B.NV_ERR_INVALID_ARG
+    assert call(rhs=0) == B.NV_ERR_INVALID_ARG
+    assert call(lhs=4) == B.NV_ERR_INVALID_ARG
+    assert call(R=0, ws_bytes=L.nv_gather_qmm_workspace_size(0, E)) == B.NV_OK
+
+
+def test_flags_argument_errors():
+    L = nvq.lib()
+    flags = C.c_uint32(0)
+    assert L.nv_gather_qmm_flags(0, C.addressof(flags), None) == B.NV_ERR_INVALID_ARG
+    assert L.nv_gather_qmm_flags(16, 0, None) == B.NV_ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding has no fallback: a missing library that cannot be built raises."""
+    monkeypatch.setattr(B, "_LIB", None)
+    monkeypatch.setattr(B._build, "LIB", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B._build, "build", lambda *a, **k: None)
+    with pytest.raises(RuntimeError, match="libnvq.so missing"):
+        B.lib()
