@@ -125,8 +125,17 @@ def nv_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: t
         _dev(t, n)
     K = x.shape[-1]
     M = x.numel() // K if K else 0
+    if codes.dim() != 2 or scales.shape != biases.shape or scales.dim() != 2:
+        raise ValueError("codes, scales and biases must be 2-D and scales/biases alike")
     N = codes.shape[-2] if transpose else codes.shape[-1] * 32 // bits
+    rows, cols = (N, K) if transpose else (K, N)
+    if tuple(codes.shape) != (rows, cols * bits // 32) or \
+            tuple(scales.shape) != (rows, cols // group_size):
+        raise ValueError(f"weights do not match x: codes {tuple(codes.shape)}, scales "
+                         f"{tuple(scales.shape)} for K={K}, N={N}, transpose={transpose}")
     y = out if out is not None else torch.empty(*x.shape[:-1], N, dtype=x.dtype, device=x.device)
+    if y.numel() != M * N or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
     _dev(y, "out")
     if scales.dtype != x.dtype:
         raise NvqError("nv_qmm", NV_ERR_UNSUPPORTED, nv_status_string(NV_ERR_UNSUPPORTED))
@@ -158,12 +167,23 @@ def nv_gather_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
     K = x.shape[-1]
     x_rows = x.numel() // K if K else 0
     E = codes.shape[0]
+    if codes.dim() != 3 or scales.dim() != 3 or scales.shape != biases.shape:
+        raise ValueError("codes, scales and biases must be [E, rows, ...] alike")
     N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    rows, cols = (N, K) if transpose else (K, N)
+    if tuple(codes.shape) != (E, rows, cols * bits // 32) or \
+            tuple(scales.shape) != (E, rows, cols // group_size):
+        raise ValueError(f"expert weights do not match x: codes {tuple(codes.shape)}, scales "
+                         f"{tuple(scales.shape)} for K={K}, N={N}, transpose={transpose}")
     R = rhs.numel()
+    if lhs is not None and lhs.numel() != R:
+        raise ValueError("lhs and rhs differ in length")
     ws_bytes = nv_gather_qmm_workspace_size(R, E)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     y = out if out is not None else torch.empty(R, N, dtype=x.dtype, device=x.device)
+    if y.numel() != R * N or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
     st = lib().nv_gather_qmm(x.data_ptr(), _DT.get(x.dtype, -1), x_rows, K, _ptr(lhs),
                              rhs.data_ptr(), R, E, N, codes.data_ptr(), scales.data_ptr(),
                              biases.data_ptr(), group_size, bits, int(transpose), int(sorted),

@@ -91,9 +91,21 @@ nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
                 return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases,
                                                     group_size, bits, y, s, sms));
         } else {
-            if (M <= NV_ROW_INDEPENDENT_ROWS && nvq::qmvt_supported_m(bits, group_size, M))
-                return from_cuda(nvq::launch_qmvt(x, M, K, N, codes, scales, biases, group_size,
-                                                  bits, y, s, sms));
+            if (M <= NV_ROW_INDEPENDENT_ROWS && nvq::qmvt_supported_m(bits, group_size, 1)) {
+                // Rows go through in chunks the kernel holds in registers; every
+                // row's arithmetic is the same in any chunk, so the chunking keeps
+                // each row's bits equal to its one-row product.
+                int64_t chunk = M;
+                while (chunk > 1 && !nvq::qmvt_supported_m(bits, group_size, chunk)) --chunk;
+                for (int64_t m0 = 0; m0 < M; m0 += chunk) {
+                    const int64_t mc = M - m0 < chunk ? M - m0 : chunk;
+                    cudaError_t e = nvq::launch_qmvt(
+                        static_cast<const uint16_t*>(x) + m0 * K, mc, K, N, codes, scales, biases,
+                        group_size, bits, static_cast<uint16_t*>(y) + m0 * N, s, sms);
+                    if (e != cudaSuccess) return NV_ERR_CUDA;
+                }
+                return NV_OK;
+            }
         }
     }
     return from_cuda(nvq::launch_qmm_simt(x, dt, M, K, N, codes, scales, biases, group_size, bits,

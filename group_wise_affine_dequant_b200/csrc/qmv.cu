@@ -99,38 +99,37 @@ __device__ __forceinline__ void x_fragments(const uint32_t* xv, uint32_t (*b)[2]
     }
 }
 
+// Asynchronous 4/8/16-byte copies global -> shared (cp.async); src_bytes = 0
+// writes zeros without reading.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void* src, bool valid) {
+    const int n = valid ? BYTES : 0;
+    if constexpr (BYTES == 16) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+    } else {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n" ::"r"(dst), "l"(src),
+                     "n"(BYTES), "r"(n));
+    }
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 template <int LW>
-__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* w) {
+__device__ __forceinline__ void lds_words(const uint32_t* p, uint32_t* w) {
     if constexpr (LW == 1) {
-        w[0] = __ldg(p);
+        w[0] = *p;
     } else if constexpr (LW == 2) {
-        uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        uint2 v = *reinterpret_cast<const uint2*>(p);
         w[0] = v.x; w[1] = v.y;
     } else {
-        uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        uint4 v = *reinterpret_cast<const uint4*>(p);
         w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     }
-}
-
-// GPS consecutive bf16 values (a slice's scales or biases for one row), packed
-// two per register.
-template <int GPS>
-__device__ __forceinline__ void load_groups(const uint16_t* p, uint32_t* v) {
-    if constexpr (GPS == 1) {
-        v[0] = __ldg(p);
-    } else if constexpr (GPS == 2) {
-        v[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
-    } else if constexpr (GPS == 4) {
-        uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
-        v[0] = q.x; v[1] = q.y;
-    } else {
-        uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    }
-}
-
-__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
-    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
 }
 
 struct QmvParams {
@@ -153,10 +152,34 @@ struct QmvParams {
 
 constexpr int kMaxWarps = 16;
 
-template <int BITS, int GS, bool GATHER>
+__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
+    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
+}
+
+// Per-thread staging of one tile (16 rows of the CTA, one warp slice): the
+// codes of the thread's two rows, then (when a slice's scales and biases are a
+// vector of >= 4 bytes per row) the four scale/bias vectors. Units are laid
+// out lane-interleaved so that the 32 lanes of a warp touch consecutive bytes.
+template <int BITS, int GS>
+struct Stage {
+    using S = Shape<BITS, GS>;
+    static constexpr int SBW = S::GPS >= 2 ? S::GPS / 2 : 0;      // words per scale vector
+    static constexpr int CODE_WORDS = 2 * S::KS * S::LW;
+    static constexpr int WPT = CODE_WORDS + 4 * SBW;               // words per thread
+    static constexpr int WORDS = 32 * WPT;                         // words per warp and stage
+    __host__ __device__ static constexpr uint32_t code_off(int q, int r, int lane) {  // r: 0 = row g, 1 = row g + 8
+        return (2 * q + r) * S::LW * 32 + lane * S::LW;
+    }
+    __host__ __device__ static constexpr uint32_t sb_off(int j, int lane) {  // j: s_a, s_b, b_a, b_b
+        return CODE_WORDS * 32 + j * SBW * 32 + lane * SBW;
+    }
+};
+
+template <int BITS, int GS, bool GATHER, int NS>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams prm) {
     using S = Shape<BITS, GS>;
-    extern __shared__ float red[];  // [nslices][rows_cap][M] partial sums
+    using ST = Stage<BITS, GS>;
+    extern __shared__ __align__(16) uint32_t smem[];  // [warps][NS][WORDS] ring, then partials
     __shared__ int64_t s_xrow[8];
     __shared__ int64_t s_yrow[8];
 
@@ -217,11 +240,51 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
     const int rows_cap = prm.rows_cap;
     const int nslices = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
     const uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
+    // Vector loads of a slice's scales need every row to start on a slice boundary.
+    const bool vec_sb = ST::SBW > 0 && K % S::KSLICE == 0;
+    uint32_t* ring = smem + static_cast<size_t>(warp) * NS * ST::WORDS;
+    float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(nwarps) * NS * ST::WORDS);
 
     for (int sl = warp; sl < nslices; sl += nwarps) {
         const int64_t kslice0 = static_cast<int64_t>(sl) * S::KSLICE;
-        // Vector loads of a slice's scales need every row to start on a slice boundary.
-        const bool full_slice = K % S::KSLICE == 0;
+        const int64_t g0 = kslice0 / GS;
+
+        // chunks of this slice inside K (all of them unless K ends mid-slice)
+        const int64_t left = (K - kslice0) / S::CK;
+        const int nq = left < S::KS ? static_cast<int>(left) : S::KS;
+        const int64_t slice_word = kslice0 / S::PER + t * S::LW;
+
+        // Enqueue the copies of tile `tile` into ring stage `st`.
+        auto issue = [&](int tile, int st) {
+            uint32_t* stage = ring + st * ST::WORDS;
+            const int64_t ra = n0 + tile * 16 + g;
+            const bool va = ra < n1, vb = ra + 8 < n1;
+            const uint32_t* pa = va ? codes + ra * wpr + slice_word : codes;
+            const uint32_t* pb = vb ? codes + (ra + 8) * wpr + slice_word : codes;
+            const uint32_t da = smem_addr(stage + ST::code_off(0, 0, lane));
+#pragma unroll
+            for (int q = 0; q < S::KS; ++q) {
+                const bool vq = q < nq;
+                cp_async<S::LW * 4>(da + 4 * (ST::code_off(q, 0, 0)), pa + (vq && va ? q * S::CW : 0), va && vq);
+                cp_async<S::LW * 4>(da + 4 * (ST::code_off(q, 1, 0)), pb + (vq && vb ? q * S::CW : 0), vb && vq);
+            }
+            if constexpr (ST::SBW > 0) {
+                if (vec_sb) {
+                    const int64_t oa = va ? ra * gpr + g0 : 0, ob = vb ? (ra + 8) * gpr + g0 : 0;
+                    const uint32_t ds = smem_addr(stage + ST::sb_off(0, lane));
+                    cp_async<ST::SBW * 4>(ds, scales + oa, va);
+                    cp_async<ST::SBW * 4>(ds + 4 * ST::SBW * 32, scales + ob, vb);
+                    cp_async<ST::SBW * 4>(ds + 8 * ST::SBW * 32, biases + oa, va);
+                    cp_async<ST::SBW * 4>(ds + 12 * ST::SBW * 32, biases + ob, vb);
+                }
+            }
+        };
+
+#pragma unroll
+        for (int i = 0; i < NS - 1; ++i) {
+            if (i < tiles) issue(i, i);
+            cp_async_commit();
+        }
 
         // ---- activations of this slice: B fragments and per-chunk sums ----
         uint32_t bfr[S::KS][S::MMAS][2];
@@ -265,31 +328,29 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
             xs[q][1] = d[1];
         }
 
-        // ---- walk the CTA's rows, 16 per tile ----
+        // ---- walk the CTA's rows, 16 per tile, NS - 1 tiles in flight ----
         for (int tile = 0; tile < tiles; ++tile) {
-            const int64_t ra = n0 + tile * 16 + g;
-            const int64_t rb = ra + 8;
+            const int tn = tile + NS - 1;
+            if (tn < tiles) issue(tn, tn % NS);
+            cp_async_commit();
+            cp_async_wait<NS - 1>();
+            const uint32_t* stage = ring + (tile % NS) * ST::WORDS;
+            const int64_t ra = n0 + tile * 16 + g, rb = ra + 8;
             const bool va = ra < n1, vb = rb < n1;
-            uint32_t wa[S::KS][S::LW], wb[S::KS][S::LW];
-            uint32_t sa[(S::GPS + 1) / 2], sb[(S::GPS + 1) / 2];
-            uint32_t ba[(S::GPS + 1) / 2], bb[(S::GPS + 1) / 2];
+
+            constexpr int SBR = ST::SBW > 0 ? ST::SBW : 1;
+            uint32_t sa[SBR], sb[SBR], ba[SBR], bb[SBR];
+            if (vec_sb) {
 #pragma unroll
-            for (int q = 0; q < S::KS; ++q) {
-                const int64_t kq = kslice0 + q * S::CK;
-                const int64_t woff = kq / S::PER + t * S::LW;
-                const bool vq = kq < K;
-                if (va && vq) load_words<S::LW>(codes + ra * wpr + woff, wa[q]);
-                else for (int j = 0; j < S::LW; ++j) wa[q][j] = 0u;
-                if (vb && vq) load_words<S::LW>(codes + rb * wpr + woff, wb[q]);
-                else for (int j = 0; j < S::LW; ++j) wb[q][j] = 0u;
-            }
-            const int64_t g0 = kslice0 / GS;
-            if (full_slice) {
-                if (va) { load_groups<S::GPS>(scales + ra * gpr + g0, sa); load_groups<S::GPS>(biases + ra * gpr + g0, ba); }
-                if (vb) { load_groups<S::GPS>(scales + rb * gpr + g0, sb); load_groups<S::GPS>(biases + rb * gpr + g0, bb); }
+                for (int i = 0; i < SBR; ++i) {
+                    sa[i] = stage[ST::sb_off(0, lane) + i];
+                    sb[i] = stage[ST::sb_off(1, lane) + i];
+                    ba[i] = stage[ST::sb_off(2, lane) + i];
+                    bb[i] = stage[ST::sb_off(3, lane) + i];
+                }
             } else {
 #pragma unroll
-                for (int i = 0; i < (S::GPS + 1) / 2; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
+                for (int i = 0; i < SBR; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
 #pragma unroll
                 for (int i = 0; i < S::GPS; ++i) {
                     if ((g0 + i) * GS < K) {
@@ -305,12 +366,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < S::KS; ++q) {
+                uint32_t wa[S::LW], wb[S::LW];
+                lds_words<S::LW>(stage + ST::code_off(q, 0, lane), wa);
+                lds_words<S::LW>(stage + ST::code_off(q, 1, lane), wb);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
                     uint32_t pa[S::NP], pb[S::NP];
-                    unpack_word<BITS>(wa[q][j], pa);
-                    unpack_word<BITS>(wb[q][j], pb);
+                    unpack_word<BITS>(wa[j], pa);
+                    unpack_word<BITS>(wb[j], pb);
 #pragma unroll
                     for (int u = 0; u < S::MPW; ++u)
                         mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
@@ -331,6 +395,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
             if (m0 < M) { base[r0 * M + m0] = acc[0]; base[(r0 + 8) * M + m0] = acc[2]; }
             if (m1 < M) { base[r0 * M + m1] = acc[1]; base[(r0 + 8) * M + m1] = acc[3]; }
         }
+        cp_async_wait<0>();
     }
     __syncthreads();
 
@@ -347,30 +412,45 @@ template <bool GATHER>
 using KernelPtr = void (*)(const QmvParams);
 
 template <bool GATHER>
-KernelPtr<GATHER> pick(int bits, int gs) {
-    if (bits == 4 && gs == 32) return qmv_kernel<4, 32, GATHER>;
-    if (bits == 4 && gs == 64) return qmv_kernel<4, 64, GATHER>;
-    if (bits == 4 && gs == 128) return qmv_kernel<4, 128, GATHER>;
-    if (bits == 8 && gs == 32) return qmv_kernel<8, 32, GATHER>;
-    if (bits == 8 && gs == 64) return qmv_kernel<8, 64, GATHER>;
-    if (bits == 8 && gs == 128) return qmv_kernel<8, 128, GATHER>;
-    if (bits == 2 && gs == 64) return qmv_kernel<2, 64, GATHER>;
-    if (bits == 2 && gs == 128) return qmv_kernel<2, 128, GATHER>;
-    return nullptr;
+struct Variant {
+    KernelPtr<GATHER> k4, k3, k2;  // ring depth 4, 3, 2
+    int words;                     // ring words per warp and stage
+};
+
+template <int BITS, int GS, bool GATHER>
+Variant<GATHER> variant() {
+    return {qmv_kernel<BITS, GS, GATHER, 4>, qmv_kernel<BITS, GS, GATHER, 3>,
+            qmv_kernel<BITS, GS, GATHER, 2>, Stage<BITS, GS>::WORDS};
+}
+
+template <bool GATHER>
+bool pick(int bits, int gs, Variant<GATHER>& v) {
+    if (bits == 4 && gs == 32) { v = variant<4, 32, GATHER>(); return true; }
+    if (bits == 4 && gs == 64) { v = variant<4, 64, GATHER>(); return true; }
+    if (bits == 4 && gs == 128) { v = variant<4, 128, GATHER>(); return true; }
+    if (bits == 8 && gs == 32) { v = variant<8, 32, GATHER>(); return true; }
+    if (bits == 8 && gs == 64) { v = variant<8, 64, GATHER>(); return true; }
+    if (bits == 8 && gs == 128) { v = variant<8, 128, GATHER>(); return true; }
+    if (bits == 2 && gs == 64) { v = variant<2, 64, GATHER>(); return true; }
+    if (bits == 2 && gs == 128) { v = variant<2, 128, GATHER>(); return true; }
+    return false;
 }
 
 int kslice_of(int bits) { return bits == 8 ? 128 : 256; }
 
-// Split N over CTAs: every SM busy, at most 128 rows a CTA, and the slice
-// partials (nslices x rows x M fp32) inside shared memory.
+constexpr size_t kSmemMax = 227 * 1024 - 256;
+
+// Split N over CTAs (every SM busy, at most 128 rows a CTA); size the slice
+// partials (nslices x rows x M fp32) and the deepest copy ring that fits.
 struct Plan {
-    int ctas, rows_cap, warps;
+    int ctas, rows_cap, warps, depth;
     size_t smem;
 };
 
-Plan plan(int64_t N, int64_t K, int M, int bits, int num_sms, bool gather) {
+Plan plan(int64_t N, int64_t K, int M, int bits, int words, int num_sms, bool gather) {
     const int64_t nslices = (K + kslice_of(bits) - 1) / kslice_of(bits);
-    const size_t smem_cap = 200 * 1024;
+    const int warps = static_cast<int>(std::min<int64_t>(kMaxWarps, nslices));
+    const size_t ring2 = static_cast<size_t>(warps) * 2 * words * 4;
     // A gather launches one set of CTAs per (expert, <= 8 pairs) problem, so
     // its CTAs take up to 128 rows each instead of spreading one matrix over
     // every SM.
@@ -380,13 +460,16 @@ Plan plan(int64_t N, int64_t K, int M, int bits, int num_sms, bool gather) {
     for (;;) {
         const int64_t rows = (N + ctas - 1) / ctas;
         const int64_t cap = (rows + 15) / 16 * 16;
-        const size_t smem = static_cast<size_t>(nslices * cap * M) * sizeof(float);
-        if (smem <= smem_cap || cap <= 16) {
+        const size_t red = static_cast<size_t>(nslices * cap * M) * sizeof(float);
+        if (red + ring2 <= kSmemMax || cap <= 16) {
             Plan p;
             p.ctas = static_cast<int>(ctas);
             p.rows_cap = static_cast<int>(cap);
-            p.warps = static_cast<int>(std::min<int64_t>(kMaxWarps, nslices));
-            p.smem = smem;
+            p.warps = warps;
+            p.depth = 2;
+            for (int d = 4; d > 2; --d)
+                if (red + static_cast<size_t>(warps) * d * words * 4 <= kSmemMax) { p.depth = d; break; }
+            p.smem = red + static_cast<size_t>(warps) * p.depth * words * 4;
             return p;
         }
         ctas = ctas * 2;
@@ -394,8 +477,9 @@ Plan plan(int64_t N, int64_t K, int M, int bits, int num_sms, bool gather) {
 }
 
 template <bool GATHER>
-cudaError_t launch(KernelPtr<GATHER> k, const Plan& p, dim3 grid, const QmvParams& prm,
+cudaError_t launch(const Variant<GATHER>& v, const Plan& p, dim3 grid, const QmvParams& prm,
                    cudaStream_t stream) {
+    KernelPtr<GATHER> k = p.depth == 4 ? v.k4 : p.depth == 3 ? v.k3 : v.k2;
     if (p.smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(p.smem));
@@ -407,14 +491,17 @@ cudaError_t launch(KernelPtr<GATHER> k, const Plan& p, dim3 grid, const QmvParam
 
 }  // namespace
 
-bool qmv_supported(int bits, int gs) { return pick<false>(bits, gs) != nullptr; }
+bool qmv_supported(int bits, int gs) {
+    Variant<false> v;
+    return pick<false>(bits, gs, v);
+}
 
 cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                        const void* scales, const void* biases, int gs, int bits, void* y,
                        cudaStream_t stream, int num_sms) {
-    auto k = pick<false>(bits, gs);
-    if (!k) return cudaErrorInvalidValue;
-    Plan p = plan(N, K, static_cast<int>(M), bits, num_sms, false);
+    Variant<false> v;
+    if (!pick<false>(bits, gs, v)) return cudaErrorInvalidValue;
+    Plan p = plan(N, K, static_cast<int>(M), bits, v.words, num_sms, false);
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -426,7 +513,7 @@ cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uin
     prm.M = static_cast<int>(M);
     prm.ctas_per_problem = p.ctas;
     prm.rows_cap = p.rows_cap;
-    return launch<false>(k, p, dim3(p.ctas, 1, 1), prm, stream);
+    return launch<false>(v, p, dim3(p.ctas, 1, 1), prm, stream);
 }
 
 cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_t* codes,
@@ -435,11 +522,11 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
                               const uint32_t* problems, const uint32_t* num_problems,
                               int64_t max_problems, int64_t E, void* y, cudaStream_t stream,
                               int num_sms) {
-    auto k = pick<true>(bits, gs);
-    if (!k) return cudaErrorInvalidValue;
+    Variant<true> v;
+    if (!pick<true>(bits, gs, v)) return cudaErrorInvalidValue;
     if (max_problems <= 0) return cudaSuccess;
     // Every problem covers all N rows of one expert for <= 8 pairs.
-    Plan p = plan(N, K, 8, bits, num_sms, true);
+    Plan p = plan(N, K, 8, bits, v.words, num_sms, true);
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -456,7 +543,7 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     prm.problems = problems;
     prm.num_problems = num_problems;
     prm.E = E;
-    return launch<true>(k, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), prm, stream);
+    return launch<true>(v, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), prm, stream);
 }
 
 }  // namespace nvq

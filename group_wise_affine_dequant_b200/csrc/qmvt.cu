@@ -168,7 +168,7 @@ qmvt_kernel(const QmvtParams prm) {
         const uint16_t* sp = prm.scales + grp;
         const uint16_t* bp = prm.biases + grp;
         // Loads in flight per thread; halved where 64 accumulators fill the registers.
-        constexpr int U = MT * COLS_T >= 64 ? 2 : 4;
+        constexpr int U = MT * COLS_T >= 64 ? 2 : MT * COLS_T > 32 ? 4 : 8;
         int64_t k = kr0 + p;
         for (; k + (U - 1) * KP < kr1; k += U * KP) {
             uint32_t wv[U][TW];

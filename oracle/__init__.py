@@ -135,6 +135,7 @@ def qmm(x, codes, scales, biases, group_size: int, bits: int, transpose: bool = 
         N = codes.shape[0]
     else:
         N = codes.shape[1] * 32 // bits
+    _check_weights(codes, scales, biases, K, N, group_size, bits, transpose)
     y = torch.empty(M, N, dtype=torch.float64)
     a = torch.empty(M, N, dtype=torch.float64)
     rc = lib.orc_qmm(x.data_ptr(), _DT[x.dtype], M, K, N, codes.data_ptr(), scales.data_ptr(),
@@ -150,6 +151,7 @@ def qmm_sampled(x, codes, scales, biases, group_size, bits, transpose, m_idx, n_
     x, codes, scales, biases = _cpu(x), _cpu(codes), _cpu(scales), _cpu(biases)
     M, K = x.shape
     N = codes.shape[0] if transpose else codes.shape[1] * 32 // bits
+    _check_weights(codes, scales, biases, K, N, group_size, bits, transpose)
     m_idx = _cpu(torch.as_tensor(m_idx, dtype=torch.int64))
     n_idx = _cpu(torch.as_tensor(n_idx, dtype=torch.int64))
     S = m_idx.numel()
@@ -161,6 +163,15 @@ def qmm_sampled(x, codes, scales, biases, group_size, bits, transpose, m_idx, n_
                              y.data_ptr(), a.data_ptr())
     _check(rc, "qmm_sampled")
     return y, a
+
+
+def _check_weights(codes, scales, biases, K, N, group_size, bits, transpose):
+    rows, cols = (N, K) if transpose else (K, N)
+    lead = tuple(codes.shape[:-2])
+    if tuple(codes.shape[-2:]) != (rows, cols * bits // 32) or \
+            tuple(scales.shape) != lead + (rows, cols // group_size) or scales.shape != biases.shape:
+        raise ValueError(f"oracle: weights {tuple(codes.shape)}/{tuple(scales.shape)} do not "
+                         f"match K={K}, N={N}, transpose={transpose}")
 
 
 def _u32(t):
@@ -177,6 +188,7 @@ def gather_qmm(x, codes, scales, biases, lhs, rhs, group_size, bits, transpose=T
     x_rows, K = x2.shape
     E = codes.shape[0]
     N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    _check_weights(codes, scales, biases, K, N, group_size, bits, transpose)
     lhs_t, rhs_t = _u32(lhs), _u32(rhs)
     R = rhs_t.numel()
     y = torch.empty(R, N, dtype=torch.float64)
@@ -198,6 +210,7 @@ def gather_qmm_sampled(x, codes, scales, biases, lhs, rhs, group_size, bits, tra
     x_rows, K = x2.shape
     E = codes.shape[0]
     N = codes.shape[1] if transpose else codes.shape[2] * 32 // bits
+    _check_weights(codes, scales, biases, K, N, group_size, bits, transpose)
     lhs_t, rhs_t = _u32(lhs), _u32(rhs)
     R = rhs_t.numel()
     r_idx = _cpu(torch.as_tensor(r_idx, dtype=torch.int64))
