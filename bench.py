@@ -322,7 +322,17 @@ def run_nvq(args):
         also[name + "_tok_s"] = round(ws * wl.T / step_s, 1)
         also[name + "_gbs"] = round(ws * wl.bytes / step_s / 1e9, 1)
         del g, wl
-    also["prefill_tflops"] = None  # tensor-core path not built yet
+    for bits, gs in W.PREFILL_VARIANTS:
+        wl = Decode(dev, N=14336, K=4096, M=2048, bits=bits, gs=gs)
+        kp = max(3, min(K, 100))
+        g = timed_graph(wl.step, kp, Wm, stream)
+        t = max_over_ranks(replay_timed(g, stream, barrier))
+        tf = ws * wl.flops / (t / 1e3 / kp) / 1e12
+        key = "prefill_tflops" if (bits, gs) == (4, 64) else f"prefill_b{bits}_g{gs}_tflops"
+        also[key] = round(tf, 1)
+        if (bits, gs) == (4, 64):
+            also["prefill_frac_of_bf16_peak"] = round(tf / pk["bf16_tflops"], 4)
+        del g, wl
 
     line = {
         "metric": METRIC,

@@ -25,7 +25,7 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_qmm", "nv_gather_qmm_workspace_size",
-           "nv_gather_qmm", "nv_gather_qmm_flags")
+           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error")
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
 _LOCK = threading.Lock()
@@ -68,6 +68,8 @@ def lib():
             L.nv_gather_qmm.restype = _i
             L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
             L.nv_gather_qmm_flags.restype = _i
+            L.nv_pipeline_error.argtypes = [_p]
+            L.nv_pipeline_error.restype = _i
             _LIB = L
         return _LIB
 
@@ -199,3 +201,11 @@ def nv_gather_qmm_flags(workspace: torch.Tensor, stream=None) -> int:
     st = lib().nv_gather_qmm_flags(workspace.data_ptr(), C.addressof(flags), _stream(stream))
     _check("nv_gather_qmm_flags", st)
     return int(flags.value)
+
+
+def nv_pipeline_error() -> int:
+    """Read and clear the kernels' pipeline timeout word (0 = no wait gave up)."""
+    code = C.c_uint32(0)
+    st = lib().nv_pipeline_error(C.addressof(code))
+    _check("nv_pipeline_error", st)
+    return int(code.value)

@@ -161,4 +161,14 @@ nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_st
     return from_cuda(cudaStreamSynchronize(s));
 }
 
+nv_status nv_pipeline_error(uint32_t* host_code) {
+    if (!host_code) return NV_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return NV_ERR_CUDA;
+    const unsigned int a = nvq::qmv_error_take();
+    const unsigned int b = nvq::tc_error_take();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return NV_ERR_CUDA;
+    *host_code = a ? a : b;
+    return NV_OK;
+}
+
 }  // extern "C"

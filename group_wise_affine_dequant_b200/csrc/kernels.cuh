@@ -12,6 +12,7 @@ cudaError_t launch_quantize_affine(const void* w, int dt, int64_t rows, int64_t 
 
 // Matrix-vector products for up to 8 rows, weights [N, K] (transpose = 1), bf16.
 bool qmv_supported(int bits, int gs);
+unsigned int qmv_error_take();  // read and clear the kernels' pipeline error word
 cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                        const void* scales, const void* biases, int gs, int bits, void* y,
                        cudaStream_t stream, int num_sms);

@@ -4,8 +4,11 @@
 // once for all rows).
 //
 // Design (sm_100a):
-//  * The weights stream from HBM exactly once per call. Each thread loads
-//    LW consecutive code words of one row with one vector load.
+//  * The weights stream from HBM exactly once per call, by TMA: each warp
+//    copies its slice of 16 rows per tile (one 2-D tensor copy, 128-byte
+//    swizzle so the fragment reads below hit distinct banks) plus the slice's
+//    scales and biases into its own ring of shared-memory stages, completing
+//    on a per-warp mbarrier, several tiles ahead of the math.
 //  * Codes become bf16 exactly: OR-ing a code (< 128) into the mantissa of 128.0
 //    gives 128 + code, two codes per 32-bit register, one LOP3 each (8-bit codes
 //    go through as their two 4-bit halves, the high half against 16 * x).
@@ -28,6 +31,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace nvq {
 namespace {
@@ -99,37 +103,8 @@ __device__ __forceinline__ void x_fragments(const uint32_t* xv, uint32_t (*b)[2]
     }
 }
 
-// Asynchronous 4/8/16-byte copies global -> shared (cp.async); src_bytes = 0
-// writes zeros without reading.
-template <int BYTES>
-__device__ __forceinline__ void cp_async(uint32_t dst, const void* src, bool valid) {
-    const int n = valid ? BYTES : 0;
-    if constexpr (BYTES == 16) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
-    } else {
-        asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n" ::"r"(dst), "l"(src),
-                     "n"(BYTES), "r"(n));
-    }
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-template <int LW>
-__device__ __forceinline__ void lds_words(const uint32_t* p, uint32_t* w) {
-    if constexpr (LW == 1) {
-        w[0] = *p;
-    } else if constexpr (LW == 2) {
-        uint2 v = *reinterpret_cast<const uint2*>(p);
-        w[0] = v.x; w[1] = v.y;
-    } else {
-        uint4 v = *reinterpret_cast<const uint4*>(p);
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    }
+__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
+    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
 }
 
 struct QmvParams {
@@ -142,6 +117,7 @@ struct QmvParams {
     int M;                   // rows (plain product)
     int ctas_per_problem;    // G: CTAs along N
     int rows_cap;            // max rows of one CTA, multiple of 16
+    int sb_tma;              // scales/biases staged by TMA (rows 16-byte aligned)
     // gather only
     const uint32_t* lhs;     // nullable
     const uint32_t* perm;
@@ -152,50 +128,61 @@ struct QmvParams {
 
 constexpr int kMaxWarps = 16;
 
-__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
-    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
-}
-
-// Per-thread staging of one tile (16 rows of the CTA, one warp slice): the
-// codes of the thread's two rows, then (when a slice's scales and biases are a
-// vector of >= 4 bytes per row) the four scale/bias vectors. Units are laid
-// out lane-interleaved so that the 32 lanes of a warp touch consecutive bytes.
+// Ring geometry of one warp: per stage, the code box (16 rows x CBYTES, TMA
+// 128-byte swizzle when CBYTES is 128) and the scale and bias boxes (16 rows x
+// SBOX bf16, unswizzled). Code stages are 1024-byte aligned.
 template <int BITS, int GS>
-struct Stage {
+struct Ring {
     using S = Shape<BITS, GS>;
-    static constexpr int SBW = S::GPS >= 2 ? S::GPS / 2 : 0;      // words per scale vector
-    static constexpr int CODE_WORDS = 2 * S::KS * S::LW;
-    static constexpr int WPT = CODE_WORDS + 4 * SBW;               // words per thread
-    static constexpr int WORDS = 32 * WPT;                         // words per warp and stage
-    __host__ __device__ static constexpr uint32_t code_off(int q, int r, int lane) {  // r: 0 = row g, 1 = row g + 8
-        return (2 * q + r) * S::LW * 32 + lane * S::LW;
-    }
-    __host__ __device__ static constexpr uint32_t sb_off(int j, int lane) {  // j: s_a, s_b, b_a, b_b
-        return CODE_WORDS * 32 + j * SBW * 32 + lane * SBW;
+    static constexpr int CBYTES = S::KSLICE * BITS / 8;          // code bytes per row and slice
+    static constexpr bool SWZ = CBYTES == 128;
+    static constexpr int CODE_STAGE = 16 * CBYTES;               // 2048 or 1024
+    static constexpr int SBOX = S::GPS > 8 ? S::GPS : 8;         // groups per scale box row
+    static constexpr int SB_STAGE = 16 * SBOX * 2;               // one of scales / biases
+    // byte offset of code word `word` of row `r` inside a code stage
+    __device__ static __forceinline__ uint32_t code_off(int r, int word) {
+        const uint32_t o = static_cast<uint32_t>(word) * 4;
+        if constexpr (SWZ) return r * 128 + ((((o >> 4) ^ (r & 7)) << 4) | (o & 15));
+        else return r * CBYTES + o;
     }
 };
 
+template <int LW>
+__device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t* w) {
+    if constexpr (LW == 1) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if constexpr (LW == 2) {
+        uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = v.x; w[1] = v.y;
+    } else {
+        uint4 v = *reinterpret_cast<const uint4*>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    }
+}
+
 template <int BITS, int GS, bool GATHER, int NS>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams prm) {
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_s,
+           const __grid_constant__ CUtensorMap map_b, const QmvParams prm) {
     using S = Shape<BITS, GS>;
-    using ST = Stage<BITS, GS>;
-    extern __shared__ __align__(16) uint32_t smem[];  // [warps][NS][WORDS] ring, then partials
+    using RG = Ring<BITS, GS>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ int64_t s_xrow[8];
     __shared__ int64_t s_yrow[8];
+    __shared__ int s_expert;
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t N = prm.N, K = prm.K;
-    const int64_t wpr = K * BITS / 32;  // code words per row
-    const int64_t gpr = K / GS;         // groups per row
+    const int64_t gpr = K / GS;  // groups per row
 
     int M;
-    const uint32_t* codes = prm.codes;
     const uint16_t* scales = prm.scales;
     const uint16_t* biases = prm.biases;
     bool zero_problem = false;
+    int expert = 0;
     if constexpr (GATHER) {
         const uint32_t p = blockIdx.y;
         if (p >= __ldg(prm.num_problems)) return;
@@ -204,7 +191,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
         M = static_cast<int>(__ldg(prm.problems + 4 * p + 2));
         zero_problem = e >= prm.E;  // pairs with an invalid id get zeros
         if (!zero_problem) {
-            codes += static_cast<int64_t>(e) * N * wpr;
+            expert = static_cast<int>(e);
             scales += static_cast<int64_t>(e) * N * gpr;
             biases += static_cast<int64_t>(e) * N * gpr;
         }
@@ -220,6 +207,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
             s_yrow[threadIdx.x] = threadIdx.x;
         }
     }
+    (void)s_expert;
     __syncthreads();
 
     const int64_t G = prm.ctas_per_problem;
@@ -236,55 +224,55 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
         return;
     }
 
+    // shared memory: [warps][NS] code stages | [warps][NS] scale+bias stages |
+    // [warps][NS] mbarriers | slice partials
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint8_t* code_ring = smem + static_cast<size_t>(warp) * NS * RG::CODE_STAGE;
+    uint8_t* sb_ring = smem + static_cast<size_t>(nwarps) * NS * RG::CODE_STAGE +
+                       static_cast<size_t>(warp) * NS * 2 * RG::SB_STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(
+        smem + static_cast<size_t>(nwarps) * NS * (RG::CODE_STAGE + 2 * RG::SB_STAGE)) + warp * NS;
+    float* red = reinterpret_cast<float*>(
+        smem + static_cast<size_t>(nwarps) * NS * (RG::CODE_STAGE + 2 * RG::SB_STAGE) +
+        static_cast<size_t>(nwarps) * NS * 8);
+
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+        mbar_init_fence();
+    }
+    __syncwarp();
+
     const int tiles = (rows + 15) / 16;
     const int rows_cap = prm.rows_cap;
     const int nslices = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
     const uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
-    // Vector loads of a slice's scales need every row to start on a slice boundary.
-    const bool vec_sb = ST::SBW > 0 && K % S::KSLICE == 0;
-    uint32_t* ring = smem + static_cast<size_t>(warp) * NS * ST::WORDS;
-    float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(nwarps) * NS * ST::WORDS);
+    const bool sb_tma = prm.sb_tma != 0;
+    const uint32_t stage_bytes = RG::CODE_STAGE + (sb_tma ? 2 * RG::SB_STAGE : 0);
+    bool ok = true;
+    uint32_t it = 0;  // this warp's tile counter across its slices (ring position)
 
-    for (int sl = warp; sl < nslices; sl += nwarps) {
+    for (int sl = warp; sl < nslices && ok; sl += nwarps) {
         const int64_t kslice0 = static_cast<int64_t>(sl) * S::KSLICE;
         const int64_t g0 = kslice0 / GS;
+        const int gbox = static_cast<int>(g0 / RG::SBOX * RG::SBOX);  // scale box start (16-B aligned)
+        const int goff = static_cast<int>(g0 - gbox);                 // slice's first group in the box
+        const int cword = static_cast<int>(kslice0 * BITS / 32);
 
-        // chunks of this slice inside K (all of them unless K ends mid-slice)
-        const int64_t left = (K - kslice0) / S::CK;
-        const int nq = left < S::KS ? static_cast<int>(left) : S::KS;
-        const int64_t slice_word = kslice0 / S::PER + t * S::LW;
-
-        // Enqueue the copies of tile `tile` into ring stage `st`.
+        // lane 0: copy tile `tile` of this slice into ring stage `st`
         auto issue = [&](int tile, int st) {
-            uint32_t* stage = ring + st * ST::WORDS;
-            const int64_t ra = n0 + tile * 16 + g;
-            const bool va = ra < n1, vb = ra + 8 < n1;
-            const uint32_t* pa = va ? codes + ra * wpr + slice_word : codes;
-            const uint32_t* pb = vb ? codes + (ra + 8) * wpr + slice_word : codes;
-            const uint32_t da = smem_addr(stage + ST::code_off(0, 0, lane));
-#pragma unroll
-            for (int q = 0; q < S::KS; ++q) {
-                const bool vq = q < nq;
-                cp_async<S::LW * 4>(da + 4 * (ST::code_off(q, 0, 0)), pa + (vq && va ? q * S::CW : 0), va && vq);
-                cp_async<S::LW * 4>(da + 4 * (ST::code_off(q, 1, 0)), pb + (vq && vb ? q * S::CW : 0), vb && vq);
-            }
-            if constexpr (ST::SBW > 0) {
-                if (vec_sb) {
-                    const int64_t oa = va ? ra * gpr + g0 : 0, ob = vb ? (ra + 8) * gpr + g0 : 0;
-                    const uint32_t ds = smem_addr(stage + ST::sb_off(0, lane));
-                    cp_async<ST::SBW * 4>(ds, scales + oa, va);
-                    cp_async<ST::SBW * 4>(ds + 4 * ST::SBW * 32, scales + ob, vb);
-                    cp_async<ST::SBW * 4>(ds + 8 * ST::SBW * 32, biases + oa, va);
-                    cp_async<ST::SBW * 4>(ds + 12 * ST::SBW * 32, biases + ob, vb);
-                }
+            uint64_t* bar = &full[st];
+            mbar_expect_tx(bar, stage_bytes);
+            const int row = static_cast<int>(n0) + tile * 16;
+            tma_load_3d(code_ring + st * RG::CODE_STAGE, &map_c, bar, cword, row, expert);
+            if (sb_tma) {
+                uint8_t* sbs = sb_ring + st * 2 * RG::SB_STAGE;
+                tma_load_3d(sbs, &map_s, bar, gbox, row, expert);
+                tma_load_3d(sbs + RG::SB_STAGE, &map_b, bar, gbox, row, expert);
             }
         };
-
-#pragma unroll
-        for (int i = 0; i < NS - 1; ++i) {
-            if (i < tiles) issue(i, i);
-            cp_async_commit();
-        }
+        const uint32_t it0 = it;
+        if (lane == 0)
+            for (int i = 0; i < NS && i < tiles; ++i) issue(i, (it0 + i) % NS);
 
         // ---- activations of this slice: B fragments and per-chunk sums ----
         uint32_t bfr[S::KS][S::MMAS][2];
@@ -328,29 +316,30 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
             xs[q][1] = d[1];
         }
 
-        // ---- walk the CTA's rows, 16 per tile, NS - 1 tiles in flight ----
-        for (int tile = 0; tile < tiles; ++tile) {
-            const int tn = tile + NS - 1;
-            if (tn < tiles) issue(tn, tn % NS);
-            cp_async_commit();
-            cp_async_wait<NS - 1>();
-            const uint32_t* stage = ring + (tile % NS) * ST::WORDS;
+        // ---- walk the CTA's rows, 16 per tile, NS tiles in flight ----
+        for (int tile = 0; tile < tiles; ++tile, ++it) {
+            const int st = static_cast<int>(it % NS);
+            if (!(ok = mbar_wait(&full[st], (it / NS) & 1, 10))) break;
+            const uint8_t* cst = code_ring + st * RG::CODE_STAGE;
             const int64_t ra = n0 + tile * 16 + g, rb = ra + 8;
             const bool va = ra < n1, vb = rb < n1;
 
-            constexpr int SBR = ST::SBW > 0 ? ST::SBW : 1;
+            constexpr int SBR = S::GPS >= 2 ? S::GPS / 2 : 1;
             uint32_t sa[SBR], sb[SBR], ba[SBR], bb[SBR];
-            if (vec_sb) {
 #pragma unroll
-                for (int i = 0; i < SBR; ++i) {
-                    sa[i] = stage[ST::sb_off(0, lane) + i];
-                    sb[i] = stage[ST::sb_off(1, lane) + i];
-                    ba[i] = stage[ST::sb_off(2, lane) + i];
-                    bb[i] = stage[ST::sb_off(3, lane) + i];
+            for (int i = 0; i < SBR; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
+            if (sb_tma) {
+                const uint16_t* ss = reinterpret_cast<const uint16_t*>(sb_ring + st * 2 * RG::SB_STAGE);
+                const uint16_t* bs = ss + RG::SB_STAGE / 2;
+#pragma unroll
+                for (int i = 0; i < S::GPS; ++i) {
+                    const int sh = (i & 1) * 16;
+                    sa[i >> 1] |= uint32_t(ss[g * RG::SBOX + goff + i]) << sh;
+                    sb[i >> 1] |= uint32_t(ss[(g + 8) * RG::SBOX + goff + i]) << sh;
+                    ba[i >> 1] |= uint32_t(bs[g * RG::SBOX + goff + i]) << sh;
+                    bb[i >> 1] |= uint32_t(bs[(g + 8) * RG::SBOX + goff + i]) << sh;
                 }
             } else {
-#pragma unroll
-                for (int i = 0; i < SBR; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
 #pragma unroll
                 for (int i = 0; i < S::GPS; ++i) {
                     if ((g0 + i) * GS < K) {
@@ -367,8 +356,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
 #pragma unroll
             for (int q = 0; q < S::KS; ++q) {
                 uint32_t wa[S::LW], wb[S::LW];
-                lds_words<S::LW>(stage + ST::code_off(q, 0, lane), wa);
-                lds_words<S::LW>(stage + ST::code_off(q, 1, lane), wb);
+                const int word = q * S::CW + t * S::LW;
+                lds_words<S::LW>(cst + RG::code_off(g, word), wa);
+                lds_words<S::LW>(cst + RG::code_off(g + 8, word), wb);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
@@ -389,13 +379,16 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
                 acc[2] = fmaf(b_b, xs[q][0], fmaf(s_b, d[2], acc[2]));
                 acc[3] = fmaf(b_b, xs[q][1], fmaf(s_b, d[3], acc[3]));
             }
+            // every lane has read the stage: refill it with tile + NS
+            __syncwarp();
+            if (lane == 0 && tile + NS < tiles) issue(tile + NS, st);
+
             const int r0 = tile * 16 + g;
             float* base = red + static_cast<int64_t>(sl) * rows_cap * M;
             const int m0 = 2 * t, m1 = 2 * t + 1;
             if (m0 < M) { base[r0 * M + m0] = acc[0]; base[(r0 + 8) * M + m0] = acc[2]; }
             if (m1 < M) { base[r0 * M + m1] = acc[1]; base[(r0 + 8) * M + m1] = acc[3]; }
         }
-        cp_async_wait<0>();
     }
     __syncthreads();
 
@@ -409,18 +402,24 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmv_kernel(const QmvParams 
 }
 
 template <bool GATHER>
-using KernelPtr = void (*)(const QmvParams);
+using KernelPtr = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const QmvParams);
 
 template <bool GATHER>
 struct Variant {
     KernelPtr<GATHER> k4, k3, k2;  // ring depth 4, 3, 2
-    int words;                     // ring words per warp and stage
+    int stage_bytes;               // code + scale + bias bytes per warp and stage
+    int code_row_bytes;            // code bytes per row and slice (TMA box row)
+    bool swizzle;
+    int sbox;                      // groups per scale box row
+    int kslice;
 };
 
 template <int BITS, int GS, bool GATHER>
 Variant<GATHER> variant() {
+    using RG = Ring<BITS, GS>;
     return {qmv_kernel<BITS, GS, GATHER, 4>, qmv_kernel<BITS, GS, GATHER, 3>,
-            qmv_kernel<BITS, GS, GATHER, 2>, Stage<BITS, GS>::WORDS};
+            qmv_kernel<BITS, GS, GATHER, 2>, RG::CODE_STAGE + 2 * RG::SB_STAGE, RG::CBYTES,
+            RG::SWZ, RG::SBOX, Shape<BITS, GS>::KSLICE};
 }
 
 template <bool GATHER>
@@ -436,21 +435,19 @@ bool pick(int bits, int gs, Variant<GATHER>& v) {
     return false;
 }
 
-int kslice_of(int bits) { return bits == 8 ? 128 : 256; }
-
-constexpr size_t kSmemMax = 227 * 1024 - 256;
+constexpr size_t kSmemMax = 227 * 1024;
 
 // Split N over CTAs (every SM busy, at most 128 rows a CTA); size the slice
-// partials (nslices x rows x M fp32) and the deepest copy ring that fits.
+// partials (nslices x rows x M fp32) and the deepest ring that fits.
 struct Plan {
     int ctas, rows_cap, warps, depth;
     size_t smem;
 };
 
-Plan plan(int64_t N, int64_t K, int M, int bits, int words, int num_sms, bool gather) {
-    const int64_t nslices = (K + kslice_of(bits) - 1) / kslice_of(bits);
+Plan plan(int64_t N, int64_t K, int M, int kslice, int stage_bytes, int num_sms, bool gather) {
+    const int64_t nslices = (K + kslice - 1) / kslice;
     const int warps = static_cast<int>(std::min<int64_t>(kMaxWarps, nslices));
-    const size_t ring2 = static_cast<size_t>(warps) * 2 * words * 4;
+    auto ring = [&](int d) { return static_cast<size_t>(warps) * d * (stage_bytes + 8) + 1024 + 256; };
     // A gather launches one set of CTAs per (expert, <= 8 pairs) problem, so
     // its CTAs take up to 128 rows each instead of spreading one matrix over
     // every SM.
@@ -461,31 +458,72 @@ Plan plan(int64_t N, int64_t K, int M, int bits, int words, int num_sms, bool ga
         const int64_t rows = (N + ctas - 1) / ctas;
         const int64_t cap = (rows + 15) / 16 * 16;
         const size_t red = static_cast<size_t>(nslices * cap * M) * sizeof(float);
-        if (red + ring2 <= kSmemMax || cap <= 16) {
+        if (red + ring(2) <= kSmemMax || cap <= 16) {
             Plan p;
             p.ctas = static_cast<int>(ctas);
             p.rows_cap = static_cast<int>(cap);
             p.warps = warps;
             p.depth = 2;
             for (int d = 4; d > 2; --d)
-                if (red + static_cast<size_t>(warps) * d * words * 4 <= kSmemMax) { p.depth = d; break; }
-            p.smem = red + static_cast<size_t>(warps) * p.depth * words * 4;
+                if (red + ring(d) <= kSmemMax) { p.depth = d; break; }
+            p.smem = red + ring(p.depth);
             return p;
         }
         ctas = ctas * 2;
     }
 }
 
+// 3-D tensor maps [E][rows][inner] over the codes, scales and biases.
 template <bool GATHER>
-cudaError_t launch(const Variant<GATHER>& v, const Plan& p, dim3 grid, const QmvParams& prm,
+bool encode_maps(const Variant<GATHER>& v, const uint32_t* codes, const void* scales,
+                 const void* biases, int64_t E, int64_t N, int64_t K, int gs, int bits,
+                 CUtensorMap* mc, CUtensorMap* ms, CUtensorMap* mb, bool* sb_tma) {
+    EncodeTiled enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int64_t wpr = K * bits / 32, gpr = K / gs;
+    {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(E)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(wpr) * 4, static_cast<cuuint64_t>(wpr * N) * 4};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(v.code_row_bytes / 4), 16, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(codes), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                v.swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    // scales/biases by TMA when their rows are 16-byte multiples
+    *sb_tma = (gpr * 2) % 16 == 0;
+    if (*sb_tma) {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(E)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(gpr) * 2, static_cast<cuuint64_t>(gpr * N) * 2};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(v.sbox), 16, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        for (int i = 0; i < 2; ++i) {
+            if (enc(i ? mb : ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void*>(i ? biases : scales), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return false;
+        }
+    } else {
+        *ms = *mc;  // unused
+        *mb = *mc;
+    }
+    return true;
+}
+
+template <bool GATHER>
+cudaError_t launch(const Variant<GATHER>& v, const Plan& p, dim3 grid, const CUtensorMap& mc,
+                   const CUtensorMap& ms, const CUtensorMap& mb, const QmvParams& prm,
                    cudaStream_t stream) {
     KernelPtr<GATHER> k = p.depth == 4 ? v.k4 : p.depth == 3 ? v.k3 : v.k2;
-    if (p.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(p.smem));
-        if (e != cudaSuccess) return e;
-    }
-    k<<<grid, p.warps * 32, p.smem, stream>>>(prm);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(p.smem));
+    if (e != cudaSuccess) return e;
+    k<<<grid, p.warps * 32, p.smem, stream>>>(mc, ms, mb, prm);
     return cudaGetLastError();
 }
 
@@ -496,12 +534,18 @@ bool qmv_supported(int bits, int gs) {
     return pick<false>(bits, gs, v);
 }
 
+unsigned int qmv_error_take() { return pipeline_error_take(); }
+
 cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                        const void* scales, const void* biases, int gs, int bits, void* y,
                        cudaStream_t stream, int num_sms) {
     Variant<false> v;
     if (!pick<false>(bits, gs, v)) return cudaErrorInvalidValue;
-    Plan p = plan(N, K, static_cast<int>(M), bits, v.words, num_sms, false);
+    CUtensorMap mc, ms, mb;
+    bool sb_tma = false;
+    if (!encode_maps(v, codes, scales, biases, 1, N, K, gs, bits, &mc, &ms, &mb, &sb_tma))
+        return cudaErrorInvalidValue;
+    Plan p = plan(N, K, static_cast<int>(M), v.kslice, v.stage_bytes, num_sms, false);
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -513,7 +557,8 @@ cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uin
     prm.M = static_cast<int>(M);
     prm.ctas_per_problem = p.ctas;
     prm.rows_cap = p.rows_cap;
-    return launch<false>(v, p, dim3(p.ctas, 1, 1), prm, stream);
+    prm.sb_tma = sb_tma ? 1 : 0;
+    return launch<false>(v, p, dim3(p.ctas, 1, 1), mc, ms, mb, prm, stream);
 }
 
 cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_t* codes,
@@ -525,8 +570,12 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     Variant<true> v;
     if (!pick<true>(bits, gs, v)) return cudaErrorInvalidValue;
     if (max_problems <= 0) return cudaSuccess;
+    CUtensorMap mc, ms, mb;
+    bool sb_tma = false;
+    if (!encode_maps(v, codes, scales, biases, E, N, K, gs, bits, &mc, &ms, &mb, &sb_tma))
+        return cudaErrorInvalidValue;
     // Every problem covers all N rows of one expert for <= 8 pairs.
-    Plan p = plan(N, K, 8, bits, v.words, num_sms, true);
+    Plan p = plan(N, K, 8, v.kslice, v.stage_bytes, num_sms, true);
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -538,12 +587,14 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     prm.M = 8;
     prm.ctas_per_problem = p.ctas;
     prm.rows_cap = p.rows_cap;
+    prm.sb_tma = sb_tma ? 1 : 0;
     prm.lhs = lhs;
     prm.perm = perm;
     prm.problems = problems;
     prm.num_problems = num_problems;
     prm.E = E;
-    return launch<true>(v, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), prm, stream);
+    return launch<true>(v, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), mc, ms, mb,
+                        prm, stream);
 }
 
 }  // namespace nvq

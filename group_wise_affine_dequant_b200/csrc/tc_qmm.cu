@@ -1,12 +1,503 @@
+// Tensor-core quantized GEMM for many rows (the tiled kernel of "Docs /
+// Quantization", section "Products on the GPU"): y[M, N] = x[M, K] . w^T, bf16
+// activations, weights [N, K] as packed codes + per-group scale and bias.
+//
+// Blackwell design (sm_100a, one CTA per SM, persistent over 128 x BN tiles):
+//   warp 0      TMA producer: the x tile (128 x 64 bf16, 128-byte swizzle) and
+//               the packed code tile (BN rows x 64 k) per k-step, into a ring
+//               of NS stages, completing on mbarriers.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (kind::f16,
+//               M = 128, N = BN, K = 16) from shared memory into a TMEM fp32
+//               accumulator, double-buffered across tiles, and frees ring
+//               stages with tcgen05.commit.
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (32 lanes each), round to
+//               bf16, store y.
+//   warps 6-13  dequantize: each thread owns one weight row of the tile; it
+//               turns its codes into bf16 w = scale * code + bias (one rounding:
+//               the code is made exact first, then one bf16 fma) and writes the
+//               row into the B tile in the canonical K-major 128-byte-swizzled
+//               layout the MMA reads.
+// The contraction runs on the tensor cores in bf16 with fp32 accumulation; the
+// dequantized weight is rounded once to bf16 (relative error <= 2^-9), and the
+// result once to bf16 on output: together within the product tolerance.
+// Every wait on an mbarrier is bounded by a timer; on expiry the kernel records
+// an error code, stops issuing work and exits after draining its copies.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
 #include "tc.cuh"
+#include "tma.cuh"
 
 namespace nvq {
+namespace {
 
-bool tc_supported(int64_t, int64_t, int64_t, int, int) { return false; }
+constexpr int BM = 128;          // rows of x per tile (TMEM lanes)
+constexpr int BK = 64;           // k per stage: one 128-byte swizzle atom of bf16
+constexpr int UMMA_K = 16;
+constexpr int kThreads = 448;    // 14 warps
+constexpr int kDequantWarp0 = 6;
+constexpr int kDequantThreads = 256;
 
-cudaError_t launch_tc_qmm(const void*, int64_t, int64_t, int64_t, const uint32_t*, const void*,
-                          const void*, int, int, void*, cudaStream_t, int) {
-    return cudaErrorNotSupported;
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes stacked along M/N (stride 1024), Blackwell descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(const void* p) {
+    const uint64_t addr = smem_u32(p);
+    return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// ---------------------------------------------------------------- dequantizer
+// One word of codes -> bf16 weights w = s * c + b for consecutive k, written
+// as 32-bit pairs out[0..PAIRS). s2 / b2: bf16x2 (s, s) and (b, b).
+template <int BITS>
+struct Dequant;
+
+template <>
+struct Dequant<4> {  // word: 8 codes -> 4 pairs
+    static constexpr int PAIRS = 4;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
+                                               float, uint32_t* out) {
+        const uint32_t v = w >> 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // bytes (w.byte_i, -, v.byte_i, -): low nibbles are codes 2i and 2i+1
+            const uint32_t sel = i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12);
+            const uint32_t r = codes_to_bf16x2(prmt(w, v, sel), 0x000F000Fu);  // 128 + c
+            out[i] = bf2_fma(s2, bf2_sub(r, 0x43004300u), b2);
+        }
+    }
+};
+
+template <>
+struct Dequant<2> {  // word: 16 codes -> 8 pairs
+    static constexpr int PAIRS = 8;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
+                                               float, uint32_t* out) {
+        const uint32_t v1 = w >> 2, v2 = w >> 4, v3 = w >> 6;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t sel = i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12);
+            const uint32_t r0 = codes_to_bf16x2(prmt(w, v1, sel), 0x00030003u);   // codes 4i, 4i+1
+            const uint32_t r1 = codes_to_bf16x2(prmt(v2, v3, sel), 0x00030003u);  // codes 4i+2, 4i+3
+            out[2 * i] = bf2_fma(s2, bf2_sub(r0, 0x43004300u), b2);
+            out[2 * i + 1] = bf2_fma(s2, bf2_sub(r1, 0x43004300u), b2);
+        }
+    }
+};
+
+template <>
+struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes
+    static constexpr int PAIRS = 2;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t, uint32_t, float s, float b,
+                                               uint32_t* out) {
+        const uint32_t magic = 0x4B000000u;  // 2^23: byte i -> 2^23 + c_i
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float c0 = __uint_as_float(prmt(w, magic, (2 * i) | 0x7440)) - 8388608.0f;
+            const float c1 = __uint_as_float(prmt(w, magic, (2 * i + 1) | 0x7440)) - 8388608.0f;
+            out[i] = f2_to_bf2(fmaf(s, c0, b), fmaf(s, c1, b));
+        }
+    }
+};
+
+struct TcParams {
+    uint16_t* y;
+    const uint16_t* scales;
+    const uint16_t* biases;
+    int64_t M, N, K;
+    int gs;
+    int bn;            // tile columns (weight rows), multiple of 32, <= 256
+    int m_tiles, n_tiles;
+    int stages;
+    uint32_t a_off, b_off, c_off, bar_off;  // shared-memory layout (bytes)
+    uint32_t b_stage_bytes, c_stage_bytes;
+    uint32_t tmem_cols;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
+              const TcParams prm) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base: the 128-byte swizzle pattern repeats every 8 rows
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NS = prm.stages;
+    const int BN = prm.bn;
+    uint8_t* a_ring = smem + prm.a_off;
+    uint8_t* b_ring = smem + prm.b_off;
+    uint8_t* c_ring = smem + prm.c_off;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.bar_off);
+    uint64_t* full_a = bars;
+    uint64_t* full_c = bars + NS;
+    uint64_t* full_b = bars + 2 * NS;
+    uint64_t* empty = bars + 3 * NS;
+    uint64_t* acc_full = bars + 4 * NS;
+    uint64_t* acc_empty = bars + 4 * NS + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * NS + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&full_c[s], 1);
+            mbar_init(&full_b[s], kDequantThreads / 32);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(prm.tmem_cols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t ksteps = prm.K / BK;
+    const int tiles = prm.m_tiles * prm.n_tiles;
+    const uint32_t a_bytes = BM * BK * 2;
+    const uint32_t c_bytes = static_cast<uint32_t>(BN) * BK * BITS / 8;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int64_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
+                for (int64_t ks = 0; ks < ksteps && ok; ++ks, ++it) {
+                    const int s = static_cast<int>(it % NS);
+                    const uint32_t use = static_cast<uint32_t>(it / NS);
+                    if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, 1))) break;
+                    mbar_expect_tx(&full_a[s], a_bytes);
+                    tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], static_cast<int>(ks * BK),
+                                mt * BM);
+                    mbar_expect_tx(&full_c[s], c_bytes);
+                    tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
+                                static_cast<int>(ks * BK * BITS / 32), nt * BN);
+                }
+            }
+            // drain: the last loads in flight land before the CTA may exit
+            for (int64_t j = it - NS; j < it; ++j) {
+                if (j < 0) continue;
+                const int s = static_cast<int>(j % NS);
+                const uint32_t use = static_cast<uint32_t>(j / NS);
+                mbar_wait(&full_a[s], use & 1, 9);
+                mbar_wait(&full_c[s], use & 1, 9);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, BN);
+            int64_t it = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+                const int a = local & 1;
+                const uint32_t ause = static_cast<uint32_t>(local >> 1);
+                if (ause > 0 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, 2))) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
+                for (int64_t ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = static_cast<int>(it % NS);
+                    const uint32_t use = static_cast<uint32_t>(it / NS);
+                    if (!(ok = mbar_wait(&full_a[s], use & 1, 3))) break;
+                    if (!(ok = mbar_wait(&full_b[s], use & 1, 4))) break;
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(a_ring + s * a_bytes);
+                    const uint64_t bd = sw128_desc(b_ring + s * prm.b_stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        // advance 16 bf16 (32 bytes) along K inside the swizzle atom
+                        tc_mma(d_tmem, ad + (kk * UMMA_K * 2 >> 4), bd + (kk * UMMA_K * 2 >> 4), idesc,
+                               (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                if (ok) tc_commit(&acc_full[a]);
+            }
+        }
+    } else if (warp < kDequantWarp0) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int row_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+            const int a = local & 1;
+            const uint32_t ause = static_cast<uint32_t>(local >> 1);
+            if (!mbar_wait(&acc_full[a], ause & 1, 5)) break;
+            tc_fence_after();
+            const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
+            const int64_t row = static_cast<int64_t>(mt) * BM + row_in_tile;
+            const int64_t col0 = static_cast<int64_t>(nt) * BN;
+            for (int j = 0; j < BN / 32; ++j) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                       static_cast<uint32_t>(a * BN + j * 32);
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                    "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                    "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                      "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                      "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+                      "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+                      "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                    : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                const int64_t c = col0 + j * 32;
+                if (row < prm.M) {
+                    uint16_t* yp = prm.y + row * prm.N + c;
+                    if (c + 32 <= prm.N && (prm.N % 8) == 0) {
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            uint4 o;
+                            o.x = f2_to_bf2(__uint_as_float(v[8 * h + 0]), __uint_as_float(v[8 * h + 1]));
+                            o.y = f2_to_bf2(__uint_as_float(v[8 * h + 2]), __uint_as_float(v[8 * h + 3]));
+                            o.z = f2_to_bf2(__uint_as_float(v[8 * h + 4]), __uint_as_float(v[8 * h + 5]));
+                            o.w = f2_to_bf2(__uint_as_float(v[8 * h + 6]), __uint_as_float(v[8 * h + 7]));
+                            *reinterpret_cast<uint4*>(yp + 8 * h) = o;
+                        }
+                    } else {
+                        for (int e = 0; e < 32; ++e)
+                            if (c + e < prm.N) yp[e] = f32_to_bf16_bits(__uint_as_float(v[e]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
+        }
+    } else {
+        // ------------------------------------------------------------ dequantize
+        const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 255
+        const int r = dt;                                 // weight row within the tile
+        const bool has_row = r < BN;
+        const int64_t gpr = prm.K / prm.gs;
+        constexpr int WPS = BK * BITS / 32;  // code words per row per k-step
+        using DQ = Dequant<BITS>;
+        int64_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            const int nt = tile / prm.m_tiles;
+            const int64_t n = static_cast<int64_t>(nt) * BN + r;
+            const bool live = has_row && n < prm.N;
+            const uint16_t* srow = prm.scales + (live ? n : 0) * gpr;
+            const uint16_t* brow = prm.biases + (live ? n : 0) * gpr;
+            for (int64_t ks = 0; ks < ksteps; ++ks, ++it) {
+                const int s = static_cast<int>(it % NS);
+                const uint32_t use = static_cast<uint32_t>(it / NS);
+                // this k-step's one or two groups (loaded before waiting for the codes)
+                const int64_t k0 = ks * BK;
+                const int64_t gfirst = k0 / prm.gs;
+                float sf[2] = {0.f, 0.f}, bf[2] = {0.f, 0.f};
+                if (live) {
+                    sf[0] = bf16_bits_to_f32(__ldg(srow + gfirst));
+                    bf[0] = bf16_bits_to_f32(__ldg(brow + gfirst));
+                    if (prm.gs < BK) {
+                        sf[1] = bf16_bits_to_f32(__ldg(srow + gfirst + 1));
+                        bf[1] = bf16_bits_to_f32(__ldg(brow + gfirst + 1));
+                    }
+                }
+                if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
+                if (has_row) {
+                    const uint32_t* crow = reinterpret_cast<const uint32_t*>(
+                        c_ring + s * prm.c_stage_bytes) + r * WPS;
+                    uint32_t w[WPS];
+#pragma unroll
+                    for (int i = 0; i < WPS; i += 4) {
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(crow + i);
+                        w[i] = v4.x; w[i + 1] = v4.y; w[i + 2] = v4.z; w[i + 3] = v4.w;
+                    }
+                    uint8_t* brow_s = b_ring + s * prm.b_stage_bytes + (r >> 3) * 1024 + (r & 7) * 128;
+                    // 8 chunks of 8 k (16 bytes) per row and k-step
+                    constexpr int WPC = 8 * BITS / 32 > 0 ? 8 * BITS / 32 : 1;  // words per chunk
+#pragma unroll
+                    for (int c = 0; c < 8; c += (BITS == 2 ? 2 : 1)) {
+                        const int gi = (prm.gs < BK && c >= 4) ? 1 : 0;  // 32-groups: chunks 4..7
+                        const float sc = sf[gi], bc = bf[gi];
+                        const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
+                        const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
+                        uint32_t out[8];
+                        if constexpr (BITS == 2) {
+                            DQ::run(w[c / 2], s2, b2, sc, bc, out);  // 16 k: chunks c, c+1
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < WPC; ++u) DQ::run(w[c * WPC + u], s2, b2, sc, bc, out + u * DQ::PAIRS);
+                        }
+#pragma unroll
+                        for (int h = 0; h < (BITS == 2 ? 2 : 1); ++h) {
+                            const int cc = c + h;
+                            uint4 o;
+                            o.x = out[4 * h]; o.y = out[4 * h + 1]; o.z = out[4 * h + 2]; o.w = out[4 * h + 3];
+                            *reinterpret_cast<uint4*>(brow_s + ((cc ^ (r & 7)) << 4)) = o;
+                        }
+                    }
+                    fence_proxy_async();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_b[s]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(prm.tmem_cols));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+int pick_bn(int64_t M, int64_t N, int num_sms) {
+    const int64_t mt = (M + BM - 1) / BM;
+    int best = 256;
+    double best_eff = -1.0;
+    for (int bn = 256; bn >= 128; bn -= 32) {
+        const int64_t tiles = mt * ((N + bn - 1) / bn);
+        const int64_t waves = (tiles + num_sms - 1) / num_sms;
+        // useful work over the work of the waves, counting padded columns
+        const double eff = static_cast<double>(M * N) /
+                           (static_cast<double>(waves * num_sms) * BM * bn);
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = bn; }
+    }
+    return best;
+}
+
+}  // namespace
+
+unsigned int tc_error_take() { return pipeline_error_take(); }
+
+bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
+    return M > 0 && N > 0 && K % BK == 0 && K >= BK && (bits == 2 || bits == 4 || bits == 8) &&
+           (gs == 32 || gs == 64 || gs == 128) && M < (int64_t(1) << 31) && N < (int64_t(1) << 31);
+}
+
+cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+                          const void* scales, const void* biases, int gs, int bits, void* y,
+                          cudaStream_t stream, int num_sms) {
+    EncodeTiled enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const int bn = pick_bn(M, N, num_sms);
+    CUtensorMap map_x, map_c;
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+        cuuint32_t box[2] = {BK, BM};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const int64_t wpr = K * bits / 32;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(BK * bits / 32), static_cast<cuuint32_t>(bn)};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&map_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    TcParams prm{};
+    prm.y = static_cast<uint16_t*>(y);
+    prm.scales = static_cast<const uint16_t*>(scales);
+    prm.biases = static_cast<const uint16_t*>(biases);
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.gs = gs;
+    prm.bn = bn;
+    prm.m_tiles = static_cast<int>((M + BM - 1) / BM);
+    prm.n_tiles = static_cast<int>((N + bn - 1) / bn);
+    const uint32_t a_stage = BM * BK * 2;                         // 16 KB, 1024-aligned
+    const uint32_t b_stage = static_cast<uint32_t>(bn) * BK * 2;  // bn * 128
+    const uint32_t c_stage = (static_cast<uint32_t>(bn) * BK * bits / 8 + 1023) / 1024 * 1024;
+    const uint32_t per_stage = a_stage + b_stage + c_stage;
+    const uint32_t budget = 227 * 1024 - 1024 - 256;
+    int stages = static_cast<int>(budget / per_stage);
+    if (stages > 6) stages = 6;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    prm.stages = stages;
+    prm.a_off = 0;
+    prm.b_off = a_stage * stages;
+    prm.c_off = prm.b_off + b_stage * stages;
+    prm.bar_off = prm.c_off + c_stage * stages;
+    prm.b_stage_bytes = b_stage;
+    prm.c_stage_bytes = c_stage;
+    prm.tmem_cols = 2 * bn <= 256 ? 256 : 512;
+    const size_t smem = prm.bar_off + (4 * stages + 4) * 8 + 16 + 1024;  // + alignment slack
+    const int tiles = prm.m_tiles * prm.n_tiles;
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    void (*k)(const CUtensorMap, const CUtensorMap, const TcParams) =
+        bits == 4 ? tc_qmm_kernel<4> : bits == 8 ? tc_qmm_kernel<8> : tc_qmm_kernel<2>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, smem, stream>>>(map_x, map_c, prm);
+    return cudaGetLastError();
 }
 
 }  // namespace nvq

@@ -149,6 +149,15 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
  * *host_flags (a HOST pointer). Synchronises `stream`. */
 nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream);
 
+/*
+ * Read and clear the sticky error word of the asynchronous (TMA / tensor-core)
+ * pipelines into *host_code (a HOST pointer): 0 when every wait inside the
+ * kernels completed; otherwise a nonzero code naming the first wait that gave
+ * up after its time limit (the kernel then stopped early, and its outputs are
+ * not valid). Synchronises the device.
+ */
+nv_status nv_pipeline_error(uint32_t* host_code);
+
 #ifdef __cplusplus
 }
 #endif

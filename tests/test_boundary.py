@@ -110,6 +110,7 @@ def test_gather_argument_errors():
 
 def test_flags_argument_errors():
     L = nvq.lib()
+    assert L.nv_pipeline_error(0) == B.NV_ERR_INVALID_ARG
     flags = C.c_uint32(0)
     assert L.nv_gather_qmm_flags(0, C.addressof(flags), None) == B.NV_ERR_INVALID_ARG
     assert L.nv_gather_qmm_flags(16, 0, None) == B.NV_ERR_INVALID_ARG

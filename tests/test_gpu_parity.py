@@ -323,3 +323,62 @@ def test_moe_gather_sorted_and_unsorted(moe_case):
     rows = torch.tensor([0, 1, 777, 2047])
     yr, a = O.gather_qmm(x, c, s, b, lhs[rows], rhs[rows], 64, 4)
     P.assert_within(y_u[rows], yr, a, BF16, "moe rows")
+
+
+# ------------------------------------------------------------------- prefill
+@pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (4, 128), (2, 64), (8, 64), (8, 32), (2, 128)])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (200, 480, 640), (9, 100, 128), (300, 1000, 512)])
+def test_prefill_small(bits, gs, M, N, K):
+    """Tensor-core tiles: ragged M (rows beyond a 128 tile), ragged N (beyond a
+    column tile), several k-steps, every width and group size."""
+    if K % gs:
+        pytest.skip("K must be a multiple of the group size")
+    _check_product(N, K, M, bits, gs, True)
+
+
+def test_prefill_deterministic_and_integer_exact():
+    w = W.normal((512, 512), 0.02, 8, "bf16")
+    c, s, b = P.to_dev(*O.quantize_affine(w, 64, 4))
+    x = W.normal((300, 512), 1.0, 9, "bf16").cuda()
+    y1 = nvq.nv_qmm(x, c, s, b, 64, 4, True)
+    y2 = nvq.nv_qmm(x, c, s, b, 64, 4, True)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    gen = torch.Generator().manual_seed(77)
+    wi = P.integer_weights(256, 512, 64, 4, gen)
+    xi = torch.randint(-2, 3, (200, 512), generator=gen)
+    xi[:, 8:] = 0  # |y| <= 8 * 2 * 15 = 240: exact in bf16
+    ci, si, bi = O.quantize_affine(wi.to(BF16), 64, 4)
+    y = _run(xi.to(BF16), ci, si, bi, 64, 4, True)
+    yr, _ = O.qmm(xi.to(BF16), ci, si, bi, 64, 4, True)
+    assert torch.equal(y.to(torch.float64), yr)
+
+
+@pytest.fixture(scope="module")
+def prefill_inputs():
+    w = W.normal((14336, 4096), 0.02, 0, "bf16")
+    x = W.activations(2048, 4096)
+    return w, x
+
+
+@pytest.mark.parametrize("bits,gs", W.PREFILL_VARIANTS)
+def test_prefill_full(prefill_inputs, bits, gs):
+    """x [2048, 4096] . W[14336, 4096]^T at the five quantizations: sampled
+    outputs and whole rows against the oracle."""
+    w, x = prefill_inputs
+    c, s, b = O.quantize_affine(w, gs, bits)
+    y = _run(x, c, s, b, gs, bits, True)
+    assert tuple(y.shape) == (2048, 14336)
+    g = torch.Generator().manual_seed(bits * 100 + gs)
+    mi = torch.randint(0, 2048, (3000,), generator=g)
+    ni = torch.randint(0, 14336, (3000,), generator=g)
+    yr, a = O.qmm_sampled(x, c, s, b, gs, bits, True, mi, ni)
+    P.assert_within(y[mi, ni], yr, a, BF16, f"prefill b{bits} g{gs} sampled")
+    for m in (0, 1337, 2047):
+        yr, a = O.qmm(x[m:m + 1], c, s, b, gs, bits, True)
+        P.assert_within(y[m:m + 1], yr, a, BF16, f"prefill b{bits} g{gs} row {m}")
+
+
+def test_pipelines_never_timed_out():
+    """No wait inside the TMA / tensor-core pipelines gave up during the tests
+    above (the sticky error word is 0)."""
+    assert nvq.nv_pipeline_error() == 0
