@@ -16,7 +16,10 @@
 //               turns its codes into bf16 w = scale * code + bias (one rounding:
 //               the code is made exact first, then one bf16 fma) and writes the
 //               row into the B tile in the canonical K-major 128-byte-swizzled
-//               layout the MMA reads.
+//               layout the MMA reads. Codes arrive swizzled (32/64-byte TMA
+//               swizzle) so the row reads hit distinct banks; scales and biases
+//               arrive by TMA in blocks of 8 groups x BN rows through a 2-slot
+//               ring that the dequant warps release.
 // The contraction runs on the tensor cores in bf16 with fp32 accumulation; the
 // dequantized weight is rounded once to bf16 (relative error <= 2^-9), and the
 // result once to bf16 on output: together within the product tolerance.
@@ -96,8 +99,17 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- dequantizer
+// Right shift as mul.hi by a runtime power of two: it runs on the FMA pipe,
+// leaving the integer pipe to the byte permutes and masks.
+__device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t m) {
+    uint32_t r;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(m));
+    return r;
+}
+
 // One word of codes -> bf16 weights w = s * c + b for consecutive k, written
-// as 32-bit pairs out[0..PAIRS). s2 / b2: bf16x2 (s, s) and (b, b).
+// as 32-bit pairs out[0..PAIRS). s2 / b2: bf16x2 (s, s) and (b, b); m2/m4/m6:
+// the multipliers 2^30, 2^28, 2^26 (right shifts by 2, 4, 6).
 template <int BITS>
 struct Dequant;
 
@@ -105,8 +117,9 @@ template <>
 struct Dequant<4> {  // word: 8 codes -> 4 pairs
     static constexpr int PAIRS = 4;
     __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
-                                               float, uint32_t* out) {
-        const uint32_t v = w >> 4;
+                                               float, uint32_t, uint32_t m4, uint32_t,
+                                               uint32_t* out) {
+        const uint32_t v = shr(w, m4);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             // bytes (w.byte_i, -, v.byte_i, -): low nibbles are codes 2i and 2i+1
@@ -121,8 +134,9 @@ template <>
 struct Dequant<2> {  // word: 16 codes -> 8 pairs
     static constexpr int PAIRS = 8;
     __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
-                                               float, uint32_t* out) {
-        const uint32_t v1 = w >> 2, v2 = w >> 4, v3 = w >> 6;
+                                               float, uint32_t m2, uint32_t m4, uint32_t m6,
+                                               uint32_t* out) {
+        const uint32_t v1 = shr(w, m2), v2 = shr(w, m4), v3 = shr(w, m6);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t sel = i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12);
@@ -138,7 +152,7 @@ template <>
 struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes
     static constexpr int PAIRS = 2;
     __device__ static __forceinline__ void run(uint32_t w, uint32_t, uint32_t, float s, float b,
-                                               uint32_t* out) {
+                                               uint32_t, uint32_t, uint32_t, uint32_t* out) {
         const uint32_t magic = 0x4B000000u;  // 2^23: byte i -> 2^23 + c_i
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -161,11 +175,15 @@ struct TcParams {
     uint32_t a_off, b_off, c_off, bar_off;  // shared-memory layout (bytes)
     uint32_t b_stage_bytes, c_stage_bytes;
     uint32_t tmem_cols;
+    uint32_t sb_off;          // scale/bias ring: 2 slots x (scales, biases) x bn x 16 bytes
+    int sb_tma;               // scales/biases by TMA (rows of 16-byte multiples)
+    uint32_t m2, m4, m6;      // shift multipliers 2^30, 2^28, 2^26
 };
 
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
+              const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_b,
               const TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base: the 128-byte swizzle pattern repeats every 8 rows
@@ -183,7 +201,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     uint64_t* empty = bars + 3 * NS;
     uint64_t* acc_full = bars + 4 * NS;
     uint64_t* acc_empty = bars + 4 * NS + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * NS + 4);
+    uint64_t* sb_full = bars + 4 * NS + 4;
+    uint64_t* sb_empty = bars + 4 * NS + 6;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * NS + 8);
+    uint8_t* sb_ring = smem + prm.sb_off;
+    const uint32_t sb_slot_bytes = 2u * BN * 16u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -195,6 +217,8 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 4);
+            mbar_init(&sb_full[a], 1);
+            mbar_init(&sb_empty[a], kDequantThreads / 32);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -210,6 +234,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     const uint32_t tmem_base = *tmem_slot;
 
     const int64_t ksteps = prm.K / BK;
+    const int sgk = 8 * prm.gs / BK;  // k-steps per block of 8 groups
     const int tiles = prm.m_tiles * prm.n_tiles;
     const uint32_t a_bytes = BM * BK * 2;
     const uint32_t c_bytes = static_cast<uint32_t>(BN) * BK * BITS / 8;
@@ -218,10 +243,22 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int64_t it = 0;
+            uint32_t blk = 0;  // scale/bias blocks issued
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
                 const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
                 for (int64_t ks = 0; ks < ksteps && ok; ++ks, ++it) {
+                    if (prm.sb_tma && ks % sgk == 0) {
+                        const int slot = blk & 1;
+                        const uint32_t u = blk >> 1;
+                        if (u > 0 && !(ok = mbar_wait(&sb_empty[slot], (u - 1) & 1, 7))) break;
+                        mbar_expect_tx(&sb_full[slot], sb_slot_bytes);
+                        uint8_t* dst = sb_ring + slot * sb_slot_bytes;
+                        const int gcol = static_cast<int>(ks / sgk * 8);
+                        tma_load_2d(dst, &map_s, &sb_full[slot], gcol, nt * BN);
+                        tma_load_2d(dst + BN * 16, &map_b, &sb_full[slot], gcol, nt * BN);
+                        ++blk;
+                    }
                     const int s = static_cast<int>(it % NS);
                     const uint32_t use = static_cast<uint32_t>(it / NS);
                     if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, 1))) break;
@@ -335,6 +372,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         constexpr int WPS = BK * BITS / 32;  // code words per row per k-step
         using DQ = Dequant<BITS>;
         int64_t it = 0;
+        uint32_t blk = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             const int nt = tile / prm.m_tiles;
@@ -345,11 +383,23 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             for (int64_t ks = 0; ks < ksteps; ++ks, ++it) {
                 const int s = static_cast<int>(it % NS);
                 const uint32_t use = static_cast<uint32_t>(it / NS);
-                // this k-step's one or two groups (loaded before waiting for the codes)
                 const int64_t k0 = ks * BK;
                 const int64_t gfirst = k0 / prm.gs;
                 float sf[2] = {0.f, 0.f}, bf[2] = {0.f, 0.f};
-                if (live) {
+                const int slot = blk & 1;
+                if (prm.sb_tma) {
+                    if (ks % sgk == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
+                    if (has_row) {
+                        const uint16_t* ss = reinterpret_cast<const uint16_t*>(sb_ring + slot * sb_slot_bytes);
+                        const int gi = static_cast<int>(gfirst % 8);
+                        sf[0] = bf16_bits_to_f32(ss[r * 8 + gi]);
+                        bf[0] = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi]);
+                        if (prm.gs < BK) {
+                            sf[1] = bf16_bits_to_f32(ss[r * 8 + gi + 1]);
+                            bf[1] = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi + 1]);
+                        }
+                    }
+                } else if (live) {
                     sf[0] = bf16_bits_to_f32(__ldg(srow + gfirst));
                     bf[0] = bf16_bits_to_f32(__ldg(brow + gfirst));
                     if (prm.gs < BK) {
@@ -359,12 +409,17 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 }
                 if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
                 if (has_row) {
-                    const uint32_t* crow = reinterpret_cast<const uint32_t*>(
-                        c_ring + s * prm.c_stage_bytes) + r * WPS;
+                    const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
                     uint32_t w[WPS];
 #pragma unroll
                     for (int i = 0; i < WPS; i += 4) {
-                        const uint4 v4 = *reinterpret_cast<const uint4*>(crow + i);
+                        // logical 16-byte chunk i/4 of row r under the code tile's swizzle
+                        const int j = i / 4;
+                        uint32_t off;
+                        if constexpr (BITS == 4) off = r * 32 + ((j ^ ((r >> 2) & 1)) << 4);
+                        else if constexpr (BITS == 8) off = r * 64 + ((j ^ ((r >> 1) & 3)) << 4);
+                        else off = r * 16;
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(cst + off);
                         w[i] = v4.x; w[i + 1] = v4.y; w[i + 2] = v4.z; w[i + 3] = v4.w;
                     }
                     uint8_t* brow_s = b_ring + s * prm.b_stage_bytes + (r >> 3) * 1024 + (r & 7) * 128;
@@ -378,10 +433,12 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                         const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
                         uint32_t out[8];
                         if constexpr (BITS == 2) {
-                            DQ::run(w[c / 2], s2, b2, sc, bc, out);  // 16 k: chunks c, c+1
+                            DQ::run(w[c / 2], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out);  // 16 k
                         } else {
 #pragma unroll
-                            for (int u = 0; u < WPC; ++u) DQ::run(w[c * WPC + u], s2, b2, sc, bc, out + u * DQ::PAIRS);
+                            for (int u = 0; u < WPC; ++u)
+                                DQ::run(w[c * WPC + u], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6,
+                                        out + u * DQ::PAIRS);
                         }
 #pragma unroll
                         for (int h = 0; h < (BITS == 2 ? 2 : 1); ++h) {
@@ -395,6 +452,10 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);
+                if (prm.sb_tma && (ks % sgk == sgk - 1 || ks == ksteps - 1)) {
+                    if (lane == 0) mbar_arrive(&sb_empty[slot]);  // this warp is done with the block
+                    ++blk;
+                }
             }
         }
     }
@@ -456,12 +517,40 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
         cuuint32_t box[2] = {static_cast<cuuint32_t>(BK * bits / 32), static_cast<cuuint32_t>(bn)};
         cuuint32_t es[2] = {1, 1};
+        // 32/64-byte swizzle of the code rows: the dequant threads' row reads
+        // then fall on distinct banks
+        const CUtensorMapSwizzle swz = bits == 4   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                       : bits == 8 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                   : CU_TENSOR_MAP_SWIZZLE_NONE;
         if (enc(&map_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides,
-                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    // scales and biases: blocks of 8 groups x bn rows, when rows are 16-byte multiples
+    CUtensorMap map_s, map_b;
+    const int64_t gpr = K / gs;
+    const bool sb_tma = (gpr * 2) % 16 == 0;
+    if (sb_tma) {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(gpr) * 2};
+        cuuint32_t box[2] = {8, static_cast<cuuint32_t>(bn)};
+        cuuint32_t es[2] = {1, 1};
+        for (int i = 0; i < 2; ++i)
+            if (enc(i ? &map_b : &map_s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(i ? biases : scales), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+    } else {
+        map_s = map_c;
+        map_b = map_c;
+    }
     TcParams prm{};
+    prm.sb_tma = sb_tma ? 1 : 0;
+    prm.m2 = 1u << 30;
+    prm.m4 = 1u << 28;
+    prm.m6 = 1u << 26;
     prm.y = static_cast<uint16_t*>(y);
     prm.scales = static_cast<const uint16_t*>(scales);
     prm.biases = static_cast<const uint16_t*>(biases);
@@ -476,7 +565,8 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     const uint32_t b_stage = static_cast<uint32_t>(bn) * BK * 2;  // bn * 128
     const uint32_t c_stage = (static_cast<uint32_t>(bn) * BK * bits / 8 + 1023) / 1024 * 1024;
     const uint32_t per_stage = a_stage + b_stage + c_stage;
-    const uint32_t budget = 227 * 1024 - 1024 - 256;
+    const uint32_t sb_ring = 2u * 2u * static_cast<uint32_t>(bn) * 16u;  // 2 slots x (s, b)
+    const uint32_t budget = 227 * 1024 - 1024 - 512 - sb_ring;
     int stages = static_cast<int>(budget / per_stage);
     if (stages > 6) stages = 6;
     if (stages < 2) return cudaErrorInvalidConfiguration;
@@ -484,19 +574,21 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     prm.a_off = 0;
     prm.b_off = a_stage * stages;
     prm.c_off = prm.b_off + b_stage * stages;
-    prm.bar_off = prm.c_off + c_stage * stages;
+    prm.sb_off = prm.c_off + c_stage * stages;
+    prm.bar_off = prm.sb_off + sb_ring;
     prm.b_stage_bytes = b_stage;
     prm.c_stage_bytes = c_stage;
     prm.tmem_cols = 2 * bn <= 256 ? 256 : 512;
-    const size_t smem = prm.bar_off + (4 * stages + 4) * 8 + 16 + 1024;  // + alignment slack
+    const size_t smem = prm.bar_off + (4 * stages + 8) * 8 + 16 + 1024;  // + alignment slack
     const int tiles = prm.m_tiles * prm.n_tiles;
     const int grid = tiles < num_sms ? tiles : num_sms;
-    void (*k)(const CUtensorMap, const CUtensorMap, const TcParams) =
+    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+              const TcParams) =
         bits == 4 ? tc_qmm_kernel<4> : bits == 8 ? tc_qmm_kernel<8> : tc_qmm_kernel<2>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, stream>>>(map_x, map_c, prm);
+    k<<<grid, kThreads, smem, stream>>>(map_x, map_c, map_s, map_b, prm);
     return cudaGetLastError();
 }
 
