@@ -57,41 +57,29 @@ struct Shape {
     static_assert(CK <= GS && GS % CK == 0, "a chunk lies inside one group");
 };
 
-// Right shifts as mul.hi by 2^(32-s): they run on the FMA pipe instead of the
-// integer ALU pipe, which the masks below already keep busy. The multipliers
-// come from kernel parameters, so the compiler cannot turn them back into shifts.
-struct Shifts {
-    uint32_t m2, m4, m6, m8, m10, m12, m14;  // 2^(32-s) for s = 2, 4, ..., 14
-};
-__device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t m) {
-    uint32_t r;
-    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(m));
-    return r;
-}
-
 // Word -> NP bf16x2 registers; MMA u of the word uses p[2u] (k-slots 2t, 2t+1)
 // and p[2u+1] (k-slots 2t+8, 2t+9).
 template <int BITS>
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* p, const Shifts& sh) {
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* p) {
     if constexpr (BITS == 4) {
         p[0] = codes_to_bf16x2(w, 0x000F000Fu);               // (c0, c4)
-        p[1] = codes_to_bf16x2(shr(w, sh.m4), 0x000F000Fu);   // (c1, c5)
-        p[2] = codes_to_bf16x2(shr(w, sh.m8), 0x000F000Fu);   // (c2, c6)
-        p[3] = codes_to_bf16x2(shr(w, sh.m12), 0x000F000Fu);  // (c3, c7)
+        p[1] = codes_to_bf16x2((w >> 4), 0x000F000Fu);   // (c1, c5)
+        p[2] = codes_to_bf16x2((w >> 8), 0x000F000Fu);   // (c2, c6)
+        p[3] = codes_to_bf16x2((w >> 12), 0x000F000Fu);  // (c3, c7)
     } else if constexpr (BITS == 8) {
         p[0] = codes_to_bf16x2(w, 0x000F000Fu);               // low halves of (c0, c2)
-        p[1] = codes_to_bf16x2(shr(w, sh.m8), 0x000F000Fu);   // low halves of (c1, c3)
-        p[2] = codes_to_bf16x2(shr(w, sh.m4), 0x000F000Fu);   // high halves of (c0, c2)
-        p[3] = codes_to_bf16x2(shr(w, sh.m12), 0x000F000Fu);  // high halves of (c1, c3)
+        p[1] = codes_to_bf16x2((w >> 8), 0x000F000Fu);   // low halves of (c1, c3)
+        p[2] = codes_to_bf16x2((w >> 4), 0x000F000Fu);   // high halves of (c0, c2)
+        p[3] = codes_to_bf16x2((w >> 12), 0x000F000Fu);  // high halves of (c1, c3)
     } else {
         p[0] = codes_to_bf16x2(w, 0x00030003u);  // (c_s, c_s+8) for s = 0..7
-        p[1] = codes_to_bf16x2(shr(w, sh.m2), 0x00030003u);
-        p[2] = codes_to_bf16x2(shr(w, sh.m4), 0x00030003u);
-        p[3] = codes_to_bf16x2(shr(w, sh.m6), 0x00030003u);
-        p[4] = codes_to_bf16x2(shr(w, sh.m8), 0x00030003u);
-        p[5] = codes_to_bf16x2(shr(w, sh.m10), 0x00030003u);
-        p[6] = codes_to_bf16x2(shr(w, sh.m12), 0x00030003u);
-        p[7] = codes_to_bf16x2(shr(w, sh.m14), 0x00030003u);
+        p[1] = codes_to_bf16x2((w >> 2), 0x00030003u);
+        p[2] = codes_to_bf16x2((w >> 4), 0x00030003u);
+        p[3] = codes_to_bf16x2((w >> 6), 0x00030003u);
+        p[4] = codes_to_bf16x2((w >> 8), 0x00030003u);
+        p[5] = codes_to_bf16x2((w >> 10), 0x00030003u);
+        p[6] = codes_to_bf16x2((w >> 12), 0x00030003u);
+        p[7] = codes_to_bf16x2((w >> 14), 0x00030003u);
     }
 }
 
@@ -136,7 +124,6 @@ struct QmvParams {
     int ctas_per_problem;    // G: CTAs along N
     int rows_cap;            // max rows of one CTA, multiple of 16
     int sb_tma;              // scales/biases staged by TMA (rows 16-byte aligned)
-    Shifts sh;
     // gather only
     const uint32_t* lhs;     // nullable
     const uint32_t* perm;
@@ -386,8 +373,8 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
                     uint32_t pa[S::NP], pb[S::NP];
-                    unpack_word<BITS>(wa[j], pa, prm.sh);
-                    unpack_word<BITS>(wb[j], pb, prm.sh);
+                    unpack_word<BITS>(wa[j], pa);
+                    unpack_word<BITS>(wb[j], pb);
 #pragma unroll
                     for (int u = 0; u < S::MPW; ++u)
                         mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
@@ -463,7 +450,6 @@ bool pick(int bits, int gs, Variant<GATHER>& v) {
 
 constexpr size_t kSmemMax = 227 * 1024;
 
-Shifts shifts() { return {1u << 30, 1u << 28, 1u << 26, 1u << 24, 1u << 22, 1u << 20, 1u << 18}; }
 
 // Split N over CTAs (every SM busy, at most 128 rows a CTA); size the slice
 // partials (nslices x rows x M fp32) and the deepest ring that fits.
@@ -586,7 +572,6 @@ cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uin
     prm.ctas_per_problem = p.ctas;
     prm.rows_cap = p.rows_cap;
     prm.sb_tma = sb_tma ? 1 : 0;
-    prm.sh = shifts();
     return launch<false>(v, p, dim3(p.ctas, 1, 1), mc, ms, mb, prm, stream);
 }
 
@@ -617,7 +602,6 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     prm.ctas_per_problem = p.ctas;
     prm.rows_cap = p.rows_cap;
     prm.sb_tma = sb_tma ? 1 : 0;
-    prm.sh = shifts();
     prm.lhs = lhs;
     prm.perm = perm;
     prm.problems = problems;

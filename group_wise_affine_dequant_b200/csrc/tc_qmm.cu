@@ -77,6 +77,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Block of 8 groups that k-step ks starts in (sgk k-steps per block).
+__device__ __forceinline__ int blk_in_tile(int ks, int sgk) { return ks / sgk; }
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -99,17 +102,11 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- dequantizer
-// Right shift as mul.hi by a runtime power of two: it runs on the FMA pipe,
-// leaving the integer pipe to the byte permutes and masks.
-__device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t m) {
-    uint32_t r;
-    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(m));
-    return r;
-}
+__device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t bits) { return w >> bits; }
 
 // One word of codes -> bf16 weights w = s * c + b for consecutive k, written
 // as 32-bit pairs out[0..PAIRS). s2 / b2: bf16x2 (s, s) and (b, b); m2/m4/m6:
-// the multipliers 2^30, 2^28, 2^26 (right shifts by 2, 4, 6).
+// the shift counts 2, 4, 6.
 template <int BITS>
 struct Dequant;
 
@@ -177,7 +174,8 @@ struct TcParams {
     uint32_t tmem_cols;
     uint32_t sb_off;          // scale/bias ring: 2 slots x (scales, biases) x bn x 16 bytes
     int sb_tma;               // scales/biases by TMA (rows of 16-byte multiples)
-    uint32_t m2, m4, m6;      // shift multipliers 2^30, 2^28, 2^26
+    uint32_t m2, m4, m6;      // shift counts 2, 4, 6
+    int lg_gs;                // log2(group size)
 };
 
 template <int BITS>
@@ -233,7 +231,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int64_t ksteps = prm.K / BK;
+    const int ksteps = static_cast<int>(prm.K / BK);
     const int sgk = 8 * prm.gs / BK;  // k-steps per block of 8 groups
     const int tiles = prm.m_tiles * prm.n_tiles;
     const uint32_t a_bytes = BM * BK * 2;
@@ -242,39 +240,40 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int64_t it = 0;
-            uint32_t blk = 0;  // scale/bias blocks issued
+            int s = 0;            // ring stage and its use count (no divisions in the loop)
+            uint32_t use = 0;
+            uint32_t blk = 0;     // scale/bias blocks issued
+            int issued = 0;       // loads issued (bounded by the drain below)
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
                 const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
-                for (int64_t ks = 0; ks < ksteps && ok; ++ks, ++it) {
-                    if (prm.sb_tma && ks % sgk == 0) {
+                int kb = 0;  // k-step within the current scale block
+                for (int ks = 0; ks < ksteps && ok; ++ks) {
+                    if (prm.sb_tma && kb == 0) {
                         const int slot = blk & 1;
                         const uint32_t u = blk >> 1;
                         if (u > 0 && !(ok = mbar_wait(&sb_empty[slot], (u - 1) & 1, 7))) break;
                         mbar_expect_tx(&sb_full[slot], sb_slot_bytes);
                         uint8_t* dst = sb_ring + slot * sb_slot_bytes;
-                        const int gcol = static_cast<int>(ks / sgk * 8);
+                        const int gcol = static_cast<int>((blk_in_tile(ks, sgk)) * 8);
                         tma_load_2d(dst, &map_s, &sb_full[slot], gcol, nt * BN);
                         tma_load_2d(dst + BN * 16, &map_b, &sb_full[slot], gcol, nt * BN);
                         ++blk;
                     }
-                    const int s = static_cast<int>(it % NS);
-                    const uint32_t use = static_cast<uint32_t>(it / NS);
+                    if (++kb == sgk) kb = 0;
                     if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, 1))) break;
                     mbar_expect_tx(&full_a[s], a_bytes);
-                    tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], static_cast<int>(ks * BK),
-                                mt * BM);
+                    tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], ks * BK, mt * BM);
                     mbar_expect_tx(&full_c[s], c_bytes);
                     tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
-                                static_cast<int>(ks * BK * BITS / 32), nt * BN);
+                                ks * BK * BITS / 32, nt * BN);
+                    ++issued;
+                    if (++s == NS) { s = 0; ++use; }
                 }
             }
             // drain: the last loads in flight land before the CTA may exit
-            for (int64_t j = it - NS; j < it; ++j) {
-                if (j < 0) continue;
-                const int s = static_cast<int>(j % NS);
-                const uint32_t use = static_cast<uint32_t>(j / NS);
+            for (int j = 0; j < NS && j < issued; ++j) {
+                if (--s < 0) { s = NS - 1; --use; }
                 mbar_wait(&full_a[s], use & 1, 9);
                 mbar_wait(&full_c[s], use & 1, 9);
             }
@@ -283,7 +282,8 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, BN);
-            int64_t it = 0;
+            int s = 0;
+            uint32_t use = 0;
             int local = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
@@ -292,9 +292,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 if (ause > 0 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, 2))) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
-                for (int64_t ks = 0; ks < ksteps; ++ks, ++it) {
-                    const int s = static_cast<int>(it % NS);
-                    const uint32_t use = static_cast<uint32_t>(it / NS);
+                for (int ks = 0; ks < ksteps; ++ks) {
                     if (!(ok = mbar_wait(&full_a[s], use & 1, 3))) break;
                     if (!(ok = mbar_wait(&full_b[s], use & 1, 4))) break;
                     tc_fence_after();
@@ -307,6 +305,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                                (ks > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
+                    if (++s == NS) { s = 0; ++use; }
                 }
                 if (ok) tc_commit(&acc_full[a]);
             }
@@ -371,27 +370,26 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         const int64_t gpr = prm.K / prm.gs;
         constexpr int WPS = BK * BITS / 32;  // code words per row per k-step
         using DQ = Dequant<BITS>;
-        int64_t it = 0;
+        int s = 0;
+        uint32_t use = 0;
         uint32_t blk = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             const int nt = tile / prm.m_tiles;
+            int kb = 0;
             const int64_t n = static_cast<int64_t>(nt) * BN + r;
             const bool live = has_row && n < prm.N;
             const uint16_t* srow = prm.scales + (live ? n : 0) * gpr;
             const uint16_t* brow = prm.biases + (live ? n : 0) * gpr;
-            for (int64_t ks = 0; ks < ksteps; ++ks, ++it) {
-                const int s = static_cast<int>(it % NS);
-                const uint32_t use = static_cast<uint32_t>(it / NS);
-                const int64_t k0 = ks * BK;
-                const int64_t gfirst = k0 / prm.gs;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int gfirst = (ks * BK) >> prm.lg_gs;
                 float sf[2] = {0.f, 0.f}, bf[2] = {0.f, 0.f};
                 const int slot = blk & 1;
                 if (prm.sb_tma) {
-                    if (ks % sgk == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
+                    if (kb == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
                     if (has_row) {
                         const uint16_t* ss = reinterpret_cast<const uint16_t*>(sb_ring + slot * sb_slot_bytes);
-                        const int gi = static_cast<int>(gfirst % 8);
+                        const int gi = gfirst & 7;
                         sf[0] = bf16_bits_to_f32(ss[r * 8 + gi]);
                         bf[0] = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi]);
                         if (prm.gs < BK) {
@@ -452,10 +450,12 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);
-                if (prm.sb_tma && (ks % sgk == sgk - 1 || ks == ksteps - 1)) {
+                if (prm.sb_tma && (kb == sgk - 1 || ks == ksteps - 1)) {
                     if (lane == 0) mbar_arrive(&sb_empty[slot]);  // this warp is done with the block
                     ++blk;
                 }
+                if (++kb == sgk) kb = 0;
+                if (++s == NS) { s = 0; ++use; }
             }
         }
     }
@@ -548,9 +548,10 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     }
     TcParams prm{};
     prm.sb_tma = sb_tma ? 1 : 0;
-    prm.m2 = 1u << 30;
-    prm.m4 = 1u << 28;
-    prm.m6 = 1u << 26;
+    prm.m2 = 2;
+    prm.m4 = 4;
+    prm.m6 = 6;
+    prm.lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
     prm.y = static_cast<uint16_t*>(y);
     prm.scales = static_cast<const uint16_t*>(scales);
     prm.biases = static_cast<const uint16_t*>(biases);
