@@ -143,7 +143,12 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
     if (e != cudaSuccess) return NV_ERR_CUDA;
     if (N == 0) return NV_OK;
-    (void)row_exact;  // every route below gives each pair the bits of its one-row product
+    // Tensor-core route: each expert's weights are read once for all its rows.
+    if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size))
+        return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
+                                               codes, scales, biases, group_size, bits, y, s, sms));
+    // Matrix-vector route (row_exact): every pair gets the bits of its one-row
+    // product nv_qmm(M = 1) with its expert's weights.
     if (dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size))
         return from_cuda(nvq::launch_qmv_gather(x, K, N, codes, scales, biases, group_size, bits,
                                                 lhs_idx, ws.perm, ws.problems, ws.num_problems,
@@ -166,8 +171,9 @@ nv_status nv_pipeline_error(uint32_t* host_code) {
     if (cudaDeviceSynchronize() != cudaSuccess) return NV_ERR_CUDA;
     const unsigned int a = nvq::qmv_error_take();
     const unsigned int b = nvq::tc_error_take();
-    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return NV_ERR_CUDA;
-    *host_code = a ? a : b;
+    const unsigned int c = nvq::tc_gather_error_take();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return NV_ERR_CUDA;
+    *host_code = a ? a : b ? b : c;
     return NV_OK;
 }
 

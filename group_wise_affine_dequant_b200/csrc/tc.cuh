@@ -14,4 +14,14 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
 // Read and clear the error word of the tensor-core kernels (synchronous).
 unsigned int tc_error_take();
 
+// Mixture-of-experts product on the tensor cores (transposed: weights as the
+// 128-row operand, each expert's gathered activation rows as N). perm/offsets
+// come from the gather router.
+bool tc_gather_supported(int64_t K, int64_t N, int bits, int gs);
+cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                             const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
+                             const uint32_t* codes, const void* scales, const void* biases, int gs,
+                             int bits, void* y, cudaStream_t stream, int num_sms);
+unsigned int tc_gather_error_take();
+
 }  // namespace nvq

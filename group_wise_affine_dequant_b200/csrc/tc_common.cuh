@@ -1,0 +1,135 @@
+// Device helpers shared by the tcgen05 kernels (sm_100a): tensor-core fences,
+// MMA issue and commit, shared-memory / instruction descriptors, bf16 pair
+// arithmetic, and the code -> bf16 weight dequantizers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "tma.cuh"
+
+namespace nvq {
+namespace tc {
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes stacked along M/N (stride 1024), Blackwell descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(const void* p) {
+    const uint64_t addr = smem_u32(p);
+    return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Block of 8 groups that k-step ks starts in (sgk k-steps per block).
+__device__ __forceinline__ int blk_in_tile(int ks, int sgk) { return ks / sgk; }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// ---------------------------------------------------------------- dequantizer
+__device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t bits) { return w >> bits; }
+
+// One word of codes -> bf16 weights w = s * c + b for consecutive k, written
+// as 32-bit pairs out[0..PAIRS). s2 / b2: bf16x2 (s, s) and (b, b); m2/m4/m6:
+// the shift counts 2, 4, 6.
+template <int BITS>
+struct Dequant;
+
+template <>
+struct Dequant<4> {  // word: 8 codes -> 4 pairs
+    static constexpr int PAIRS = 4;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
+                                               float, uint32_t, uint32_t m4, uint32_t,
+                                               uint32_t* out) {
+        const uint32_t v = shr(w, m4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // bytes (w.byte_i, -, v.byte_i, -): low nibbles are codes 2i and 2i+1
+            const uint32_t sel = i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12);
+            const uint32_t r = codes_to_bf16x2(prmt(w, v, sel), 0x000F000Fu);  // 128 + c
+            out[i] = bf2_fma(s2, bf2_sub(r, 0x43004300u), b2);
+        }
+    }
+};
+
+template <>
+struct Dequant<2> {  // word: 16 codes -> 8 pairs
+    static constexpr int PAIRS = 8;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
+                                               float, uint32_t m2, uint32_t m4, uint32_t m6,
+                                               uint32_t* out) {
+        const uint32_t v1 = shr(w, m2), v2 = shr(w, m4), v3 = shr(w, m6);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t sel = i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12);
+            const uint32_t r0 = codes_to_bf16x2(prmt(w, v1, sel), 0x00030003u);   // codes 4i, 4i+1
+            const uint32_t r1 = codes_to_bf16x2(prmt(v2, v3, sel), 0x00030003u);  // codes 4i+2, 4i+3
+            out[2 * i] = bf2_fma(s2, bf2_sub(r0, 0x43004300u), b2);
+            out[2 * i + 1] = bf2_fma(s2, bf2_sub(r1, 0x43004300u), b2);
+        }
+    }
+};
+
+template <>
+struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes
+    static constexpr int PAIRS = 2;
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t, uint32_t, float s, float b,
+                                               uint32_t, uint32_t, uint32_t, uint32_t* out) {
+        const uint32_t magic = 0x4B000000u;  // 2^23: byte i -> 2^23 + c_i
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float c0 = __uint_as_float(prmt(w, magic, (2 * i) | 0x7440)) - 8388608.0f;
+            const float c1 = __uint_as_float(prmt(w, magic, (2 * i + 1) | 0x7440)) - 8388608.0f;
+            out[i] = f2_to_bf2(fmaf(s, c0, b), fmaf(s, c1, b));
+        }
+    }
+};
+
+}  // namespace tc
+}  // namespace nvq

@@ -251,9 +251,12 @@ def test_gather_page_example(dt):
     P.assert_within(y, yr, a, x.dtype, "page example")
 
 
-@pytest.mark.parametrize("bits,gs", [(4, 64), (8, 32), (2, 128), (4, 128)])
-def test_gather_ragged(bits, gs):
-    """37 pairs over 5 experts (one empty, one with 17 pairs), random token map."""
+@pytest.mark.parametrize("bits,gs", [(4, 64), (8, 32), (2, 128), (4, 128), (4, 32), (8, 128)])
+@pytest.mark.parametrize("row_exact", [False, True])
+def test_gather_ragged(bits, gs, row_exact):
+    """37 pairs over 5 experts (one empty, one with 17 pairs), random token map:
+    both routes within tolerance of the oracle; under row_exact every pair
+    equals its one-row product with its expert's weights, bit for bit."""
     g = torch.Generator().manual_seed(41)
     E, N, K = 5, 200, 512
     w = W.normal((E, N, K), 0.02, 2, "bf16")
@@ -261,15 +264,32 @@ def test_gather_ragged(bits, gs):
     c, s, b = O.quantize_affine(w, gs, bits)
     rhs = torch.tensor([0] * 9 + [2] * 17 + [3] * 4 + [4] * 7)[torch.randperm(37, generator=g)]
     lhs = torch.randint(0, 23, (37,), generator=g)
-    y, flags = _gather(x, c, s, b, rhs, lhs, gs, bits)
+    y, flags = _gather(x, c, s, b, rhs, lhs, gs, bits, row_exact=row_exact)
     assert flags == 0
     yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, gs, bits)
-    P.assert_within(y, yr, a, BF16, "ragged gather")
-    # each pair equals its one-row product with its expert's weights
-    for r in range(37):
-        e, t = int(rhs[r]), int(lhs[r])
-        one = _run(x[t:t + 1], c[e], s[e], b[e], gs, bits, True)
-        assert torch.equal(one[0].view(torch.int16), y[r].view(torch.int16)), r
+    P.assert_within(y, yr, a, BF16, f"ragged gather row_exact={row_exact}")
+    if row_exact:
+        for r in range(37):
+            e, t = int(rhs[r]), int(lhs[r])
+            one = _run(x[t:t + 1], c[e], s[e], b[e], gs, bits, True)
+            assert torch.equal(one[0].view(torch.int16), y[r].view(torch.int16)), r
+
+
+def test_gather_many_pairs_per_expert():
+    """An expert with more pairs than one tensor-core pass holds (600 > 256)
+    and an expert whose weight rows end mid-tile (N = 300)."""
+    E, N, K = 3, 300, 256
+    w = W.normal((E, N, K), 0.02, 4, "bf16")
+    x = W.normal((700, K), 1.0, 5, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    g = torch.Generator().manual_seed(3)
+    rhs = torch.cat([torch.full((600,), 1), torch.full((40,), 2), torch.full((5,), 0)])
+    rhs = rhs[torch.randperm(645, generator=g)]
+    lhs = torch.randint(0, 700, (645,), generator=g)
+    y, flags = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    assert flags == 0
+    yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, 64, 4)
+    P.assert_within(y, yr, a, BF16, "many pairs")
 
 
 def test_gather_flags_and_invalid_ids():
@@ -319,6 +339,10 @@ def test_moe_gather_sorted_and_unsorted(moe_case):
     n_idx = torch.randint(0, 1536, (4096,), generator=g)
     yr, a = O.gather_qmm_sampled(x, c, s, b, lhs, rhs, 64, 4, True, r_idx, n_idx)
     P.assert_within(y_u[r_idx, n_idx], yr, a, BF16, "moe sampled")
+    # the row-exact route on the same workload
+    y_x, f_x = _gather(x, c, s, b, rhs, lhs, 64, 4, row_exact=True)
+    assert f_x == 0
+    P.assert_within(y_x[r_idx, n_idx], yr, a, BF16, "moe sampled, row_exact")
     # whole rows for a few pairs
     rows = torch.tensor([0, 1, 777, 2047])
     yr, a = O.gather_qmm(x, c, s, b, lhs[rows], rhs[rows], 64, 4)
