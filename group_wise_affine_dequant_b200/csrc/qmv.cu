@@ -36,7 +36,13 @@
 namespace nvq {
 namespace {
 
-template <int BITS, int GS>
+// MMA k-steps per warp slice. 8 keeps a warp's activation fragments at 16
+// registers, so 32 warps (64 registers each) fit an SM: twice the warps of a
+// 16-step slice to hide the latency of the unpack -> MMA -> scale chain.
+constexpr int kSteps = 8;
+constexpr int kMaxWarps = 32;
+
+template <int BITS, int GS, int STEPS = kSteps>
 struct Shape {
     static constexpr int PER = 32 / BITS;                // codes per word
     static constexpr int GW = GS * BITS / 32;            // words per group
@@ -46,7 +52,7 @@ struct Shape {
     static constexpr int CW = 4 * LW;                    // words per chunk (one lane quad)
     static constexpr int CK = CW * PER;                  // k per chunk
     static constexpr int MMAS = LW * MPW;                // MMAs per chunk
-    static constexpr int KS = 16 / MMAS;                 // chunks per warp slice
+    static constexpr int KS = STEPS / MMAS > 0 ? STEPS / MMAS : 1;  // chunks per warp slice
     static constexpr int KSLICE = KS * CK;               // k per warp slice
     static constexpr int GPS = KSLICE / GS > 0 ? KSLICE / GS : 1;  // groups per slice
     static constexpr int CPG = GS / CK;                  // chunks per group
@@ -132,7 +138,6 @@ struct QmvParams {
     int64_t E;
 };
 
-constexpr int kMaxWarps = 16;
 
 // Ring geometry of one warp: per stage, the code box (16 rows x CBYTES, TMA
 // 128-byte swizzle when CBYTES is 128) and the scale and bias boxes (16 rows x
@@ -141,14 +146,16 @@ template <int BITS, int GS>
 struct Ring {
     using S = Shape<BITS, GS>;
     static constexpr int CBYTES = S::KSLICE * BITS / 8;          // code bytes per row and slice
-    static constexpr bool SWZ = CBYTES == 128;
+    static constexpr bool SWZ = CBYTES >= 32;   // TMA swizzle span = row bytes (32/64/128)
     static constexpr int CODE_STAGE = 16 * CBYTES;               // 2048 or 1024
     static constexpr int SBOX = S::GPS > 8 ? S::GPS : 8;         // groups per scale box row
     static constexpr int SB_STAGE = 16 * SBOX * 2;               // one of scales / biases
     // byte offset of code word `word` of row `r` inside a code stage
     __device__ static __forceinline__ uint32_t code_off(int r, int word) {
         const uint32_t o = static_cast<uint32_t>(word) * 4;
-        if constexpr (SWZ) return r * 128 + ((((o >> 4) ^ (r & 7)) << 4) | (o & 15));
+        if constexpr (CBYTES == 128) return r * 128 + ((((o >> 4) ^ (r & 7)) << 4) | (o & 15));
+        else if constexpr (CBYTES == 64) return r * 64 + ((((o >> 4) ^ ((r >> 1) & 3)) << 4) | (o & 15));
+        else if constexpr (CBYTES == 32) return r * 32 + ((((o >> 4) ^ ((r >> 2) & 1)) << 4) | (o & 15));
         else return r * CBYTES + o;
     }
 };
@@ -422,7 +429,7 @@ struct Variant {
     KernelPtr<GATHER> k4, k3, k2;  // ring depth 4, 3, 2
     int stage_bytes;               // code + scale + bias bytes per warp and stage
     int code_row_bytes;            // code bytes per row and slice (TMA box row)
-    bool swizzle;
+    int swizzle_bytes;             // 0, 32, 64 or 128
     int sbox;                      // groups per scale box row
     int kslice;
 };
@@ -432,7 +439,7 @@ Variant<GATHER> variant() {
     using RG = Ring<BITS, GS>;
     return {qmv_kernel<BITS, GS, GATHER, 4>, qmv_kernel<BITS, GS, GATHER, 3>,
             qmv_kernel<BITS, GS, GATHER, 2>, RG::CODE_STAGE + 2 * RG::SB_STAGE, RG::CBYTES,
-            RG::SWZ, RG::SBOX, Shape<BITS, GS>::KSLICE};
+            RG::SWZ ? RG::CBYTES : 0, RG::SBOX, Shape<BITS, GS>::KSLICE};
 }
 
 template <bool GATHER>
@@ -503,7 +510,10 @@ bool encode_maps(const Variant<GATHER>& v, const uint32_t* codes, const void* sc
         cuuint32_t es[3] = {1, 1, 1};
         if (enc(mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(codes), dims, strides, box,
                 es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                v.swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                v.swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                : v.swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                : v.swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                        : CU_TENSOR_MAP_SWIZZLE_NONE,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
