@@ -25,7 +25,7 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_qmm", "nv_gather_qmm_workspace_size",
-           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error")
+           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error")
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
 _LOCK = threading.Lock()
@@ -68,6 +68,8 @@ def lib():
             L.nv_gather_qmm.restype = _i
             L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
             L.nv_gather_qmm_flags.restype = _i
+            L.nv_last_cuda_error.argtypes = []
+            L.nv_last_cuda_error.restype = C.c_char_p
             L.nv_pipeline_error.argtypes = [_p]
             L.nv_pipeline_error.restype = _i
             _LIB = L
@@ -80,7 +82,10 @@ def nv_status_string(status: int) -> str:
 
 def _check(fn: str, status: int):
     if status != NV_OK:
-        raise NvqError(fn, status, nv_status_string(status))
+        text = nv_status_string(status)
+        if status == NV_ERR_CUDA:
+            text += f" ({lib().nv_last_cuda_error().decode()})"
+        raise NvqError(fn, status, text)
 
 
 def _stream(stream) -> int:

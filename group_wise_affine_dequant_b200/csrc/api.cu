@@ -22,8 +22,13 @@ nv_status check_quant(int gs, int bits) {
 
 bool valid_dtype(nv_dtype dt) { return dt == NV_F32 || dt == NV_BF16; }
 
+// The last CUDA error a call of this thread returned as NV_ERR_CUDA
+// (diagnostics for nv_last_cuda_error).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
 nv_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return NV_OK;
+    t_last_cuda_error = e;
     return NV_ERR_CUDA;
 }
 
@@ -102,7 +107,7 @@ nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
                     cudaError_t e = nvq::launch_qmvt(
                         static_cast<const uint16_t*>(x) + m0 * K, mc, K, N, codes, scales, biases,
                         group_size, bits, static_cast<uint16_t*>(y) + m0 * N, s, sms);
-                    if (e != cudaSuccess) return NV_ERR_CUDA;
+                    if (e != cudaSuccess) return from_cuda(e);
                 }
                 return NV_OK;
             }
@@ -141,7 +146,7 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     const int sms = sm_count();
     nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
     cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
-    if (e != cudaSuccess) return NV_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     if (N == 0) return NV_OK;
     // Tensor-core route: each expert's weights are read once for all its rows.
     if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size))
@@ -164,6 +169,10 @@ nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_st
         cudaSuccess)
         return NV_ERR_CUDA;
     return from_cuda(cudaStreamSynchronize(s));
+}
+
+const char* nv_last_cuda_error(void) {
+    return cudaGetErrorName(t_last_cuda_error);
 }
 
 nv_status nv_pipeline_error(uint32_t* host_code) {

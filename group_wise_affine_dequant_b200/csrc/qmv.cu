@@ -455,7 +455,9 @@ bool pick(int bits, int gs, Variant<GATHER>& v) {
     return false;
 }
 
-constexpr size_t kSmemMax = 227 * 1024;
+// Dynamic shared memory budget: the per-block limit (227 KB) less the kernel's
+// static shared memory (the row maps and the 1024-byte alignment of the ring).
+constexpr size_t kSmemMax = 227 * 1024 - 2048;
 
 
 // Split N over CTAs (every SM busy, at most 128 rows a CTA); size the slice

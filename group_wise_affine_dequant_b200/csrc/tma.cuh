@@ -51,14 +51,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity; false (and the error word
 // set to `code`) if it did not complete within kWaitLimitNs or another wait of
 // the launch already gave up.
+// The time limit and the error word are checked once every 256 polls only: a
+// global load on every poll would flood the memory pipeline of a spinning warp.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned code) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    for (;;) {
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
-            atomicCAS(&g_pipeline_error, 0u, code);
-            return false;
+        if ((i & 255u) == 0) {
+            if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
+                atomicCAS(&g_pipeline_error, 0u, code);
+                return false;
+            }
         }
     }
 }

@@ -158,6 +158,10 @@ nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_st
  */
 nv_status nv_pipeline_error(uint32_t* host_code);
 
+/* Name of the CUDA error behind the last NV_ERR_CUDA this thread received
+ * (static storage; "cudaSuccess" if none). Diagnostics only. */
+const char* nv_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
