@@ -25,7 +25,8 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_qmm", "nv_gather_qmm_workspace_size",
-           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error")
+           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error",
+           "nv_gather_qmm_noalloc")
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
 _LOCK = threading.Lock()
@@ -68,6 +69,9 @@ def lib():
             L.nv_gather_qmm.restype = _i
             L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
             L.nv_gather_qmm_flags.restype = _i
+            L.nv_gather_qmm_noalloc.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p,
+                                                 _p, _p, _i, _i, _i, _i, _i, _p, _p]
+            L.nv_gather_qmm_noalloc.restype = _i
             L.nv_last_cuda_error.argtypes = []
             L.nv_last_cuda_error.restype = C.c_char_p
             L.nv_pipeline_error.argtypes = [_p]

@@ -21,9 +21,12 @@
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is a DEVICE pointer (unless stated otherwise) owned
- *     by the caller; the library allocates no device memory, keeps no state
- *     between calls and never synchronises the stream. All work is enqueued on
- *     `stream` (NULL = the legacy default stream), in call order.
+ *     by the caller; the library allocates no device memory and never
+ *     synchronises the stream (except nv_gather_qmm_flags and
+ *     nv_pipeline_error, whose job is to read a word back). The only state kept
+ *     between calls is the sticky pipeline error word (nv_pipeline_error) and
+ *     the fixed routing array of nv_gather_qmm_noalloc. All work is enqueued
+ *     on `stream` (NULL = the legacy default stream), in call order.
  *   - Device pointers must be 16-byte aligned.
  *   - Argument errors are found on the host before anything is launched and
  *     are returned synchronously: NV_ERR_INVALID_ARG (a shape, pointer or
@@ -157,6 +160,28 @@ nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_st
  * not valid). Synchronises the device.
  */
 nv_status nv_pipeline_error(uint32_t* host_code);
+
+/*
+ * nv_gather_qmm without a workspace argument, for callers that cannot allocate
+ * device memory (a host runtime that owns all memory and forbids allocation
+ * on its hot path, a plugin without an allocator, a real-time loop where
+ * cudaMalloc may block). The pages have no counterpart: this is an addition of
+ * this library. Arguments and results as nv_gather_qmm.
+ * The routing tables live in one fixed device array built into the library
+ * (about 200 KB, kept on every GPU that loads the library until exit):
+ * R <= 32768 pairs and E <= 256 experts, else NV_ERR_WORKSPACE before any
+ * launch. The first call on a device looks the array's address up (with that
+ * device current) and should come before any stream capture. Every call
+ * shares the array: calls that may overlap on the GPU race and must be
+ * serialised by the caller (one stream, or events). Nothing in the array needs
+ * to start at zero (each call writes every entry it reads). No device memory
+ * is allocated or freed.
+ */
+nv_status nv_gather_qmm_noalloc(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
+                                const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R,
+                                int64_t E, int64_t N, const uint32_t* codes, const void* scales,
+                                const void* biases, int group_size, int bits, int transpose,
+                                int sorted, int row_exact, void* y, nv_stream_t stream);
 
 /* Name of the CUDA error behind the last NV_ERR_CUDA this thread received
  * (static storage; "cudaSuccess" if none). Diagnostics only. */
