@@ -127,9 +127,17 @@ struct QmvParams {
     uint16_t* y;             // bf16 [*, N]
     int64_t N, K;
     int M;                   // rows (plain product)
-    int ctas_per_problem;    // G: CTAs along N
+    int ctas_per_problem;    // G: CTAs along N; CTA c takes rows_q + (c < rows_r) rows
+    int rows_q, rows_r;      // N / G and N % G
     int rows_cap;            // max rows of one CTA, multiple of 16
-    int sb_tma;              // scales/biases staged by TMA (rows 16-byte aligned)
+    int rows_max;            // max rows of one CTA (height of the scale/bias block)
+    // Scales and biases: 2 = the CTA's whole block by TMA once (nbox boxes of
+    // 2^sbw_log-byte rows along the groups, each in a `region`-byte area,
+    // swizzled like the code tiles); 1 = per tile with the codes; 0 = loads.
+    int sb_mode;
+    int sbw_log, nbox;
+    uint32_t region;
+    uint32_t off_sb, off_bar, off_red;  // shared-memory layout (bytes)
     // gather only
     const uint32_t* lhs;     // nullable
     const uint32_t* perm;
@@ -160,6 +168,17 @@ struct Ring {
     }
 };
 
+// Byte offset of group column `gc` of row `r` inside one scale/bias box region
+// with rows of 2^sbw_log bytes, under the TMA swizzle of that row width.
+__device__ __forceinline__ uint32_t sb_block_off(int r, int gc, int sbw_log) {
+    const uint32_t o = static_cast<uint32_t>(gc) * 2;
+    uint32_t c = o >> 4;
+    if (sbw_log == 7) c ^= r & 7;
+    else if (sbw_log == 6) c ^= (r >> 1) & 3;
+    else if (sbw_log == 5) c ^= (r >> 2) & 1;
+    return (static_cast<uint32_t>(r) << sbw_log) + (c << 4) + (o & 15);
+}
+
 template <int LW>
 __device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t* w) {
     if constexpr (LW == 1) {
@@ -173,7 +192,18 @@ __device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t* w) {
     }
 }
 
-template <int BITS, int GS, bool GATHER, int NS>
+// One lane of the warp, chosen by the hardware (all lanes must take part).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// M1: the call has one activation row (only column 0 of the MMA is live). The
+// arithmetic of every stored output is the same as in the general form.
+template <int BITS, int GS, bool GATHER, int NS, bool M1>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_s,
            const __grid_constant__ CUtensorMap map_b, const QmvParams prm) {
@@ -182,10 +212,11 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ int64_t s_xrow[8];
     __shared__ int64_t s_yrow[8];
-    __shared__ int s_expert;
 
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
+    // warp index as a warp-uniform value, so that the TMA operands derived from
+    // it stay in uniform registers
+    const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
     const int nwarps = blockDim.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t N = prm.N, K = prm.K;
@@ -196,7 +227,9 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     const uint16_t* biases = prm.biases;
     bool zero_problem = false;
     int expert = 0;
+    pdl_launch_dependents();
     if constexpr (GATHER) {
+        pdl_wait();  // the routing tables come from the previous kernel
         const uint32_t p = blockIdx.y;
         if (p >= __ldg(prm.num_problems)) return;
         const uint32_t e = __ldg(prm.problems + 4 * p);
@@ -214,19 +247,50 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             s_xrow[threadIdx.x] = prm.lhs ? __ldg(prm.lhs + pair) : pair;
         }
     } else {
-        M = prm.M;
+        // The weights are not written by kernels of this library's stream
+        // order that could still run, but the previous kernel may be anything:
+        // only L2 prefetches (coherent) touch memory before the wait.
+        {
+            const int cta = static_cast<int>(blockIdx.x);
+            const int r0 = cta * prm.rows_q + min(cta, prm.rows_r);
+            const int nrows = prm.rows_q + (cta < prm.rows_r ? 1 : 0);
+            const int nsl = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
+            // the first ring's worth of tiles of the warp's first slice
+            // (prefetching everything floods HBM while the previous kernel
+            // still streams its own tiles)
+            const int w = static_cast<int>(threadIdx.x >> 5);
+            if ((threadIdx.x & 31) == 0 && w < nsl) {
+                {
+                    const int cw = w * S::KSLICE * BITS / 32;
+                    const int gb = w * S::KSLICE / GS / RG::SBOX * RG::SBOX;
+                    for (int i = 0; i < NS && i * 16 < nrows; ++i) {
+                        tma_prefetch_3d(&map_c, cw, r0 + i * 16, 0);
+                        if (prm.sb_mode == 1) {
+                            tma_prefetch_3d(&map_s, gb, r0 + i * 16, 0);
+                            tma_prefetch_3d(&map_b, gb, r0 + i * 16, 0);
+                        }
+                    }
+                    if (prm.sb_mode == 2 && w < prm.nbox) {
+                        const int gcol = w << (prm.sbw_log - 1);
+                        tma_prefetch_3d(&map_s, gcol, r0, 0);
+                        tma_prefetch_3d(&map_b, gcol, r0, 0);
+                    }
+                }
+            }
+        }
+        pdl_wait();  // x may come from the previous kernel; y may still be read by it
+        M = M1 ? 1 : prm.M;
         if (threadIdx.x < M) {
             s_xrow[threadIdx.x] = threadIdx.x;
             s_yrow[threadIdx.x] = threadIdx.x;
         }
     }
-    (void)s_expert;
     __syncthreads();
 
-    const int64_t G = prm.ctas_per_problem;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * N / G;
-    const int64_t n1 = static_cast<int64_t>(blockIdx.x + 1) * N / G;
-    const int rows = static_cast<int>(n1 - n0);
+    const int cta = static_cast<int>(blockIdx.x);
+    const int64_t n0 = static_cast<int64_t>(cta) * prm.rows_q + min(cta, prm.rows_r);
+    const int rows = prm.rows_q + (cta < prm.rows_r ? 1 : 0);
+    const int64_t n1 = n0 + rows;
     if (rows <= 0) return;
 
     if (zero_problem) {
@@ -237,62 +301,90 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         return;
     }
 
-    // shared memory: [warps][NS] code stages | [warps][NS] scale+bias stages |
-    // [warps][NS] mbarriers | slice partials
+    // shared memory: [warps][NS] code stages | scale+bias block (mode 2) or
+    // [warps][NS] scale+bias stages (mode 1) | [warps][NS] + 1 mbarriers |
+    // slice partials
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int sb_mode = prm.sb_mode;
     uint8_t* code_ring = smem + static_cast<size_t>(warp) * NS * RG::CODE_STAGE;
-    uint8_t* sb_ring = smem + static_cast<size_t>(nwarps) * NS * RG::CODE_STAGE +
-                       static_cast<size_t>(warp) * NS * 2 * RG::SB_STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(
-        smem + static_cast<size_t>(nwarps) * NS * (RG::CODE_STAGE + 2 * RG::SB_STAGE)) + warp * NS;
-    float* red = reinterpret_cast<float*>(
-        smem + static_cast<size_t>(nwarps) * NS * (RG::CODE_STAGE + 2 * RG::SB_STAGE) +
-        static_cast<size_t>(nwarps) * NS * 8);
+    uint8_t* sb_base = smem + prm.off_sb;
+    uint8_t* sb_ring = sb_base + static_cast<size_t>(warp) * NS * 2 * RG::SB_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.off_bar);
+    uint64_t* full = bars + warp * NS;
+    uint64_t* sb_full = bars + nwarps * NS;
+    float* red = reinterpret_cast<float*>(smem + prm.off_red);
 
     if (lane == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+        if (warp == 0) mbar_init(sb_full, 1);
         mbar_init_fence();
     }
-    __syncwarp();
+    __syncthreads();
+    if (sb_mode == 2 && warp == 0 && elect_one()) {
+        // the CTA's scales and biases: rows [n0, n0 + rows_max), all groups
+        const uint32_t box = static_cast<uint32_t>(prm.rows_max) << prm.sbw_log;
+        mbar_expect_tx(sb_full, 2u * prm.nbox * box);
+        for (int bi = 0; bi < prm.nbox; ++bi) {
+            const int gcol = bi << (prm.sbw_log - 1);
+            tma_load_3d(sb_base + bi * prm.region, &map_s, sb_full, gcol, static_cast<int>(n0), expert);
+            tma_load_3d(sb_base + (prm.nbox + bi) * prm.region, &map_b, sb_full, gcol,
+                        static_cast<int>(n0), expert);
+        }
+    }
 
     const int tiles = (rows + 15) / 16;
     const int rows_cap = prm.rows_cap;
     const int nslices = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
     const uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
-    const bool sb_tma = prm.sb_tma != 0;
-    const uint32_t stage_bytes = RG::CODE_STAGE + (sb_tma ? 2 * RG::SB_STAGE : 0);
+    const uint32_t stage_bytes = RG::CODE_STAGE + (sb_mode == 1 ? 2 * RG::SB_STAGE : 0);
+    const int row0 = static_cast<int>(n0);
+    const int MC = M1 ? 1 : M;  // columns kept per row in the slice partials
+
+    // byte offsets of this lane's code words inside a stage (rows g and g + 8)
+    uint32_t offa[S::KS], offb[S::KS];
+#pragma unroll
+    for (int q = 0; q < S::KS; ++q) {
+        offa[q] = RG::code_off(g, q * S::CW + t * S::LW);
+        offb[q] = RG::code_off(g + 8, q * S::CW + t * S::LW);
+    }
+
     bool ok = true;
-    uint32_t it = 0;  // this warp's tile counter across its slices (ring position)
+    int st = 0;       // ring stage of this warp's next tile
+    uint32_t ph = 0;  // and the parity of its current use
 
     for (int sl = warp; sl < nslices && ok; sl += nwarps) {
-        const int64_t kslice0 = static_cast<int64_t>(sl) * S::KSLICE;
-        const int64_t g0 = kslice0 / GS;
-        const int gbox = static_cast<int>(g0 / RG::SBOX * RG::SBOX);  // scale box start (16-B aligned)
-        const int goff = static_cast<int>(g0 - gbox);                 // slice's first group in the box
-        const int cword = static_cast<int>(kslice0 * BITS / 32);
+        const int kslice0 = sl * S::KSLICE;
+        const int g0 = kslice0 / GS;
+        const int gbox = g0 / RG::SBOX * RG::SBOX;  // scale box start (16-B aligned)
+        const int goff = g0 - gbox;                 // slice's first group in the box
+        const int cword = kslice0 * BITS / 32;
 
-        // lane 0: copy tile `tile` of this slice into ring stage `st`
-        auto issue = [&](int tile, int st) {
-            uint64_t* bar = &full[st];
+        // one lane: copy tile `tile` of this slice into ring stage `s`
+        auto issue = [&](int tile, int s) {
+            uint64_t* bar = &full[s];
             mbar_expect_tx(bar, stage_bytes);
-            const int row = static_cast<int>(n0) + tile * 16;
-            tma_load_3d(code_ring + st * RG::CODE_STAGE, &map_c, bar, cword, row, expert);
-            if (sb_tma) {
-                uint8_t* sbs = sb_ring + st * 2 * RG::SB_STAGE;
+            const int row = row0 + tile * 16;
+            tma_load_3d(code_ring + s * RG::CODE_STAGE, &map_c, bar, cword, row, expert);
+            if (sb_mode == 1) {
+                uint8_t* sbs = sb_ring + s * 2 * RG::SB_STAGE;
                 tma_load_3d(sbs, &map_s, bar, gbox, row, expert);
                 tma_load_3d(sbs + RG::SB_STAGE, &map_b, bar, gbox, row, expert);
             }
         };
-        const uint32_t it0 = it;
-        if (lane == 0)
-            for (int i = 0; i < NS && i < tiles; ++i) issue(i, (it0 + i) % NS);
+        if (elect_one()) {
+            int s = st;
+            for (int i = 0; i < NS && i < tiles; ++i) {
+                issue(i, s);
+                if (++s == NS) s = 0;
+            }
+        }
 
         // ---- activations of this slice: B fragments and per-chunk sums ----
         uint32_t bfr[S::KS][S::MMAS][2];
         float xs[S::KS][2];
 #pragma unroll
         for (int q = 0; q < S::KS; ++q) {
-            const int64_t kq = kslice0 + q * S::CK;
+            const int64_t kq = static_cast<int64_t>(kslice0) + q * S::CK;
             const bool valid = kq < K && g < M;
 #pragma unroll
             for (int j = 0; j < S::LW; ++j) {
@@ -329,22 +421,40 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             xs[q][1] = d[1];
         }
 
+        const int oa = (g * RG::SBOX + goff) * 2, ob = ((g + 8) * RG::SBOX + goff) * 2;
+        const int sbgmask = (1 << (prm.sbw_log - 1)) - 1;  // group columns per box - 1
+        float* red_sl = red + sl * rows_cap * MC;
+
         // ---- walk the CTA's rows, 16 per tile, NS tiles in flight ----
-        for (int tile = 0; tile < tiles; ++tile, ++it) {
-            const int st = static_cast<int>(it % NS);
-            if (!(ok = mbar_wait(&full[st], (it / NS) & 1, 10))) break;
+        for (int tile = 0; tile < tiles; ++tile) {
+            if (!(ok = mbar_wait(&full[st], ph, 10))) break;
             const uint8_t* cst = code_ring + st * RG::CODE_STAGE;
-            const int64_t ra = n0 + tile * 16 + g, rb = ra + 8;
-            const bool va = ra < n1, vb = rb < n1;
 
             constexpr int SBR = S::GPS >= 2 ? S::GPS / 2 : 1;
             uint32_t sa[SBR], sb[SBR], ba[SBR], bb[SBR];
 #pragma unroll
             for (int i = 0; i < SBR; ++i) { sa[i] = sb[i] = ba[i] = bb[i] = 0u; }
-            if (sb_tma) {
+            if (sb_mode == 2) {
+                if (tile == 0 && sl == warp && !(ok = mbar_wait(sb_full, 0, 11))) break;
+                const int r_a = tile * 16 + g;
+                const uint32_t oa2 = sb_block_off(r_a, g0 & sbgmask, prm.sbw_log);
+                const uint32_t ob2 = sb_block_off(r_a + 8, g0 & sbgmask, prm.sbw_log);
+                const uint8_t* ss = sb_base + (g0 >> (prm.sbw_log - 1)) * prm.region;
+                const uint8_t* bs = ss + prm.nbox * prm.region;
+                if constexpr (S::GPS == 1) {
+                    sa[0] = *reinterpret_cast<const uint16_t*>(ss + oa2);
+                    sb[0] = *reinterpret_cast<const uint16_t*>(ss + ob2);
+                    ba[0] = *reinterpret_cast<const uint16_t*>(bs + oa2);
+                    bb[0] = *reinterpret_cast<const uint16_t*>(bs + ob2);
+                } else {
+                    lds_words<SBR>(ss + oa2, sa);
+                    lds_words<SBR>(ss + ob2, sb);
+                    lds_words<SBR>(bs + oa2, ba);
+                    lds_words<SBR>(bs + ob2, bb);
+                }
+            } else if (sb_mode == 1) {
                 const uint8_t* ss = sb_ring + st * 2 * RG::SB_STAGE;
                 const uint8_t* bs = ss + RG::SB_STAGE;
-                const int oa = (g * RG::SBOX + goff) * 2, ob = ((g + 8) * RG::SBOX + goff) * 2;
                 if constexpr (S::GPS == 1) {
                     sa[0] = *reinterpret_cast<const uint16_t*>(ss + oa);
                     sb[0] = *reinterpret_cast<const uint16_t*>(ss + ob);
@@ -357,9 +467,11 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                     lds_words<SBR>(bs + ob, bb);
                 }
             } else {
+                const int64_t ra = n0 + tile * 16 + g, rb = ra + 8;
+                const bool va = ra < n1, vb = rb < n1;
 #pragma unroll
                 for (int i = 0; i < S::GPS; ++i) {
-                    if ((g0 + i) * GS < K) {
+                    if ((g0 + i) * static_cast<int64_t>(GS) < K) {
                         const int sh = (i & 1) * 16;
                         if (va) { sa[i >> 1] |= uint32_t(__ldg(scales + ra * gpr + g0 + i)) << sh;
                                   ba[i >> 1] |= uint32_t(__ldg(biases + ra * gpr + g0 + i)) << sh; }
@@ -373,9 +485,8 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
             for (int q = 0; q < S::KS; ++q) {
                 uint32_t wa[S::LW], wb[S::LW];
-                const int word = q * S::CW + t * S::LW;
-                lds_words<S::LW>(cst + RG::code_off(g, word), wa);
-                lds_words<S::LW>(cst + RG::code_off(g + 8, word), wb);
+                lds_words<S::LW>(cst + offa[q], wa);
+                lds_words<S::LW>(cst + offb[q], wb);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
@@ -394,30 +505,45 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                 // columns 2t (every call) and 2t + 1 (only when a second row exists)
                 acc[0] = fmaf(b_a, xs[q][0], fmaf(s_a, d[0], acc[0]));
                 acc[2] = fmaf(b_b, xs[q][0], fmaf(s_b, d[2], acc[2]));
-                if (M > 1) {
+                if (!M1) {
                     acc[1] = fmaf(b_a, xs[q][1], fmaf(s_a, d[1], acc[1]));
                     acc[3] = fmaf(b_b, xs[q][1], fmaf(s_b, d[3], acc[3]));
                 }
             }
             // every lane has read the stage: refill it with tile + NS
             __syncwarp();
-            if (lane == 0 && tile + NS < tiles) issue(tile + NS, st);
+            if (tile + NS < tiles && elect_one()) issue(tile + NS, st);
+            if (++st == NS) { st = 0; ph ^= 1u; }
 
             const int r0 = tile * 16 + g;
-            float* base = red + static_cast<int64_t>(sl) * rows_cap * M;
-            const int m0 = 2 * t, m1 = 2 * t + 1;
-            if (m0 < M) { base[r0 * M + m0] = acc[0]; base[(r0 + 8) * M + m0] = acc[2]; }
-            if (m1 < M) { base[r0 * M + m1] = acc[1]; base[(r0 + 8) * M + m1] = acc[3]; }
+            if (M1) {
+                if (t == 0) { red_sl[r0] = acc[0]; red_sl[r0 + 8] = acc[2]; }
+            } else {
+                const int m0 = 2 * t, m1 = 2 * t + 1;
+                if (m0 < M) { red_sl[r0 * M + m0] = acc[0]; red_sl[(r0 + 8) * M + m0] = acc[2]; }
+                if (m1 < M) { red_sl[r0 * M + m1] = acc[1]; red_sl[(r0 + 8) * M + m1] = acc[3]; }
+            }
         }
     }
     __syncthreads();
 
-    // ---- fixed-order reduction over the slices ----
-    for (int i = threadIdx.x; i < rows * M; i += blockDim.x) {
-        const int m = i / rows, r = i % rows;
-        float v = red[static_cast<int64_t>(r) * M + m];
-        for (int sl = 1; sl < nslices; ++sl) v += red[(static_cast<int64_t>(sl) * rows_cap + r) * M + m];
-        prm.y[s_yrow[m] * N + n0 + r] = f32_to_bf16_bits(v);
+    // ---- fixed-order reduction over the slices: four interleaved chains
+    // (slices j, j + 4, j + 8, ...), then (c0 + c1) + (c2 + c3) ----
+    const int slice_stride = rows_cap * MC;
+    for (int m = 0; m < MC; ++m) {
+        for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+            const float* p = red + r * MC + m;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j < nslices) c[j] = p[j * slice_stride];
+            for (int sl = 4; sl < nslices; sl += 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (sl + j < nslices) c[j] += p[(sl + j) * slice_stride];
+            }
+            prm.y[s_yrow[m] * N + n0 + r] = f32_to_bf16_bits((c[0] + c[1]) + (c[2] + c[3]));
+        }
     }
 }
 
@@ -426,8 +552,9 @@ using KernelPtr = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorM
 
 template <bool GATHER>
 struct Variant {
-    KernelPtr<GATHER> k4, k3, k2;  // ring depth 4, 3, 2
-    int stage_bytes;               // code + scale + bias bytes per warp and stage
+    KernelPtr<GATHER> k[2][3];     // [one activation row][ring depth 4, 3, 2]
+    int code_stage;                // code bytes per warp and stage
+    int sb_stage;                  // bytes of one per-tile scale (or bias) box
     int code_row_bytes;            // code bytes per row and slice (TMA box row)
     int swizzle_bytes;             // 0, 32, 64 or 128
     int sbox;                      // groups per scale box row
@@ -437,9 +564,21 @@ struct Variant {
 template <int BITS, int GS, bool GATHER>
 Variant<GATHER> variant() {
     using RG = Ring<BITS, GS>;
-    return {qmv_kernel<BITS, GS, GATHER, 4>, qmv_kernel<BITS, GS, GATHER, 3>,
-            qmv_kernel<BITS, GS, GATHER, 2>, RG::CODE_STAGE + 2 * RG::SB_STAGE, RG::CBYTES,
-            RG::SWZ ? RG::CBYTES : 0, RG::SBOX, Shape<BITS, GS>::KSLICE};
+    Variant<GATHER> v{};
+    v.k[0][0] = qmv_kernel<BITS, GS, GATHER, 4, false>;
+    v.k[0][1] = qmv_kernel<BITS, GS, GATHER, 3, false>;
+    v.k[0][2] = qmv_kernel<BITS, GS, GATHER, 2, false>;
+    // a gather problem's row count is only known on the device
+    v.k[1][0] = GATHER ? v.k[0][0] : qmv_kernel<BITS, GS, GATHER, 4, !GATHER>;
+    v.k[1][1] = GATHER ? v.k[0][1] : qmv_kernel<BITS, GS, GATHER, 3, !GATHER>;
+    v.k[1][2] = GATHER ? v.k[0][2] : qmv_kernel<BITS, GS, GATHER, 2, !GATHER>;
+    v.code_stage = RG::CODE_STAGE;
+    v.sb_stage = RG::SB_STAGE;
+    v.code_row_bytes = RG::CBYTES;
+    v.swizzle_bytes = RG::SWZ ? RG::CBYTES : 0;
+    v.sbox = RG::SBOX;
+    v.kslice = Shape<BITS, GS>::KSLICE;
+    return v;
 }
 
 template <bool GATHER>
@@ -460,17 +599,24 @@ bool pick(int bits, int gs, Variant<GATHER>& v) {
 constexpr size_t kSmemMax = 227 * 1024 - 2048;
 
 
-// Split N over CTAs (every SM busy, at most 128 rows a CTA); size the slice
-// partials (nslices x rows x M fp32) and the deepest ring that fits.
+// Split N over CTAs (every SM busy, at most 128 rows a CTA); choose how the
+// scales and biases reach shared memory and the deepest ring that fits next to
+// the slice partials (nslices x rows x M fp32).
 struct Plan {
-    int ctas, rows_cap, warps, depth;
+    int ctas, rows_cap, rows_max, warps, depth;
+    int sb_mode, sbw_log, nbox;
+    uint32_t region, off_sb, off_bar, off_red;
     size_t smem;
 };
 
-Plan plan(int64_t N, int64_t K, int M, int kslice, int stage_bytes, int num_sms, bool gather) {
+static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Plan plan(int64_t N, int64_t K, int M, int gs, int kslice, int code_stage, int sb_stage,
+          int num_sms, bool gather) {
     const int64_t nslices = (K + kslice - 1) / kslice;
     const int warps = static_cast<int>(std::min<int64_t>(kMaxWarps, nslices));
-    auto ring = [&](int d) { return static_cast<size_t>(warps) * d * (stage_bytes + 8) + 1024 + 256; };
+    const int64_t gpr = K / gs;
+    const bool sb_aligned = (gpr * 2) % 16 == 0;  // rows of scales are 16-byte multiples
     // A gather launches one set of CTAs per (expert, <= 8 pairs) problem, so
     // its CTAs take up to 128 rows each instead of spreading one matrix over
     // every SM.
@@ -481,26 +627,53 @@ Plan plan(int64_t N, int64_t K, int M, int kslice, int stage_bytes, int num_sms,
         const int64_t rows = (N + ctas - 1) / ctas;
         const int64_t cap = (rows + 15) / 16 * 16;
         const size_t red = static_cast<size_t>(nslices * cap * M) * sizeof(float);
-        if (red + ring(2) <= kSmemMax || cap <= 16) {
-            Plan p;
-            p.ctas = static_cast<int>(ctas);
-            p.rows_cap = static_cast<int>(cap);
-            p.warps = warps;
-            p.depth = 2;
-            for (int d = 4; d > 2; --d)
-                if (red + ring(d) <= kSmemMax) { p.depth = d; break; }
-            p.smem = red + ring(p.depth);
-            return p;
+        Plan p{};
+        p.ctas = static_cast<int>(ctas);
+        p.rows_cap = static_cast<int>(cap);
+        p.rows_max = static_cast<int>(rows);
+        p.warps = warps;
+        // layout for ring depth d with `sb_stage_bytes` of scales per stage and
+        // `block` bytes of scale block; true if it fits
+        auto fit = [&](int d, size_t sb_stage_bytes, size_t block) {
+            const size_t codes = static_cast<size_t>(warps) * d * code_stage;
+            const size_t sb = block + static_cast<size_t>(warps) * d * sb_stage_bytes;
+            const size_t bars = round_up(static_cast<size_t>(warps * d + 1) * 8, 16);
+            p.depth = d;
+            p.off_sb = static_cast<uint32_t>(codes);
+            p.off_bar = static_cast<uint32_t>(codes + sb);
+            p.off_red = static_cast<uint32_t>(codes + sb + bars);
+            p.smem = 1024 + codes + sb + bars + red;
+            return p.smem <= kSmemMax;
+        };
+        // mode 2: the CTA's block of scales and biases, loaded once
+        if (sb_aligned && rows <= 256 && (gpr >= 64 || gpr == 8 || gpr == 16 || gpr == 32)) {
+            p.sb_mode = 2;
+            const int sbw = gpr >= 64 ? 128 : static_cast<int>(gpr) * 2;
+            p.sbw_log = sbw == 128 ? 7 : sbw == 64 ? 6 : sbw == 32 ? 5 : 4;
+            p.nbox = gpr >= 64 ? static_cast<int>((gpr + 63) / 64) : 1;
+            // the box holds rows_max rows; the region spans every row a tile can
+            // address (rows_cap), so reads past the CTA's rows stay inside it
+            p.region = static_cast<uint32_t>(round_up(static_cast<size_t>(cap) * sbw, 1024));
+            for (int d = 4; d >= 2; --d)
+                if (fit(d, 0, 2u * p.nbox * p.region)) return p;
         }
+        // mode 1: scales and biases per tile with the codes; mode 0: plain loads
+        p.sb_mode = sb_aligned ? 1 : 0;
+        p.sbw_log = 4;
+        p.nbox = 0;
+        p.region = 0;
+        for (int d = 4; d >= 2; --d)
+            if (fit(d, sb_aligned ? 2 * sb_stage : 0, 0)) return p;
+        if (cap <= 16) return p;  // nothing smaller to try: launch fails loudly
         ctas = ctas * 2;
     }
 }
 
 // 3-D tensor maps [E][rows][inner] over the codes, scales and biases.
 template <bool GATHER>
-bool encode_maps(const Variant<GATHER>& v, const uint32_t* codes, const void* scales,
-                 const void* biases, int64_t E, int64_t N, int64_t K, int gs, int bits,
-                 CUtensorMap* mc, CUtensorMap* ms, CUtensorMap* mb, bool* sb_tma) {
+bool encode_maps(const Variant<GATHER>& v, const Plan& p, const uint32_t* codes,
+                 const void* scales, const void* biases, int64_t E, int64_t N, int64_t K, int gs,
+                 int bits, CUtensorMap* mc, CUtensorMap* ms, CUtensorMap* mb) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return false;
     const int64_t wpr = K * bits / 32, gpr = K / gs;
@@ -519,38 +692,73 @@ bool encode_maps(const Variant<GATHER>& v, const uint32_t* codes, const void* sc
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
-    // scales/biases by TMA when their rows are 16-byte multiples
-    *sb_tma = (gpr * 2) % 16 == 0;
-    if (*sb_tma) {
-        cuuint64_t dims[3] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N),
-                              static_cast<cuuint64_t>(E)};
-        cuuint64_t strides[2] = {static_cast<cuuint64_t>(gpr) * 2, static_cast<cuuint64_t>(gpr * N) * 2};
-        cuuint32_t box[3] = {static_cast<cuuint32_t>(v.sbox), 16, 1};
-        cuuint32_t es[3] = {1, 1, 1};
-        for (int i = 0; i < 2; ++i) {
-            if (enc(i ? mb : ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                    const_cast<void*>(i ? biases : scales), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-                return false;
-        }
-    } else {
+    if (p.sb_mode == 0) {
         *ms = *mc;  // unused
         *mb = *mc;
+        return true;
+    }
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(gpr) * 2, static_cast<cuuint64_t>(gpr * N) * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(v.sbox), 16, 1};
+    CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (p.sb_mode == 2) {  // whole rows of the CTA, 2^sbw_log bytes of groups per box
+        box[0] = 1u << (p.sbw_log - 1);
+        box[1] = static_cast<cuuint32_t>(p.rows_max);
+        swz = p.sbw_log == 7   ? CU_TENSOR_MAP_SWIZZLE_128B
+              : p.sbw_log == 6 ? CU_TENSOR_MAP_SWIZZLE_64B
+              : p.sbw_log == 5 ? CU_TENSOR_MAP_SWIZZLE_32B
+                               : CU_TENSOR_MAP_SWIZZLE_NONE;
+    }
+    cuuint32_t es[3] = {1, 1, 1};
+    for (int i = 0; i < 2; ++i) {
+        if (enc(i ? mb : ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                const_cast<void*>(i ? biases : scales), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
     }
     return true;
+}
+
+static void set_plan(QmvParams& prm, const Plan& p, int64_t N) {
+    prm.ctas_per_problem = p.ctas;
+    prm.rows_q = static_cast<int>(N / p.ctas);
+    prm.rows_r = static_cast<int>(N % p.ctas);
+    prm.rows_cap = p.rows_cap;
+    prm.rows_max = p.rows_max;
+    prm.sb_mode = p.sb_mode;
+    prm.sbw_log = p.sbw_log;
+    prm.nbox = p.nbox;
+    prm.region = p.region;
+    prm.off_sb = p.off_sb;
+    prm.off_bar = p.off_bar;
+    prm.off_red = p.off_red;
 }
 
 template <bool GATHER>
 cudaError_t launch(const Variant<GATHER>& v, const Plan& p, dim3 grid, const CUtensorMap& mc,
                    const CUtensorMap& ms, const CUtensorMap& mb, const QmvParams& prm,
                    cudaStream_t stream) {
-    KernelPtr<GATHER> k = p.depth == 4 ? v.k4 : p.depth == 3 ? v.k3 : v.k2;
+    const int one = prm.M == 1 ? 1 : 0;
+    KernelPtr<GATHER> k = v.k[one][p.depth == 4 ? 0 : p.depth == 3 ? 1 : 2];
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(p.smem));
     if (e != cudaSuccess) return e;
-    k<<<grid, p.warps * 32, p.smem, stream>>>(mc, ms, mb, prm);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the kernel may start while the previous
+    // kernel on the stream drains; it waits (griddepcontrol.wait) before it
+    // reads anything but weights (prefetched into L2) or writes anything.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(static_cast<unsigned>(p.warps * 32), 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, mc, ms, mb, prm);
 }
 
 }  // namespace
@@ -567,11 +775,11 @@ cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uin
                        cudaStream_t stream, int num_sms) {
     Variant<false> v;
     if (!pick<false>(bits, gs, v)) return cudaErrorInvalidValue;
+    const Plan p = plan(N, K, static_cast<int>(M), gs, v.kslice, v.code_stage, v.sb_stage, num_sms,
+                        false);
     CUtensorMap mc, ms, mb;
-    bool sb_tma = false;
-    if (!encode_maps(v, codes, scales, biases, 1, N, K, gs, bits, &mc, &ms, &mb, &sb_tma))
+    if (!encode_maps(v, p, codes, scales, biases, 1, N, K, gs, bits, &mc, &ms, &mb))
         return cudaErrorInvalidValue;
-    Plan p = plan(N, K, static_cast<int>(M), v.kslice, v.stage_bytes, num_sms, false);
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -581,9 +789,7 @@ cudaError_t launch_qmv(const void* x, int64_t M, int64_t K, int64_t N, const uin
     prm.N = N;
     prm.K = K;
     prm.M = static_cast<int>(M);
-    prm.ctas_per_problem = p.ctas;
-    prm.rows_cap = p.rows_cap;
-    prm.sb_tma = sb_tma ? 1 : 0;
+    set_plan(prm, p, N);
     return launch<false>(v, p, dim3(p.ctas, 1, 1), mc, ms, mb, prm, stream);
 }
 
@@ -596,12 +802,11 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     Variant<true> v;
     if (!pick<true>(bits, gs, v)) return cudaErrorInvalidValue;
     if (max_problems <= 0) return cudaSuccess;
-    CUtensorMap mc, ms, mb;
-    bool sb_tma = false;
-    if (!encode_maps(v, codes, scales, biases, E, N, K, gs, bits, &mc, &ms, &mb, &sb_tma))
-        return cudaErrorInvalidValue;
     // Every problem covers all N rows of one expert for <= 8 pairs.
-    Plan p = plan(N, K, 8, v.kslice, v.stage_bytes, num_sms, true);
+    const Plan p = plan(N, K, 8, gs, v.kslice, v.code_stage, v.sb_stage, num_sms, true);
+    CUtensorMap mc, ms, mb;
+    if (!encode_maps(v, p, codes, scales, biases, E, N, K, gs, bits, &mc, &ms, &mb))
+        return cudaErrorInvalidValue;
     QmvParams prm{};
     prm.x = static_cast<const uint16_t*>(x);
     prm.codes = codes;
@@ -611,9 +816,7 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     prm.N = N;
     prm.K = K;
     prm.M = 8;
-    prm.ctas_per_problem = p.ctas;
-    prm.rows_cap = p.rows_cap;
-    prm.sb_tma = sb_tma ? 1 : 0;
+    set_plan(prm, p, N);
     prm.lhs = lhs;
     prm.perm = perm;
     prm.problems = problems;

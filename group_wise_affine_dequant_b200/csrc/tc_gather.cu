@@ -37,10 +37,12 @@ using namespace tc;
 constexpr int WM = 128;          // weight rows per unit (TMEM lanes)
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
-constexpr int kMaxPairs = 256;   // pairs per pass (TMEM columns of one accumulator)
-constexpr int kThreads = 448;
-constexpr int kDequantWarp0 = 6;
-constexpr int kDequantThreads = 256;
+constexpr int kMaxPairs = 128;   // pairs per pass (TMEM columns of one accumulator)
+constexpr int kEpilogueWarp0 = 2;
+constexpr int kXWarp = 6;        // activation-row producer
+constexpr int kDequantWarp0 = 7; // warps 7-22: dequantize, four threads per weight row
+constexpr int kDequantThreads = 512;
+constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
 
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int col, int r0, int r1, int r2, int r3) {
@@ -62,11 +64,19 @@ struct GParams {
     int64_t N, K, E;
     int gs, lg_gs;
     int wtiles;                 // ceil(N / 128)
-    int stages;
-    uint32_t a_off, x_off, c_off, sb_off, idx_off, bar_off;
+    int dx, dc, da;             // depths: gathered activations, codes, dequantized weights
+    uint32_t x_off, c_off, a_off, sb_off, idx_off, bar_off;
     uint32_t c_stage_bytes;
     int sb_tma;
     uint32_t m2, m4, m6;        // shift counts 2, 4, 6
+};
+
+struct RingPos {
+    int s = 0;
+    uint32_t use = 0;
+    __device__ __forceinline__ void next(int depth) {
+        if (++s == depth) { s = 0; ++use; }
+    }
 };
 
 template <int BITS>
@@ -77,45 +87,45 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int NS = prm.stages;
+    const int DX = prm.dx, DC = prm.dc, DA = prm.da;
     constexpr uint32_t A_STAGE = WM * BK * 2;            // 16 KB
-    constexpr uint32_t X_STAGE = kMaxPairs * BK * 2;     // 32 KB
+    constexpr uint32_t X_STAGE = kMaxPairs * BK * 2;     // 16 KB
     uint8_t* a_ring = smem + prm.a_off;
     uint8_t* x_ring = smem + prm.x_off;
     uint8_t* c_ring = smem + prm.c_off;
     uint8_t* sb_ring = smem + prm.sb_off;
     int* s_rows = reinterpret_cast<int*>(smem + prm.idx_off);  // activation row per pair
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.bar_off);
-    uint64_t* full_x = bars;            // gathered activations (TMA)
-    uint64_t* full_c = bars + NS;       // codes (TMA)
-    uint64_t* full_a = bars + 2 * NS;   // dequantized weights (dequant warps)
-    uint64_t* empty = bars + 3 * NS;    // stage consumed (tcgen05.commit)
-    uint64_t* acc_full = bars + 4 * NS;
-    uint64_t* acc_empty = bars + 4 * NS + 2;
-    uint64_t* sb_full = bars + 4 * NS + 4;
-    uint64_t* sb_empty = bars + 4 * NS + 6;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * NS + 8);
+    uint64_t* full_x = bars;
+    uint64_t* empty_x = full_x + DX;
+    uint64_t* full_c = empty_x + DX;
+    uint64_t* empty_c = full_c + DC;
+    uint64_t* full_a = empty_c + DC;
+    uint64_t* empty_a = full_a + DA;
+    uint64_t* acc_full = empty_a + DA;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* sb_full = acc_empty + 2;
+    uint64_t* sb_empty = sb_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sb_empty + 2);
     constexpr uint32_t SB_SLOT = 2u * WM * 16u;
+    constexpr int kDequantWarps = kDequantThreads / 32;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&full_x[s], 1);
-            mbar_init(&full_c[s], 1);
-            mbar_init(&full_a[s], kDequantThreads / 32);
-            mbar_init(&empty[s], 1);
-        }
+        for (int i = 0; i < DX; ++i) { mbar_init(&full_x[i], 1); mbar_init(&empty_x[i], 1); }
+        for (int i = 0; i < DC; ++i) { mbar_init(&full_c[i], 1); mbar_init(&empty_c[i], kDequantWarps); }
+        for (int i = 0; i < DA; ++i) { mbar_init(&full_a[i], kDequantWarps); mbar_init(&empty_a[i], 1); }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 4);
             mbar_init(&sb_full[a], 1);
-            mbar_init(&sb_empty[a], kDequantThreads / 32);
+            mbar_init(&sb_empty[a], kDequantWarps);
         }
         mbar_init_fence();
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(512));
+                     "r"(2 * kMaxPairs));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -137,9 +147,47 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     };
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        int s = 0;
-        uint32_t use = 0, blk = 0;
+        // -------------------------------------------- producer: codes, scales
+        if (lane == 0) {
+            RingPos c;
+            uint32_t blk = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int e, wt, first, count;
+                unit_pairs(u, e, wt, first, count);
+                for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
+                    int kb = 0;
+                    for (int ks = 0; ks < ksteps && ok; ++ks) {
+                        if (prm.sb_tma && kb == 0) {
+                            const int slot = blk & 1;
+                            const uint32_t bu = blk >> 1;
+                            if (bu > 0 && !(ok = mbar_wait(&sb_empty[slot], (bu - 1) & 1, 27))) break;
+                            mbar_expect_tx(&sb_full[slot], SB_SLOT);
+                            uint8_t* dst = sb_ring + slot * SB_SLOT;
+                            const int gcol = blk_in_tile(ks, sgk) * 8;
+                            tma_load_3d(dst, &map_s, &sb_full[slot], gcol, wt * WM, e);
+                            tma_load_3d(dst + WM * 16, &map_b, &sb_full[slot], gcol, wt * WM, e);
+                            ++blk;
+                        }
+                        if (++kb == sgk) kb = 0;
+                        if (c.use > 0 && !(ok = mbar_wait(&empty_c[c.s], (c.use - 1) & 1, 21))) break;
+                        mbar_expect_tx(&full_c[c.s], WM * BK * BITS / 8);
+                        tma_load_3d(c_ring + c.s * prm.c_stage_bytes, &map_c, &full_c[c.s],
+                                    ks * BK * BITS / 32, wt * WM, e);
+                        ++issued;
+                        c.next(DC);
+                    }
+                }
+            }
+            for (int j = 0; j < DC && j < issued; ++j) {  // drain the last copies
+                if (--c.s < 0) { c.s = DC - 1; --c.use; }
+                mbar_wait(&full_c[c.s], c.use & 1, 29);
+            }
+        }
+    } else if (warp == kXWarp) {
+        // -------------------------------------------- producer: activation rows
+        RingPos x;
         int issued = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -157,49 +205,31 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    int kb = 0;
                     for (int ks = 0; ks < ksteps && ok; ++ks) {
-                        if (prm.sb_tma && kb == 0) {
-                            const int slot = blk & 1;
-                            const uint32_t bu = blk >> 1;
-                            if (bu > 0 && !(ok = mbar_wait(&sb_empty[slot], (bu - 1) & 1, 27))) break;
-                            mbar_expect_tx(&sb_full[slot], SB_SLOT);
-                            uint8_t* dst = sb_ring + slot * SB_SLOT;
-                            const int gcol = blk_in_tile(ks, sgk) * 8;
-                            tma_load_3d(dst, &map_s, &sb_full[slot], gcol, wt * WM, e);
-                            tma_load_3d(dst + WM * 16, &map_b, &sb_full[slot], gcol, wt * WM, e);
-                            ++blk;
-                        }
-                        if (++kb == sgk) kb = 0;
-                        if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, 21))) break;
-                        mbar_expect_tx(&full_c[s], WM * BK * BITS / 8);
-                        tma_load_3d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
-                                    ks * BK * BITS / 32, wt * WM, e);
-                        mbar_expect_tx(&full_x[s], static_cast<uint32_t>(groups4) * 4 * BK * 2);
-                        uint8_t* xd = x_ring + s * X_STAGE;
+                        if (x.use > 0 && !(ok = mbar_wait(&empty_x[x.s], (x.use - 1) & 1, 31))) break;
+                        mbar_expect_tx(&full_x[x.s], static_cast<uint32_t>(groups4) * 4 * BK * 2);
+                        uint8_t* xd = x_ring + x.s * X_STAGE;
                         for (int g4 = 0; g4 < groups4; ++g4)
-                            tma_gather4(xd + g4 * 4 * BK * 2, &map_x, &full_x[s], ks * BK,
+                            tma_gather4(xd + g4 * 4 * BK * 2, &map_x, &full_x[x.s], ks * BK,
                                         s_rows[4 * g4], s_rows[4 * g4 + 1], s_rows[4 * g4 + 2],
                                         s_rows[4 * g4 + 3]);
                         ++issued;
-                        if (++s == NS) { s = 0; ++use; }
+                        x.next(DX);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             }
         }
         if (lane == 0) {
-            for (int j = 0; j < NS && j < issued; ++j) {  // drain the last copies
-                if (--s < 0) { s = NS - 1; --use; }
-                mbar_wait(&full_c[s], use & 1, 29);
-                mbar_wait(&full_x[s], use & 1, 29);
+            for (int j = 0; j < DX && j < issued; ++j) {
+                if (--x.s < 0) { x.s = DX - 1; --x.use; }
+                mbar_wait(&full_x[x.s], x.use & 1, 30);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int s = 0;
-            uint32_t use = 0;
+            RingPos x, a;
             int local = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -209,29 +239,31 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                     const int cn = min(kMaxPairs, count - p0);
                     const int npad = (cn + 15) / 16 * 16;
                     const uint32_t idesc = idesc_bf16(WM, npad);
-                    const int a = local & 1;
+                    const int acc = local & 1;
                     const uint32_t ause = static_cast<uint32_t>(local >> 1);
-                    if (ause > 0 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, 22))) break;
+                    if (ause > 0 && !(ok = mbar_wait(&acc_empty[acc], (ause - 1) & 1, 22))) break;
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kMaxPairs);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kMaxPairs);
                     for (int ks = 0; ks < ksteps; ++ks) {
-                        if (!(ok = mbar_wait(&full_a[s], use & 1, 23))) break;
-                        if (!(ok = mbar_wait(&full_x[s], use & 1, 24))) break;
+                        if (!(ok = mbar_wait(&full_a[a.s], a.use & 1, 23))) break;
+                        if (!(ok = mbar_wait(&full_x[x.s], x.use & 1, 24))) break;
                         tc_fence_after();
-                        const uint64_t ad = sw128_desc(a_ring + s * A_STAGE);
-                        const uint64_t bd = sw128_desc(x_ring + s * X_STAGE);
+                        const uint64_t ad = sw128_desc(a_ring + a.s * A_STAGE);
+                        const uint64_t bd = sw128_desc(x_ring + x.s * X_STAGE);
 #pragma unroll
                         for (int kk = 0; kk < BK / UMMA_K; ++kk)
                             tc_mma(d_tmem, ad + (kk * UMMA_K * 2 >> 4), bd + (kk * UMMA_K * 2 >> 4), idesc,
                                    (ks > 0 || kk > 0) ? 1u : 0u);
-                        tc_commit(&empty[s]);
-                        if (++s == NS) { s = 0; ++use; }
+                        tc_commit(&empty_a[a.s]);
+                        tc_commit(&empty_x[x.s]);
+                        a.next(DA);
+                        x.next(DX);
                     }
-                    if (ok) tc_commit(&acc_full[a]);
+                    if (ok) tc_commit(&acc_full[acc]);
                 }
             }
         }
-    } else if (warp < kDequantWarp0) {
+    } else if (warp < kEpilogueWarp0 + 4) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         const int wrow = q * 32 + lane;  // weight row within the unit = TMEM lane
@@ -243,14 +275,14 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
             const int64_t n = static_cast<int64_t>(wt) * WM + wrow;
             for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs, ++local) {
                 const int cn = min(kMaxPairs, count - p0);
-                const int a = local & 1;
+                const int acc = local & 1;
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
-                if (!(ok = mbar_wait(&acc_full[a], ause & 1, 25))) break;
+                if (!(ok = mbar_wait(&acc_full[acc], ause & 1, 25))) break;
                 tc_fence_after();
                 for (int c0 = 0; c0 < cn; c0 += 16) {
                     uint32_t v[16];
                     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                           static_cast<uint32_t>(a * kMaxPairs + c0);
+                                           static_cast<uint32_t>(acc * kMaxPairs + c0);
                     asm volatile(
                         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
                         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -270,20 +302,19 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[a]);
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
             }
         }
-    } else {
+    } else if (warp >= kDequantWarp0) {
         // ------------------------------------------------------------ dequantize
-        const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 255
-        const int r = dt >> 1;                            // weight row within the unit
-        const int half = dt & 1;                          // chunks 4*half .. 4*half+3
-        constexpr int WPS = BK * BITS / 32;               // code words per row per k-step
-        constexpr int WPH = WPS / 2;                      // ... per half
+        const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 511
+        const int r = dt >> 2;                            // weight row within the unit
+        const int qt = dt & 3;                            // k chunks 2*qt, 2*qt + 1 (16 k)
+        constexpr int WPQ = BK * BITS / 32 / 4;           // code words per quarter row
         using DQ = Dequant<BITS>;
         const int64_t gpr = prm.K / prm.gs;
-        int s = 0;
-        uint32_t use = 0, blk = 0;
+        RingPos c, a;
+        uint32_t blk = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int e, wt, first, count;
@@ -297,8 +328,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                 for (int ks = 0; ks < ksteps; ++ks) {
                     const int gfirst = (ks * BK) >> prm.lg_gs;
                     const int slot = blk & 1;
-                    // this thread's chunks lie in one group unless groups are 32 wide
-                    const int gsel = (prm.gs < BK) ? half : 0;
+                    const int gsel = (prm.gs < BK) ? (qt >> 1) : 0;  // 32-wide groups: two per k-step
                     float sc = 0.f, bc = 0.f;
                     if (prm.sb_tma) {
                         if (kb == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 28))) break;
@@ -310,58 +340,55 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                         sc = bf16_bits_to_f32(__ldg(srow + gfirst + gsel));
                         bc = bf16_bits_to_f32(__ldg(brow + gfirst + gsel));
                     }
-                    if (!(ok = mbar_wait(&full_c[s], use & 1, 26))) break;
-                    // codes of row r, this half: 16 bytes (4-bit), 32 (8-bit) or 8 (2-bit)
-                    const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
-                    uint32_t w[WPH];
+                    // this thread's quarter row of codes, then release the code stage
+                    if (!(ok = mbar_wait(&full_c[c.s], c.use & 1, 26))) break;
+                    const uint8_t* cst = c_ring + c.s * prm.c_stage_bytes;
+                    uint32_t w[WPQ];
                     if constexpr (BITS == 4) {
-                        const uint32_t off = r * 32 + ((half ^ ((r >> 2) & 1)) << 4);
+                        const uint32_t off = r * 32 + ((((qt >> 1) ^ ((r >> 2) & 1))) << 4) + (qt & 1) * 8;
+                        const uint2 v2 = *reinterpret_cast<const uint2*>(cst + off);
+                        w[0] = v2.x; w[1] = v2.y;
+                    } else if constexpr (BITS == 8) {
+                        const uint32_t off = r * 64 + ((qt ^ ((r >> 1) & 3)) << 4);
                         const uint4 v4 = *reinterpret_cast<const uint4*>(cst + off);
                         w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
-                    } else if constexpr (BITS == 8) {
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j = 2 * half + jj;
-                            const uint32_t off = r * 64 + ((j ^ ((r >> 1) & 3)) << 4);
-                            const uint4 v4 = *reinterpret_cast<const uint4*>(cst + off);
-                            w[4 * jj] = v4.x; w[4 * jj + 1] = v4.y; w[4 * jj + 2] = v4.z; w[4 * jj + 3] = v4.w;
-                        }
                     } else {
-                        const uint2 v2 = *reinterpret_cast<const uint2*>(cst + r * 16 + half * 8);
-                        w[0] = v2.x; w[1] = v2.y;
+                        w[0] = *reinterpret_cast<const uint32_t*>(cst + r * 16 + qt * 4);
                     }
-                    uint8_t* arow = a_ring + s * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty_c[c.s]);
+                    c.next(DC);
+                    if (a.use > 0 && !(ok = mbar_wait(&empty_a[a.s], (a.use - 1) & 1, 32))) break;
+                    uint8_t* arow = a_ring + a.s * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
-                    constexpr int WPC = BITS == 2 ? 1 : 8 * BITS / 32;  // words per 16-byte chunk (2-bit: 2 chunks per word)
+                    uint32_t out[8];
+                    if constexpr (BITS == 2) {
+                        DQ::run(w[0], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out);  // 16 k
+                    } else if constexpr (BITS == 4) {
+                        DQ::run(w[0], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out);
+                        DQ::run(w[1], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + 4);
+                    } else {
 #pragma unroll
-                    for (int cw = 0; cw < (BITS == 2 ? 2 : 4); ++cw) {
-                        uint32_t out[8];
-                        if constexpr (BITS == 2) {
-                            DQ::run(w[cw], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out);
-                        } else {
+                        for (int uu = 0; uu < 4; ++uu)
+                            DQ::run(w[uu], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + 2 * uu);
+                    }
 #pragma unroll
-                            for (int uu = 0; uu < WPC; ++uu)
-                                DQ::run(w[cw * WPC + uu], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6,
-                                        out + uu * DQ::PAIRS);
-                        }
-#pragma unroll
-                        for (int h = 0; h < (BITS == 2 ? 2 : 1); ++h) {
-                            const int c = 4 * half + (BITS == 2 ? 2 * cw + h : cw);
-                            uint4 o;
-                            o.x = out[4 * h]; o.y = out[4 * h + 1]; o.z = out[4 * h + 2]; o.w = out[4 * h + 3];
-                            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = o;
-                        }
+                    for (int h = 0; h < 2; ++h) {
+                        const int ch = 2 * qt + h;
+                        uint4 o;
+                        o.x = out[4 * h]; o.y = out[4 * h + 1]; o.z = out[4 * h + 2]; o.w = out[4 * h + 3];
+                        *reinterpret_cast<uint4*>(arow + ((ch ^ (r & 7)) << 4)) = o;
                     }
                     fence_proxy_async();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&full_a[s]);
+                    if (lane == 0) mbar_arrive(&full_a[a.s]);
+                    a.next(DA);
                     if (prm.sb_tma && (kb == sgk - 1 || ks == ksteps - 1)) {
                         if (lane == 0) mbar_arrive(&sb_empty[slot]);
                         ++blk;
                     }
                     if (++kb == sgk) kb = 0;
-                    if (++s == NS) { s = 0; ++use; }
                 }
             }
         }
@@ -371,7 +398,8 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(2 * kMaxPairs));
     }
 }
 
@@ -464,20 +492,28 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     const uint32_t c_stage = (static_cast<uint32_t>(WM) * BK * bits / 8 + 1023) / 1024 * 1024;
     const uint32_t sb_ring = 2u * 2u * WM * 16u;
     const uint32_t idx = kMaxPairs * 4;
-    const uint32_t per_stage = a_stage + x_stage + c_stage;
-    const uint32_t budget = 227 * 1024 - 1024 - 512 - sb_ring - idx;
-    int stages = static_cast<int>(budget / per_stage);
-    if (stages > 4) stages = 4;
-    if (stages < 2) return cudaErrorInvalidConfiguration;
-    prm.stages = stages;
+    int dx = 6, dc = 8, da = 2;
+    auto bytes = [&]() {
+        return static_cast<size_t>(x_stage) * dx + static_cast<size_t>(c_stage) * dc +
+               static_cast<size_t>(a_stage) * da + sb_ring + idx +
+               static_cast<size_t>(2 * (dx + dc + da) + 8) * 8 + 16;
+    };
+    const size_t budget = 227 * 1024 - 2048 - 1024;
+    while (bytes() > budget && (dx > 2 || dc > 2)) {
+        if (dc >= dx && dc > 2) --dc; else --dx;
+    }
+    if (bytes() > budget) return cudaErrorInvalidConfiguration;
+    prm.dx = dx;
+    prm.dc = dc;
+    prm.da = da;
     prm.a_off = 0;
-    prm.x_off = a_stage * stages;
-    prm.c_off = prm.x_off + x_stage * stages;
-    prm.sb_off = prm.c_off + c_stage * stages;
+    prm.x_off = a_stage * da;
+    prm.c_off = prm.x_off + x_stage * dx;
+    prm.sb_off = prm.c_off + c_stage * dc;
     prm.idx_off = prm.sb_off + sb_ring;
     prm.bar_off = prm.idx_off + idx;
     prm.c_stage_bytes = c_stage;
-    const size_t smem = prm.bar_off + (4 * stages + 8) * 8 + 16 + 1024;
+    const size_t smem = bytes() + 1024;
     const int units = static_cast<int>(E) * prm.wtiles;
     const int grid = units < num_sms ? units : num_sms;
     void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GParams) =
