@@ -48,21 +48,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that lets the hardware suspend the thread for up to `hint_ns`
+// (until the phase completes or the hint expires), so a waiting warp does not
+// take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase with the given parity; false (and the error word
 // set to `code`) if it did not complete within kWaitLimitNs or another wait of
-// the launch already gave up.
-// The time limit and the error word are checked once every 256 polls only: a
-// global load on every poll would flood the memory pipeline of a spinning warp.
+// the launch already gave up. After a first plain poll the thread sleeps in
+// try_wait with a 100 us hint, and the time limit and error word are checked
+// between sleeps.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned code) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0) {
-            if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
-                atomicCAS(&g_pipeline_error, 0u, code);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
+            atomicCAS(&g_pipeline_error, 0u, code);
+            return false;
         }
     }
 }
