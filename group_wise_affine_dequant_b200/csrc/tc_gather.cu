@@ -17,11 +17,11 @@
 //               accumulator.
 //   warps 2-5   epilogue: TMEM lane = weight row, column = pair; each column is
 //               stored to its pair's output row (32 lanes -> 64 contiguous bytes).
-//   warps 6-7   copy the pairs' activation rows with cp.async (16 bytes per
+//   warps 6-13  copy the pairs' activation rows with cp.async (16 bytes per
 //               thread per row and k-step) into the 128-byte-swizzled B layout;
 //               each thread fences its completed copies into the async proxy
 //               before it arrives on the stage's barrier.
-//   warps 8-23  dequantize, four threads per weight row (16 k each), straight
+//   warps 14-21 dequantize, two threads per weight row (32 k each), straight
 //               into tensor memory (tcgen05.st): the MMA reads A from TMEM, so
 //               the dequantized tile costs no shared-memory bandwidth, and
 //               eight A stages fit beside the two accumulators.
@@ -45,10 +45,10 @@ constexpr int BK = 64;
 constexpr int UMMA_K = 16;
 constexpr int kMaxPairs = 128;   // pairs per pass (TMEM columns of one accumulator)
 constexpr int kEpilogueWarp0 = 2;
-constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6 and 7
-constexpr int kXThreads = 64;
-constexpr int kDequantWarp0 = 8; // warps 8-23: dequantize, four threads per weight row
-constexpr int kDequantThreads = 512;
+constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-13
+constexpr int kXThreads = 256;
+constexpr int kDequantWarp0 = 14; // warps 14-21: dequantize, two threads per weight row
+constexpr int kDequantThreads = 256;
 constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
 constexpr uint32_t kStage = 16384;  // one 128-row x 128-byte tile
 constexpr int kDA = 8;              // dequantized-weight stages, in TMEM after the accumulators
@@ -119,7 +119,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     uint64_t* sb_full = acc_empty + 2;
     uint64_t* sb_empty = sb_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sb_empty + 2);
-    // [kMaxPairs / 8][kXThreads]: x element offsets of each loader thread's rows
+    // [kMaxPairs / (kXThreads / 8)][kXThreads]: x element offsets of each loader thread's rows
     uint32_t* s_xoff = reinterpret_cast<uint32_t*>(smem + prm.row_off);
     constexpr int kDequantWarps = kDequantThreads / 32;
 
@@ -282,9 +282,10 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         }
     } else if (warp < kDequantWarp0) {
         // ------------------------------------------- activation rows (cp.async)
-        // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 8 j of every
+        // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 32 j of every
         // k-step. Stages are completed in order, LAG k-steps behind the copies.
-        const int xt = threadIdx.x - kXWarp0 * 32;  // 0 .. 63
+        const int xt = threadIdx.x - kXWarp0 * 32;  // 0 .. kXThreads - 1
+        constexpr int RS = kXThreads / 8;            // row stride between a thread's rows
         const int ch = xt & 7, r0 = xt >> 3;
         const int lag = DX - 1 < 4 ? DX - 1 : 4;
         RingPos x, done;  // next stage to fill, next stage to complete
@@ -301,11 +302,11 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
             unit_pairs(u, e, wt, first, count);
             for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
                 const int cn = min(kMaxPairs, count - p0);
-                const int nr = cn > r0 ? (cn - r0 + 7) / 8 : 0;  // rows of this thread
+                const int nr = cn > r0 ? (cn - r0 + RS - 1) / RS : 0;  // rows of this thread
                 // offsets of this thread's rows, once per pass, into its own slots
                 // of shared memory (no other thread reads them: no barrier)
                 for (int j = 0; j < nr; ++j) {
-                    const uint32_t pair = __ldg(prm.perm + first + p0 + r0 + 8 * j);
+                    const uint32_t pair = __ldg(prm.perm + first + p0 + r0 + RS * j);
                     const uint32_t row = prm.lhs ? __ldg(prm.lhs + pair) : pair;
                     s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K) + ch * 8;
                 }
@@ -313,7 +314,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (x.use > 0 && !(ok = mbar_wait(&empty_x[x.s], (x.use - 1) & 1, 31))) break;
                     uint8_t* dst = x_ring + x.s * kStage;
                     for (int j = 0; j < nr; ++j) {
-                        const int r = r0 + 8 * j;
+                        const int r = r0 + RS * j;
                         cp_async16(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4),
                                    prm.x + s_xoff[j * kXThreads + xt] + ks * BK);
                     }
@@ -335,9 +336,9 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     } else {
         // ------------------------------------------------------------ dequantize
         // warp w writes TMEM lanes 32 (w % 4) ..: row = its lane there; the
-        // four warps of each lane quarter take the four 16-k quarters of a k-step
+        // two warps of each lane quarter take the two 32-k halves of a k-step
         const int r = 32 * (warp & 3) + lane;                 // weight row within the unit
-        const int qt = (warp - kDequantWarp0) >> 2;           // k 16 qt .. 16 qt + 15
+        const int hf = (warp - kDequantWarp0) >> 2;           // k 32 hf .. 32 hf + 31
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         using DQ = Dequant<BITS>;
         RingPos c, a;
@@ -356,26 +357,32 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         gb = (ks * BK) >> prm.lg_gs;  // first group of the block
                     }
                     const uint8_t* ss = sb_ring + slot * prm.sb_slot;
-                    const int gc = ((ks * BK + 16 * qt) >> prm.lg_gs) - gb;
+                    // 32 k of one group (groups are 32-k aligned multiples of 32)
+                    const int gc = ((ks * BK + 32 * hf) >> prm.lg_gs) - gb;
                     const uint32_t so = sb_swz(r, gc, prm.lg_sbw);
                     const float sc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
                     const float bc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
                     if (kc == 0 && !(ok = mbar_wait(&full_c[c.s], c.use & 1, 26))) break;
-                    // this thread's 16 k of row r: part kc of the 128-byte code row
+                    // this thread's 32 k of row r: part kc of the 128-byte code row
                     const uint8_t* crow = c_ring + c.s * kStage + r * 128;
-                    uint32_t w[BITS / 2 > 0 ? BITS / 2 : 1];
+                    constexpr int NW = BITS;  // code words per 32 k
+                    uint32_t w[NW];
                     if constexpr (BITS == 4) {
-                        const int o = kc * 32 + qt * 8;
-                        const uint2 v2 = *reinterpret_cast<const uint2*>(
-                            crow + ((((o >> 4) ^ (r & 7))) << 4) + (o & 15));
-                        w[0] = v2.x; w[1] = v2.y;
-                    } else if constexpr (BITS == 8) {
-                        const int o = kc * 64 + qt * 16;
-                        const uint4 v4 = *reinterpret_cast<const uint4*>(crow + ((((o >> 4) ^ (r & 7))) << 4));
+                        const int o = kc * 32 + hf * 16;
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
                         w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+                    } else if constexpr (BITS == 8) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int o = kc * 64 + hf * 32 + h * 16;
+                            const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
+                            w[4 * h] = v4.x; w[4 * h + 1] = v4.y; w[4 * h + 2] = v4.z; w[4 * h + 3] = v4.w;
+                        }
                     } else {
-                        const int o = kc * 16 + qt * 4;
-                        w[0] = *reinterpret_cast<const uint32_t*>(crow + ((((o >> 4) ^ (r & 7))) << 4) + (o & 15));
+                        const int o = kc * 16 + hf * 8;
+                        const uint2 v2 = *reinterpret_cast<const uint2*>(
+                            crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
+                        w[0] = v2.x; w[1] = v2.y;
                     }
                     const bool last_part = (kc == spk - 1) || (ks == ksteps - 1);
                     if (last_part) {
@@ -388,18 +395,11 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     tc_fence_after();
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
-                    uint32_t out[8];
-                    if constexpr (BITS == 2) {
-                        DQ::run(w[0], s2, b2, sc, bc, 2u, 4u, 6u, out);  // 16 k
-                    } else if constexpr (BITS == 4) {
-                        DQ::run(w[0], s2, b2, sc, bc, 2u, 4u, 6u, out);
-                        DQ::run(w[1], s2, b2, sc, bc, 2u, 4u, 6u, out + 4);
-                    } else {
+                    uint32_t out[16];
 #pragma unroll
-                        for (int uu = 0; uu < 4; ++uu)
-                            DQ::run(w[uu], s2, b2, sc, bc, 2u, 4u, 6u, out + 2 * uu);
-                    }
-                    tmem_st_x8(tmem_base + lane_addr + 2 * kMaxPairs + 32 * a.s + 8 * qt, out);
+                    for (int i = 0; i < NW; ++i)
+                        DQ::run(w[i], s2, b2, sc, bc, 2u, 4u, 6u, out + i * DQ::PAIRS);
+                    tmem_st_x16(tmem_base + lane_addr + 2 * kMaxPairs + 32 * a.s + 16 * hf, out);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_a[a.s]);
@@ -501,7 +501,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     const size_t sb_ring = 2u * static_cast<size_t>(prm.sb_slot);
     int dx = 8, dc = 3;
     auto bytes = [&]() {
-        return static_cast<size_t>(kStage) * (dx + dc) + sb_ring + kMaxPairs / 8 * kXThreads * 4 +
+        return static_cast<size_t>(kStage) * (dx + dc) + sb_ring + kMaxPairs * 8 * 4 +
                static_cast<size_t>(2 * (dx + dc + kDA) + 8) * 8 + 16;
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
@@ -517,7 +517,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.a_off = 0;  // A stages live in TMEM
     prm.sb_off = prm.c_off + kStage * dc;
     prm.row_off = prm.sb_off + static_cast<uint32_t>(sb_ring);
-    prm.bar_off = prm.row_off + kMaxPairs / 8 * kXThreads * 4;
+    prm.bar_off = prm.row_off + kMaxPairs * 8 * 4;
     const size_t smem = bytes() + 1024;
     const int units = static_cast<int>(E) * prm.wtiles;
     const int grid = units < num_sms ? units : num_sms;
