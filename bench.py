@@ -153,25 +153,32 @@ def replay_timed(graphs, stream, barrier):
     return start.elapsed_time(end)
 
 
-def kernel_hash():
+# Sources of each profiled kernel (its .cu file and the headers it includes).
+KERNEL_SOURCES = {
+    "qmv_decode_b4_g64": ["csrc/qmv.cu", "csrc/common.cuh", "csrc/kernels.cuh", "csrc/tma.cuh",
+                          "../include/nvq.h"],
+}
+
+
+def kernel_hash(kernel_key: str = "qmv_decode_b4_g64"):
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "group_wise_affine_dequant_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
+    pkg = os.path.join(ROOT, "group_wise_affine_dequant_b200")
+    for f in KERNEL_SOURCES[kernel_key]:
+        with open(os.path.normpath(os.path.join(pkg, f)), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel_key: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources."""
+    the current sources of that kernel."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("src_hash") != kernel_hash():
+    if not e or e.get("src_hash") != kernel_hash(kernel_key):
         return None
     return e.get("dram_bytes_per_launch")
 

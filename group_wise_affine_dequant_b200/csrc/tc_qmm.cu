@@ -12,8 +12,8 @@
 //               stages with tcgen05.commit.
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (32 lanes each), round to
 //               bf16, store y.
-//   warps 6-13  dequantize: each thread owns one weight row of the tile; it
-//               turns its codes into bf16 w = scale * code + bias (one rounding:
+//   warps 6-21  dequantize: two threads per weight row of the tile (32 k
+//               each); they turn codes into bf16 w = scale * code + bias (one rounding:
 //               the code is made exact first, then one bf16 fma) and writes the
 //               row into the B tile in the canonical K-major 128-byte-swizzled
 //               layout the MMA reads. Codes arrive swizzled (32/64-byte TMA
@@ -41,9 +41,9 @@ using namespace tc;
 constexpr int BM = 128;          // rows of x per tile (TMEM lanes)
 constexpr int BK = 64;           // k per stage: one 128-byte swizzle atom of bf16
 constexpr int UMMA_K = 16;
-constexpr int kThreads = 448;    // 14 warps
 constexpr int kDequantWarp0 = 6;
-constexpr int kDequantThreads = 256;
+constexpr int kDequantThreads = 512;  // two threads per weight row (32 k each)
+constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
 
 struct TcParams {
     uint16_t* y;
@@ -249,11 +249,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ dequantize
-        const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 255
-        const int r = dt;                                 // weight row within the tile
+        const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 511
+        const int r = dt >> 1;                            // weight row within the tile
+        const int h = dt & 1;                             // k 32 h .. 32 h + 31 of the k-step
         const bool has_row = r < BN;
         const int64_t gpr = prm.K / prm.gs;
-        constexpr int WPS = BK * BITS / 32;  // code words per row per k-step
         using DQ = Dequant<BITS>;
         int s = 0;
         uint32_t use = 0;
@@ -267,69 +267,54 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             const uint16_t* srow = prm.scales + (live ? n : 0) * gpr;
             const uint16_t* brow = prm.biases + (live ? n : 0) * gpr;
             for (int ks = 0; ks < ksteps; ++ks) {
-                const int gfirst = (ks * BK) >> prm.lg_gs;
-                float sf[2] = {0.f, 0.f}, bf[2] = {0.f, 0.f};
+                // 32 k lie in one group (groups are 32-k aligned multiples of 32)
+                const int g = ((ks * BK + 32 * h) >> prm.lg_gs);
+                float sc = 0.f, bc = 0.f;
                 const int slot = blk & 1;
                 if (prm.sb_tma) {
                     if (kb == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
                     if (has_row) {
                         const uint16_t* ss = reinterpret_cast<const uint16_t*>(sb_ring + slot * sb_slot_bytes);
-                        const int gi = gfirst & 7;
-                        sf[0] = bf16_bits_to_f32(ss[r * 8 + gi]);
-                        bf[0] = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi]);
-                        if (prm.gs < BK) {
-                            sf[1] = bf16_bits_to_f32(ss[r * 8 + gi + 1]);
-                            bf[1] = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi + 1]);
-                        }
+                        const int gi = g & 7;
+                        sc = bf16_bits_to_f32(ss[r * 8 + gi]);
+                        bc = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi]);
                     }
                 } else if (live) {
-                    sf[0] = bf16_bits_to_f32(__ldg(srow + gfirst));
-                    bf[0] = bf16_bits_to_f32(__ldg(brow + gfirst));
-                    if (prm.gs < BK) {
-                        sf[1] = bf16_bits_to_f32(__ldg(srow + gfirst + 1));
-                        bf[1] = bf16_bits_to_f32(__ldg(brow + gfirst + 1));
-                    }
+                    sc = bf16_bits_to_f32(__ldg(srow + g));
+                    bc = bf16_bits_to_f32(__ldg(brow + g));
                 }
                 if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
                 if (has_row) {
                     const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
-                    uint32_t w[WPS];
+                    constexpr int NW = BITS;  // code words per 32 k
+                    uint32_t w[NW];
+                    if constexpr (BITS == 4) {
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(cst + r * 32 + ((h ^ ((r >> 2) & 1)) << 4));
+                        w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+                    } else if constexpr (BITS == 8) {
 #pragma unroll
-                    for (int i = 0; i < WPS; i += 4) {
-                        // logical 16-byte chunk i/4 of row r under the code tile's swizzle
-                        const int j = i / 4;
-                        uint32_t off;
-                        if constexpr (BITS == 4) off = r * 32 + ((j ^ ((r >> 2) & 1)) << 4);
-                        else if constexpr (BITS == 8) off = r * 64 + ((j ^ ((r >> 1) & 3)) << 4);
-                        else off = r * 16;
-                        const uint4 v4 = *reinterpret_cast<const uint4*>(cst + off);
-                        w[i] = v4.x; w[i + 1] = v4.y; w[i + 2] = v4.z; w[i + 3] = v4.w;
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int j = 2 * h + jj;
+                            const uint4 v4 = *reinterpret_cast<const uint4*>(cst + r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+                            w[4 * jj] = v4.x; w[4 * jj + 1] = v4.y; w[4 * jj + 2] = v4.z; w[4 * jj + 3] = v4.w;
+                        }
+                    } else {
+                        const uint2 v2 = *reinterpret_cast<const uint2*>(cst + r * 16 + h * 8);
+                        w[0] = v2.x; w[1] = v2.y;
                     }
                     uint8_t* brow_s = b_ring + s * prm.b_stage_bytes + (r >> 3) * 1024 + (r & 7) * 128;
-                    // 8 chunks of 8 k (16 bytes) per row and k-step
-                    constexpr int WPC = 8 * BITS / 32 > 0 ? 8 * BITS / 32 : 1;  // words per chunk
+                    const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
+                    const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
+                    uint32_t out[16];
 #pragma unroll
-                    for (int c = 0; c < 8; c += (BITS == 2 ? 2 : 1)) {
-                        const int gi = (prm.gs < BK && c >= 4) ? 1 : 0;  // 32-groups: chunks 4..7
-                        const float sc = sf[gi], bc = bf[gi];
-                        const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
-                        const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
-                        uint32_t out[8];
-                        if constexpr (BITS == 2) {
-                            DQ::run(w[c / 2], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out);  // 16 k
-                        } else {
+                    for (int i = 0; i < NW; ++i)
+                        DQ::run(w[i], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + i * DQ::PAIRS);
+                    // chunks 4 h .. 4 h + 3 (8 k each) of the row, under the 128-byte swizzle
 #pragma unroll
-                            for (int u = 0; u < WPC; ++u)
-                                DQ::run(w[c * WPC + u], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6,
-                                        out + u * DQ::PAIRS);
-                        }
-#pragma unroll
-                        for (int h = 0; h < (BITS == 2 ? 2 : 1); ++h) {
-                            const int cc = c + h;
-                            uint4 o;
-                            o.x = out[4 * h]; o.y = out[4 * h + 1]; o.z = out[4 * h + 2]; o.w = out[4 * h + 3];
-                            *reinterpret_cast<uint4*>(brow_s + ((cc ^ (r & 7)) << 4)) = o;
-                        }
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 o;
+                        o.x = out[4 * c]; o.y = out[4 * c + 1]; o.z = out[4 * c + 2]; o.w = out[4 * c + 3];
+                        *reinterpret_cast<uint4*>(brow_s + (((4 * h + c) ^ (r & 7)) << 4)) = o;
                     }
                     fence_proxy_async();
                 }
