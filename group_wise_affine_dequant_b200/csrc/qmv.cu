@@ -9,16 +9,25 @@
 //    swizzle so the fragment reads below hit distinct banks) plus the slice's
 //    scales and biases into its own ring of shared-memory stages, completing
 //    on a per-warp mbarrier, several tiles ahead of the math.
-//  * Codes become bf16 exactly: OR-ing a code (< 128) into the mantissa of 128.0
-//    gives 128 + code, two codes per 32-bit register, one LOP3 each (8-bit codes
-//    go through as their two 4-bit halves, the high half against 16 * x).
-//  * The multiply-adds run on the tensor cores (mma.sync m16n8k16): A = 16 weight
-//    rows x 16 k of codes, B = the activations (one column per activation row,
-//    up to 8), fp32 accumulation. Which physical k feeds which MMA k-slot is
-//    chosen so that each thread's loaded words feed its own A fragments; the
-//    activations are permuted the same way once, in registers.
-//  * Scale and bias are applied per group outside the MMA:
-//        sum_k x_k w_k = s * sum_k x_k (128 + c_k) + (b - 128 s) * sum_k x_k,
+//  * Codes become fp16 exactly with one mask each: OR-ing a code field into the
+//    mantissa of 1024.0 gives 1024 + c * 2^p for a field p bits above the
+//    mantissa's base (fp16 has 10 mantissa bits, so a 4-bit word needs one
+//    shift and four masks, an 8-bit word one shift and two masks).
+//  * The multiply-adds run on the tensor cores (mma.sync m16n8k16, fp16 in,
+//    fp32 accumulate): A = 16 weight rows x 16 k of codes, B = the activations
+//    (one column per activation row, up to 8). Which physical k feeds which MMA
+//    k-slot is chosen so that each thread's loaded words feed its own A
+//    fragments; the activations are permuted the same way once, in registers,
+//    and the activation of a slot holding c * 2^p is divided by 2^p.
+//  * Activations enter as fp16 after an exact power-of-two scaling 2^-e per
+//    slice and activation row (largest magnitude brought to [1, 2): no
+//    overflow, and every value within 2^-10 of that maximum converts exactly
+//    even after the division by a slot's code scale); the slice's partial
+//    sums are multiplied back by 2^e. Small integer activations stay exact
+//    through the fp32 sums.
+//  * Scale and bias are applied per group outside the MMA, with the 1024s
+//    removed by an MMA over the same rounded activations:
+//        sum_k x_k w_k = s * (D - 1024-sum) + b * sum_k x_k,
 //    so every product x * code is exact and only the group sums round.
 //  * A warp owns a k-slice of 16 MMA k-steps (256 k at 2/4 bits, 128 at 8) and
 //    keeps its activations in registers while it walks the rows of its CTA.
@@ -42,13 +51,13 @@ namespace {
 constexpr int kSteps = 16;
 constexpr int kMaxWarps = 16;
 
-template <int BITS, int GS, int STEPS = kSteps>
+template <int BITS, int GS, int STEPS = (BITS == 8 ? kSteps / 2 : kSteps)>
 struct Shape {
     static constexpr int PER = 32 / BITS;                // codes per word
     static constexpr int GW = GS * BITS / 32;            // words per group
     static constexpr int LW = GW / 4 < 4 ? GW / 4 : 4;   // words per thread per row per chunk
-    static constexpr int MPW = BITS == 2 ? 4 : 2;        // MMAs per word
-    static constexpr int NP = 2 * MPW;                   // bf16x2 registers per unpacked word
+    static constexpr int MPW = BITS == 2 ? 4 : BITS == 4 ? 2 : 1;  // MMAs per word
+    static constexpr int NP = 2 * MPW;                   // fp16x2 registers per unpacked word
     static constexpr int CW = 4 * LW;                    // words per chunk (one lane quad)
     static constexpr int CK = CW * PER;                  // k per chunk
     static constexpr int MMAS = LW * MPW;                // MMAs per chunk
@@ -56,62 +65,87 @@ struct Shape {
     static constexpr int KSLICE = KS * CK;               // k per warp slice
     static constexpr int GPS = KSLICE / GS > 0 ? KSLICE / GS : 1;  // groups per slice
     static constexpr int CPG = GS / CK;                  // chunks per group
-    static constexpr int XMMA = BITS == 8 ? 1 : MPW;     // MMAs per word whose B is x itself
-    // sum_k x (128 + c) = sum x c + OFF sum x; 8-bit codes add 128 twice, once x16.
-    static constexpr float OFF = BITS == 8 ? 2176.0f : 128.0f;
     static_assert(LW >= 1, "group too small for this kernel");
     static_assert(CK <= GS && GS % CK == 0, "a chunk lies inside one group");
 };
 
-// Word -> NP bf16x2 registers; MMA u of the word uses p[2u] (k-slots 2t, 2t+1)
-// and p[2u+1] (k-slots 2t+8, 2t+9).
-template <int BITS>
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* p) {
-    if constexpr (BITS == 4) {
-        p[0] = codes_to_bf16x2(w, 0x000F000Fu);               // (c0, c4)
-        p[1] = codes_to_bf16x2((w >> 4), 0x000F000Fu);   // (c1, c5)
-        p[2] = codes_to_bf16x2((w >> 8), 0x000F000Fu);   // (c2, c6)
-        p[3] = codes_to_bf16x2((w >> 12), 0x000F000Fu);  // (c3, c7)
-    } else if constexpr (BITS == 8) {
-        p[0] = codes_to_bf16x2(w, 0x000F000Fu);               // low halves of (c0, c2)
-        p[1] = codes_to_bf16x2((w >> 8), 0x000F000Fu);   // low halves of (c1, c3)
-        p[2] = codes_to_bf16x2((w >> 4), 0x000F000Fu);   // high halves of (c0, c2)
-        p[3] = codes_to_bf16x2((w >> 12), 0x000F000Fu);  // high halves of (c1, c3)
-    } else {
-        p[0] = codes_to_bf16x2(w, 0x00030003u);  // (c_s, c_s+8) for s = 0..7
-        p[1] = codes_to_bf16x2((w >> 2), 0x00030003u);
-        p[2] = codes_to_bf16x2((w >> 4), 0x00030003u);
-        p[3] = codes_to_bf16x2((w >> 6), 0x00030003u);
-        p[4] = codes_to_bf16x2((w >> 8), 0x00030003u);
-        p[5] = codes_to_bf16x2((w >> 10), 0x00030003u);
-        p[6] = codes_to_bf16x2((w >> 12), 0x00030003u);
-        p[7] = codes_to_bf16x2((w >> 14), 0x00030003u);
-    }
+// (v & mask) | 1024.0 in both fp16 halves: 1024 + the masked field.
+__device__ __forceinline__ uint32_t codes_to_f16x2(uint32_t v, uint32_t mask) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(0x64006400u));
+    return r;
 }
 
-// The activations matching unpack_word: b[u][0..1] for MMA u of a word whose
-// first k is k0. xv holds x[k0 .. k0 + PER) as bf16 pairs.
+// Word -> NP fp16x2 registers (1024 + c * 2^p); MMA u of the word uses p[2u]
+// (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). kScale[i] = 2^p of
+// register i (the activation of that slot pair is divided by it): scale(i).
 template <int BITS>
-__device__ __forceinline__ void x_fragments(const uint32_t* xv, uint32_t (*b)[2]) {
-    if constexpr (BITS == 4) {
-        b[0][0] = pair_lo(xv[0], xv[2]);  // (x0, x4)
-        b[0][1] = pair_hi(xv[0], xv[2]);  // (x1, x5)
-        b[1][0] = pair_lo(xv[1], xv[3]);  // (x2, x6)
-        b[1][1] = pair_hi(xv[1], xv[3]);  // (x3, x7)
-    } else if constexpr (BITS == 8) {
-        b[0][0] = pair_lo(xv[0], xv[1]);  // (x0, x2)
-        b[0][1] = pair_hi(xv[0], xv[1]);  // (x1, x3)
-        const __nv_bfloat162 sixteen = __floats2bfloat162_rn(16.0f, 16.0f);
-        __nv_bfloat162 h0 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&b[0][0]), sixteen);
-        __nv_bfloat162 h1 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&b[0][1]), sixteen);
-        b[1][0] = *reinterpret_cast<uint32_t*>(&h0);
-        b[1][1] = *reinterpret_cast<uint32_t*>(&h1);
-    } else {
+struct Unpack;
+
+template <>
+struct Unpack<4> {  // (c0,c4) (c1,c5)*16 (c2,c6) (c3,c7)*16
+    // 2^p of register i, and the code index of its low half (high = +4)
+    __host__ __device__ static constexpr float scale(int i) { return (i & 1) ? 16.f : 1.f; }
+    __host__ __device__ static constexpr int lo(int i) { return i; }
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
+        const uint32_t v = w >> 8;
+        p[0] = codes_to_f16x2(w, 0x000F000Fu);
+        p[1] = codes_to_f16x2(w, 0x00F000F0u);
+        p[2] = codes_to_f16x2(v, 0x000F000Fu);
+        p[3] = codes_to_f16x2(v, 0x00F000F0u);
+    }
+};
+
+template <>
+struct Unpack<8> {  // (c0,c2) (c1,c3)
+    __host__ __device__ static constexpr float scale(int) { return 1.f; }
+    __host__ __device__ static constexpr int lo(int i) { return i; }  // high = +2
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
+        p[0] = codes_to_f16x2(w, 0x00FF00FFu);
+        p[1] = codes_to_f16x2(w >> 8, 0x00FF00FFu);
+    }
+};
+
+template <>
+struct Unpack<2> {  // (c_i, c_i+8) * 4^i for i < 5, then c5..c7 from w >> 10
+    __host__ __device__ static constexpr float scale(int i) {
+        return i < 5 ? static_cast<float>(1 << (2 * i)) : static_cast<float>(1 << (2 * (i - 5)));
+    }
+    __host__ __device__ static constexpr int lo(int i) { return i; }  // high = +8
+    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
+        const uint32_t v = w >> 10;
+        p[0] = codes_to_f16x2(w, 0x00030003u);
+        p[1] = codes_to_f16x2(w, 0x000C000Cu);
+        p[2] = codes_to_f16x2(w, 0x00300030u);
+        p[3] = codes_to_f16x2(w, 0x00C000C0u);
+        p[4] = codes_to_f16x2(w, 0x03000300u);
+        p[5] = codes_to_f16x2(v, 0x00030003u);
+        p[6] = codes_to_f16x2(v, 0x000C000Cu);
+        p[7] = codes_to_f16x2(v, 0x00300030u);
+    }
+};
+
+__device__ __forceinline__ float bf16_elem(const uint32_t* xv, int i) {
+    return __uint_as_float((i & 1) ? (xv[i >> 1] & 0xFFFF0000u) : (xv[i >> 1] << 16));
+}
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ uint32_t h2_const(float v) { return f2_to_h2(v, v); }
+
+// The activations matching Unpack: b[u][0..1] for MMA u of a word whose first k
+// is k0, from xv = x[k0 .. k0 + PER) as bf16 pairs, times f = 2^-e and divided
+// by the slot's code scale.
+template <int BITS>
+__device__ __forceinline__ void x_fragments(const uint32_t* xv, float f, uint32_t (*b)[2]) {
+    using U = Unpack<BITS>;
+    constexpr int HI = 32 / BITS / 2;  // code index distance between the halves
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            b[u][0] = pair_lo(xv[u], xv[4 + u]);  // (x_2u, x_2u+8)
-            b[u][1] = pair_hi(xv[u], xv[4 + u]);  // (x_2u+1, x_2u+9)
-        }
+    for (int i = 0; i < 2 * (BITS == 2 ? 4 : BITS == 4 ? 2 : 1); ++i) {
+        const float m = f / U::scale(i);
+        b[i >> 1][i & 1] = f2_to_h2(bf16_elem(xv, U::lo(i)) * m, bf16_elem(xv, U::lo(i) + HI) * m);
     }
 }
 
@@ -335,7 +369,6 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     const int tiles = (rows + 15) / 16;
     const int rows_cap = prm.rows_cap;
     const int nslices = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
-    const uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
     const uint32_t stage_bytes = RG::CODE_STAGE + (sb_mode == 1 ? 2 * RG::SB_STAGE : 0);
     const int row0 = static_cast<int>(n0);
     const int MC = M1 ? 1 : M;  // columns kept per row in the slice partials
@@ -380,8 +413,8 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         }
 
         // ---- activations of this slice: B fragments and per-chunk sums ----
-        uint32_t bfr[S::KS][S::MMAS][2];
-        float xs[S::KS][2];
+        uint32_t xall[S::KS][S::LW][S::PER / 2];
+        float xmax = 0.f;  // largest |x| of this lane's part of the slice
 #pragma unroll
         for (int q = 0; q < S::KS; ++q) {
             const int64_t kq = static_cast<int64_t>(kslice0) + q * S::CK;
@@ -389,7 +422,7 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
             for (int j = 0; j < S::LW; ++j) {
                 const int64_t k0 = kq + (t * S::LW + j) * S::PER;
-                uint32_t xv[S::PER / 2];
+                uint32_t* xv = xall[q][j];
                 if (valid) {
                     const uint16_t* xp = prm.x + s_xrow[g] * K + k0;
                     if constexpr (S::PER == 4) {
@@ -407,18 +440,46 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
                     for (int h = 0; h < S::PER / 2; ++h) xv[h] = 0u;
                 }
-                x_fragments<BITS>(xv, &bfr[q][j * S::MPW]);
+#pragma unroll
+                for (int h = 0; h < S::PER / 2; ++h) {
+                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xv[h] << 16)));
+                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xv[h] & 0xFFFF0000u)));
+                }
             }
-            // sum of this chunk's activations, per activation row: an MMA with A = 1.
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+        }
+        // per activation row (lane quad g): 2^-e brings max |x| to [1, 2)
+        xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 1));
+        xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 2));
+        int e = 0;
+        if (xmax > 0.f) e = min(max(static_cast<int>((__float_as_uint(xmax) >> 23) & 0xFF) - 127, -100), 100);
+        const float f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+        // 2^e of the activation rows of this lane's D columns 2t and 2t + 1
+        const int e0 = __shfl_sync(0xffffffffu, e, 8 * t), e1 = __shfl_sync(0xffffffffu, e, 8 * t + 4);
+        const float ef0 = __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+        const float ef1 = __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+
+        uint32_t bfr[S::KS][S::MMAS][2];
+        float xoff[S::KS][2], xsum[S::KS][2];  // per chunk and column: 1024-sum, sum of x
+        const uint32_t k1024 = 0x64006400u;      // fp16x2 (1024, 1024)
+#pragma unroll
+        for (int q = 0; q < S::KS; ++q) {
+#pragma unroll
+            for (int j = 0; j < S::LW; ++j) x_fragments<BITS>(xall[q][j], f, &bfr[q][j * S::MPW]);
+            float d1[4] = {0.f, 0.f, 0.f, 0.f}, d0[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < S::LW; ++j)
 #pragma unroll
-                for (int u = 0; u < S::XMMA; ++u)
-                    mma_bf16_16816(d, kOnes, kOnes, kOnes, kOnes, bfr[q][j * S::MPW + u][0],
-                                   bfr[q][j * S::MPW + u][1]);
-            xs[q][0] = d[0];
-            xs[q][1] = d[1];
+                for (int u = 0; u < S::MPW; ++u) {
+                    const uint32_t* b2 = bfr[q][j * S::MPW + u];
+                    mma_f16_16816(d1, k1024, k1024, k1024, k1024, b2[0], b2[1]);
+                    const uint32_t lo = h2_const(Unpack<BITS>::scale(2 * u));
+                    const uint32_t hi = h2_const(Unpack<BITS>::scale(2 * u + 1));
+                    mma_f16_16816(d0, lo, lo, hi, hi, b2[0], b2[1]);
+                }
+            xoff[q][0] = d1[0];
+            xoff[q][1] = d1[1];
+            xsum[q][0] = d0[0];
+            xsum[q][1] = d0[1];
         }
 
         const int oa = (g * RG::SBOX + goff) * 2, ob = ((g + 8) * RG::SBOX + goff) * 2;
@@ -491,23 +552,22 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
                     uint32_t pa[S::NP], pb[S::NP];
-                    unpack_word<BITS>(wa[j], pa);
-                    unpack_word<BITS>(wb[j], pb);
+                    Unpack<BITS>::run(wa[j], pa);
+                    Unpack<BITS>::run(wb[j], pb);
 #pragma unroll
                     for (int u = 0; u < S::MPW; ++u)
-                        mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
-                                       bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
+                        mma_f16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
+                                      bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
                 }
                 const int gi = q / S::CPG;
                 const float s_a = group_value(sa, gi), s_b = group_value(sb, gi);
-                const float b_a = fmaf(-S::OFF, s_a, group_value(ba, gi));
-                const float b_b = fmaf(-S::OFF, s_b, group_value(bb, gi));
+                const float b_a = group_value(ba, gi), b_b = group_value(bb, gi);
                 // columns 2t (every call) and 2t + 1 (only when a second row exists)
-                acc[0] = fmaf(b_a, xs[q][0], fmaf(s_a, d[0], acc[0]));
-                acc[2] = fmaf(b_b, xs[q][0], fmaf(s_b, d[2], acc[2]));
+                acc[0] = fmaf(b_a, xsum[q][0], fmaf(s_a, d[0] - xoff[q][0], acc[0]));
+                acc[2] = fmaf(b_b, xsum[q][0], fmaf(s_b, d[2] - xoff[q][0], acc[2]));
                 if (!M1) {
-                    acc[1] = fmaf(b_a, xs[q][1], fmaf(s_a, d[1], acc[1]));
-                    acc[3] = fmaf(b_b, xs[q][1], fmaf(s_b, d[3], acc[3]));
+                    acc[1] = fmaf(b_a, xsum[q][1], fmaf(s_a, d[1] - xoff[q][1], acc[1]));
+                    acc[3] = fmaf(b_b, xsum[q][1], fmaf(s_b, d[3] - xoff[q][1], acc[3]));
                 }
             }
             // every lane has read the stage: refill it with tile + NS
@@ -516,12 +576,13 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             if (++st == NS) { st = 0; ph ^= 1u; }
 
             const int r0 = tile * 16 + g;
+            // undo the activations' 2^-e (exact)
             if (M1) {
-                if (t == 0) { red_sl[r0] = acc[0]; red_sl[r0 + 8] = acc[2]; }
+                if (t == 0) { red_sl[r0] = acc[0] * ef0; red_sl[r0 + 8] = acc[2] * ef0; }
             } else {
                 const int m0 = 2 * t, m1 = 2 * t + 1;
-                if (m0 < M) { red_sl[r0 * M + m0] = acc[0]; red_sl[(r0 + 8) * M + m0] = acc[2]; }
-                if (m1 < M) { red_sl[r0 * M + m1] = acc[1]; red_sl[(r0 + 8) * M + m1] = acc[3]; }
+                if (m0 < M) { red_sl[r0 * M + m0] = acc[0] * ef0; red_sl[(r0 + 8) * M + m0] = acc[2] * ef0; }
+                if (m1 < M) { red_sl[r0 * M + m1] = acc[1] * ef1; red_sl[(r0 + 8) * M + m1] = acc[3] * ef1; }
             }
         }
     }
