@@ -292,24 +292,27 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             // the first ring's worth of tiles of the warp's first slice
             // (prefetching everything floods HBM while the previous kernel
             // still streams its own tiles)
+            // (every warp's first tile and the scale block first, then the rest)
             const int w = static_cast<int>(threadIdx.x >> 5);
-            if ((threadIdx.x & 31) == 0 && w < nsl) {
-                {
-                    const int cw = w * S::KSLICE * BITS / 32;
-                    const int gb = w * S::KSLICE / GS / RG::SBOX * RG::SBOX;
-                    for (int i = 0; i < NS && i * 16 < nrows; ++i) {
+            const bool lead = (threadIdx.x & 31) == 0 && w < nsl;
+            const int cw = w * S::KSLICE * BITS / 32;
+            const int gb = w * S::KSLICE / GS / RG::SBOX * RG::SBOX;
+            for (int phase = 0; phase < 2; ++phase) {
+                if (lead) {
+                    for (int i = phase; i < (phase ? NS : 1) && i * 16 < nrows; ++i) {
                         tma_prefetch_3d(&map_c, cw, r0 + i * 16, 0);
                         if (prm.sb_mode == 1) {
                             tma_prefetch_3d(&map_s, gb, r0 + i * 16, 0);
                             tma_prefetch_3d(&map_b, gb, r0 + i * 16, 0);
                         }
                     }
-                    if (prm.sb_mode == 2 && w < prm.nbox) {
+                    if (phase == 0 && prm.sb_mode == 2 && w < prm.nbox) {
                         const int gcol = w << (prm.sbw_log - 1);
                         tma_prefetch_3d(&map_s, gcol, r0, 0);
                         tma_prefetch_3d(&map_b, gcol, r0, 0);
                     }
                 }
+                if (phase == 0) __syncthreads();
             }
         }
         pdl_wait();  // x may come from the previous kernel; y may still be read by it
@@ -404,11 +407,17 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                 tma_load_3d(sbs + RG::SB_STAGE, &map_b, bar, gbox, row, expert);
             }
         };
+        // Fill the ring. On the first slice every warp queues its first tile,
+        // then (after a CTA barrier) the rest, so that the SM's copy queue
+        // holds every warp's first tile ahead of any second tile.
+        const bool first_slice = sl == warp;
+        if (elect_one()) issue(0, st);
+        if (first_slice) __syncthreads();
         if (elect_one()) {
             int s = st;
-            for (int i = 0; i < NS && i < tiles; ++i) {
-                issue(i, s);
+            for (int i = 1; i < NS && i < tiles; ++i) {
                 if (++s == NS) s = 0;
+                issue(i, s);
             }
         }
 
