@@ -228,7 +228,7 @@ def gather_qmm_sampled(x, codes, scales, biases, lhs, rhs, group_size, bits, tra
     return y, a
 
 
-# Acceptance bounds (spec tolerance): |y - y_ref| <= rel * a + 1e-5 with
+# Acceptance bounds of the products: |y - y_ref| <= rel * a + 1e-5 with
 # rel = 4e-3 for bf16 activations and 1e-5 for fp32.
 TOL_REL = {torch.bfloat16: 4e-3, torch.float32: 1e-5}
 TOL_ABS = 1e-5

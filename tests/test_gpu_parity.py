@@ -3,7 +3,7 @@
 Sizes: small cases span several tiles, slices and a ragged tail; the full
 workloads (decode, transposed decode, few-row, mixture of experts) are checked
 in full where the oracle takes seconds and on sampled outputs otherwise.
-Tolerance (north-star): |y - y_ref| <= 4e-3 * sum_k |x_k w_k| + 1e-5 for bf16
+Tolerance: |y - y_ref| <= 4e-3 * sum_k |x_k w_k| + 1e-5 for bf16
 activations, 1e-5 relative for fp32. Codes, scales and biases: bit-exact.
 """
 import pytest
