@@ -11,6 +11,27 @@
 #include "tma.cuh"
 
 namespace nvq {
+
+// A bounded wait (as mbar_wait) for waits expected to be long (an epilogue waiting
+// for a whole tile's accumulation, a producer waiting for a free stage): after
+// the first failed poll the thread sleeps between polls, doubling the sleep up
+// to max_ns, so that it takes almost no issue slots from the working warps.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, unsigned code,
+                                                  uint32_t max_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    uint32_t ns = 32;
+    for (;;) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        ns = ns * 2 < max_ns ? ns * 2 : max_ns;
+        if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
+            atomicCAS(&g_pipeline_error, 0u, code);
+            return false;
+        }
+    }
+}
+
 namespace tc {
 
 __device__ __forceinline__ void tc_fence_before() {

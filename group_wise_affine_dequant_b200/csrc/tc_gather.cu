@@ -174,7 +174,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         if (kb == 0) {
                             const int slot = blk & 1;
                             const uint32_t bu = blk >> 1;
-                            if (bu > 0 && !(ok = mbar_wait(&sb_empty[slot], (bu - 1) & 1, 27))) break;
+                            if (bu > 0 && !(ok = mbar_wait_backoff(&sb_empty[slot], (bu - 1) & 1, 27, 512))) break;
                             const uint32_t half = static_cast<uint32_t>(prm.sb_slot) / 2;
                             mbar_expect_tx(&sb_full[slot], static_cast<uint32_t>(prm.sb_slot));
                             uint8_t* dst = sb_ring + slot * prm.sb_slot;
@@ -185,7 +185,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         }
                         if (++kb == sgk) kb = 0;
                         if (kc == 0) {
-                            if (c.use > 0 && !(ok = mbar_wait(&empty_c[c.s], (c.use - 1) & 1, 21))) break;
+                            if (c.use > 0 && !(ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 21, 512))) break;
                             mbar_expect_tx(&full_c[c.s], kStage);
                             tma_load_3d(c_ring + c.s * kStage, &map_c, &full_c[c.s], ks * BK * BITS / 32,
                                         wt * WM, e);
@@ -216,7 +216,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     const uint32_t idesc = idesc_bf16(WM, npad);
                     const int acc = local & 1;
                     const uint32_t ause = static_cast<uint32_t>(local >> 1);
-                    if (ause > 0 && !(ok = mbar_wait(&acc_empty[acc], (ause - 1) & 1, 22))) break;
+                    if (ause > 0 && !(ok = mbar_wait_backoff(&acc_empty[acc], (ause - 1) & 1, 22, 256))) break;
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kMaxPairs);
                     for (int ks = 0; ks < ksteps; ++ks) {
@@ -252,7 +252,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                 const int cn = min(kMaxPairs, count - p0);
                 const int acc = local & 1;
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
-                if (!(ok = mbar_wait(&acc_full[acc], ause & 1, 25))) break;
+                if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
                 for (int c0 = 0; c0 < cn; c0 += 16) {
                     uint32_t v[16];
@@ -311,7 +311,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K) + ch * 8;
                 }
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    if (x.use > 0 && !(ok = mbar_wait(&empty_x[x.s], (x.use - 1) & 1, 31))) break;
+                    if (x.use > 0 && !(ok = mbar_wait_backoff(&empty_x[x.s], (x.use - 1) & 1, 31, 256))) break;
                     uint8_t* dst = x_ring + x.s * kStage;
                     for (int j = 0; j < nr; ++j) {
                         const int r = r0 + RS * j;
@@ -353,7 +353,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                 for (int ks = 0; ks < ksteps; ++ks) {
                     const int slot = blk & 1;
                     if (kb == 0) {
-                        if (!(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 28))) break;
+                        if (!(ok = mbar_wait_backoff(&sb_full[slot], (blk >> 1) & 1, 28, 256))) break;
                         gb = (ks * BK) >> prm.lg_gs;  // first group of the block
                     }
                     const uint8_t* ss = sb_ring + slot * prm.sb_slot;
@@ -391,7 +391,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         c.next(DC);
                     }
                     if (++kc == spk) kc = 0;
-                    if (a.use > 0 && !(ok = mbar_wait(&empty_a[a.s], (a.use - 1) & 1, 32))) break;
+                    if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;

@@ -203,7 +203,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
             const int a = local & 1;
             const uint32_t ause = static_cast<uint32_t>(local >> 1);
-            if (!mbar_wait(&acc_full[a], ause & 1, 5)) break;
+            if (!mbar_wait_backoff(&acc_full[a], ause & 1, 5, 2048)) break;
             tc_fence_after();
             const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
             const int64_t row = static_cast<int64_t>(mt) * BM + row_in_tile;
