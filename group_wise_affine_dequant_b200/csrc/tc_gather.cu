@@ -6,15 +6,16 @@
 // gathered activation rows as the N side (16 .. 128 columns). Every weight tile
 // is read from HBM once and used for all of the expert's rows.
 //
-// Work unit: (expert e, 128 weight rows); a unit's pairs are taken in passes of
-// at most 128. Roles, per CTA (persistent):
+// Work unit: (expert e, 256 weight rows = two 128-row tiles that share every
+// activation stage); a unit's pairs are taken in passes of at most 64. Roles,
+// per CTA (persistent):
 //   warp 0      one lane streams the code tiles by TMA, 128 rows x 128 bytes
 //               (several k-steps) per copy, into a ring released by the
 //               dequantizing warps once they have read them; scales and biases
 //               arrive per unit in blocks of up to 64 groups (swizzled boxes).
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (M = 128,
-//               N = pairs rounded up to 16, K = 16) into a double-buffered TMEM
-//               accumulator.
+//               N = pairs rounded up to 16, K = 16), one per tile, into a
+//               double-buffered TMEM accumulator (64 columns per tile).
 //   warps 2-5   epilogue: TMEM lane = weight row, column = pair; each column is
 //               stored to its pair's output row (32 lanes -> 64 contiguous bytes).
 //   warps 6-13  copy the pairs' activation rows with cp.async (16 bytes per
@@ -22,9 +23,10 @@
 //               each thread fences its completed copies into the async proxy
 //               before it arrives on the stage's barrier.
 //   warps 14-21 dequantize, two threads per weight row (32 k each), straight
-//               into tensor memory (tcgen05.st): the MMA reads A from TMEM, so
-//               the dequantized tile costs no shared-memory bandwidth, and
-//               eight A stages fit beside the two accumulators.
+//               into tensor memory (tcgen05.st), both tiles of the unit: the
+//               MMA reads A from TMEM, so the dequantized tiles cost no
+//               shared-memory bandwidth, and four A stages fit beside the two
+//               accumulators.
 // Waits are bounded by a timer like the other pipelines.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -40,19 +42,25 @@ namespace {
 
 using namespace tc;
 
-constexpr int WM = 128;          // weight rows per unit (TMEM lanes)
+constexpr int WM = 128;          // weight rows per tile (TMEM lanes)
+constexpr int kTiles = 2;        // weight tiles per unit: every activation stage serves both
+constexpr int UW = WM * kTiles;  // weight rows per unit
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
-constexpr int kMaxPairs = 128;   // pairs per pass (TMEM columns of one accumulator)
+constexpr int kMaxPairs = 64;    // pairs per pass (TMEM columns of one tile's accumulator)
 constexpr int kEpilogueWarp0 = 2;
 constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-13
 constexpr int kXThreads = 256;
 constexpr int kDequantWarp0 = 14; // warps 14-21: dequantize, two threads per weight row
 constexpr int kDequantThreads = 256;
 constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
-constexpr uint32_t kStage = 16384;  // one 128-row x 128-byte tile
-constexpr int kDA = 8;              // dequantized-weight stages, in TMEM after the accumulators
-constexpr uint32_t kTmemCols = 512; // 2 x 128 accumulator columns + 8 x 32 A columns
+constexpr uint32_t kXStage = kMaxPairs * 128;  // activation stage: kMaxPairs rows x 64 k
+constexpr uint32_t kCStage = UW * 128;         // code stage: the unit's rows x 128 code bytes
+constexpr int kAccCols = kTiles * kMaxPairs;   // accumulator columns of one pass
+constexpr int kACols = kTiles * 32;            // TMEM columns of one A stage (64 k per tile)
+constexpr int kDA = 4;                         // A stages, in TMEM after the accumulators
+constexpr uint32_t kTmemCols = 512;
+static_assert(2 * kAccCols + kDA * kACols <= static_cast<int>(kTmemCols), "TMEM budget");
 
 struct GParams {
     uint16_t* y;                // [R, N]
@@ -62,7 +70,7 @@ struct GParams {
     const uint32_t* offsets;    // [E + 2]
     int64_t N, K, E;
     int lg_gs;
-    int wtiles;                 // ceil(N / 128)
+    int wunits;                 // ceil(N / UW)
     int spk;                    // k-steps per code stage (128-byte code rows)
     int sbg, lg_sbw;            // groups per scale/bias box; log2 of its row bytes
     int sb_slot;                // bytes of one slot (scales + biases)
@@ -149,11 +157,11 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     const int ksteps = static_cast<int>(prm.K / BK);
     const int spk = prm.spk;
     const int sgk = (prm.sbg << prm.lg_gs) / BK;  // k-steps per scale/bias block
-    const int units = static_cast<int>(prm.E) * prm.wtiles;
+    const int units = static_cast<int>(prm.E) * prm.wunits;
 
     auto unit_pairs = [&](int u, int& e, int& wt, int& first, int& count) {
-        e = u / prm.wtiles;
-        wt = u - e * prm.wtiles;
+        e = u / prm.wunits;
+        wt = u - e * prm.wunits;
         first = static_cast<int>(__ldg(prm.offsets + e));
         count = static_cast<int>(__ldg(prm.offsets + e + 1)) - first;
     };
@@ -179,16 +187,16 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                             mbar_expect_tx(&sb_full[slot], static_cast<uint32_t>(prm.sb_slot));
                             uint8_t* dst = sb_ring + slot * prm.sb_slot;
                             const int gcol = (ks * BK) >> prm.lg_gs;
-                            tma_load_3d(dst, &map_s, &sb_full[slot], gcol, wt * WM, e);
-                            tma_load_3d(dst + half, &map_b, &sb_full[slot], gcol, wt * WM, e);
+                            tma_load_3d(dst, &map_s, &sb_full[slot], gcol, wt * UW, e);
+                            tma_load_3d(dst + half, &map_b, &sb_full[slot], gcol, wt * UW, e);
                             ++blk;
                         }
                         if (++kb == sgk) kb = 0;
                         if (kc == 0) {
                             if (c.use > 0 && !(ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 21, 512))) break;
-                            mbar_expect_tx(&full_c[c.s], kStage);
-                            tma_load_3d(c_ring + c.s * kStage, &map_c, &full_c[c.s], ks * BK * BITS / 32,
-                                        wt * WM, e);
+                            mbar_expect_tx(&full_c[c.s], kCStage);
+                            tma_load_3d(c_ring + c.s * kCStage, &map_c, &full_c[c.s], ks * BK * BITS / 32,
+                                        wt * UW, e);
                             ++issued;
                             c.next(DC);
                         }
@@ -218,17 +226,19 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     const uint32_t ause = static_cast<uint32_t>(local >> 1);
                     if (ause > 0 && !(ok = mbar_wait_backoff(&acc_empty[acc], (ause - 1) & 1, 22, 256))) break;
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kMaxPairs);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
                     for (int ks = 0; ks < ksteps; ++ks) {
                         if (!(ok = mbar_wait(&full_a[a.s], a.use & 1, 23))) break;
                         if (!(ok = mbar_wait(&full_x[x.s], x.use & 1, 24))) break;
                         tc_fence_after();
-                        const uint32_t at = tmem_base + 2 * kMaxPairs + 32 * a.s;  // A stage columns
-                        const uint64_t bd = sw128_desc(x_ring + x.s * kStage);
+                        const uint32_t at = tmem_base + 2 * kAccCols + kACols * a.s;  // A stage columns
+                        const uint64_t bd = sw128_desc(x_ring + x.s * kXStage);
 #pragma unroll
-                        for (int kk = 0; kk < BK / UMMA_K; ++kk)  // 16 k = 8 TMEM columns of A
-                            tc_mma_ts(d_tmem, at + kk * (UMMA_K / 2), bd + (kk * UMMA_K * 2 >> 4), idesc,
-                                      (ks > 0 || kk > 0) ? 1u : 0u);
+                        for (int tt = 0; tt < kTiles; ++tt)  // both tiles against the same activations
+#pragma unroll
+                            for (int kk = 0; kk < BK / UMMA_K; ++kk)  // 16 k = 8 TMEM columns of A
+                                tc_mma_ts(d_tmem + tt * kMaxPairs, at + tt * 32 + kk * (UMMA_K / 2),
+                                          bd + (kk * UMMA_K * 2 >> 4), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                         tc_commit(&empty_a[a.s]);
                         tc_commit(&empty_x[x.s]);
                         a.next(DA);
@@ -241,23 +251,24 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     } else if (warp < kEpilogueWarp0 + 4) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int wrow = q * 32 + lane;  // weight row within the unit = TMEM lane
         int local = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int e, wt, first, count;
             unit_pairs(u, e, wt, first, count);
-            const int64_t n = static_cast<int64_t>(wt) * WM + wrow;
             for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs, ++local) {
                 const int cn = min(kMaxPairs, count - p0);
                 const int acc = local & 1;
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
                 if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
+                for (int tt = 0; tt < kTiles; ++tt)
                 for (int c0 = 0; c0 < cn; c0 += 16) {
+                    // weight row of the unit = tile * 128 + TMEM lane
+                    const int64_t n = static_cast<int64_t>(wt) * UW + tt * WM + q * 32 + lane;
                     uint32_t v[16];
                     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                           static_cast<uint32_t>(acc * kMaxPairs + c0);
+                                           static_cast<uint32_t>(acc * kAccCols + tt * kMaxPairs + c0);
                     asm volatile(
                         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
                         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -312,7 +323,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                 }
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if (x.use > 0 && !(ok = mbar_wait_backoff(&empty_x[x.s], (x.use - 1) & 1, 31, 256))) break;
-                    uint8_t* dst = x_ring + x.s * kStage;
+                    uint8_t* dst = x_ring + x.s * kXStage;
                     for (int j = 0; j < nr; ++j) {
                         const int r = r0 + RS * j;
                         cp_async16(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4),
@@ -359,30 +370,36 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     const uint8_t* ss = sb_ring + slot * prm.sb_slot;
                     // 32 k of one group (groups are 32-k aligned multiples of 32)
                     const int gc = ((ks * BK + 32 * hf) >> prm.lg_gs) - gb;
-                    const uint32_t so = sb_swz(r, gc, prm.lg_sbw);
-                    const float sc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
-                    const float bc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
                     if (kc == 0 && !(ok = mbar_wait(&full_c[c.s], c.use & 1, 26))) break;
-                    // this thread's 32 k of row r: part kc of the 128-byte code row
-                    const uint8_t* crow = c_ring + c.s * kStage + r * 128;
+                    // this thread's 32 k of row r of each tile: part kc of the code rows
                     constexpr int NW = BITS;  // code words per 32 k
-                    uint32_t w[NW];
-                    if constexpr (BITS == 4) {
-                        const int o = kc * 32 + hf * 16;
-                        const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                        w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
-                    } else if constexpr (BITS == 8) {
+                    uint32_t w[kTiles][NW];
+                    float sc[kTiles], bc[kTiles];
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int o = kc * 64 + hf * 32 + h * 16;
+                    for (int tt = 0; tt < kTiles; ++tt) {
+                        const int rr = tt * WM + r;  // row within the unit
+                        const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
+                        sc[tt] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
+                        bc[tt] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
+                        const uint8_t* crow = c_ring + c.s * kCStage + rr * 128;
+                        if constexpr (BITS == 4) {
+                            const int o = kc * 32 + hf * 16;
                             const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                            w[4 * h] = v4.x; w[4 * h + 1] = v4.y; w[4 * h + 2] = v4.z; w[4 * h + 3] = v4.w;
+                            w[tt][0] = v4.x; w[tt][1] = v4.y; w[tt][2] = v4.z; w[tt][3] = v4.w;
+                        } else if constexpr (BITS == 8) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int o = kc * 64 + hf * 32 + h * 16;
+                                const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
+                                w[tt][4 * h] = v4.x; w[tt][4 * h + 1] = v4.y;
+                                w[tt][4 * h + 2] = v4.z; w[tt][4 * h + 3] = v4.w;
+                            }
+                        } else {
+                            const int o = kc * 16 + hf * 8;
+                            const uint2 v2 = *reinterpret_cast<const uint2*>(
+                                crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
+                            w[tt][0] = v2.x; w[tt][1] = v2.y;
                         }
-                    } else {
-                        const int o = kc * 16 + hf * 8;
-                        const uint2 v2 = *reinterpret_cast<const uint2*>(
-                            crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
-                        w[0] = v2.x; w[1] = v2.y;
                     }
                     const bool last_part = (kc == spk - 1) || (ks == ksteps - 1);
                     if (last_part) {
@@ -393,13 +410,16 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (++kc == spk) kc = 0;
                     if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
-                    const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
-                    const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
-                    uint32_t out[16];
 #pragma unroll
-                    for (int i = 0; i < NW; ++i)
-                        DQ::run(w[i], s2, b2, sc, bc, 2u, 4u, 6u, out + i * DQ::PAIRS);
-                    tmem_st_x16(tmem_base + lane_addr + 2 * kMaxPairs + 32 * a.s + 16 * hf, out);
+                    for (int tt = 0; tt < kTiles; ++tt) {
+                        const uint32_t s2 = (__float_as_uint(sc[tt]) >> 16) * 0x00010001u;
+                        const uint32_t b2 = (__float_as_uint(bc[tt]) >> 16) * 0x00010001u;
+                        uint32_t out[16];
+#pragma unroll
+                        for (int i = 0; i < NW; ++i)
+                            DQ::run(w[tt][i], s2, b2, sc[tt], bc[tt], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                        tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + 32 * tt + 16 * hf, out);
+                    }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_a[a.s]);
@@ -455,22 +475,22 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
         cuuint64_t dims[3] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(E)};
         cuuint64_t strides[2] = {static_cast<cuuint64_t>(wpr) * 4, static_cast<cuuint64_t>(wpr * N) * 4};
-        cuuint32_t box[3] = {32, WM, 1};
+        cuuint32_t box[3] = {32, UW, 1};
         cuuint32_t es[3] = {1, 1, 1};
         if (enc(&map_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(codes), dims, strides,
                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    // scale/bias boxes: up to 64 groups (128 bytes) per row, swizzled by row width
-    const int sbg = gpr >= 64 ? 64 : static_cast<int>(gpr);
+    // scale/bias boxes: up to 32 groups (64 bytes) per row, swizzled by row width
+    const int sbg = gpr >= 32 ? 32 : static_cast<int>(gpr);
     const int sbw = sbg * 2;
     const int lg_sbw = sbw == 128 ? 7 : sbw == 64 ? 6 : sbw == 32 ? 5 : 4;
     {
         cuuint64_t dims[3] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(E)};
         cuuint64_t strides[2] = {static_cast<cuuint64_t>(gpr) * 2, static_cast<cuuint64_t>(gpr * N) * 2};
-        cuuint32_t box[3] = {static_cast<cuuint32_t>(sbg), WM, 1};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(sbg), UW, 1};
         cuuint32_t es[3] = {1, 1, 1};
         const CUtensorMapSwizzle swz = lg_sbw == 7   ? CU_TENSOR_MAP_SWIZZLE_128B
                                        : lg_sbw == 6 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -493,33 +513,32 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.K = K;
     prm.E = E;
     prm.lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
-    prm.wtiles = static_cast<int>((N + WM - 1) / WM);
+    prm.wunits = static_cast<int>((N + UW - 1) / UW);
     prm.spk = 128 / (BK * bits / 8);  // k-steps per 128-byte code row: 8, 4, 2
     prm.sbg = sbg;
     prm.lg_sbw = lg_sbw;
-    prm.sb_slot = 2 * WM * sbw;
+    prm.sb_slot = 2 * UW * sbw;
     const size_t sb_ring = 2u * static_cast<size_t>(prm.sb_slot);
-    int dx = 8, dc = 3;
+    int dx = 8, dc = 2;
     auto bytes = [&]() {
-        return static_cast<size_t>(kStage) * (dx + dc) + sb_ring + kMaxPairs * 8 * 4 +
+        return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kCStage) * dc + sb_ring +
+               kMaxPairs * 8 * 4 +
                static_cast<size_t>(2 * (dx + dc + kDA) + 8) * 8 + 16;
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
-    while (bytes() > budget && (dx > 3 || dc > 2)) {
-        if (dx > 3) --dx; else --dc;
-    }
+    while (bytes() > budget && dx > 3) --dx;
     if (bytes() > budget) return cudaErrorInvalidConfiguration;
     prm.dx = dx;
     prm.dc = dc;
     prm.da = kDA;
     prm.x_off = 0;
-    prm.c_off = kStage * dx;
+    prm.c_off = kXStage * dx;
     prm.a_off = 0;  // A stages live in TMEM
-    prm.sb_off = prm.c_off + kStage * dc;
+    prm.sb_off = prm.c_off + kCStage * dc;
     prm.row_off = prm.sb_off + static_cast<uint32_t>(sb_ring);
     prm.bar_off = prm.row_off + kMaxPairs * 8 * 4;
     const size_t smem = bytes() + 1024;
-    const int units = static_cast<int>(E) * prm.wtiles;
+    const int units = static_cast<int>(E) * prm.wunits;
     const int grid = units < num_sms ? units : num_sms;
     void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GParams) =
         bits == 4 ? tc_gather_kernel<4> : bits == 8 ? tc_gather_kernel<8> : tc_gather_kernel<2>;
