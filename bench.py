@@ -64,6 +64,24 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(v: float, ws: int, device) -> float:
+    """The largest of every rank's value (every rank gets it): the job's time
+    is its slowest replica's. A collective on `device` (cuda for NCCL, cpu
+    for gloo); a plain return on one rank."""
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(ws: int, units_per_step: float, steps: int, ms_max: float) -> float:
+    """Whole-job rate of N independent replicas: the units all ranks processed
+    divided by the slowest rank's time (per second)."""
+    return ws * units_per_step * steps / (ms_max / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi samples of the SM clock and throttle reasons while running."""
 
@@ -275,12 +293,8 @@ def run_nvq(args):
         if ws > 1:
             dist.barrier(device_ids=[local])
 
-    def max_over_ranks(v: float) -> float:
-        if ws == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ms(v: float) -> float:
+        return max_over_ranks(v, ws, dev)
 
     pk, pk_kind = peaks()
     K, Wm = args.steps, args.warmup
@@ -295,18 +309,18 @@ def run_nvq(args):
         while time.time() < t_end:
             replay_timed(graphs, stream, lambda: None)
     del graphs
-    ms = max_over_ranks(ms)
+    ms = max_ms(ms)
     per_step_s = ms / 1e3 / K
-    value = ws * dec.bytes / per_step_s / 1e9
+    value = replica_rate(ws, dec.bytes, K, ms) / 1e9
     achieved = dec.bytes / per_step_s / 1e9  # one launch per step on this rank
     clocks = clk.summary()
 
     # ---- end to end through host buffers
     e2e = DecodeE2E(dev)
     graphs = timed_graph(e2e.step, K, Wm, stream)
-    ms_e2e = max_over_ranks(replay_timed(graphs, stream, barrier))
+    ms_e2e = max_ms(replay_timed(graphs, stream, barrier))
     del graphs
-    e2e_value = ws * e2e.bytes / (ms_e2e / 1e3 / K) / 1e9
+    e2e_value = replica_rate(ws, e2e.bytes, K, ms_e2e) / 1e9
 
     # ---- the other workloads, same rules (fewer steps)
     also = {}
@@ -318,23 +332,22 @@ def run_nvq(args):
                      ("fewrow_m8_4096x4096_gbs", lambda: Decode(dev, N=4096, M=8))):
         wl = mk()
         g = timed_graph(wl.step, ks, Wm, stream)
-        t = max_over_ranks(replay_timed(g, stream, barrier))
-        also[name] = round(ws * wl.bytes / (t / 1e3 / ks) / 1e9, 1)
+        t = max_ms(replay_timed(g, stream, barrier))
+        also[name] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
         del g, wl
     for name, srt in (("gather_sorted", True), ("gather_unsorted", False)):
         wl = Gather(dev, srt)
         g = timed_graph(wl.step, ks, Wm, stream)
-        t = max_over_ranks(replay_timed(g, stream, barrier))
-        step_s = t / 1e3 / ks
-        also[name + "_tok_s"] = round(ws * wl.T / step_s, 1)
-        also[name + "_gbs"] = round(ws * wl.bytes / step_s / 1e9, 1)
+        t = max_ms(replay_timed(g, stream, barrier))
+        also[name + "_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
+        also[name + "_gbs"] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
         del g, wl
     for bits, gs in W.PREFILL_VARIANTS:
         wl = Decode(dev, N=14336, K=4096, M=2048, bits=bits, gs=gs)
         kp = max(3, min(K, 100))
         g = timed_graph(wl.step, kp, Wm, stream)
-        t = max_over_ranks(replay_timed(g, stream, barrier))
-        tf = ws * wl.flops / (t / 1e3 / kp) / 1e12
+        t = max_ms(replay_timed(g, stream, barrier))
+        tf = replica_rate(ws, wl.flops, kp, t) / 1e12
         key = "prefill_tflops" if (bits, gs) == (4, 64) else f"prefill_b{bits}_g{gs}_tflops"
         also[key] = round(tf, 1)
         if (bits, gs) == (4, 64):
