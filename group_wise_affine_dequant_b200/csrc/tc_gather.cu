@@ -18,12 +18,12 @@
 //               double-buffered TMEM accumulator (64 columns per tile).
 //   warps 2-5   epilogue: TMEM lane = weight row, column = pair; each column is
 //               stored to its pair's output row (32 lanes -> 64 contiguous bytes).
-//   warps 6-13  copy the pairs' activation rows with cp.async (16 bytes per
+//   warps 6-9   copy the pairs' activation rows with cp.async (16 bytes per
 //               thread per row and k-step) into the 128-byte-swizzled B layout;
 //               each thread fences its completed copies into the async proxy
 //               before it arrives on the stage's barrier.
-//   warps 14-21 dequantize, two threads per weight row (32 k each), straight
-//               into tensor memory (tcgen05.st), both tiles of the unit: the
+//   warps 10-25 dequantize, one thread per (weight row, 32 k) of each tile,
+//               straight into tensor memory (tcgen05.st): the
 //               MMA reads A from TMEM, so the dequantized tiles cost no
 //               shared-memory bandwidth, and four A stages fit beside the two
 //               accumulators.
@@ -49,10 +49,10 @@ constexpr int BK = 64;
 constexpr int UMMA_K = 16;
 constexpr int kMaxPairs = 64;    // pairs per pass (TMEM columns of one tile's accumulator)
 constexpr int kEpilogueWarp0 = 2;
-constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-13
-constexpr int kXThreads = 256;
-constexpr int kDequantWarp0 = 14; // warps 14-21: dequantize, two threads per weight row
-constexpr int kDequantThreads = 256;
+constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-9
+constexpr int kXThreads = 128;
+constexpr int kDequantWarp0 = 10; // warps 10-25: dequantize, one tile and 32 k per thread
+constexpr int kDequantThreads = 512;
 constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
 constexpr uint32_t kXStage = kMaxPairs * 128;  // activation stage: kMaxPairs rows x 64 k
 constexpr uint32_t kCStage = UW * 128;         // code stage: the unit's rows x 128 code bytes
@@ -293,7 +293,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         }
     } else if (warp < kDequantWarp0) {
         // ------------------------------------------- activation rows (cp.async)
-        // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 32 j of every
+        // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 16 j of every
         // k-step. Stages are completed in order, LAG k-steps behind the copies.
         const int xt = threadIdx.x - kXWarp0 * 32;  // 0 .. kXThreads - 1
         constexpr int RS = kXThreads / 8;            // row stride between a thread's rows
@@ -347,9 +347,12 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     } else {
         // ------------------------------------------------------------ dequantize
         // warp w writes TMEM lanes 32 (w % 4) ..: row = its lane there; the
-        // two warps of each lane quarter take the two 32-k halves of a k-step
-        const int r = 32 * (warp & 3) + lane;                 // weight row within the unit
-        const int hf = (warp - kDequantWarp0) >> 2;           // k 32 hf .. 32 hf + 31
+        // four warps of each lane quarter take (tile, 32-k half) of a k-step
+        const int r = 32 * (warp & 3) + lane;                 // weight row within a tile
+        const int dw = warp - kDequantWarp0;                  // 0 .. 15
+        const int tt = (dw >> 2) & 1;                         // tile of the unit
+        const int hf = dw >> 3;                               // k 32 hf .. 32 hf + 31
+        const int rr = tt * WM + r;                           // row within the unit
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         using DQ = Dequant<BITS>;
         RingPos c, a;
@@ -371,34 +374,30 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     // 32 k of one group (groups are 32-k aligned multiples of 32)
                     const int gc = ((ks * BK + 32 * hf) >> prm.lg_gs) - gb;
                     if (kc == 0 && !(ok = mbar_wait(&full_c[c.s], c.use & 1, 26))) break;
-                    // this thread's 32 k of row r of each tile: part kc of the code rows
+                    // this thread's 32 k of its row: part kc of the code rows
                     constexpr int NW = BITS;  // code words per 32 k
-                    uint32_t w[kTiles][NW];
-                    float sc[kTiles], bc[kTiles];
-#pragma unroll
-                    for (int tt = 0; tt < kTiles; ++tt) {
-                        const int rr = tt * WM + r;  // row within the unit
-                        const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
-                        sc[tt] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
-                        bc[tt] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
+                    uint32_t w[NW];
+                    const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
+                    const float sc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
+                    const float bc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
+                    {
                         const uint8_t* crow = c_ring + c.s * kCStage + rr * 128;
                         if constexpr (BITS == 4) {
                             const int o = kc * 32 + hf * 16;
                             const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                            w[tt][0] = v4.x; w[tt][1] = v4.y; w[tt][2] = v4.z; w[tt][3] = v4.w;
+                            w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
                         } else if constexpr (BITS == 8) {
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
                                 const int o = kc * 64 + hf * 32 + h * 16;
                                 const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                                w[tt][4 * h] = v4.x; w[tt][4 * h + 1] = v4.y;
-                                w[tt][4 * h + 2] = v4.z; w[tt][4 * h + 3] = v4.w;
+                                w[4 * h] = v4.x; w[4 * h + 1] = v4.y; w[4 * h + 2] = v4.z; w[4 * h + 3] = v4.w;
                             }
                         } else {
                             const int o = kc * 16 + hf * 8;
                             const uint2 v2 = *reinterpret_cast<const uint2*>(
                                 crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
-                            w[tt][0] = v2.x; w[tt][1] = v2.y;
+                            w[0] = v2.x; w[1] = v2.y;
                         }
                     }
                     const bool last_part = (kc == spk - 1) || (ks == ksteps - 1);
@@ -410,14 +409,13 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (++kc == spk) kc = 0;
                     if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int tt = 0; tt < kTiles; ++tt) {
-                        const uint32_t s2 = (__float_as_uint(sc[tt]) >> 16) * 0x00010001u;
-                        const uint32_t b2 = (__float_as_uint(bc[tt]) >> 16) * 0x00010001u;
+                    {
+                        const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
+                        const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
                         uint32_t out[16];
 #pragma unroll
                         for (int i = 0; i < NW; ++i)
-                            DQ::run(w[tt][i], s2, b2, sc[tt], bc[tt], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                            DQ::run(w[i], s2, b2, sc, bc, 2u, 4u, 6u, out + i * DQ::PAIRS);
                         tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + 32 * tt + 16 * hf, out);
                     }
                     tc_fence_before();
