@@ -178,12 +178,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and with whitespace collapsed: a comment
+    edit does not change the kernel the counters were taken on."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_hash(kernel_key: str = "qmv_decode_b4_g64"):
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "group_wise_affine_dequant_b200")
     for f in KERNEL_SOURCES[kernel_key]:
-        with open(os.path.normpath(os.path.join(pkg, f)), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.normpath(os.path.join(pkg, f)), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

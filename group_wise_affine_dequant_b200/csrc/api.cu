@@ -152,8 +152,8 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size))
         return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
                                                codes, scales, biases, group_size, bits, y, s, sms));
-    // Matrix-vector route (row_exact): every pair gets the bits of its one-row
-    // product nv_qmm(M = 1) with its expert's weights.
+    // Matrix-vector route (row_exact): every pair's output is bitwise equal to
+    // nv_qmm(M = 1) of that row with its expert's weights.
     if (dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size))
         return from_cuda(nvq::launch_qmv_gather(x, K, N, codes, scales, biases, group_size, bits,
                                                 lhs_idx, ws.perm, ws.problems, ws.num_problems,

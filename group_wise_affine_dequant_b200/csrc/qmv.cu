@@ -1,7 +1,7 @@
 // Quantized matrix-vector products for 1 to 8 rows of bf16 activations,
 // weights stored [N, K] ("Docs / Quantization", sections "Affine" and "Products
-// on the GPU": matrix-vector kernels for few rows, reading each weight group
-// once for all rows).
+// on the GPU": small row counts go to matrix-vector kernels, and every weight
+// group is read once however many rows there are).
 //
 // Design (sm_100a):
 //  * The weights stream from HBM exactly once per call, by TMA: each warp
@@ -34,8 +34,9 @@
 //    Each CTA owns a contiguous range of rows (N split evenly over the SMs) and
 //    reduces the slices in a fixed order through shared memory.
 //  * Every output (row n, activation row m) is computed by the same sequence
-//    of operations whatever M is, so an M-row call gives each row the bits of
-//    its one-row call (row exactness, nuvec crate docs, "Determinism").
+//    of operations whatever M is, so each row of an M-row call is bitwise equal
+//    to a call with that row alone (row exactness, nuvec crate docs,
+//    "Determinism").
 #include <algorithm>
 
 #include "common.cuh"

@@ -2,9 +2,9 @@
  * nvq.h: C ABI of the group-wise affine quantized products for NVIDIA B200 (sm_100a).
  *
  * The format (nuvec documentation, "Docs / Quantization", section "Affine"):
- * each row of a weight matrix is cut into groups of group_size consecutive
- * values (32, 64 or 128). Each group has one scale and one bias, and each value
- * becomes an integer code of `bits` bits packed into uint32 words, so that
+ * a weight row is divided into runs of group_size consecutive values (32, 64
+ * or 128); a run stores one scale and one bias, and every value is stored as a
+ * `bits`-wide unsigned integer, several to a uint32 word, with
  *     w ~= scale * code + bias.
  * Code j of a word sits at bits [j*bits, (j+1)*bits). Scales and biases have
  * the weights' dtype (nuvec crate docs, "Structs": Quantized). This library
@@ -65,10 +65,11 @@ typedef enum nv_dtype {
     NV_BF16 = 1  /* bfloat16 */
 } nv_dtype;
 
-/* Products with at most this many rows give each row the bits of its one-row
- * product under row_exact (nuvec crate docs: constant ROW_INDEPENDENT_ROWS and
- * function with_row_exact; "Docs / Quantization", section "Products on the
- * GPU": "up to 8 rows"). */
+/* Largest row count for which row_exact holds: each row's output is then
+ * bitwise equal to a one-row call (nuvec crate docs: constant
+ * ROW_INDEPENDENT_ROWS and function with_row_exact; "Docs / Quantization",
+ * section "Products on the GPU", which sends at most 8 rows to the
+ * matrix-vector kernels). */
 #define NV_ROW_INDEPENDENT_ROWS 8
 
 /* Device anomaly flags written by nv_gather_qmm into its workspace. */
@@ -80,8 +81,8 @@ typedef enum nv_dtype {
 const char* nv_status_string(nv_status s);
 
 /*
- * Affine quantizer ("Docs / Quantization", section "Affine", and its example
- * w.quantize(Quant::affine(64, 4))).
+ * Affine quantizer ("Docs / Quantization", section "Affine", and its first
+ * example: affine mode, group size 64, 4 bits).
  *
  * w       [rows, cols] in `dt` (NV_F32 or NV_BF16), grouped along cols.
  * codes   uint32 [rows, cols * bits / 32] (output).
@@ -124,8 +125,8 @@ size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E);
 
 /*
  * Mixture-of-experts product ("Docs / Quantization", section "Mixture of
- * experts": gather_qmm multiplies each row by the expert chosen for it without
- * gathering the weights first).
+ * experts": every row is multiplied by its own expert's quantized weights,
+ * read in place, with no gathered copy of the weights).
  *
  * x        [x_rows, K] in `dt`.
  * lhs_idx  uint32 [R] or NULL: pair r reads row lhs_idx[r] of x (NULL: row r).
@@ -136,8 +137,8 @@ size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E);
  * sorted   = 1 is the caller's promise that rhs_idx never decreases (the
  *   option sorted_indices); a broken promise is flagged (NV_FLAG_NOT_SORTED)
  *   and the result is still correct.
- * row_exact = 1: each row gets the bits of its one-row product nv_qmm(M = 1)
- *   with its expert's weights.
+ * row_exact = 1: each row's output is bitwise equal to nv_qmm(M = 1) of that
+ *   row with its expert's weights.
  * workspace: device memory of at least nv_gather_qmm_workspace_size(R, E)
  *   bytes, 16-byte aligned, owned by the caller; its contents on entry do not
  *   matter. Calls that share a workspace must not overlap on the GPU.

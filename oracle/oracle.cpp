@@ -6,15 +6,16 @@
 // CUDA library, and the CUDA library never calls it.
 //
 // Sources (nuvec documentation pages):
-//   [Q-Affine]   "Docs / Quantization", section "Affine": groups of group_size
-//                values along each row, one scale and one bias per group,
-//                bits-wide integer codes packed into uint32 words,
-//                w ~= scale * code + bias; 4-bit/g64 is about 4.5 bits/weight.
+//   [Q-Affine]   "Docs / Quantization", section "Affine": a row is cut into
+//                runs of group_size values; each run carries a scale and a
+//                bias; every value is stored as a small unsigned integer, many
+//                to a 32-bit word; w is approximately scale * code + bias;
+//                4-bit codes with 64-value groups cost roughly 4.5 bits each.
 //   [Q-Example]  same section, the example: quantize W [out, in], then
 //                quantized_matmul(q, transpose=true) is x . w^T.
 //   [Q-Products] "Docs / Quantization", section "Products on the GPU".
 //   [Q-MoE]      "Docs / Quantization", section "Mixture of experts":
-//                gather_qmm multiplies each row by the expert chosen for it.
+//                in gather_qmm every row meets the weights of its own expert.
 //   [Crate-Quantized] nuvec crate docs, "Structs": Quantized holds uint32
 //                codes, one scale per group in the weights' dtype, biases.
 //
