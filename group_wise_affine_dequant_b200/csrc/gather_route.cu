@@ -13,6 +13,7 @@
 // segments and get their per-expert bases from a scan of per-warp histograms.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace nvq {
 namespace {
@@ -65,6 +66,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1) gather_route_kernel(
     __shared__ uint32_t s_flags;
     const int NB = E + 1;  // buckets: experts, then "invalid"
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the grouped product may launch now; it waits for this grid to finish
+    // before it reads the tables
+    pdl_launch_dependents();
 
     for (int i = threadIdx.x; i < kRouteWarps * NB; i += kRouteThreads) hist[i] = 0;
     if (threadIdx.x == 0) s_flags = 0;

@@ -48,6 +48,7 @@ constexpr int UW = WM * kTiles;  // weight rows per unit
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
 constexpr int kMaxPairs = 64;    // pairs per pass (TMEM columns of one tile's accumulator)
+static_assert(kMaxPairs == 64, "the epilogue keeps two pair ids per lane");
 constexpr int kEpilogueWarp0 = 2;
 constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-9
 constexpr int kXThreads = 128;
@@ -149,15 +150,28 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
     const int ksteps = static_cast<int>(prm.K / BK);
     const int spk = prm.spk;
     const int sgk = (prm.sbg << prm.lg_gs) / BK;  // k-steps per scale/bias block
     const int units = static_cast<int>(prm.E) * prm.wunits;
+
+    // The launch may overlap the routing kernel (programmatic dependent
+    // launch): until the wait below, touch nothing it writes. The weights of
+    // the CTA's first unit do not depend on the routing, so their first code
+    // stages and scale/bias block are prefetched into L2 meanwhile.
+    if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < units) {
+        const int e = static_cast<int>(blockIdx.x) / prm.wunits;
+        const int row = (static_cast<int>(blockIdx.x) - e * prm.wunits) * UW;
+        const int words = static_cast<int>(prm.K * BITS / 32);
+        for (int i = 0; i < DC && i * 32 < words; ++i) tma_prefetch_3d(&map_c, i * 32, row, e);
+        tma_prefetch_3d(&map_s, 0, row, e);
+        tma_prefetch_3d(&map_b, 0, row, e);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // the routing tables (offsets, perm) come from the previous kernel
 
     auto unit_pairs = [&](int u, int& e, int& wt, int& first, int& count) {
         e = u / prm.wunits;
@@ -260,6 +274,14 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                 const int cn = min(kMaxPairs, count - p0);
                 const int acc = local & 1;
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
+                // output rows of the pass's pairs, loaded while the products
+                // run: lane l holds those of columns l and l + 32
+                uint32_t prow[kMaxPairs / 32];
+#pragma unroll
+                for (int h = 0; h < kMaxPairs / 32; ++h) {
+                    const int c = h * 32 + lane;
+                    prow[h] = c < cn ? __ldg(prm.perm + first + p0 + c) : 0u;
+                }
                 if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
                 for (int tt = 0; tt < kTiles; ++tt)
@@ -277,13 +299,13 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                           "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
                         : "r"(taddr));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    const uint32_t rows = (c0 >> 5) ? prow[1] : prow[0];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        if (c0 + j < cn && n < prm.N) {
-                            const uint32_t pair = __ldg(prm.perm + first + p0 + c0 + j);
+                        const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
+                        if (c0 + j < cn && n < prm.N)
                             prm.y[static_cast<int64_t>(pair) * prm.N + n] =
                                 f32_to_bf16_bits(__uint_as_float(v[j]));
-                        }
                     }
                 }
                 tc_fence_before();
@@ -432,6 +454,16 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         }
     }
 
+    // pairs whose expert or token id is out of range (the router's last
+    // bucket) get zero rows
+    {
+        const int64_t first = __ldg(prm.offsets + prm.E), last = __ldg(prm.offsets + prm.E + 1);
+        for (int64_t i = first + blockIdx.x; i < last; i += gridDim.x) {
+            uint16_t* row = prm.y + static_cast<int64_t>(__ldg(prm.perm + i)) * prm.N;
+            for (int64_t n = threadIdx.x; n < prm.N; n += blockDim.x) row[n] = 0;
+        }
+    }
+
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -439,15 +471,6 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(kTmemCols));
     }
-}
-
-// Pairs whose expert or token id is out of range (bucket E of the router) get
-// zero rows.
-__global__ void zero_invalid_pairs(uint16_t* y, const uint32_t* perm, const uint32_t* offsets,
-                                   int64_t E, int64_t N) {
-    const int64_t first = offsets[E], last = offsets[E + 1];
-    for (int64_t i = first + blockIdx.x; i < last; i += gridDim.x)
-        for (int64_t n = threadIdx.x; n < N; n += blockDim.x) y[static_cast<int64_t>(perm[i]) * N + n] = 0;
 }
 
 }  // namespace
@@ -543,11 +566,20 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, stream>>>(map_c, map_s, map_b, prm);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    zero_invalid_pairs<<<64, 256, 0, stream>>>(static_cast<uint16_t*>(y), perm, offsets, E, N);
-    return cudaGetLastError();
+    // Programmatic dependent launch on the routing kernel: the CTAs set up
+    // (barriers, tensor memory, L2 prefetch of their first weights) while the
+    // routing runs and wait for its tables with griddepcontrol.wait.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, map_c, map_s, map_b, prm);
 }
 
 }  // namespace nvq
