@@ -8,7 +8,8 @@ a 4-bit, group-64 decode product y = x . w^T with x [1, 4096] bf16 and
 W [14336, 4096] (Llama-8B MLP shape), i.e. one nv_qmm call. The JSON line
 reports HBM GB/s of algorithmic bytes (codes + scales + biases + x + y); the
 other workloads (8-bit and transposed decode, few rows, prefill, mixture of
-experts) are measured in the same run and reported under "also".
+experts, dequantization to bf16) are measured in the same run and reported
+under "also".
 
 Timing: W untimed warm-up steps, then K timed steps captured in CUDA graphs and
 bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
@@ -252,6 +253,28 @@ class DecodeE2E(Decode):
         self.yh.copy_(self.y, non_blocking=True)
 
 
+class Dequant:
+    """w = scale * code + bias for W [N, K] (4-bit g64 codes) into bf16."""
+
+    def __init__(self, dev, N=14336, K=4096, bits=4, gs=64):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        self.bits, self.gs = bits, gs
+        w = W.normal((N, K), 0.02, 0, "bf16").to(dev)
+        c, s, b = nvq.nv_quantize_affine(w, gs, bits)
+        del w
+        wbytes = qbytes(N, K, bits, gs)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))
+        self.ws = [(c.clone(), s.clone(), b.clone()) for _ in range(self.copies)]
+        self.out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        self.bytes = wbytes + N * K * 2
+
+    def step(self, i):
+        c, s, b = self.ws[i % self.copies]
+        self.nvq.nv_dequantize_affine(c, s, b, self.gs, self.bits, out=self.out)
+
+
 class Gather:
     """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4."""
 
@@ -344,6 +367,13 @@ def run_nvq(args):
         t = max_ms(replay_timed(g, stream, barrier))
         also[name] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
         del g, wl
+    wl = Dequant(dev)
+    g = timed_graph(wl.step, ks, Wm, stream)
+    t = max_ms(replay_timed(g, stream, barrier))
+    dq = replica_rate(ws, wl.bytes, ks, t) / 1e9
+    also["dequantize_14336x4096_b4g64_bf16_gbs"] = round(dq, 1)
+    also["dequantize_frac_of_hbm"] = round(dq / ws / pk["hbm_gbs"], 4)
+    del g, wl
     for name, srt in (("gather_sorted", True), ("gather_unsorted", False)):
         wl = Gather(dev, srt)
         g = timed_graph(wl.step, ks, Wm, stream)

@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     nv_gather_qmm,
     nv_gather_qmm_flags,
     nv_gather_qmm_workspace_size,
+    nv_dequantize_affine,
     nv_pipeline_error,
     nv_qmm,
     nv_quantize_affine,

@@ -24,7 +24,8 @@ NV_FLAG_NOT_SORTED = 0x2
 NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
-EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_qmm", "nv_gather_qmm_workspace_size",
+EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_dequantize_affine", "nv_qmm",
+           "nv_gather_qmm_workspace_size",
            "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error",
            "nv_gather_qmm_noalloc")
 
@@ -60,6 +61,8 @@ def lib():
             L.nv_status_string.restype = C.c_char_p
             L.nv_quantize_affine.argtypes = [_p, _i, _i64, _i64, _i, _i, _p, _p, _p, _p]
             L.nv_quantize_affine.restype = _i
+            L.nv_dequantize_affine.argtypes = [_p, _p, _p, _i, _i64, _i64, _i, _i, _p, _p]
+            L.nv_dequantize_affine.restype = _i
             L.nv_qmm.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i, _p, _p]
             L.nv_qmm.restype = _i
             L.nv_gather_qmm_workspace_size.argtypes = [_i64, _i64]
@@ -126,6 +129,32 @@ def nv_quantize_affine(w: torch.Tensor, group_size: int = 64, bits: int = 4, str
                                   _stream(stream))
     _check("nv_quantize_affine", st)
     return codes, scales, biases
+
+
+def nv_dequantize_affine(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                         group_size: int = 64, bits: int = 4, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """w = scale * code + bias [..., rows, cols] in the scales' dtype, from the
+    layout nv_quantize_affine writes (codes [..., rows, cols * bits / 32])."""
+    for t, n in ((codes, "codes"), (scales, "scales"), (biases, "biases")):
+        _dev(t, n)
+    if scales.shape != biases.shape or scales.dtype != biases.dtype or codes.dim() < 1:
+        raise ValueError("scales and biases must match, codes must have a last axis")
+    cols = codes.shape[-1] * 32 // bits
+    rows = codes.numel() // codes.shape[-1] if codes.shape[-1] else 0
+    if tuple(scales.shape) != (*codes.shape[:-1], cols // group_size):
+        raise ValueError(f"scales {tuple(scales.shape)} do not match codes {tuple(codes.shape)} "
+                         f"at group_size {group_size}, bits {bits}")
+    w = out if out is not None else torch.empty(*codes.shape[:-1], cols, dtype=scales.dtype,
+                                                device=codes.device)
+    if w.numel() != rows * cols or w.dtype != scales.dtype:
+        raise ValueError("out has the wrong size or dtype")
+    _dev(w, "out")
+    st = lib().nv_dequantize_affine(codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                                    _DT.get(scales.dtype, -1), rows, cols, group_size, bits,
+                                    w.data_ptr(), _stream(stream))
+    _check("nv_dequantize_affine", st)
+    return w
 
 
 def nv_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,

@@ -13,11 +13,18 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-nv_status check_quant(int gs, int bits) {
-    if (bits == 1 || bits == 3 || bits == 5 || bits == 6) return NV_ERR_UNSUPPORTED;
-    if (bits != 2 && bits != 4 && bits != 8) return NV_ERR_INVALID_ARG;
+// Widths the quantizer and dequantizer take: 1, 2, 4, 8 (they divide 32).
+nv_status check_codes(int gs, int bits) {
+    if (bits == 3 || bits == 5 || bits == 6) return NV_ERR_UNSUPPORTED;
+    if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return NV_ERR_INVALID_ARG;
     if (gs != 32 && gs != 64 && gs != 128) return NV_ERR_INVALID_ARG;
     return NV_OK;
+}
+
+// Widths the products take: 2, 4, 8 (1-bit codes have no product kernels).
+nv_status check_quant(int gs, int bits) {
+    if (bits == 1) return NV_ERR_UNSUPPORTED;
+    return check_codes(gs, bits);
 }
 
 bool valid_dtype(nv_dtype dt) { return dt == NV_F32 || dt == NV_BF16; }
@@ -59,7 +66,7 @@ nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t c
                              int group_size, int bits, uint32_t* codes, void* scales,
                              void* biases, nv_stream_t stream) {
     if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
-    nv_status st = check_quant(group_size, bits);
+    nv_status st = check_codes(group_size, bits);
     if (st != NV_OK) return st;
     if (rows < 0 || cols <= 0 || cols % group_size != 0) return NV_ERR_INVALID_ARG;
     if (rows == 0) return NV_OK;
@@ -68,6 +75,21 @@ nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t c
         return NV_ERR_INVALID_ARG;
     return from_cuda(nvq::launch_quantize_affine(w, dt, rows, cols, group_size, bits, codes,
                                                  scales, biases, stream, sm_count()));
+}
+
+nv_status nv_dequantize_affine(const uint32_t* codes, const void* scales, const void* biases,
+                               nv_dtype dt, int64_t rows, int64_t cols, int group_size,
+                               int bits, void* w, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    nv_status st = check_codes(group_size, bits);
+    if (st != NV_OK) return st;
+    if (rows < 0 || cols <= 0 || cols % group_size != 0) return NV_ERR_INVALID_ARG;
+    if (rows == 0) return NV_OK;
+    if (!w || !codes || !scales || !biases) return NV_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases))
+        return NV_ERR_INVALID_ARG;
+    return from_cuda(nvq::launch_dequantize_affine(codes, scales, biases, dt, rows, cols,
+                                                   group_size, bits, w, stream, sm_count()));
 }
 
 nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,

@@ -1,0 +1,126 @@
+// Dequantizer ("Docs / Quantization", section "Affine": every value is stored
+// as a small unsigned code with a scale and a bias per group, w ~ scale *
+// code + bias; the nuvec crate docs list `dequantize` beside the quantizer).
+//
+// The codes of every row are one flat run of words, and a group never crosses
+// a row (cols is a multiple of the group size, and a word's 32 / bits codes
+// never cross a group), so word i of the whole array holds the values
+// [i * per_word, (i + 1) * per_word) of the flat output and belongs to group
+// (i * per_word) / group_size of the flat scale and bias arrays. The kernel is
+// therefore a flat map over words: each thread takes four consecutive words
+// (one 16-byte load), writes their values with 8- to 16-byte stores, and
+// strides over the array. Every value is one fused multiply-add in fp32,
+// scale * code + bias rounded once, then stored in the output dtype (bf16 by
+// round-to-nearest-even). HBM-bound: bytes moved per weight are bits / 8
+// (codes) + 4 / group_size or 8 / group_size (scale and bias) + the output
+// element size.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace nvq {
+namespace {
+
+// Exact fp32 value of a code below 2^23: its bits under the mantissa of 2^23,
+// minus 2^23.
+__device__ __forceinline__ float code_f32(uint32_t c) {
+    return __uint_as_float(0x4B000000u | c) - 8388608.0f;
+}
+
+// Values of one word, stored at out (16-byte aligned for bf16 at 4 bits and
+// wider outputs, 8-byte for 8-bit codes to bf16).
+template <int DT, int BITS>
+__device__ __forceinline__ void word_out(uint32_t w, float s, float b, void* out) {
+    constexpr int PER = 32 / BITS;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    if constexpr (DT == NV_BF16) {
+        uint32_t v[PER / 2];
+#pragma unroll
+        for (int j = 0; j < PER / 2; ++j) {
+            const float lo = fmaf(s, code_f32((w >> (2 * j * BITS)) & MASK), b);
+            const float hi = fmaf(s, code_f32((w >> ((2 * j + 1) * BITS)) & MASK), b);
+            v[j] = static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
+                   (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+        }
+        if constexpr (PER / 2 >= 4) {
+            uint4* o = reinterpret_cast<uint4*>(out);
+#pragma unroll
+            for (int q = 0; q < PER / 8; ++q) o[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+            *reinterpret_cast<uint2*>(out) = make_uint2(v[0], v[1]);
+        }
+    } else {
+        float v[PER];
+#pragma unroll
+        for (int j = 0; j < PER; ++j) v[j] = fmaf(s, code_f32((w >> (j * BITS)) & MASK), b);
+        float4* o = reinterpret_cast<float4*>(out);
+#pragma unroll
+        for (int q = 0; q < PER / 4; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+template <int DT, int BITS>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restrict__ codes,
+                                                         const void* __restrict__ scales,
+                                                         const void* __restrict__ biases,
+                                                         int64_t words, int lg_gs,
+                                                         void* __restrict__ out) {
+    constexpr int PER = 32 / BITS;
+    constexpr int ESZ = DT == NV_F32 ? 4 : 2;
+    char* o = static_cast<char*>(out);
+    const int64_t chunks = words / 4;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+         c += stride) {
+        const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(codes) + c);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t i = 4 * c + q;
+            const int64_t g = (i * PER) >> lg_gs;
+            word_out<DT, BITS>(w[q], load_elem<DT>(scales, g), load_elem<DT>(biases, g),
+                               o + i * PER * ESZ);
+        }
+    }
+    // the last words % 4 words, one per thread of the first block
+    if (blockIdx.x == 0 && threadIdx.x < words - 4 * chunks) {
+        const int64_t i = 4 * chunks + threadIdx.x;
+        const int64_t g = (i * PER) >> lg_gs;
+        word_out<DT, BITS>(__ldg(codes + i), load_elem<DT>(scales, g), load_elem<DT>(biases, g),
+                           o + i * PER * ESZ);
+    }
+}
+
+template <int DT>
+cudaError_t launch_dt(const uint32_t* codes, const void* scales, const void* biases,
+                      int64_t words, int gs, int bits, void* out, cudaStream_t stream,
+                      int num_sms) {
+    const int lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
+    const int threads = 256;
+    int64_t blocks = (words / 4 + threads - 1) / threads;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const dim3 grid(static_cast<unsigned>(blocks));
+    switch (bits) {
+        case 1: dequantize_kernel<DT, 1><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
+        case 2: dequantize_kernel<DT, 2><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
+        case 4: dequantize_kernel<DT, 4><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
+        case 8: dequantize_kernel<DT, 8><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dequantize_affine(const uint32_t* codes, const void* scales,
+                                     const void* biases, int dt, int64_t rows, int64_t cols,
+                                     int gs, int bits, void* out, cudaStream_t stream,
+                                     int num_sms) {
+    const int64_t words = rows * (cols * bits / 32);
+    if (words == 0) return cudaSuccess;
+    return dt == NV_F32 ? launch_dt<NV_F32>(codes, scales, biases, words, gs, bits, out, stream, num_sms)
+                        : launch_dt<NV_BF16>(codes, scales, biases, words, gs, bits, out, stream, num_sms);
+}
+
+}  // namespace nvq

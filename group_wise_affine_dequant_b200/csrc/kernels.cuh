@@ -10,6 +10,12 @@ cudaError_t launch_quantize_affine(const void* w, int dt, int64_t rows, int64_t 
                                    int bits, uint32_t* codes, void* scales, void* biases,
                                    cudaStream_t stream, int num_sms);
 
+// w_hat = scale * code + bias for every code, in the scales' dtype.
+cudaError_t launch_dequantize_affine(const uint32_t* codes, const void* scales,
+                                     const void* biases, int dt, int64_t rows, int64_t cols,
+                                     int gs, int bits, void* out, cudaStream_t stream,
+                                     int num_sms);
+
 // Matrix-vector products for up to 8 rows, weights [N, K] (transpose = 1), bf16.
 bool qmv_supported(int bits, int gs);
 unsigned int qmv_error_take();  // read and clear the kernels' pipeline error word

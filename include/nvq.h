@@ -8,7 +8,8 @@
  *     w ~= scale * code + bias.
  * Code j of a word sits at bits [j*bits, (j+1)*bits). Scales and biases have
  * the weights' dtype (nuvec crate docs, "Structs": Quantized). This library
- * supports bits 2, 4 and 8.
+ * quantizes and dequantizes at bits 1, 2, 4 and 8 (the widths that divide 32)
+ * and runs products at bits 2, 4 and 8.
  *
  * Layouts (all dense, row-major, no padding):
  *   weights [rows, cols], grouped along cols:
@@ -93,12 +94,31 @@ const char* nv_status_string(nv_status s);
  *   a constant group (scale == 0) gets code 0; scale and bias are stored in
  *   `dt` (bf16 by round-to-nearest-even). The minimum of a group holding both
  *   -0 and +0 is -0, the maximum +0. Inputs must be finite.
- * group_size in {32, 64, 128}; bits in {2, 4, 8}; cols % group_size == 0.
- * Other bit widths return NV_ERR_UNSUPPORTED.
+ * group_size in {32, 64, 128}; bits in {1, 2, 4, 8}; cols % group_size == 0.
+ * Bits 3, 5 and 6 return NV_ERR_UNSUPPORTED (no packing of widths that do not
+ * divide 32 is specified), any other width NV_ERR_INVALID_ARG.
  */
 nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t cols,
                              int group_size, int bits, uint32_t* codes, void* scales,
                              void* biases, nv_stream_t stream);
+
+/*
+ * Dequantizer: the weights back from their codes ("Docs / Quantization",
+ * section "Affine": w ~= scale * code + bias; the nuvec crate docs list
+ * dequantize beside the quantizer).
+ *
+ * codes   uint32 [rows, cols * bits / 32]; scales, biases `dt` [rows,
+ *         cols / group_size] (inputs, the layout nv_quantize_affine writes).
+ * w       `dt` [rows, cols] (output): w[r, c] = scale * code + bias, one fp32
+ *         fused multiply-add (rounded once), stored in `dt` (bf16 by
+ *         round-to-nearest-even). Deterministic and exact up to that rounding.
+ * dt in {NV_F32, NV_BF16}; group_size in {32, 64, 128}; bits in {1, 2, 4, 8};
+ * cols % group_size == 0; rows == 0 is a no-op returning NV_OK. Bits 3, 5, 6
+ * return NV_ERR_UNSUPPORTED.
+ */
+nv_status nv_dequantize_affine(const uint32_t* codes, const void* scales, const void* biases,
+                               nv_dtype dt, int64_t rows, int64_t cols, int group_size,
+                               int bits, void* w, nv_stream_t stream);
 
 /*
  * Quantized product ("Docs / Quantization", sections "Affine" (example
@@ -114,6 +134,7 @@ nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t c
  *   row's result equals, bit for bit, the same call with that row alone (M = 1).
  * Routing is a pure function of (M, N, K, dt, group_size, bits, transpose,
  * row_exact): matrix-vector kernels for M <= 8, tensor-core tiles above.
+ * bits in {2, 4, 8}; 1-bit codes return NV_ERR_UNSUPPORTED here.
  * M == 0 or N == 0 is a no-op returning NV_OK.
  */
 nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,

@@ -124,6 +124,22 @@ def dequantize(codes, scales, biases, group_size: int, bits: int, lib=None) -> t
     return out
 
 
+def dequantize_stored(codes, scales, biases, group_size: int, bits: int, lib=None) -> torch.Tensor:
+    """The dequantized weights as stored in the scales' dtype ("Docs /
+    Quantization", section "Affine": w ~= scale * code + bias).
+
+    Reading (the pages fix no precision for this step): scale * code + bias is
+    evaluated exactly and rounded once to fp32 (one fused multiply-add), then
+    stored in the dtype (bf16: round to nearest, ties to even). The exact value
+    is the fp64 result of ``dequantize``: scale * code has at most 32
+    significant bits, so the sum with the bias is exact in fp64 whenever the
+    two are within ~20 binades of each other (true of every quantized group,
+    whose codes span the bias's range); torch's fp64 -> fp32 and fp32 -> bf16
+    conversions round to nearest even."""
+    wh = dequantize(codes, scales, biases, group_size, bits, lib=lib)
+    return wh.to(torch.float32).to(_cpu(scales).dtype)
+
+
 def qmm(x, codes, scales, biases, group_size: int, bits: int, transpose: bool = True, lib=None):
     """fp64 (y, a) for x [M, K]; weights [N, K] (transpose) or [K, N].
 

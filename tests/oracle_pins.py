@@ -126,6 +126,37 @@ def pin_handbuilt_groups(lib):
             assert got[1].tolist() == _cycle(codes[::-1], gs), (name, dt)
 
 
+def pin_dequantize_stored_rounding(lib):
+    """The stored dequantized value is scale * code + bias rounded once to fp32,
+    then to the dtype with ties to even (the reading the dequantizer follows):
+    * bf16, scale 2^-9, bias 1: codes 1, 2, 3 give 1 + 2^-9 (below half a bf16
+      step: 1), 1 + 2^-8 (exactly half: the even neighbour 1), 1 + 3 * 2^-9
+      (above half: 1 + 2^-7);
+    * fp32, scale 1 + 2^-23, bias -3, code 3: the exact value 3 * 2^-23 is an
+      fp32 number, so one rounding keeps it (a product rounded first would give
+      3 + 2^-21 and then 2^-21);
+    * scale 1 and bias 0 return the codes, in both dtypes."""
+    words = torch.tensor([[1 | (2 << 8) | (3 << 16)]], dtype=torch.int32)  # 8-bit codes 1, 2, 3, 0
+    s = torch.tensor([[2.0 ** -9]], dtype=torch.bfloat16)
+    b = torch.tensor([[1.0]], dtype=torch.bfloat16)
+    got = O.dequantize_stored(torch.cat([words] * 8, 1), s, b, 32, 8, lib=lib)
+    assert got.dtype == torch.bfloat16
+    assert got[0, :4].to(torch.float64).tolist() == [1.0, 1.0, 1.0 + 2.0 ** -7, 1.0], got[0, :4]
+    s32 = torch.tensor([[1.0 + 2.0 ** -23]], dtype=torch.float32)
+    b32 = torch.tensor([[-3.0]], dtype=torch.float32)
+    w3 = torch.full((1, 8), 3 | (3 << 8) | (3 << 16) | (3 << 24), dtype=torch.int32)
+    got = O.dequantize_stored(w3, s32, b32, 32, 8, lib=lib)
+    assert got.dtype == torch.float32 and (got == 3 * 2.0 ** -23).all(), got
+    for bits, codes, word in pack_word_cases():
+        gs = 32
+        words = torch.zeros(1, gs * bits // 32, dtype=torch.int32)
+        words[0, 0] = word - 2 ** 32 if word >= 2 ** 31 else word
+        for dt in (torch.float32, torch.bfloat16):
+            one, zero = torch.ones(1, 1, dtype=dt), torch.zeros(1, 1, dtype=dt)
+            wh = O.dequantize_stored(words, one, zero, gs, bits, lib=lib)
+            assert wh.dtype == dt and wh[0, :len(codes)].tolist() == [float(c) for c in codes]
+
+
 def pin_signed_zero_extremes(lib):
     """A group whose smallest values are -0 and +0 (in either order) has bias -0;
     one whose largest are -0 and +0 has its range measured to +0."""

@@ -79,6 +79,23 @@ def test_quantize_argument_errors():
     assert q(16, 1, 4, 64, 64, 4, 0, 16, 16, None) == B.NV_ERR_INVALID_ARG
     assert q(24, 1, 4, 64, 64, 4, 16, 16, 16, None) == B.NV_ERR_INVALID_ARG
     assert q(16, 1, 0, 64, 64, 4, 16, 16, 16, None) == B.NV_OK
+    assert q(16, 1, 0, 64, 64, 1, 16, 16, 16, None) == B.NV_OK  # 1-bit codes: quantizer only
+    assert q(16, 1, 4, 64, 64, 7, 16, 16, 16, None) == B.NV_ERR_INVALID_ARG
+
+
+def test_dequantize_argument_errors():
+    d = nvq.lib().nv_dequantize_affine
+    # codes, scales, biases, dt, rows, cols, group_size, bits, w, stream
+    assert d(16, 16, 16, 1, 4, 64, 64, 3, 16, None) == B.NV_ERR_UNSUPPORTED
+    assert d(16, 16, 16, 1, 4, 64, 64, 7, 16, None) == B.NV_ERR_INVALID_ARG
+    assert d(16, 16, 16, 7, 4, 64, 64, 4, 16, None) == B.NV_ERR_UNSUPPORTED
+    assert d(16, 16, 16, 1, 4, 96, 64, 4, 16, None) == B.NV_ERR_INVALID_ARG   # cols % group
+    assert d(16, 16, 16, 1, 4, 64, 48, 4, 16, None) == B.NV_ERR_INVALID_ARG   # group size
+    assert d(16, 16, 16, 1, -1, 64, 64, 4, 16, None) == B.NV_ERR_INVALID_ARG
+    assert d(0, 16, 16, 1, 4, 64, 64, 4, 16, None) == B.NV_ERR_INVALID_ARG
+    assert d(16, 16, 16, 1, 4, 64, 64, 4, 0, None) == B.NV_ERR_INVALID_ARG
+    assert d(24, 16, 16, 1, 4, 64, 64, 4, 16, None) == B.NV_ERR_INVALID_ARG  # misaligned
+    assert d(16, 16, 16, 1, 0, 64, 64, 1, 16, None) == B.NV_OK                # empty
 
 
 def test_gather_argument_errors():
