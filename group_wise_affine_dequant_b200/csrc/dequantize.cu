@@ -7,13 +7,14 @@
 // never cross a group), so word i of the whole array holds the values
 // [i * per_word, (i + 1) * per_word) of the flat output and belongs to group
 // (i * per_word) / group_size of the flat scale and bias arrays. The kernel is
-// therefore a flat map over words: each thread takes four consecutive words
-// (one 16-byte load), writes their values with 8- to 16-byte stores, and
-// strides over the array. Every value is one fused multiply-add in fp32,
-// scale * code + bias rounded once, then stored in the output dtype (bf16 by
-// round-to-nearest-even). HBM-bound: bytes moved per weight are bits / 8
-// (codes) + 4 / group_size or 8 / group_size (scale and bias) + the output
-// element size.
+// therefore a flat map over words: a warp takes 128 consecutive words per
+// step, lane l the words 32 q + l (q < 4), so that every load and store
+// instruction of the warp covers one contiguous run; it writes each word's
+// values with 8- to 16-byte stores and strides over the array. Every value is
+// one fused multiply-add in fp32, scale * code + bias rounded once, then
+// stored in the output dtype (bf16 by round-to-nearest-even). HBM-bound:
+// bytes moved per weight are bits / 8 (codes) + 4 / group_size or
+// 8 / group_size (scale and bias) + the output element size.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -67,26 +68,28 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restr
     constexpr int PER = 32 / BITS;
     constexpr int ESZ = DT == NV_F32 ? 4 : 2;
     char* o = static_cast<char*>(out);
-    const int64_t chunks = words / 4;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
-         c += stride) {
-        const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(codes) + c);
-        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // A warp takes 128 consecutive words per step, lane l the words 32 q + l:
+    // each load and each store instruction of the warp covers one contiguous
+    // run (128 code bytes in; 32 words' outputs out).
+    for (int64_t base = warp * 128; base < words; base += nwarps * 128) {
+        uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int64_t i = 4 * c + q;
-            const int64_t g = (i * PER) >> lg_gs;
-            word_out<DT, BITS>(w[q], load_elem<DT>(scales, g), load_elem<DT>(biases, g),
-                               o + i * PER * ESZ);
+            const int64_t i = base + 32 * q + lane;
+            w[q] = i < words ? __ldg(codes + i) : 0u;
         }
-    }
-    // the last words % 4 words, one per thread of the first block
-    if (blockIdx.x == 0 && threadIdx.x < words - 4 * chunks) {
-        const int64_t i = 4 * chunks + threadIdx.x;
-        const int64_t g = (i * PER) >> lg_gs;
-        word_out<DT, BITS>(__ldg(codes + i), load_elem<DT>(scales, g), load_elem<DT>(biases, g),
-                           o + i * PER * ESZ);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t i = base + 32 * q + lane;
+            if (i < words) {
+                const int64_t g = (i * PER) >> lg_gs;
+                word_out<DT, BITS>(w[q], load_elem<DT>(scales, g), load_elem<DT>(biases, g),
+                                   o + i * PER * ESZ);
+            }
+        }
     }
 }
 
@@ -96,7 +99,7 @@ cudaError_t launch_dt(const uint32_t* codes, const void* scales, const void* bia
                       int num_sms) {
     const int lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
     const int threads = 256;
-    int64_t blocks = (words / 4 + threads - 1) / threads;
+    int64_t blocks = (words / 4 + threads - 1) / threads;  // four words per thread
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
