@@ -278,8 +278,9 @@ class Dequant:
 class Gather:
     """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4."""
 
-    def __init__(self, dev, sorted_pairs: bool):
+    def __init__(self, dev, sorted_pairs: bool, row_exact: bool = False):
         import group_wise_affine_dequant_b200 as nvq
+        self.row_exact = row_exact
         self.nvq = nvq
         m = W.MOE
         self.E, self.N, self.K, self.T = m["E"], m["N"], m["K"], m["tokens"]
@@ -307,7 +308,7 @@ class Gather:
     def step(self, i):
         c, s, b = self.ws[i % self.copies]
         self.nvq.nv_gather_qmm(self.x, c, s, b, self.rhs, self.lhs, 64, 4, True, self.sorted,
-                               False, workspace=self.wsp, out=self.y)
+                               self.row_exact, workspace=self.wsp, out=self.y)
 
 
 # --------------------------------------------------------------------------- arms
@@ -374,8 +375,9 @@ def run_nvq(args):
     also["dequantize_14336x4096_b4g64_bf16_gbs"] = round(dq, 1)
     also["dequantize_frac_of_hbm"] = round(dq / ws / pk["hbm_gbs"], 4)
     del g, wl
-    for name, srt in (("gather_sorted", True), ("gather_unsorted", False)):
-        wl = Gather(dev, srt)
+    for name, srt, rx in (("gather_sorted", True, False), ("gather_unsorted", False, False),
+                          ("gather_row_exact", False, True)):
+        wl = Gather(dev, srt, rx)
         g = timed_graph(wl.step, ks, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
         also[name + "_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
