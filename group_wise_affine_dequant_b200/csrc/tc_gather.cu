@@ -2,17 +2,19 @@
 // "Mixture of experts": with rows sorted by expert, a grouped kernel reads each
 // expert's weights once). Each expert sees a handful of rows (tens), so the
 // product is computed transposed: D^T = W_e . X_e^T with the expert's weights as
-// the 128-row MMA operand A (dequantized into shared memory) and the expert's
-// gathered activation rows as the N side (16 .. 128 columns). Every weight tile
-// is read from HBM once and used for all of the expert's rows.
+// the 128-row MMA operand A (dequantized into tensor memory) and the expert's
+// gathered activation rows as the N side (16 .. 64 columns per pass). Every
+// weight tile is read from HBM once and used for all of the expert's rows.
 //
 // Work unit: (expert e, 256 weight rows = two 128-row tiles that share every
-// activation stage); a unit's pairs are taken in passes of at most 64. Roles,
-// per CTA (persistent):
-//   warp 0      one lane streams the code tiles by TMA, 128 rows x 128 bytes
+// activation stage); a unit's pairs are taken in passes of at most 64. The
+// kernel is the programmatic dependent of the routing kernel: it sets up and
+// prefetches its first weights into L2 before waiting for the routing tables.
+// Roles, per CTA (persistent):
+//   warp 0      one lane streams the code tiles by TMA, 256 rows x 128 bytes
 //               (several k-steps) per copy, into a ring released by the
 //               dequantizing warps once they have read them; scales and biases
-//               arrive per unit in blocks of up to 64 groups (swizzled boxes).
+//               arrive per unit in blocks of up to 32 groups (swizzled boxes).
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (M = 128,
 //               N = pairs rounded up to 16, K = 16), one per tile, into a
 //               double-buffered TMEM accumulator (64 columns per tile).
@@ -27,7 +29,9 @@
 //               MMA reads A from TMEM, so the dequantized tiles cost no
 //               shared-memory bandwidth, and four A stages fit beside the two
 //               accumulators.
-// Waits are bounded by a timer like the other pipelines.
+// At the end every CTA writes zero rows for its share of the pairs whose
+// expert or token id is out of range. Waits are bounded by a timer like the
+// other pipelines.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
