@@ -292,6 +292,33 @@ def test_gather_many_pairs_per_expert():
     P.assert_within(y, yr, a, BF16, "many pairs")
 
 
+def test_gather_back_to_back_share_a_workspace():
+    """Eight calls queued on one stream without synchronising, each with its
+    own routing and output but one workspace: every call's routing kernel must
+    wait for the previous grouped kernel (which still reads the tables) and
+    every grouped kernel for its own routing (a programmatic dependent
+    launch). Each output is checked against the oracle afterwards."""
+    E, N, K, T = 6, 256, 512, 40
+    w = W.normal((E, N, K), 0.02, 6, "bf16")
+    x = W.normal((T, K), 1.0, 7, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    dc, ds, db, dx = c.cuda(), s.cuda(), b.cuda(), x.cuda()
+    g = torch.Generator().manual_seed(11)
+    R = 96
+    ws = torch.empty(nvq.nv_gather_qmm_workspace_size(R, E), dtype=torch.uint8, device="cuda")
+    calls = []
+    for i in range(8):
+        rhs = torch.randint(0, E if i % 2 else 2, (R,), generator=g)  # skewed, then spread
+        lhs = torch.randint(0, T, (R,), generator=g)
+        y = nvq.nv_gather_qmm(dx, dc, ds, db, rhs.to(torch.int32).cuda(), lhs.to(torch.int32).cuda(),
+                              64, 4, True, False, False, workspace=ws)
+        calls.append((rhs, lhs, y))
+    torch.cuda.synchronize()
+    for i, (rhs, lhs, y) in enumerate(calls):
+        yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, 64, 4)
+        P.assert_within(y.cpu(), yr, a, BF16, f"back-to-back call {i}")
+
+
 def test_gather_flags_and_invalid_ids():
     E, N, K = 4, 64, 128
     w = W.normal((E, N, K), 0.02, 2, "bf16")
