@@ -16,7 +16,9 @@ bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
 events on the launching stream; max over ranks. The weights rotate over enough
 copies that the set touched between two uses of a copy exceeds the L2 cache.
 Multi-GPU runs are independent replicas (the product does not shard here):
-value = bytes processed by all ranks / max time.
+value = bytes processed by all ranks / max time. After timing, each workload's
+own output is checked against plain torch arithmetic on the GPU
+(`output_check` in the JSON line).
 """
 from __future__ import annotations
 
@@ -81,6 +83,56 @@ def replica_rate(ws: int, units_per_step: float, steps: int, ms_max: float) -> f
     """Whole-job rate of N independent replicas: the units all ranks processed
     divided by the slowest rank's time (per second)."""
     return ws * units_per_step * steps / (ms_max / 1e3)
+
+
+# ------------------------------------------------------------ output checks
+# Each timed workload's own output is checked after timing against plain torch
+# arithmetic on the GPU (codes unpacked with shifts and masks, fp32 products):
+# a sanity check of the timed run, independent of the library's kernels. The
+# parity proper is the test suite's comparison with the oracle.
+def unpack_dequant(codes, scales, biases, gs, bits):
+    """w = scale * code + bias in fp32, [..., rows, cols], with torch ops."""
+    per = 32 // bits
+    c = codes.to(torch.int64) & 0xFFFFFFFF
+    sh = torch.arange(per, device=codes.device, dtype=torch.int64) * bits
+    v = ((c.unsqueeze(-1) >> sh) & ((1 << bits) - 1)).flatten(-2).to(torch.float32)
+    return v * scales.float().repeat_interleave(gs, -1) + biases.float().repeat_interleave(gs, -1)
+
+
+def worst_ratio(y, x, w):
+    """max |y - x.w^T| / (4e-3 * sum|x||w| + 1e-5); <= 1 passes (bf16 tolerance)."""
+    ref = x.float() @ w.T
+    tol = 4e-3 * (x.float().abs() @ w.abs().T) + 1e-5
+    return float(((y.float() - ref).abs() / tol).max())
+
+
+def check_decode(wl, rows=None):
+    c, s, b = wl.ws[0]
+    w = unpack_dequant(c, s, b, wl.gs, wl.bits)
+    if not wl.t:  # stored [K, N]: the product is x . w
+        w = w.T
+    x, y = wl.x, wl.y
+    if rows is not None:
+        x, y = x[rows], y[rows]
+    return worst_ratio(y, x, w)
+
+
+def check_gather(wl, samples=64):
+    c, s, b = wl.ws[0]
+    g = torch.Generator(device="cpu").manual_seed(5)
+    pick = torch.randperm(wl.R, generator=g)[:samples].tolist()
+    worst = 0.0
+    for r in pick:
+        e, t = int(wl.rhs[r]), int(wl.lhs[r])
+        w = unpack_dequant(c[e], s[e], b[e], 64, 4)
+        worst = max(worst, worst_ratio(wl.y[r:r + 1], wl.x[t:t + 1], w))
+    return worst
+
+
+def check_dequant(wl):
+    c, s, b = wl.ws[0]
+    ref = unpack_dequant(c, s, b, wl.gs, wl.bits).to(wl.out.dtype)
+    return 0.0 if torch.equal(ref, wl.out) else float("inf")
 
 
 class ClockSampler:
@@ -342,6 +394,7 @@ def run_nvq(args):
         while time.time() < t_end:
             replay_timed(graphs, stream, lambda: None)
     del graphs
+    checks = {"decode": round(check_decode(dec), 4)}
     ms = max_ms(ms)
     per_step_s = ms / 1e3 / K
     value = replica_rate(ws, dec.bytes, K, ms) / 1e9
@@ -367,6 +420,7 @@ def run_nvq(args):
         g = timed_graph(wl.step, ks, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
         also[name] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
+        checks[name.replace("_gbs", "")] = round(check_decode(wl), 4)
         del g, wl
     wl = Dequant(dev)
     g = timed_graph(wl.step, ks, Wm, stream)
@@ -374,6 +428,7 @@ def run_nvq(args):
     dq = replica_rate(ws, wl.bytes, ks, t) / 1e9
     also["dequantize_14336x4096_b4g64_bf16_gbs"] = round(dq, 1)
     also["dequantize_frac_of_hbm"] = round(dq / ws / pk["hbm_gbs"], 4)
+    checks["dequantize"] = check_dequant(wl)
     del g, wl
     for name, srt, rx in (("gather_sorted", True, False), ("gather_unsorted", False, False),
                           ("gather_row_exact", False, True)):
@@ -382,6 +437,7 @@ def run_nvq(args):
         t = max_ms(replay_timed(g, stream, barrier))
         also[name + "_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
         also[name + "_gbs"] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
+        checks[name] = round(check_gather(wl), 4)
         del g, wl
     for bits, gs in W.PREFILL_VARIANTS:
         wl = Decode(dev, N=14336, K=4096, M=2048, bits=bits, gs=gs)
@@ -393,6 +449,7 @@ def run_nvq(args):
         also[key] = round(tf, 1)
         if (bits, gs) == (4, 64):
             also["prefill_frac_of_bf16_peak"] = round(tf / pk["bf16_tflops"], 4)
+        checks[key.replace("_tflops", "")] = round(check_decode(wl, rows=torch.arange(0, 2048, 128)), 4)
         del g, wl
 
     line = {
@@ -423,6 +480,10 @@ def run_nvq(args):
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"]},
         "also": also,
+        "output_check": {"rule": "worst |y - torch fp32 reference| / (4e-3 sum|x w| + 1e-5) per timed "
+                                 "workload (prefill: 16 rows; gather: 64 pairs; dequantize: 0 = bitwise "
+                                 "equal); <= 1 passes",
+                         "worst": checks, "pass": all(v <= 1.0 for v in checks.values())},
         "cpu_baseline": None,
     }
     if ws == 1 and rank == 0 and not args.no_cpu_baseline:
