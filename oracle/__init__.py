@@ -63,6 +63,8 @@ def _bind(lib):
     lib.orc_gather_qmm_sampled.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p,
                                            _p, _p, _i, _i, _i, _i, _i64, _p, _p, _p, _p]
     lib.orc_gather_qmm_sampled.restype = _i
+    lib.orc_gather_mm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _i, _p, _p]
+    lib.orc_gather_mm.restype = _i
     return lib
 
 
@@ -215,6 +217,28 @@ def gather_qmm(x, codes, scales, biases, lhs, rhs, group_size, bits, transpose=T
                             _DT[scales.dtype], group_size, bits, int(transpose), y.data_ptr(),
                             a.data_ptr())
     _check(rc, "gather_qmm")
+    return y, a
+
+
+def gather_mm(x, w, lhs, rhs, lib=None):
+    """fp64 (y, a) [R, N]: row r = x[lhs[r]] times full-precision expert
+    w[rhs[r]] ([E, N, K], transposed product; lhs None: identity)."""
+    lib = lib or load()
+    x, w = _cpu(x), _cpu(w)
+    x2 = x.reshape(-1, x.shape[-1])
+    x_rows, K = x2.shape
+    E, N = w.shape[0], w.shape[1]
+    if w.dim() != 3 or w.shape[2] != K:
+        raise ValueError(f"oracle: experts {tuple(w.shape)} do not match K={K}")
+    lhs_t, rhs_t = _u32(lhs), _u32(rhs)
+    R = rhs_t.numel()
+    y = torch.empty(R, N, dtype=torch.float64)
+    a = torch.empty(R, N, dtype=torch.float64)
+    w = w.contiguous()
+    rc = lib.orc_gather_mm(x2.contiguous().data_ptr(), _DT[x.dtype], x_rows, K,
+                           None if lhs_t is None else lhs_t.data_ptr(), rhs_t.data_ptr(), R, E, N,
+                           w.data_ptr(), _DT[w.dtype], y.data_ptr(), a.data_ptr())
+    _check(rc, "gather_mm")
     return y, a
 
 

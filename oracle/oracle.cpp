@@ -315,4 +315,33 @@ int orc_gather_qmm_sampled(const void* x, int xdtype, int64_t x_rows, int64_t K,
     return 0;
 }
 
+// Gather with full-precision experts [Q-MoE: every row meets the weights of
+// its own expert; crate docs: gather_mm beside gather_qmm]:
+// y[r, n] = sum_k x[lhs[r], k] * w[rhs[r], n, k], w [E, N, K] in `wdtype`,
+// fp64, sequential in k; a[r, n] = sum_k |x * w|. Returns -1 if an index is
+// out of range.
+int orc_gather_mm(const void* x, int xdtype, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                  const uint32_t* rhs, int64_t R, int64_t E, int64_t N, const void* w,
+                  int wdtype, double* y, double* a) {
+    for (int64_t r = 0; r < R; ++r) {
+        int64_t t = lhs ? (int64_t)lhs[r] : r;
+        if (t >= x_rows || (int64_t)rhs[r] >= E) return -1;
+    }
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            const int64_t t = lhs ? (int64_t)lhs[r] : r;
+            const int64_t wrow = ((int64_t)rhs[r] * N + n) * K;
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = load_value(x, xdtype, t * K + k) * load_value(w, wdtype, wrow + k);
+                acc += p;
+                mag += std::fabs(p);
+            }
+            y[r * N + n] = acc;
+            a[r * N + n] = mag;
+        }
+    return 0;
+}
+
 }  // extern "C"

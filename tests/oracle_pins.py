@@ -378,6 +378,40 @@ def pin_gather(lib):
         raise AssertionError("expert id 8 of 8 experts accepted")
 
 
+def pin_gather_mm(lib):
+    """gather_mm with full-precision experts: integer x and weights give exact
+    integer rows equal to an int64 brute force per pair; scaled-identity
+    experts return (e + 1) times the selected x row, with sum |x w| the same
+    multiple of |x|; out-of-range ids are refused."""
+    g = torch.Generator().manual_seed(37)
+    E, N, K, T = 5, 24, 128, 9
+    for dt in (torch.float32, torch.bfloat16):
+        wi = torch.randint(-8, 9, (E, N, K), generator=g)
+        xi = torch.randint(-2, 3, (T, K), generator=g)
+        lhs = torch.randint(0, T, (17,), generator=g)
+        rhs = torch.randint(0, E, (17,), generator=g)
+        y, a = O.gather_mm(xi.to(dt), wi.to(dt), lhs, rhs, lib=lib)
+        for r in range(17):
+            t, e = int(lhs[r]), int(rhs[r])
+            ref = (wi[e] * xi[t]).sum(-1)          # int64, exact
+            assert torch.equal(y[r], ref.to(torch.float64)), (dt, r)
+            assert torch.equal(a[r], (wi[e] * xi[t]).abs().sum(-1).to(torch.float64)), (dt, r)
+    eye = torch.stack([torch.eye(K) * (e + 1) for e in range(E)])  # [E, K, K]
+    x = torch.randn(T, K, generator=g).to(torch.bfloat16)
+    rhs = torch.tensor([0, 4, 2, 2, 1])
+    y, a = O.gather_mm(x[:5], eye.to(torch.bfloat16), None, rhs, lib=lib)
+    for r in range(5):
+        mult = float(rhs[r]) + 1.0
+        assert torch.equal(y[r], x[r].double() * mult), r
+        assert torch.equal(a[r], x[r].double().abs() * mult), r
+    try:
+        O.gather_mm(x, eye, None, torch.tensor([0, 5]), lib=lib)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("expert id 5 of 5 experts accepted")
+
+
 def pin_sampled_match_full(lib):
     """The sampled product entry points agree with the full ones."""
     g = torch.Generator().manual_seed(31)

@@ -47,6 +47,12 @@ MUTANTS = [
     ("signed zero by order", "if (v < mn || (v == mn && std::signbit(v))) mn = v;",
      "if (v < mn) mn = v;"),
     ("constant group top code", "uint32_t q = 0;", "uint32_t q = (uint32_t)levels;"),
+    ("gather_mm wrong expert", "const int64_t wrow = ((int64_t)rhs[r] * N + n) * K;",
+     "const int64_t wrow = ((int64_t)rhs[R - 1 - r] * N + n) * K;"),
+    ("gather_mm ignores lhs", "const int64_t t = lhs ? (int64_t)lhs[r] : r;",
+     "const int64_t t = r % x_rows;"),
+    ("gather_mm transposed expert", "load_value(w, wdtype, wrow + k)",
+     "load_value(w, wdtype, (int64_t)rhs[r] * N * K + k * N + n)"),
 ]
 
 RUNNER = r"""
