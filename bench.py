@@ -8,8 +8,8 @@ a 4-bit, group-64 decode product y = x . w^T with x [1, 4096] bf16 and
 W [14336, 4096] (Llama-8B MLP shape), i.e. one nv_qmm call. The JSON line
 reports HBM GB/s of algorithmic bytes (codes + scales + biases + x + y); the
 other workloads (8-bit and transposed decode, few rows, prefill, mixture of
-experts, dequantization to bf16) are measured in the same run and reported
-under "also".
+experts with 4-bit and with bf16 weights, dequantization to bf16) are
+measured in the same run and reported under "also".
 
 Timing: W untimed warm-up steps, then K timed steps captured in CUDA graphs and
 bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
@@ -327,6 +327,45 @@ class Dequant:
         self.nvq.nv_dequantize_affine(c, s, b, self.gs, self.bits, out=self.out)
 
 
+class GatherMM:
+    """Mixture of experts with full-precision bf16 experts [64, 1536, 2048]."""
+
+    def __init__(self, dev):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        m = W.MOE
+        self.E, self.N, self.K, self.T = m["E"], m["N"], m["K"], m["tokens"]
+        w = W.normal((self.E, self.N, self.K), 0.02, 0, "bf16").to(dev)
+        wbytes = w.numel() * 2
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))
+        self.ws = [w] + [w.clone() for _ in range(self.copies - 1)]
+        ids = W.expert_ids(self.T, self.E, m["top_k"], 2)
+        lhs, rhs = W.flatten_pairs(ids)
+        self.lhs = lhs.to(torch.int32).to(dev)
+        self.rhs = rhs.to(torch.int32).to(dev)
+        self.R = rhs.numel()
+        self.x = W.normal((self.T, self.K), 1.0, 1, "bf16").to(dev)
+        self.y = torch.empty(self.R, self.N, dtype=torch.bfloat16, device=dev)
+        self.wsp = torch.empty(nvq.nv_gather_qmm_workspace_size(self.R, self.E), dtype=torch.uint8,
+                               device=dev)
+        self.bytes = wbytes + self.T * self.K * 2 + self.R * self.N * 2 + self.R * 8
+
+    def step(self, i):
+        self.nvq.nv_gather_mm(self.x, self.ws[i % self.copies], self.rhs, self.lhs,
+                              workspace=self.wsp, out=self.y)
+
+
+def check_gather_mm(wl, samples=64):
+    g = torch.Generator(device="cpu").manual_seed(5)
+    pick = torch.randperm(wl.R, generator=g)[:samples].tolist()
+    worst = 0.0
+    for r in pick:
+        e, t = int(wl.rhs[r]), int(wl.lhs[r])
+        worst = max(worst, worst_ratio(wl.y[r:r + 1], wl.x[t:t + 1], wl.ws[0][e].float()))
+    return worst
+
+
 class Gather:
     """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4."""
 
@@ -439,6 +478,15 @@ def run_nvq(args):
         also[name + "_gbs"] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
         checks[name] = round(check_gather(wl), 4)
         del g, wl
+    wl = GatherMM(dev)
+    g = timed_graph(wl.step, ks, Wm, stream)
+    t = max_ms(replay_timed(g, stream, barrier))
+    also["gather_mm_bf16_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
+    gm = replica_rate(ws, wl.bytes, ks, t) / 1e9
+    also["gather_mm_bf16_gbs"] = round(gm, 1)
+    also["gather_mm_frac_of_hbm"] = round(gm / ws / pk["hbm_gbs"], 4)
+    checks["gather_mm_bf16"] = round(check_gather_mm(wl), 4)
+    del g, wl
     for bits, gs in W.PREFILL_VARIANTS:
         wl = Decode(dev, N=14336, K=4096, M=2048, bits=bits, gs=gs)
         kp = max(3, min(K, 100))

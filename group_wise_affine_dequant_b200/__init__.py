@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     NV_ROW_INDEPENDENT_ROWS,
     NvqError,
     lib,
+    nv_gather_mm,
     nv_gather_qmm,
     nv_gather_qmm_flags,
     nv_gather_qmm_workspace_size,

@@ -25,7 +25,7 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_dequantize_affine", "nv_qmm",
-           "nv_gather_qmm_workspace_size",
+           "nv_gather_qmm_workspace_size", "nv_gather_mm",
            "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error",
            "nv_gather_qmm_noalloc")
 
@@ -70,6 +70,9 @@ def lib():
             L.nv_gather_qmm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _p,
                                         _i, _i, _i, _i, _i, _p, _sz, _p, _p]
             L.nv_gather_qmm.restype = _i
+            L.nv_gather_mm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _i, _p,
+                                       _sz, _p, _p]
+            L.nv_gather_mm.restype = _i
             L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
             L.nv_gather_qmm_flags.restype = _i
             L.nv_gather_qmm_noalloc.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p,
@@ -231,6 +234,40 @@ def nv_gather_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
                              workspace.numel() * workspace.element_size(), y.data_ptr(),
                              _stream(stream))
     _check("nv_gather_qmm", st)
+    return y
+
+
+def nv_gather_mm(x: torch.Tensor, w: torch.Tensor, rhs: torch.Tensor,
+                 lhs: torch.Tensor | None = None, sorted: bool = False,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Row r of the result is x[lhs[r]] times full-precision expert w[rhs[r]]
+    (transposed: w [E, N, K] bf16, y[r] = x[lhs[r]] . w[rhs[r]]^T)."""
+    for t, n in ((x, "x"), (w, "w"), (rhs, "rhs")):
+        _dev(t, n)
+    if lhs is not None:
+        _dev(lhs, "lhs")
+    K = x.shape[-1]
+    x_rows = x.numel() // K if K else 0
+    if w.dim() != 3 or w.shape[2] != K:
+        raise ValueError(f"experts {tuple(w.shape)} do not match x (K={K})")
+    E, N = w.shape[0], w.shape[1]
+    if w.dtype != x.dtype:
+        raise NvqError("nv_gather_mm", NV_ERR_UNSUPPORTED, nv_status_string(NV_ERR_UNSUPPORTED))
+    R = rhs.numel()
+    if lhs is not None and lhs.numel() != R:
+        raise ValueError("lhs and rhs differ in length")
+    ws_bytes = nv_gather_qmm_workspace_size(R, E)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
+    y = out if out is not None else torch.empty(R, N, dtype=x.dtype, device=x.device)
+    if y.numel() != R * N or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
+    st = lib().nv_gather_mm(x.data_ptr(), _DT.get(x.dtype, -1), x_rows, K, _ptr(lhs),
+                            rhs.data_ptr(), R, E, N, w.data_ptr(), int(sorted),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            y.data_ptr(), _stream(stream))
+    _check("nv_gather_mm", st)
     return y
 
 

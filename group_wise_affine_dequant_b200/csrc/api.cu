@@ -184,6 +184,31 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
                                              scales, biases, group_size, bits, transpose, y, s));
 }
 
+nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
+                       const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R, int64_t E,
+                       int64_t N, const void* w, int sorted, void* workspace,
+                       size_t workspace_bytes, void* y, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    if (x_rows < 0 || K <= 0 || R < 0 || E <= 0 || N < 0) return NV_ERR_INVALID_ARG;
+    if (R > (int64_t(1) << 31) - 1) return NV_ERR_INVALID_ARG;
+    if (E > nvq::kMaxExperts) return NV_ERR_UNSUPPORTED;
+    if (dt != NV_BF16 || !nvq::tc_gather_mm_supported(K, N > 0 ? N : 1)) return NV_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace)) return NV_ERR_WORKSPACE;
+    if (workspace_bytes < nvq::gather_workspace_bytes(R, E)) return NV_ERR_WORKSPACE;
+    if (R == 0) return NV_OK;
+    if (!x || !rhs_idx || !w || !y) return NV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y) || !aligned16(rhs_idx) ||
+        (lhs_idx && !aligned16(lhs_idx)))
+        return NV_ERR_INVALID_ARG;
+    cudaStream_t s = stream;
+    nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
+    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (N == 0) return NV_OK;
+    return from_cuda(nvq::launch_tc_gather_mm(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N, w,
+                                              y, s, sm_count()));
+}
+
 nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream) {
     if (!workspace || !aligned16(workspace) || !host_flags) return NV_ERR_INVALID_ARG;
     cudaStream_t s = stream;
@@ -203,8 +228,10 @@ nv_status nv_pipeline_error(uint32_t* host_code) {
     const unsigned int a = nvq::qmv_error_take();
     const unsigned int b = nvq::tc_error_take();
     const unsigned int c = nvq::tc_gather_error_take();
-    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return NV_ERR_CUDA;
-    *host_code = a ? a : b ? b : c;
+    const unsigned int d = nvq::tc_gather_mm_error_take();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu || d == 0xFFFFFFFFu)
+        return NV_ERR_CUDA;
+    *host_code = a ? a : b ? b : c ? c : d;
     return NV_OK;
 }
 

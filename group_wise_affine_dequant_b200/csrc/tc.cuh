@@ -24,4 +24,11 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
                              int bits, void* y, cudaStream_t stream, int num_sms);
 unsigned int tc_gather_error_take();
 
+// The same grouped product with full-precision (bf16) experts [E, N, K].
+bool tc_gather_mm_supported(int64_t K, int64_t N);
+cudaError_t launch_tc_gather_mm(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                                const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
+                                const void* w, void* y, cudaStream_t stream, int num_sms);
+unsigned int tc_gather_mm_error_take();
+
 }  // namespace nvq

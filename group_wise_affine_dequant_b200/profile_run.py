@@ -5,7 +5,8 @@
 WORKLOAD is one of decode (x[1,4096] . W[14336,4096]^T, 4-bit g64), decode8
 (the same at 8 bits), gather (64 experts [1536,2048] 4-bit g64, 512 tokens x
 top-4, unsorted), prefill (x[2048,4096] . W[14336,4096]^T, 4-bit g64),
-dequant (W[14336,4096] 4-bit g64 codes to bf16). The
+dequant (W[14336,4096] 4-bit g64 codes to bf16), gather_mm (the mixture of
+experts with bf16 experts). The
 workloads are bench.py's (same shapes, seeds and weight-copy rotation); the
 launches are plain stream launches (no graphs), so that a profiler sees one
 kernel per product (two plus the router for a gather). Prints the mean time per
@@ -37,6 +38,8 @@ def make(name: str, dev):
         return bench.Decode(dev, N=14336, K=4096, M=2048, bits=4, gs=64)
     if name == "dequant":
         return bench.Dequant(dev)
+    if name == "gather_mm":
+        return bench.GatherMM(dev)
     raise SystemExit(f"unknown workload {name!r}")
 
 

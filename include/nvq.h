@@ -170,8 +170,25 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
                         int group_size, int bits, int transpose, int sorted, int row_exact,
                         void* workspace, size_t workspace_bytes, void* y, nv_stream_t stream);
 
-/* Copy the anomaly flags of the last nv_gather_qmm that used `workspace` into
- * *host_flags (a HOST pointer). Synchronises `stream`. */
+/*
+ * Mixture-of-experts product with full-precision experts, gather_mm (the
+ * unquantized companion of gather_qmm; "Docs / Quantization", section
+ * "Mixture of experts", and the nuvec crate docs).
+ *
+ * x, lhs_idx, rhs_idx, sorted, workspace, y: as for nv_gather_qmm (the same
+ *   routing and workspace size; nv_gather_qmm_flags reads its flags).
+ * w        bf16 [E, N, K]: expert e's weights, row n = output feature n.
+ * y[r, n] = sum_k x[lhs[r], k] * w[rhs[r], n, k], fp32 accumulation, stored
+ *   in bf16; pairs with an out-of-range id get zero rows and a flag.
+ * dt must be NV_BF16 and K a multiple of 64 (NV_ERR_UNSUPPORTED otherwise).
+ */
+nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
+                       const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R, int64_t E,
+                       int64_t N, const void* w, int sorted, void* workspace,
+                       size_t workspace_bytes, void* y, nv_stream_t stream);
+
+/* Copy the anomaly flags of the last nv_gather_qmm (or nv_gather_mm) that used
+ * `workspace` into *host_flags (a HOST pointer). Synchronises `stream`. */
 nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream);
 
 /*

@@ -125,6 +125,34 @@ def test_gather_argument_errors():
     assert call(R=0, ws_bytes=L.nv_gather_qmm_workspace_size(0, E)) == B.NV_OK
 
 
+def test_gather_mm_argument_errors():
+    L = nvq.lib()
+    R, E = 2048, 64
+    need = L.nv_gather_qmm_workspace_size(R, E)
+
+    def call(ws=16, ws_bytes=need, **kw):
+        a = dict(x=16, dt=1, x_rows=512, K=2048, lhs=16, rhs=16, R=R, E=E, N=1536, w=16,
+                 sorted=0, y=16)
+        a.update(kw)
+        return L.nv_gather_mm(a["x"], a["dt"], a["x_rows"], a["K"], a["lhs"], a["rhs"], a["R"],
+                              a["E"], a["N"], a["w"], a["sorted"], ws, ws_bytes, a["y"], None)
+
+    assert call(ws_bytes=need - 1) == B.NV_ERR_WORKSPACE
+    assert call(ws=0) == B.NV_ERR_WORKSPACE
+    assert call(ws=8) == B.NV_ERR_WORKSPACE
+    assert call(dt=0) == B.NV_ERR_UNSUPPORTED        # fp32 experts: not implemented
+    assert call(dt=7) == B.NV_ERR_UNSUPPORTED
+    assert call(K=100) == B.NV_ERR_UNSUPPORTED       # K not a multiple of 64
+    assert call(E=0) == B.NV_ERR_INVALID_ARG
+    assert call(R=-1) == B.NV_ERR_INVALID_ARG
+    assert call(E=5000, ws_bytes=L.nv_gather_qmm_workspace_size(R, 5000)) == B.NV_ERR_UNSUPPORTED
+    assert call(rhs=0) == B.NV_ERR_INVALID_ARG
+    assert call(w=0) == B.NV_ERR_INVALID_ARG
+    assert call(w=24) == B.NV_ERR_INVALID_ARG        # misaligned
+    assert call(lhs=4) == B.NV_ERR_INVALID_ARG
+    assert call(R=0, ws_bytes=L.nv_gather_qmm_workspace_size(0, E)) == B.NV_OK
+
+
 def test_flags_argument_errors():
     L = nvq.lib()
     assert L.nv_pipeline_error(0) == B.NV_ERR_INVALID_ARG
