@@ -7,14 +7,16 @@
 // weight tile is read from HBM once and used for all of the expert's rows.
 //
 // Work unit: (expert e, 256 weight rows = two 128-row tiles that share every
-// activation stage); a unit's pairs are taken in passes of at most 64. The
+// activation stage); a unit's pairs are taken in passes of at most 64, and K
+// in steps of 128 (every pipeline handshake moves a 128-k slab: 16 MMAs, 16 KB
+// of codes at 4 bits, 16 KB of activations per k-step). The
 // kernel is the programmatic dependent of the routing kernel: it sets up and
 // prefetches its first weights into L2 before waiting for the routing tables.
 // Roles, per CTA (persistent):
 //   warp 0      one lane streams the code tiles by TMA, 256 rows x 128 bytes
 //               (several k-steps) per copy, into a ring released by the
 //               dequantizing warps once they have read them; scales and biases
-//               arrive per unit in blocks of up to 32 groups (swizzled boxes).
+//               arrive per unit in blocks of up to 16 groups (swizzled boxes).
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (M = 128,
 //               N = pairs rounded up to 16, K = 16), one per tile, into a
 //               double-buffered TMEM accumulator (64 columns per tile).
@@ -24,11 +26,11 @@
 //               thread per row and k-step) into the 128-byte-swizzled B layout;
 //               each thread fences its completed copies into the async proxy
 //               before it arrives on the stage's barrier.
-//   warps 10-25 dequantize, one thread per (weight row, 32 k) of each tile,
-//               straight into tensor memory (tcgen05.st): the
-//               MMA reads A from TMEM, so the dequantized tiles cost no
-//               shared-memory bandwidth, and four A stages fit beside the two
-//               accumulators.
+//   warps 10-25 dequantize, one thread per (weight row, 64 k) of each tile
+//               (two runs of 32 k, each inside one group), straight into
+//               tensor memory (tcgen05.st): the MMA reads A from TMEM, so the
+//               dequantized tiles cost no shared-memory bandwidth, and two
+//               128-k A stages fit beside the two accumulators.
 // At the end every CTA writes zero rows for its share of the pairs whose
 // expert or token id is out of range. Waits are bounded by a timer like the
 // other pipelines.
@@ -49,21 +51,24 @@ using namespace tc;
 constexpr int WM = 128;          // weight rows per tile (TMEM lanes)
 constexpr int kTiles = 2;        // weight tiles per unit: every activation stage serves both
 constexpr int UW = WM * kTiles;  // weight rows per unit
-constexpr int BK = 64;
+constexpr int BK = 128;
 constexpr int UMMA_K = 16;
 constexpr int kMaxPairs = 64;    // pairs per pass (TMEM columns of one tile's accumulator)
 static_assert(kMaxPairs == 64, "the epilogue keeps two pair ids per lane");
 constexpr int kEpilogueWarp0 = 2;
 constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-9
 constexpr int kXThreads = 128;
-constexpr int kDequantWarp0 = 10; // warps 10-25: dequantize, one tile and 32 k per thread
+constexpr int kDequantWarp0 = 10; // warps 10-25: dequantize, one tile and 64 k per thread
 constexpr int kDequantThreads = 512;
 constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;
-constexpr uint32_t kXStage = kMaxPairs * 128;  // activation stage: kMaxPairs rows x 64 k
+constexpr uint32_t kXStage = kMaxPairs * BK * 2;  // activation stage: kMaxPairs rows x BK k (two swizzle atoms)
+constexpr int kXChunks = BK * 2 / 16;         // 16-byte pieces of a row per k-step
+constexpr int kXRS = kXThreads / kXChunks;    // rows a pass of the loader threads covers
+constexpr uint32_t kXoffBytes = kMaxPairs / kXRS * kXThreads * 4;
 constexpr uint32_t kCStage = UW * 128;         // code stage: the unit's rows x 128 code bytes
 constexpr int kAccCols = kTiles * kMaxPairs;   // accumulator columns of one pass
-constexpr int kACols = kTiles * 32;            // TMEM columns of one A stage (64 k per tile)
-constexpr int kDA = 4;                         // A stages, in TMEM after the accumulators
+constexpr int kACols = kTiles * (BK / 2);      // TMEM columns of one A stage (BK k per tile)
+constexpr int kDA = 2;                         // A stages, in TMEM after the accumulators
 constexpr uint32_t kTmemCols = 512;
 static_assert(2 * kAccCols + kDA * kACols <= static_cast<int>(kTmemCols), "TMEM budget");
 
@@ -254,9 +259,11 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
 #pragma unroll
                         for (int tt = 0; tt < kTiles; ++tt)  // both tiles against the same activations
 #pragma unroll
-                            for (int kk = 0; kk < BK / UMMA_K; ++kk)  // 16 k = 8 TMEM columns of A
-                                tc_mma_ts(d_tmem + tt * kMaxPairs, at + tt * 32 + kk * (UMMA_K / 2),
-                                          bd + (kk * UMMA_K * 2 >> 4), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < BK / UMMA_K; ++kk)  // 16 k = 8 TMEM columns of A; B: 4 per 128-byte atom
+                                tc_mma_ts(d_tmem + tt * kMaxPairs, at + tt * (BK / 2) + kk * (UMMA_K / 2),
+                                          bd + static_cast<uint64_t>((kk >> 2) * (kMaxPairs * 128 >> 4)) +
+                                              (((kk & 3) * UMMA_K * 2) >> 4),
+                                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                         tc_commit(&empty_a[a.s]);
                         tc_commit(&empty_x[x.s]);
                         a.next(DA);
@@ -322,9 +329,9 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 16 j of every
         // k-step. Stages are completed in order, LAG k-steps behind the copies.
         const int xt = threadIdx.x - kXWarp0 * 32;  // 0 .. kXThreads - 1
-        constexpr int RS = kXThreads / 8;            // row stride between a thread's rows
-        const int ch = xt & 7, r0 = xt >> 3;
-        const int lag = DX - 1 < 4 ? DX - 1 : 4;
+        constexpr int RS = kXRS;                     // row stride between a thread's rows
+        const int ch = xt % kXChunks, r0 = xt / kXChunks;
+        const int lag = DX - 1 < 3 ? DX - 1 : 3;
         RingPos x, done;  // next stage to fill, next stage to complete
         int pending = 0;
         bool ok = true;
@@ -352,7 +359,8 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     uint8_t* dst = x_ring + x.s * kXStage;
                     for (int j = 0; j < nr; ++j) {
                         const int r = r0 + RS * j;
-                        cp_async16(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4),
+                        cp_async16(dst + (ch >> 3) * (kMaxPairs * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                                       (((ch & 7) ^ (r & 7)) << 4),
                                    prm.x + s_xoff[j * kXThreads + xt] + ks * BK);
                     }
                     cp_async_commit();
@@ -397,33 +405,35 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         gb = (ks * BK) >> prm.lg_gs;  // first group of the block
                     }
                     const uint8_t* ss = sb_ring + slot * prm.sb_slot;
-                    // 32 k of one group (groups are 32-k aligned multiples of 32)
-                    const int gc = ((ks * BK + 32 * hf) >> prm.lg_gs) - gb;
                     if (kc == 0 && !(ok = mbar_wait(&full_c[c.s], c.use & 1, 26))) break;
-                    // this thread's 32 k of its row: part kc of the code rows
+                    // this thread's 64 k of its row (part kc of the code rows), as two
+                    // runs of 32 k, each inside one group (groups are multiples of 32)
                     constexpr int NW = BITS;  // code words per 32 k
-                    uint32_t w[NW];
-                    const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
-                    const float sc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
-                    const float bc = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
-                    {
+                    uint32_t w[2][NW];
+                    float sc[2], bc[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int gc = ((ks * BK + 64 * hf + 32 * h2) >> prm.lg_gs) - gb;
+                        const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
+                        sc[h2] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
+                        bc[h2] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
                         const uint8_t* crow = c_ring + c.s * kCStage + rr * 128;
+                        const int o = kc * (BK * BITS / 8) + (64 * hf + 32 * h2) * BITS / 8;
                         if constexpr (BITS == 4) {
-                            const int o = kc * 32 + hf * 16;
                             const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                            w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+                            w[h2][0] = v4.x; w[h2][1] = v4.y; w[h2][2] = v4.z; w[h2][3] = v4.w;
                         } else if constexpr (BITS == 8) {
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
-                                const int o = kc * 64 + hf * 32 + h * 16;
-                                const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
-                                w[4 * h] = v4.x; w[4 * h + 1] = v4.y; w[4 * h + 2] = v4.z; w[4 * h + 3] = v4.w;
+                                const uint4 v4 = *reinterpret_cast<const uint4*>(
+                                    crow + ((((o >> 4) + h) ^ (r & 7)) << 4));
+                                w[h2][4 * h] = v4.x; w[h2][4 * h + 1] = v4.y;
+                                w[h2][4 * h + 2] = v4.z; w[h2][4 * h + 3] = v4.w;
                             }
                         } else {
-                            const int o = kc * 16 + hf * 8;
                             const uint2 v2 = *reinterpret_cast<const uint2*>(
                                 crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
-                            w[0] = v2.x; w[1] = v2.y;
+                            w[h2][0] = v2.x; w[h2][1] = v2.y;
                         }
                     }
                     const bool last_part = (kc == spk - 1) || (ks == ksteps - 1);
@@ -435,14 +445,17 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (++kc == spk) kc = 0;
                     if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
-                    {
-                        const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
-                        const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const uint32_t s2 = (__float_as_uint(sc[h2]) >> 16) * 0x00010001u;
+                        const uint32_t b2 = (__float_as_uint(bc[h2]) >> 16) * 0x00010001u;
                         uint32_t out[16];
 #pragma unroll
                         for (int i = 0; i < NW; ++i)
-                            DQ::run(w[i], s2, b2, sc, bc, 2u, 4u, 6u, out + i * DQ::PAIRS);
-                        tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + 32 * tt + 16 * hf, out);
+                            DQ::run(w[h2][i], s2, b2, sc[h2], bc[h2], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                        tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + (BK / 2) * tt +
+                                        32 * hf + 16 * h2,
+                                    out);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -508,7 +521,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
             return cudaErrorInvalidValue;
     }
     // scale/bias boxes: up to 32 groups (64 bytes) per row, swizzled by row width
-    const int sbg = gpr >= 32 ? 32 : static_cast<int>(gpr);
+    const int sbg = gpr >= 16 ? 16 : static_cast<int>(gpr);
     const int sbw = sbg * 2;
     const int lg_sbw = sbw == 128 ? 7 : sbw == 64 ? 6 : sbw == 32 ? 5 : 4;
     {
@@ -544,10 +557,10 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.lg_sbw = lg_sbw;
     prm.sb_slot = 2 * UW * sbw;
     const size_t sb_ring = 2u * static_cast<size_t>(prm.sb_slot);
-    int dx = 8, dc = 2;
+    int dx = 7, dc = 2;
     auto bytes = [&]() {
         return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kCStage) * dc + sb_ring +
-               kMaxPairs * 8 * 4 +
+               kXoffBytes +
                static_cast<size_t>(2 * (dx + dc + kDA) + 8) * 8 + 16;
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
@@ -561,7 +574,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.a_off = 0;  // A stages live in TMEM
     prm.sb_off = prm.c_off + kCStage * dc;
     prm.row_off = prm.sb_off + static_cast<uint32_t>(sb_ring);
-    prm.bar_off = prm.row_off + kMaxPairs * 8 * 4;
+    prm.bar_off = prm.row_off + kXoffBytes;
     const size_t smem = bytes() + 1024;
     const int units = static_cast<int>(E) * prm.wunits;
     const int grid = units < num_sms ? units : num_sms;
