@@ -171,7 +171,9 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     if (e != cudaSuccess) return from_cuda(e);
     if (N == 0) return NV_OK;
     // Tensor-core route: each expert's weights are read once for all its rows.
-    if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size))
+    // (the tensor-core kernel keeps 32-bit element offsets into x)
+    if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size) &&
+        x_rows * K < (int64_t(1) << 32))
         return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
                                                codes, scales, biases, group_size, bits, y, s, sms));
     // Matrix-vector route (row_exact): every pair's output is bitwise equal to
@@ -193,6 +195,7 @@ nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     if (R > (int64_t(1) << 31) - 1) return NV_ERR_INVALID_ARG;
     if (E > nvq::kMaxExperts) return NV_ERR_UNSUPPORTED;
     if (dt != NV_BF16 || !nvq::tc_gather_mm_supported(K, N > 0 ? N : 1)) return NV_ERR_UNSUPPORTED;
+    if (x_rows * K >= (int64_t(1) << 32)) return NV_ERR_UNSUPPORTED;  // 32-bit offsets into x
     if (!workspace || !aligned16(workspace)) return NV_ERR_WORKSPACE;
     if (workspace_bytes < nvq::gather_workspace_bytes(R, E)) return NV_ERR_WORKSPACE;
     if (R == 0) return NV_OK;

@@ -180,7 +180,8 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
  * w        bf16 [E, N, K]: expert e's weights, row n = output feature n.
  * y[r, n] = sum_k x[lhs[r], k] * w[rhs[r], n, k], fp32 accumulation, stored
  *   in bf16; pairs with an out-of-range id get zero rows and a flag.
- * dt must be NV_BF16 and K a multiple of 64 (NV_ERR_UNSUPPORTED otherwise).
+ * dt must be NV_BF16, K a multiple of 64 and x_rows * K below 2^32
+ * (NV_ERR_UNSUPPORTED otherwise).
  */
 nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
                        const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R, int64_t E,

@@ -151,6 +151,7 @@ def test_gather_mm_argument_errors():
     assert call(w=24) == B.NV_ERR_INVALID_ARG        # misaligned
     assert call(lhs=4) == B.NV_ERR_INVALID_ARG
     assert call(R=0, ws_bytes=L.nv_gather_qmm_workspace_size(0, E)) == B.NV_OK
+    assert call(x_rows=1 << 21) == B.NV_ERR_UNSUPPORTED  # x_rows * K = 2^32 elements
 
 
 def test_flags_argument_errors():
