@@ -65,6 +65,9 @@ def _bind(lib):
     lib.orc_gather_qmm_sampled.restype = _i
     lib.orc_gather_mm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _i, _p, _p]
     lib.orc_gather_mm.restype = _i
+    lib.orc_moe_swiglu.argtypes = [_p, _i, _i64, _i64, _p, _p, _i, _i64, _i64,
+                                   _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p]
+    lib.orc_moe_swiglu.restype = _i
     return lib
 
 
@@ -239,6 +242,33 @@ def gather_mm(x, w, lhs, rhs, lib=None):
                            None if lhs_t is None else lhs_t.data_ptr(), rhs_t.data_ptr(), R, E, N,
                            w.data_ptr(), _DT[w.dtype], y.data_ptr(), a.data_ptr())
     _check(rc, "gather_mm")
+    return y, a
+
+
+def moe_swiglu(x, gate, up, down, ids, rw, group_size, bits, lib=None):
+    """fp64 (y, a) [T, K]: each token's top-k experts, weighted by rw, of the
+    SwiGLU block down(silu(x . gate^T) * (x . up^T)). gate and up are quantized
+    (codes, scales, biases) of [E, I, K] weights, down of [E, K, I]; ids and rw
+    are [T, topk]."""
+    lib = lib or load()
+    x = _cpu(x).contiguous()
+    T, K = x.shape
+    (gc, gsc, gb), (uc, usc, ub), (dc, dsc, db) = [tuple(_cpu(t).contiguous() for t in q)
+                                                    for q in (gate, up, down)]
+    E, I = gc.shape[0], gc.shape[1]
+    if tuple(dc.shape[:2]) != (E, K) or tuple(uc.shape) != tuple(gc.shape):
+        raise ValueError("oracle: gate/up [E, I, K] and down [E, K, I] do not agree")
+    ids_t = _u32(ids).reshape(T, -1).contiguous()
+    rw_t = _cpu(torch.as_tensor(rw, dtype=torch.float32)).reshape(T, -1).contiguous()
+    topk = ids_t.shape[1]
+    y = torch.empty(T, K, dtype=torch.float64)
+    a = torch.empty(T, K, dtype=torch.float64)
+    rc = lib.orc_moe_swiglu(x.data_ptr(), _DT[x.dtype], T, K, ids_t.data_ptr(), rw_t.data_ptr(),
+                            topk, E, I, gc.data_ptr(), gsc.data_ptr(), gb.data_ptr(), uc.data_ptr(),
+                            usc.data_ptr(), ub.data_ptr(), dc.data_ptr(), dsc.data_ptr(),
+                            db.data_ptr(), _DT[gsc.dtype], group_size, bits, y.data_ptr(),
+                            a.data_ptr())
+    _check(rc, "moe_swiglu")
     return y, a
 
 

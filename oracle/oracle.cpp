@@ -344,4 +344,69 @@ int orc_gather_mm(const void* x, int xdtype, int64_t x_rows, int64_t K, const ui
     return 0;
 }
 
+// Mixture-of-experts block with a SwiGLU expert [Q-MoE; the routed pass of
+// gate, up and down products], every product through quantized weights:
+//   for token t and each of its top-k (expert e = ids[t, j], weight rw[t, j]):
+//     g_i = sum_k x[t, k] * wg_hat[e, i, k],  u_i = sum_k x[t, k] * wu_hat[e, i, k]
+//     h_i = silu(g_i) * u_i,  silu(z) = z / (1 + exp(-z))
+//     y[t, n] += rw[t, j] * sum_i h_i * wd_hat[e, n, i]
+// Gate and up weights are [E, I, K] grouped along K, down weights [E, K, I]
+// grouped along I; all share one group size, width and scale dtype. fp64
+// throughout, sums in index order; a[t, n] = sum_j |rw| sum_i |h_i * wd_hat|.
+// Returns -1 on an out-of-range expert id or a bad quantization.
+int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32_t* ids,
+                   const float* rw, int topk, int64_t E, int64_t I,
+                   const uint32_t* g_codes, const void* g_scales, const void* g_biases,
+                   const uint32_t* u_codes, const void* u_scales, const void* u_biases,
+                   const uint32_t* d_codes, const void* d_scales, const void* d_biases,
+                   int sdtype, int gs, int bits, double* y, double* a) {
+    if (!valid_quant(K, gs, bits) || !valid_quant(I, gs, bits) || topk < 1) return -1;
+    for (int64_t i = 0; i < T * topk; ++i)
+        if ((int64_t)ids[i] >= E) return -1;
+    const size_t sz = sdtype == DT_F32 ? 4 : 2;
+    const int64_t gu_words = I * K * bits / 32, gu_groups = I * K / gs;   // per expert
+    const int64_t d_words = K * I * bits / 32, d_groups = K * I / gs;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double* yt = y + t * K;
+        double* at = a + t * K;
+        for (int64_t n = 0; n < K; ++n) { yt[n] = 0.0; at[n] = 0.0; }
+        double* h = new double[I];
+        for (int j = 0; j < topk; ++j) {
+            const int64_t e = (int64_t)ids[t * topk + j];
+            const double w = (double)rw[t * topk + j];
+            const uint32_t* gc = g_codes + e * gu_words;
+            const uint32_t* uc = u_codes + e * gu_words;
+            const char* gsc = (const char*)g_scales + (size_t)(e * gu_groups) * sz;
+            const char* gbi = (const char*)g_biases + (size_t)(e * gu_groups) * sz;
+            const char* usc = (const char*)u_scales + (size_t)(e * gu_groups) * sz;
+            const char* ubi = (const char*)u_biases + (size_t)(e * gu_groups) * sz;
+            for (int64_t i = 0; i < I; ++i) {
+                double g = 0.0, u = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    const double xv = load_value(x, xdtype, t * K + k);
+                    g += xv * dequant_at(gc, gsc, gbi, sdtype, i, k, K, gs, bits);
+                    u += xv * dequant_at(uc, usc, ubi, sdtype, i, k, K, gs, bits);
+                }
+                h[i] = g / (1.0 + std::exp(-g)) * u;
+            }
+            const uint32_t* dc = d_codes + e * d_words;
+            const char* dsc = (const char*)d_scales + (size_t)(e * d_groups) * sz;
+            const char* dbi = (const char*)d_biases + (size_t)(e * d_groups) * sz;
+            for (int64_t n = 0; n < K; ++n) {
+                double acc = 0.0, mag = 0.0;
+                for (int64_t i = 0; i < I; ++i) {
+                    const double p = h[i] * dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits);
+                    acc += p;
+                    mag += std::fabs(p);
+                }
+                yt[n] += w * acc;
+                at[n] += std::fabs(w) * mag;
+            }
+        }
+        delete[] h;
+    }
+    return 0;
+}
+
 }  // extern "C"

@@ -412,6 +412,65 @@ def pin_gather_mm(lib):
         raise AssertionError("expert id 5 of 5 experts accepted")
 
 
+def _pack_codes(codes: torch.Tensor, bits: int) -> torch.Tensor:
+    """Pack integer codes [..., cols] into int32 words, code j at bits [j*bits, (j+1)*bits)."""
+    per = 32 // bits
+    c = codes.to(torch.int64).reshape(*codes.shape[:-1], -1, per)
+    word = (c << (torch.arange(per, dtype=torch.int64) * bits)).sum(-1)
+    return torch.where(word >= 2 ** 31, word - 2 ** 32, word).to(torch.int32)
+
+
+def pin_moe_swiglu(lib):
+    """The MoE SwiGLU block against closed forms, with integer data (scale
+    +-1, bias 0): silu(z) - silu(-z) = z and silu(z) + silu(-z) = z tanh(z/2),
+    so y(G) - y(-G) is the exact integer routed sum of (x G^T) * (x U^T) times
+    D^T (int64 brute force) and y(G) + y(-G) the same with g tanh(g/2) for g;
+    a zero gate gives zero; doubling the routing weights doubles y; the top-k
+    order does not matter; an out-of-range expert id is refused."""
+    g = torch.Generator().manual_seed(53)
+    E, I, K, T, top, gs, bits = 3, 64, 64, 5, 2, 32, 4
+    Gc = torch.randint(0, 4, (E, I, K), generator=g)
+    Uc = torch.randint(0, 4, (E, I, K), generator=g)
+    Dc = torch.randint(0, 16, (E, K, I), generator=g)
+    x = torch.randint(-2, 3, (T, K), generator=g).to(torch.bfloat16)
+    ids = torch.stack([torch.randperm(E, generator=g)[:top] for _ in range(T)])
+    rw = torch.randint(-2, 3, (T, top), generator=g).to(torch.float32)
+    one = lambda shape, v: torch.full(shape, float(v), dtype=torch.bfloat16)  # noqa: E731
+    q = lambda c, sign: (_pack_codes(c, bits), one((*c.shape[:-1], c.shape[-1] // gs), sign),  # noqa: E731
+                         one((*c.shape[:-1], c.shape[-1] // gs), 0))
+    G, Gn, U, D = q(Gc, 1), q(Gc, -1), q(Uc, 1), q(Dc, 1)
+    yp, a = O.moe_swiglu(x, G, U, D, ids, rw, gs, bits, lib=lib)
+    ym, _ = O.moe_swiglu(x, Gn, U, D, ids, rw, gs, bits, lib=lib)
+    xi = x.to(torch.int64)
+    odd = torch.zeros(T, K, dtype=torch.int64)
+    even = torch.zeros(T, K, dtype=torch.float64)
+    for t in range(T):
+        for j in range(top):
+            e, w = int(ids[t, j]), int(rw[t, j])
+            gv = Gc[e] @ xi[t]                      # [I], exact
+            uv = Uc[e] @ xi[t]
+            odd[t] += w * (Dc[e] @ (gv * uv))
+            gf = gv.to(torch.float64)
+            th = torch.tensor([math.tanh(v / 2) for v in gf.tolist()], dtype=torch.float64)
+            even[t] += w * (Dc[e].to(torch.float64) @ (gf * th * uv.to(torch.float64)))
+    tol = 1e-12 * (a + 1)
+    assert ((yp - ym) - odd.to(torch.float64)).abs().le(tol).all(), "odd part"
+    assert ((yp + ym) - even).abs().le(tol).all(), "even part"
+    Z = q(torch.zeros_like(Gc), 1)
+    y0, _ = O.moe_swiglu(x, Z, U, D, ids, rw, gs, bits, lib=lib)
+    assert (y0 == 0).all(), "zero gate"
+    y2, _ = O.moe_swiglu(x, G, U, D, ids, 2 * rw, gs, bits, lib=lib)
+    assert torch.equal(y2, 2 * yp), "routing weights scale the output"
+    ys, _ = O.moe_swiglu(x, G, U, D, ids.flip(1), rw.flip(1), gs, bits, lib=lib)
+    assert (ys - yp).abs().le(tol).all(), "top-k order"
+    try:
+        O.moe_swiglu(x, G, U, D, torch.full((T, top), E), rw, gs, bits, lib=lib)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("expert id E accepted")
+
+
 def pin_sampled_match_full(lib):
     """The sampled product entry points agree with the full ones."""
     g = torch.Generator().manual_seed(31)

@@ -53,6 +53,12 @@ MUTANTS = [
      "const int64_t t = r % x_rows;"),
     ("gather_mm transposed expert", "load_value(w, wdtype, wrow + k)",
      "load_value(w, wdtype, (int64_t)rhs[r] * N * K + k * N + n)"),
+    ("silu sign", "h[i] = g / (1.0 + std::exp(-g)) * u;", "h[i] = g / (1.0 + std::exp(g)) * u;"),
+    ("gate and up swapped", "h[i] = g / (1.0 + std::exp(-g)) * u;",
+     "h[i] = u / (1.0 + std::exp(-u)) * g;"),
+    ("routing weight dropped", "yt[n] += w * acc;", "yt[n] += acc;"),
+    ("down transposed", "dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits)",
+     "dequant_at(dc, dsc, dbi, sdtype, i, n, K, gs, bits)"),
 ]
 
 RUNNER = r"""
