@@ -52,6 +52,8 @@ def _bind(lib):
     lib.orc_quantize_affine.restype = _i
     lib.orc_dequantize.argtypes = [_p, _p, _p, _i, _i64, _i64, _i, _i, _p]
     lib.orc_dequantize.restype = _i
+    lib.orc_dequantize_stored.argtypes = [_p, _p, _p, _i, _i64, _i64, _i, _i, _p]
+    lib.orc_dequantize_stored.restype = _i
     lib.orc_qmm.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i, _p, _p]
     lib.orc_qmm.restype = _i
     lib.orc_qmm_sampled.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i,
@@ -131,18 +133,24 @@ def dequantize(codes, scales, biases, group_size: int, bits: int, lib=None) -> t
 
 def dequantize_stored(codes, scales, biases, group_size: int, bits: int, lib=None) -> torch.Tensor:
     """The dequantized weights as stored in the scales' dtype ("Docs /
-    Quantization", section "Affine": w ~= scale * code + bias).
+    Quantization", section "Affine": w ~= scale * code + bias; the nuvec crate
+    docs, Quantized: scales in the weights' dtype).
 
-    Reading (the pages fix no precision for this step): scale * code + bias is
-    evaluated exactly and rounded once to fp32 (one fused multiply-add), then
-    stored in the dtype (bf16: round to nearest, ties to even). The exact value
-    is the fp64 result of ``dequantize``: scale * code has at most 32
-    significant bits, so the sum with the bias is exact in fp64 whenever the
-    two are within ~20 binades of each other (true of every quantized group,
-    whose codes span the bias's range); torch's fp64 -> fp32 and fp32 -> bf16
-    conversions round to nearest even."""
-    wh = dequantize(codes, scales, biases, group_size, bits, lib=lib)
-    return wh.to(torch.float32).to(_cpu(scales).dtype)
+    Reading (the pages fix no precision for this step): the exact value
+    scale * code + bias rounded once, to nearest with ties to even, to the
+    dtype. oracle.cpp computes that single rounding exactly (two-sum, then a
+    rounding to odd at fp64 precision, then the dtype's rounding)."""
+    lib = lib or load()
+    codes, scales, biases = _cpu(codes), _cpu(scales), _cpu(biases)
+    cols = codes.shape[-1] * 32 // bits
+    rows = codes.numel() // codes.shape[-1]
+    dt = scales.dtype
+    out = torch.empty(*codes.shape[:-1], cols, dtype=torch.float32 if dt == torch.float32
+                      else torch.int16)
+    rc = lib.orc_dequantize_stored(codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                                   _DT[dt], rows, cols, group_size, bits, out.data_ptr())
+    _check(rc, "dequantize_stored")
+    return out if dt == torch.float32 else out.view(torch.bfloat16)
 
 
 def qmm(x, codes, scales, biases, group_size: int, bits: int, transpose: bool = True, lib=None):

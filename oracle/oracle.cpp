@@ -106,6 +106,57 @@ double dequant_at(const uint32_t* codes, const void* scales, const void* biases,
     return s * (double)code_at(codes, row, col, cols, bits) + b;
 }
 
+// ---- the stored dequantized value [Q-Affine, Crate-Quantized] --------------
+// The dequantized weight, as the dequantizer stores it, is the exact value
+// scale * code + bias rounded once (to nearest, ties to even) to the scales'
+// dtype. Steps:
+//   1. p = scale * code is exact in fp64 (at most 24 + 8 significant bits);
+//   2. p + bias = sum + err exactly (the two-sum of Knuth), sum rounded;
+//   3. the round-to-odd value of the exact sum at fp64 precision: sum itself
+//      when err == 0, else whichever of sum and its neighbour towards err has
+//      an odd last bit;
+//   4. that value rounded to nearest even at the dtype's precision. A
+//      rounding to odd at 53 bits followed by a rounding to at most 51 bits
+//      equals a single rounding of the exact value (the odd bit records that
+//      the exact value lies strictly between the two 53-bit neighbours).
+double round_to_odd_sum(double p, double b) {
+    const double sum = p + b;
+    const double bb = sum - p;
+    const double err = (p - (sum - bb)) + (b - bb);
+    if (err == 0.0 || !std::isfinite(sum)) return sum;
+    uint64_t u;
+    std::memcpy(&u, &sum, 8);
+    if (u & 1u) return sum;
+    return std::nextafter(sum, err > 0.0 ? INFINITY : -INFINITY);
+}
+
+// fp64 -> bf16 bit pattern, round to nearest even at 8 significant bits
+// (quantum 2^-133 below the smallest normal 2^-126), infinity past the largest
+// finite value. Written from the format: 1 sign, 8 exponent, 7 fraction bits.
+uint16_t f64_to_bf16(double d) {
+    const uint16_t sign = std::signbit(d) ? 0x8000u : 0u;
+    const double a = std::fabs(d);
+    if (a == 0.0) return sign;
+    if (!std::isfinite(a)) return (uint16_t)(sign | 0x7F80u);
+    int e = 0;
+    std::frexp(a, &e);                  // a = m * 2^e, m in [0.5, 1)
+    int q = e - 8;                      // exponent of the last kept bit
+    if (q < -133) q = -133;
+    const double r = std::ldexp(std::nearbyint(std::ldexp(a, -q)), q);  // ties to even
+    if (r >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    const float f = (float)r;           // exact: r has at most 8 significant bits
+    uint32_t bits;
+    std::memcpy(&bits, &f, 4);
+    return (uint16_t)(sign | (bits >> 16));
+}
+
+// fp64 -> fp32, round to nearest even (the conversion of the default mode),
+// infinity past the largest finite value.
+float f64_to_f32(double d) {
+    if (std::isfinite(d) && std::fabs(d) >= 0x1p128) return std::signbit(d) ? -INFINITY : INFINITY;
+    return (float)d;
+}
+
 bool valid_quant(int64_t cols, int gs, int bits) {
     if (gs != 32 && gs != 64 && gs != 128) return false;
     if (bits != 1 && bits != 2 && bits != 4 && bits != 8) return false;
@@ -223,6 +274,24 @@ int orc_dequantize(const uint32_t* codes, const void* scales, const void* biases
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t c = 0; c < cols; ++c)
             out[r * cols + c] = dequant_at(codes, scales, biases, sdtype, r, c, cols, gs, bits);
+    return 0;
+}
+
+// The dequantized weights as stored: out[r, c] = scale * code + bias rounded
+// once to the scales' dtype (see round_to_odd_sum) [Q-Affine, Crate-Quantized].
+int orc_dequantize_stored(const uint32_t* codes, const void* scales, const void* biases,
+                          int sdtype, int64_t rows, int64_t cols, int gs, int bits, void* out) {
+    if (!valid_quant(cols, gs, bits)) return -1;
+    if (std::fegetround() != FE_TONEAREST) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            const int64_t g = r * (cols / gs) + c / gs;
+            const double p = load_value(scales, sdtype, g) * (double)code_at(codes, r, c, cols, bits);
+            const double v = round_to_odd_sum(p, load_value(biases, sdtype, g));
+            if (sdtype == DT_F32) ((float*)out)[r * cols + c] = f64_to_f32(v);
+            else ((uint16_t*)out)[r * cols + c] = f64_to_bf16(v);
+        }
     return 0;
 }
 

@@ -127,15 +127,30 @@ def pin_handbuilt_groups(lib):
 
 
 def pin_dequantize_stored_rounding(lib):
-    """The stored dequantized value is scale * code + bias rounded once to fp32,
-    then to the dtype with ties to even (the reading the dequantizer follows):
+    """The stored dequantized value is the exact scale * code + bias rounded
+    once, to nearest with ties to even, to the dtype (the reading the
+    dequantizer follows):
     * bf16, scale 2^-9, bias 1: codes 1, 2, 3 give 1 + 2^-9 (below half a bf16
       step: 1), 1 + 2^-8 (exactly half: the even neighbour 1), 1 + 3 * 2^-9
       (above half: 1 + 2^-7);
+    * bf16, scale 37, code 7: 37 * 7 = 259 lies exactly halfway between the
+      bf16 neighbours 258 and 260. With bias -2^-20 the exact value
+      259 - 2^-20 is below the halfway point, so one rounding gives 258; an
+      fp32 step first (fp32 spacing 2^-15 there) would land on 259 and the tie
+      would go to the even 260. With bias -2^-60 even an fp64 step lands on 259
+      (fp64 spacing 2^-44): the single rounding still gives 258;
     * fp32, scale 1 + 2^-23, bias -3, code 3: the exact value 3 * 2^-23 is an
       fp32 number, so one rounding keeps it (a product rounded first would give
       3 + 2^-21 and then 2^-21);
     * scale 1 and bias 0 return the codes, in both dtypes."""
+    w7 = torch.tensor([[7]], dtype=torch.int32).repeat(1, 8)  # 8-bit codes 7, 0, 0, 0
+    s37 = torch.tensor([[37.0]], dtype=torch.bfloat16)
+    for b_exp in (-20, -60):
+        bb = torch.tensor([[-(2.0 ** b_exp)]], dtype=torch.bfloat16)
+        assert float(bb[0, 0]) == -(2.0 ** b_exp)
+        got = O.dequantize_stored(w7, s37, bb, 32, 8, lib=lib)
+        assert float(got[0, 0]) == 258.0, (b_exp, got[0, 0])
+        assert float(got[0, 1]) == -(2.0 ** b_exp), got[0, 1]
     words = torch.tensor([[1 | (2 << 8) | (3 << 16)]], dtype=torch.int32)  # 8-bit codes 1, 2, 3, 0
     s = torch.tensor([[2.0 ** -9]], dtype=torch.bfloat16)
     b = torch.tensor([[1.0]], dtype=torch.bfloat16)

@@ -57,6 +57,11 @@ MUTANTS = [
     ("gate and up swapped", "h[i] = g / (1.0 + std::exp(-g)) * u;",
      "h[i] = u / (1.0 + std::exp(-u)) * g;"),
     ("routing weight dropped", "yt[n] += w * acc;", "yt[n] += acc;"),
+    ("stored value rounded through fp32",
+     "const double v = round_to_odd_sum(p, load_value(biases, sdtype, g));",
+     "const double v = (double)(float)(p + load_value(biases, sdtype, g));"),
+    ("stored value rounded through fp64", "if (err == 0.0 || !std::isfinite(sum)) return sum;",
+     "return sum;"),
     ("down transposed", "dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits)",
      "dequant_at(dc, dsc, dbi, sdtype, i, n, K, gs, bits)"),
 ]
