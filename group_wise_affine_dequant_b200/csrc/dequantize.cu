@@ -11,10 +11,11 @@
 // step, lane l the words 32 q + l (q < 4), so that every load and store
 // instruction of the warp covers one contiguous run; it writes each word's
 // values with 8- to 16-byte stores and strides over the array. Every value is
-// one fused multiply-add in fp32, scale * code + bias rounded once, then
-// stored in the output dtype (bf16 by round-to-nearest-even). HBM-bound:
-// bytes moved per weight are bits / 8 (codes) + 4 / group_size or
-// 8 / group_size (scale and bias) + the output element size.
+// the exact scale * code + bias rounded once to the output dtype: one fp32
+// fused multiply-add for fp32 outputs, one bf16 fused multiply-add (on codes
+// held exactly as bf16, every integer below 256 being a bf16 number) for bf16
+// outputs. HBM-bound: bytes moved per weight are bits / 8 (codes) +
+// 4 / group_size or 8 / group_size (scale and bias) + the output element size.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -27,20 +28,43 @@ __device__ __forceinline__ float code_f32(uint32_t c) {
     return __uint_as_float(0x4B000000u | c) - 8388608.0f;
 }
 
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // Values of one word, stored at out (16-byte aligned for bf16 at 4 bits and
-// wider outputs, 8-byte for 8-bit codes to bf16).
+// wider outputs, 8-byte for 8-bit codes to bf16). s2, b2: (s, s) and (b, b)
+// as bf16 pairs (bf16 outputs only).
 template <int DT, int BITS>
-__device__ __forceinline__ void word_out(uint32_t w, float s, float b, void* out) {
+__device__ __forceinline__ void word_out(uint32_t w, float s, float b, uint32_t s2, uint32_t b2,
+                                         void* out) {
     constexpr int PER = 32 / BITS;
     constexpr uint32_t MASK = (1u << BITS) - 1u;
     if constexpr (DT == NV_BF16) {
         uint32_t v[PER / 2];
 #pragma unroll
         for (int j = 0; j < PER / 2; ++j) {
-            const float lo = fmaf(s, code_f32((w >> (2 * j * BITS)) & MASK), b);
-            const float hi = fmaf(s, code_f32((w >> ((2 * j + 1) * BITS)) & MASK), b);
-            v[j] = static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
-                   (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+            const uint32_t lo = (w >> (2 * j * BITS)) & MASK;
+            const uint32_t hi = (w >> ((2 * j + 1) * BITS)) & MASK;
+            uint32_t c2;  // (lo, hi) as exact bf16
+            if constexpr (BITS == 8) {
+                c2 = f2_to_bf2(code_f32(lo), code_f32(hi));
+            } else {  // 128 + c for c < 128 (bf16's unit at 128 is 1), minus 128
+                c2 = bf2_sub(lo | (hi << 16) | 0x43004300u, 0x43004300u);
+            }
+            v[j] = bf2_fma(s2, c2, b2);
         }
         if constexpr (PER / 2 >= 4) {
             uint4* o = reinterpret_cast<uint4*>(out);
@@ -86,8 +110,10 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restr
             const int64_t i = base + 32 * q + lane;
             if (i < words) {
                 const int64_t g = (i * PER) >> lg_gs;
-                word_out<DT, BITS>(w[q], load_elem<DT>(scales, g), load_elem<DT>(biases, g),
-                                   o + i * PER * ESZ);
+                const float s = load_elem<DT>(scales, g), b = load_elem<DT>(biases, g);
+                const uint32_t s2 = (__float_as_uint(s) >> 16) * 0x00010001u;
+                const uint32_t b2 = (__float_as_uint(b) >> 16) * 0x00010001u;
+                word_out<DT, BITS>(w[q], s, b, s2, b2, o + i * PER * ESZ);
             }
         }
     }

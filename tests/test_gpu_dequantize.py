@@ -47,7 +47,7 @@ def test_dequantize_bit_exact(bits, gs, dt):
 
 def test_dequantize_rounding_cases():
     """The oracle's rounding pins, run on the GPU: ties to even in the bf16
-    store, one rounding of scale * code + bias in fp32."""
+    store, one rounding of the exact scale * code + bias."""
     words = torch.tensor([[1 | (2 << 8) | (3 << 16)]], dtype=torch.int32).repeat(1, 8)
     s, b = torch.tensor([[2.0 ** -9]], dtype=BF16), torch.tensor([[1.0]], dtype=BF16)
     got = _gpu_dequantize(words, s, b, 32, 8)
@@ -57,6 +57,18 @@ def test_dequantize_rounding_cases():
     s32, b32 = torch.tensor([[1.0 + 2.0 ** -23]]), torch.tensor([[-3.0]])
     got = _gpu_dequantize(w3, s32, b32, 32, 8)
     assert (got == 3 * 2.0 ** -23).all(), got
+    # 37 * 7 = 259 is a bf16 tie; the exact 259 - 2^-20 (or - 2^-60) rounds once to 258
+    w7 = torch.tensor([[7 | (7 << 8) | (7 << 16) | (7 << 24)]], dtype=torch.int32).repeat(1, 8)
+    for e in (-20, -60):
+        s37, bb = torch.tensor([[37.0]], dtype=BF16), torch.tensor([[-(2.0 ** e)]], dtype=BF16)
+        got = _gpu_dequantize(w7, s37, bb, 32, 8)
+        assert (got.float() == 258.0).all(), (e, got)
+        assert torch.equal(_bits_of(got), _bits_of(O.dequantize_stored(w7, s37, bb, 32, 8)))
+    # the same tie through 4-bit codes (exact bf16 codes by the 128 + c form)
+    w4 = torch.full((1, 4), 0x77777777, dtype=torch.int32)
+    s37, bb = torch.tensor([[37.0]], dtype=BF16), torch.tensor([[-(2.0 ** -20)]], dtype=BF16)
+    got = _gpu_dequantize(w4, s37, bb, 32, 4)
+    assert (got.float() == 258.0).all(), got
 
 
 def test_dequantize_stack_of_matrices():
