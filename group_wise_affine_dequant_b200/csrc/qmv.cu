@@ -9,26 +9,30 @@
 //    swizzle so the fragment reads below hit distinct banks) plus the slice's
 //    scales and biases into its own ring of shared-memory stages, completing
 //    on a per-warp mbarrier, several tiles ahead of the math.
-//  * Codes become fp16 exactly with one mask each: OR-ing a code field into the
-//    mantissa of 1024.0 gives 1024 + c * 2^p for a field p bits above the
-//    mantissa's base (fp16 has 10 mantissa bits, so a 4-bit word needs one
-//    shift and four masks, an 8-bit word one shift and two masks).
-//  * The multiply-adds run on the tensor cores (mma.sync m16n8k16, fp16 in,
+//  * Codes become bf16 exactly with one mask each: OR-ing a field worth
+//    c * 2^p <= 127 into the mantissa of 128.0 gives 128 + c * 2^p (bf16 holds
+//    every integer below 256). A 4-bit word takes three shifts and four masks;
+//    an 8-bit code is split into its two nibbles (c = lo + 16 hi), which are
+//    unpacked like two 4-bit codes; a 2-bit word takes two shifts and eight
+//    masks.
+//  * The multiply-adds run on the tensor cores (mma.sync m16n8k16, bf16 in,
 //    fp32 accumulate): A = 16 weight rows x 16 k of codes, B = the activations
 //    (one column per activation row, up to 8). Which physical k feeds which MMA
 //    k-slot is chosen so that each thread's loaded words feed its own A
 //    fragments; the activations are permuted the same way once, in registers,
-//    and the activation of a slot holding c * 2^p is divided by 2^p.
-//  * Activations enter as fp16 after an exact power-of-two scaling 2^-e per
-//    slice and activation row (largest magnitude brought to [1, 2): no
-//    overflow, and every value within 2^-10 of that maximum converts exactly
-//    even after the division by a slot's code scale); the slice's partial
-//    sums are multiplied back by 2^e. Small integer activations stay exact
-//    through the fp32 sums.
-//  * Scale and bias are applied per group outside the MMA, with the 1024s
-//    removed by an MMA over the same rounded activations:
-//        sum_k x_k w_k = s * (D - 1024-sum) + b * sum_k x_k,
-//    so every product x * code is exact and only the group sums round.
+//    and the activation of a slot holding c * 2^p is multiplied by 2^-p (by 2
+//    for the high nibble of an 8-bit code held as 8 hi).
+//  * Activations enter the MMA as bf16, the type they arrive in: bf16 has the
+//    exponent range of fp32, so no value is rounded or flushed on the way in.
+//    Only a slice whose largest magnitude reaches 2^100 is first multiplied by
+//    2^-(e - 100) (e its exponent), which keeps every fp32 sum finite, and its
+//    partial sums are multiplied back by 2^(e - 100); both steps are exact.
+//    Every product x * code is therefore exact for every finite bf16 input
+//    (down to the bf16 subnormals), and only fp32 sums round.
+//  * Scale and bias are applied per group outside the MMA, with the 128s
+//    removed by an MMA over the same activations:
+//        sum_k x_k w_k = s * (D - 128-sum) + b * sum_k x_k,
+//    so only the group sums round.
 //  * A warp owns a k-slice of 16 MMA k-steps (256 k at 2/4 bits, 128 at 8) and
 //    keeps its activations in registers while it walks the rows of its CTA.
 //    Each CTA owns a contiguous range of rows (N split evenly over the SMs) and
@@ -52,12 +56,12 @@ namespace {
 constexpr int kSteps = 16;
 constexpr int kMaxWarps = 16;
 
-template <int BITS, int GS, int STEPS = (BITS == 8 ? kSteps / 2 : kSteps)>
+template <int BITS, int GS, int STEPS = kSteps>
 struct Shape {
     static constexpr int PER = 32 / BITS;                // codes per word
     static constexpr int GW = GS * BITS / 32;            // words per group
     static constexpr int LW = GW / 4 < 4 ? GW / 4 : 4;   // words per thread per row per chunk
-    static constexpr int MPW = BITS == 2 ? 4 : BITS == 4 ? 2 : 1;  // MMAs per word
+    static constexpr int MPW = BITS == 2 ? 4 : 2;       // MMAs per word
     static constexpr int NP = 2 * MPW;                   // fp16x2 registers per unpacked word
     static constexpr int CW = 4 * LW;                    // words per chunk (one lane quad)
     static constexpr int CK = CW * PER;                  // k per chunk
@@ -70,83 +74,82 @@ struct Shape {
     static_assert(CK <= GS && GS % CK == 0, "a chunk lies inside one group");
 };
 
-// (v & mask) | 1024.0 in both fp16 halves: 1024 + the masked field.
-__device__ __forceinline__ uint32_t codes_to_f16x2(uint32_t v, uint32_t mask) {
-    uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(mask), "r"(0x64006400u));
-    return r;
-}
-
-// Word -> NP fp16x2 registers (1024 + c * 2^p); MMA u of the word uses p[2u]
-// (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). kScale[i] = 2^p of
-// register i (the activation of that slot pair is divided by it): scale(i).
+// Word -> NP bf16x2 registers of 128 + (code field); MMA u of the word uses
+// p[2u] (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). For register i:
+//   lo(i), hi(i)  the codes of the word behind its low and high halves;
+//   mul(i)        the factor of the activations in its slots (2^-p, or 2 for
+//                 the high nibble of an 8-bit code, held as 8 hi);
+//   sumw(i)       the A constant of the x-sum MMA: sum over slots of
+//                 sumw * mul * x counts every activation exactly once.
 template <int BITS>
 struct Unpack;
 
 template <>
-struct Unpack<4> {  // (c0,c4) (c1,c5)*16 (c2,c6) (c3,c7)*16
-    // 2^p of register i, and the code index of its low half (high = +4)
-    __host__ __device__ static constexpr float scale(int i) { return (i & 1) ? 16.f : 1.f; }
+struct Unpack<4> {  // (c0,c4) (c1,c5)*8 (c2,c6) (c3,c7)*8
     __host__ __device__ static constexpr int lo(int i) { return i; }
+    __host__ __device__ static constexpr int hi(int i) { return i + 4; }
+    __host__ __device__ static constexpr float mul(int i) { return (i & 1) ? 0.125f : 1.f; }
+    __host__ __device__ static constexpr float sumw(int i) { return (i & 1) ? 8.f : 1.f; }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
-        const uint32_t v = w >> 8;
-        p[0] = codes_to_f16x2(w, 0x000F000Fu);
-        p[1] = codes_to_f16x2(w, 0x00F000F0u);
-        p[2] = codes_to_f16x2(v, 0x000F000Fu);
-        p[3] = codes_to_f16x2(v, 0x00F000F0u);
+        p[0] = codes_to_bf16x2(w, 0x000F000Fu);
+        p[1] = codes_to_bf16x2(w >> 1, 0x00780078u);
+        p[2] = codes_to_bf16x2(w >> 8, 0x000F000Fu);
+        p[3] = codes_to_bf16x2(w >> 9, 0x00780078u);
     }
 };
 
 template <>
-struct Unpack<8> {  // (c0,c2) (c1,c3)
-    __host__ __device__ static constexpr float scale(int) { return 1.f; }
-    __host__ __device__ static constexpr int lo(int i) { return i; }  // high = +2
+struct Unpack<8> {  // nibbles: (c0 lo, c2 lo) (c0 hi, c2 hi)*8 (c1 lo, c3 lo) (c1 hi, c3 hi)*8
+    __host__ __device__ static constexpr int lo(int i) { return i >> 1; }
+    __host__ __device__ static constexpr int hi(int i) { return (i >> 1) + 2; }
+    __host__ __device__ static constexpr float mul(int i) { return (i & 1) ? 2.f : 1.f; }
+    __host__ __device__ static constexpr float sumw(int i) { return (i & 1) ? 0.f : 1.f; }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
-        p[0] = codes_to_f16x2(w, 0x00FF00FFu);
-        p[1] = codes_to_f16x2(w >> 8, 0x00FF00FFu);
+        Unpack<4>::run(w, p);  // the same fields: nibble j at bits 4j
     }
 };
 
 template <>
-struct Unpack<2> {  // (c_i, c_i+8) * 4^i for i < 5, then c5..c7 from w >> 10
-    __host__ __device__ static constexpr float scale(int i) {
-        return i < 5 ? static_cast<float>(1 << (2 * i)) : static_cast<float>(1 << (2 * (i - 5)));
+struct Unpack<2> {  // (c_i, c_i+8) * (1, 4, 16, 1, 4, 16, 1, 4)
+    __host__ __device__ static constexpr int lo(int i) { return i; }
+    __host__ __device__ static constexpr int hi(int i) { return i + 8; }
+    __host__ __device__ static constexpr float sumw(int i) {
+        return static_cast<float>(1 << (2 * (i % 3)));
     }
-    __host__ __device__ static constexpr int lo(int i) { return i; }  // high = +8
+    __host__ __device__ static constexpr float mul(int i) { return 1.f / sumw(i); }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
-        const uint32_t v = w >> 10;
-        p[0] = codes_to_f16x2(w, 0x00030003u);
-        p[1] = codes_to_f16x2(w, 0x000C000Cu);
-        p[2] = codes_to_f16x2(w, 0x00300030u);
-        p[3] = codes_to_f16x2(w, 0x00C000C0u);
-        p[4] = codes_to_f16x2(w, 0x03000300u);
-        p[5] = codes_to_f16x2(v, 0x00030003u);
-        p[6] = codes_to_f16x2(v, 0x000C000Cu);
-        p[7] = codes_to_f16x2(v, 0x00300030u);
+        const uint32_t v = w >> 6, u = w >> 12;
+        p[0] = codes_to_bf16x2(w, 0x00030003u);
+        p[1] = codes_to_bf16x2(w, 0x000C000Cu);
+        p[2] = codes_to_bf16x2(w, 0x00300030u);
+        p[3] = codes_to_bf16x2(v, 0x00030003u);
+        p[4] = codes_to_bf16x2(v, 0x000C000Cu);
+        p[5] = codes_to_bf16x2(v, 0x00300030u);
+        p[6] = codes_to_bf16x2(u, 0x00030003u);
+        p[7] = codes_to_bf16x2(u, 0x000C000Cu);
     }
 };
 
 __device__ __forceinline__ float bf16_elem(const uint32_t* xv, int i) {
     return __uint_as_float((i & 1) ? (xv[i >> 1] & 0xFFFF0000u) : (xv[i >> 1] << 16));
 }
-__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+__device__ __forceinline__ uint32_t f2_to_bf2x(float lo, float hi) {
     uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
-__device__ __forceinline__ uint32_t h2_const(float v) { return f2_to_h2(v, v); }
+__device__ __forceinline__ uint32_t bf2_const(float v) { return f2_to_bf2x(v, v); }
 
 // The activations matching Unpack: b[u][0..1] for MMA u of a word whose first k
-// is k0, from xv = x[k0 .. k0 + PER) as bf16 pairs, times f = 2^-e and divided
-// by the slot's code scale.
+// is k0, from xv = x[k0 .. k0 + PER) as bf16 pairs, times f (a power of two)
+// and the slot's factor: exact products of powers of two, exact in bf16.
 template <int BITS>
 __device__ __forceinline__ void x_fragments(const uint32_t* xv, float f, uint32_t (*b)[2]) {
     using U = Unpack<BITS>;
-    constexpr int HI = 32 / BITS / 2;  // code index distance between the halves
 #pragma unroll
-    for (int i = 0; i < 2 * (BITS == 2 ? 4 : BITS == 4 ? 2 : 1); ++i) {
-        const float m = f / U::scale(i);
-        b[i >> 1][i & 1] = f2_to_h2(bf16_elem(xv, U::lo(i)) * m, bf16_elem(xv, U::lo(i) + HI) * m);
+    for (int i = 0; i < 2 * (BITS == 2 ? 4 : 2); ++i) {
+        const float m = f * U::mul(i);
+        b[i >> 1][i & 1] = f2_to_bf2x(bf16_elem(xv, U::lo(i)) * m, bf16_elem(xv, U::hi(i)) * m);
     }
 }
 
@@ -179,6 +182,7 @@ struct QmvParams {
     const uint32_t* problems;      // [P][4] = (expert, start, count, 0)
     const uint32_t* num_problems;
     int64_t E;
+    uint32_t problem0;       // problem of blockIdx.y = 0 (launches of <= 65535 problems)
 };
 
 
@@ -265,7 +269,7 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     pdl_launch_dependents();
     if constexpr (GATHER) {
         pdl_wait();  // the routing tables come from the previous kernel
-        const uint32_t p = blockIdx.y;
+        const uint32_t p = prm.problem0 + blockIdx.y;
         if (p >= __ldg(prm.num_problems)) return;
         const uint32_t e = __ldg(prm.problems + 4 * p);
         const uint32_t start = __ldg(prm.problems + 4 * p + 1);
@@ -457,20 +461,21 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                 }
             }
         }
-        // per activation row (lane quad g): 2^-e brings max |x| to [1, 2)
+        // per activation row (lane quad g): a slice whose largest |x| reaches
+        // 2^100 is brought below 2^101 by 2^-es (exact); the rest keep es = 0
         xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 1));
         xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 2));
-        int e = 0;
-        if (xmax > 0.f) e = min(max(static_cast<int>((__float_as_uint(xmax) >> 23) & 0xFF) - 127, -100), 100);
-        const float f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
-        // 2^e of the activation rows of this lane's D columns 2t and 2t + 1
-        const int e0 = __shfl_sync(0xffffffffu, e, 8 * t), e1 = __shfl_sync(0xffffffffu, e, 8 * t + 4);
+        const int ex = static_cast<int>((__float_as_uint(xmax) >> 23) & 0xFF) - 127;
+        const int es = ex > 100 ? ex - 100 : 0;  // 0 .. 28
+        const float f = __uint_as_float(static_cast<uint32_t>(127 - es) << 23);  // 2^-es
+        // 2^es of the activation rows of this lane's D columns 2t and 2t + 1
+        const int e0 = __shfl_sync(0xffffffffu, es, 8 * t), e1 = __shfl_sync(0xffffffffu, es, 8 * t + 4);
         const float ef0 = __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
         const float ef1 = __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
 
         uint32_t bfr[S::KS][S::MMAS][2];
-        float xoff[S::KS][2], xsum[S::KS][2];  // per chunk and column: 1024-sum, sum of x
-        const uint32_t k1024 = 0x64006400u;      // fp16x2 (1024, 1024)
+        float xoff[S::KS][2], xsum[S::KS][2];  // per chunk and column: 128-sum, sum of x
+        const uint32_t k128 = 0x43004300u;       // bf16x2 (128, 128)
 #pragma unroll
         for (int q = 0; q < S::KS; ++q) {
 #pragma unroll
@@ -481,10 +486,10 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < S::MPW; ++u) {
                     const uint32_t* b2 = bfr[q][j * S::MPW + u];
-                    mma_f16_16816(d1, k1024, k1024, k1024, k1024, b2[0], b2[1]);
-                    const uint32_t lo = h2_const(Unpack<BITS>::scale(2 * u));
-                    const uint32_t hi = h2_const(Unpack<BITS>::scale(2 * u + 1));
-                    mma_f16_16816(d0, lo, lo, hi, hi, b2[0], b2[1]);
+                    mma_bf16_16816(d1, k128, k128, k128, k128, b2[0], b2[1]);
+                    const uint32_t lo = bf2_const(Unpack<BITS>::sumw(2 * u));
+                    const uint32_t hi = bf2_const(Unpack<BITS>::sumw(2 * u + 1));
+                    mma_bf16_16816(d0, lo, lo, hi, hi, b2[0], b2[1]);
                 }
             xoff[q][0] = d1[0];
             xoff[q][1] = d1[1];
@@ -566,7 +571,7 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                     Unpack<BITS>::run(wb[j], pb);
 #pragma unroll
                     for (int u = 0; u < S::MPW; ++u)
-                        mma_f16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
+                        mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
                                       bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
                 }
                 const int gi = q / S::CPG;
@@ -586,7 +591,7 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             if (++st == NS) { st = 0; ph ^= 1u; }
 
             const int r0 = tile * 16 + g;
-            // undo the activations' 2^-e (exact)
+            // undo the activations' 2^-es (exact)
             if (M1) {
                 if (t == 0) { red_sl[r0] = acc[0] * ef0; red_sl[r0 + 8] = acc[2] * ef0; }
             } else {
@@ -893,8 +898,18 @@ cudaError_t launch_qmv_gather(const void* x, int64_t K, int64_t N, const uint32_
     prm.problems = problems;
     prm.num_problems = num_problems;
     prm.E = E;
-    return launch<true>(v, p, dim3(p.ctas, static_cast<unsigned>(max_problems), 1), mc, ms, mb,
-                        prm, stream);
+    // The problem count is known only on the device; max_problems bounds it.
+    // gridDim.y is limited to 65535, so larger bounds take several launches,
+    // each covering the next 65535 problems (blocks past the count return).
+    constexpr int64_t kMaxGridY = 65535;
+    for (int64_t p0 = 0; p0 < max_problems; p0 += kMaxGridY) {
+        const int64_t np = std::min(kMaxGridY, max_problems - p0);
+        prm.problem0 = static_cast<uint32_t>(p0);
+        cudaError_t e = launch<true>(v, p, dim3(p.ctas, static_cast<unsigned>(np), 1), mc, ms, mb,
+                                     prm, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace nvq
