@@ -51,6 +51,13 @@ cudaError_t launch_gather_simt(const void* x, int dt, int64_t x_rows, int64_t K,
                                const void* biases, int gs, int bits, int transpose, void* y,
                                cudaStream_t stream);
 
+// Self-test of the bounded pipeline waits: one wait on a barrier nothing
+// completes gives up after limit_ns and records kSelftestWaitCode in the error
+// word that selftest_error_take() reads and clears.
+constexpr unsigned int kSelftestWaitCode = 0x5E;
+cudaError_t launch_pipeline_selftest(uint64_t limit_ns, cudaStream_t stream);
+unsigned int selftest_error_take();
+
 // Largest expert count the single-CTA router handles (its histograms live in
 // shared memory).
 constexpr int64_t kMaxExperts = 1023;

@@ -25,7 +25,7 @@ __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity
         __nanosleep(ns);
         if (mbar_try_wait(bar, parity)) return true;
         ns = ns * 2 < max_ns ? ns * 2 : max_ns;
-        if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
             atomicCAS(&g_pipeline_error, 0u, code);
             return false;
         }

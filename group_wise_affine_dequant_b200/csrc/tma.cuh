@@ -9,8 +9,10 @@
 namespace nvq {
 
 // Sticky error word of the asynchronous pipelines of one source file: nonzero
-// when a wait gave up (the value names the wait). Each file that includes this
-// header has its own word and exposes a reader built on pipeline_error_take().
+// when a wait gave up (the value names the wait). Device code only writes it
+// (the first code wins); no wait reads it, so a wait that gave up in one launch
+// never shortens a wait of another launch. Each file that includes this header
+// has its own word and exposes a reader built on pipeline_error_take().
 static __device__ unsigned int g_pipeline_error = 0;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
@@ -63,16 +65,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 // Bounded wait for the phase with the given parity; false (and the error word
-// set to `code`) if it did not complete within kWaitLimitNs or another wait of
-// the launch already gave up. After a first plain poll the thread sleeps in
-// try_wait with a 100 us hint, and the time limit and error word are checked
-// between sleeps.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned code) {
+// set to `code`, if it was still 0) if the phase did not complete within
+// limit_ns. After a first plain poll the thread sleeps in try_wait with a
+// 100 us hint (at most limit_ns), checking the time limit between sleeps.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    const uint32_t hint = limit_ns < 100000u ? static_cast<uint32_t>(limit_ns) : 100000u;
     for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs || *(volatile unsigned*)&g_pipeline_error) {
+        if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+        if (globaltimer() - t0 > limit_ns) {
             atomicCAS(&g_pipeline_error, 0u, code);
             return false;
         }

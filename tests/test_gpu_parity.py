@@ -433,3 +433,29 @@ def test_pipelines_never_timed_out():
     """No wait inside the TMA / tensor-core pipelines gave up during the tests
     above (the sticky error word is 0)."""
     assert nvq.nv_pipeline_error() == 0
+
+
+def test_bounded_wait_gives_up_reports_and_leaves_the_next_call_correct():
+    """A wait on a barrier that nothing completes gives up after its limit
+    (here 50 ms, measured by CUDA events around it), records its code, and
+    the kernel returns: the context stays usable and the next product is
+    correct and reports no error."""
+    import time
+    assert nvq.nv_pipeline_error() == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record()
+    nvq.nv_pipeline_selftest(50000)
+    e1.record()
+    assert nvq.nv_pipeline_error() == 0x5E
+    assert time.time() - t0 < 10.0
+    assert e0.elapsed_time(e1) >= 49.0, e0.elapsed_time(e1)
+    assert nvq.nv_pipeline_error() == 0  # read and cleared
+    nvq.nv_pipeline_selftest(1)
+    assert nvq.nv_pipeline_error() == 0x5E
+    # the next products run normally (the recorded code does not cut them short)
+    nvq.nv_pipeline_selftest(1000)
+    _check_product(1000, 640, 1, 4, 64, True)
+    _check_product(300, 512, 40, 4, 64, True)
+    assert nvq.nv_pipeline_error() == 0x5E  # the self-test's code, nothing else
+    assert nvq.nv_pipeline_error() == 0
