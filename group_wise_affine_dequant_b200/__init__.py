@@ -15,7 +15,10 @@ from .binding import (  # noqa: F401
     nv_gather_qmm_workspace_size,
     nv_dequantize_affine,
     nv_pipeline_error,
+    nv_pipeline_selftest,
     nv_qmm,
+    nv_qmm_batched,
+    nv_qmm_splits,
     nv_quantize_affine,
     nv_status_string,
 )

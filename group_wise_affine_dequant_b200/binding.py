@@ -25,8 +25,10 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_dequantize_affine", "nv_qmm",
+           "nv_qmm_batched", "nv_qmm_splits",
            "nv_gather_qmm_workspace_size", "nv_gather_mm",
-           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_last_cuda_error",
+           "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_pipeline_selftest",
+           "nv_last_cuda_error",
            "nv_gather_qmm_noalloc")
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
@@ -65,6 +67,11 @@ def lib():
             L.nv_dequantize_affine.restype = _i
             L.nv_qmm.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _i, _p, _p]
             L.nv_qmm.restype = _i
+            L.nv_qmm_batched.argtypes = [_p, _i, _i64, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i,
+                                         _p, _p]
+            L.nv_qmm_batched.restype = _i
+            L.nv_qmm_splits.argtypes = [_i64, _i64, _i64, _i, _i, _i, _i]
+            L.nv_qmm_splits.restype = _i
             L.nv_gather_qmm_workspace_size.argtypes = [_i64, _i64]
             L.nv_gather_qmm_workspace_size.restype = _sz
             L.nv_gather_qmm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _p,
@@ -82,6 +89,8 @@ def lib():
             L.nv_last_cuda_error.restype = C.c_char_p
             L.nv_pipeline_error.argtypes = [_p]
             L.nv_pipeline_error.restype = _i
+            L.nv_pipeline_selftest.argtypes = [C.c_uint32, _p]
+            L.nv_pipeline_selftest.restype = _i
             _LIB = L
         return _LIB
 
@@ -189,6 +198,45 @@ def nv_qmm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: t
     return y
 
 
+def nv_qmm_batched(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                   biases: torch.Tensor, group_size: int = 64, bits: int = 4,
+                   transpose: bool = True, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """x [B, L, K]: B items of L rows with the same weights; y [B, L, N]. Item b
+    is bitwise equal to nv_qmm(x[b]) (routing and split-K per item)."""
+    for t, n in ((x, "x"), (codes, "codes"), (scales, "scales"), (biases, "biases")):
+        _dev(t, n)
+    if x.dim() != 3:
+        raise ValueError("x must be [B, L, K]")
+    B, L, K = x.shape
+    if codes.dim() != 2 or scales.shape != biases.shape or scales.dim() != 2:
+        raise ValueError("codes, scales and biases must be 2-D and scales/biases alike")
+    N = codes.shape[-2] if transpose else codes.shape[-1] * 32 // bits
+    rows, cols = (N, K) if transpose else (K, N)
+    if tuple(codes.shape) != (rows, cols * bits // 32) or \
+            tuple(scales.shape) != (rows, cols // group_size):
+        raise ValueError(f"weights do not match x: codes {tuple(codes.shape)}, scales "
+                         f"{tuple(scales.shape)} for K={K}, N={N}, transpose={transpose}")
+    y = out if out is not None else torch.empty(B, L, N, dtype=x.dtype, device=x.device)
+    if y.numel() != B * L * N or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
+    _dev(y, "out")
+    if scales.dtype != x.dtype:
+        raise NvqError("nv_qmm_batched", NV_ERR_UNSUPPORTED, nv_status_string(NV_ERR_UNSUPPORTED))
+    st = lib().nv_qmm_batched(x.data_ptr(), _DT.get(x.dtype, -1), B, L, K, N, codes.data_ptr(),
+                              scales.data_ptr(), biases.data_ptr(), group_size, bits,
+                              int(transpose), y.data_ptr(), _stream(stream))
+    _check("nv_qmm_batched", st)
+    return y
+
+
+def nv_qmm_splits(M: int, K: int, N: int, bits: int = 4, group_size: int = 64,
+                  transpose: bool = True, dtype=torch.bfloat16) -> int:
+    """K-partitions nv_qmm uses for an M-row product (1: no split)."""
+    return int(lib().nv_qmm_splits(M, K, N, bits, group_size, int(transpose),
+                                   _DT.get(dtype, -1)))
+
+
 def nv_gather_qmm_workspace_size(R: int, E: int) -> int:
     return int(lib().nv_gather_qmm_workspace_size(R, E))
 
@@ -284,3 +332,10 @@ def nv_pipeline_error() -> int:
     st = lib().nv_pipeline_error(C.addressof(code))
     _check("nv_pipeline_error", st)
     return int(code.value)
+
+
+def nv_pipeline_selftest(limit_us: int = 1000, stream=None) -> None:
+    """Enqueue one wait on a barrier nothing completes; it gives up after
+    limit_us and records code 0x5E (read it with nv_pipeline_error)."""
+    st = lib().nv_pipeline_selftest(int(limit_us), _stream(stream))
+    _check("nv_pipeline_selftest", st)

@@ -139,6 +139,66 @@ nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
                                           transpose, y, s));
 }
 
+nv_status nv_qmm_batched(const void* x, nv_dtype dt, int64_t B, int64_t L, int64_t K, int64_t N,
+                         const uint32_t* codes, const void* scales, const void* biases,
+                         int group_size, int bits, int transpose, void* y, nv_stream_t stream) {
+    if (!valid_dtype(dt)) return NV_ERR_UNSUPPORTED;
+    nv_status st = check_quant(group_size, bits);
+    if (st != NV_OK) return st;
+    if (B < 0 || L < 0 || K <= 0 || N < 0) return NV_ERR_INVALID_ARG;
+    if ((transpose ? K : N) % group_size != 0) return NV_ERR_INVALID_ARG;
+    if (L > 0 && B > (int64_t(1) << 40) / L) return NV_ERR_INVALID_ARG;
+    const int64_t M = B * L;
+    if (M == 0 || N == 0) return NV_OK;
+    if (!x || !codes || !scales || !biases || !y) return NV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases) ||
+        !aligned16(y))
+        return NV_ERR_INVALID_ARG;
+    // Routing by one item's rows L (crate docs, "Determinism": batch items of
+    // quantized products get their solo bits, the split-K partitions counted
+    // per item). Every route below computes each row with the same operations
+    // as the item's own call, whatever the batch around it.
+    cudaStream_t s = stream;
+    const int sms = sm_count();
+    if (dt == NV_BF16) {
+        if (transpose) {
+            if (L <= NV_ROW_INDEPENDENT_ROWS && nvq::qmv_supported(bits, group_size)) {
+                for (int64_t m0 = 0; m0 < M; m0 += NV_ROW_INDEPENDENT_ROWS) {
+                    const int64_t mc = M - m0 < NV_ROW_INDEPENDENT_ROWS ? M - m0 : NV_ROW_INDEPENDENT_ROWS;
+                    cudaError_t e = nvq::launch_qmv(static_cast<const uint16_t*>(x) + m0 * K, mc, K, N,
+                                                    codes, scales, biases, group_size, bits,
+                                                    static_cast<uint16_t*>(y) + m0 * N, s, sms);
+                    if (e != cudaSuccess) return from_cuda(e);
+                }
+                return NV_OK;
+            }
+            if (L > NV_ROW_INDEPENDENT_ROWS && nvq::tc_supported(M, K, N, bits, group_size))
+                return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases, group_size,
+                                                    bits, y, s, sms, L));
+        } else if (L <= NV_ROW_INDEPENDENT_ROWS && nvq::qmvt_supported_m(bits, group_size, 1)) {
+            int64_t chunk = NV_ROW_INDEPENDENT_ROWS;
+            while (chunk > 1 && !nvq::qmvt_supported_m(bits, group_size, chunk)) --chunk;
+            for (int64_t m0 = 0; m0 < M; m0 += chunk) {
+                const int64_t mc = M - m0 < chunk ? M - m0 : chunk;
+                cudaError_t e = nvq::launch_qmvt(static_cast<const uint16_t*>(x) + m0 * K, mc, K, N,
+                                                 codes, scales, biases, group_size, bits,
+                                                 static_cast<uint16_t*>(y) + m0 * N, s, sms);
+                if (e != cudaSuccess) return from_cuda(e);
+            }
+            return NV_OK;
+        }
+    }
+    return from_cuda(nvq::launch_qmm_simt(x, dt, M, K, N, codes, scales, biases, group_size, bits,
+                                          transpose, y, s));
+}
+
+int nv_qmm_splits(int64_t M, int64_t K, int64_t N, int bits, int group_size, int transpose,
+                  nv_dtype dt) {
+    if (dt != NV_BF16 || !transpose || M <= NV_ROW_INDEPENDENT_ROWS) return 1;
+    if (!nvq::tc_supported(M, K, N, bits, group_size)) return 1;
+    return nvq::tc_splits(M, K, N, sm_count());
+}
+
 size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E) {
     if (R < 0 || E < 0) return 0;
     return nvq::gather_workspace_bytes(R, E);
@@ -171,9 +231,9 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     if (e != cudaSuccess) return from_cuda(e);
     if (N == 0) return NV_OK;
     // Tensor-core route: each expert's weights are read once for all its rows.
-    // (the tensor-core kernel keeps 32-bit element offsets into x)
+    // (the tensor-core kernel keeps 32-bit offsets into x in 16-byte units)
     if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size) &&
-        x_rows * K < (int64_t(1) << 32))
+        x_rows * K < (int64_t(1) << 35))
         return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
                                                codes, scales, biases, group_size, bits, y, s, sms));
     // Matrix-vector route (row_exact): every pair's output is bitwise equal to
@@ -195,7 +255,7 @@ nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
     if (R > (int64_t(1) << 31) - 1) return NV_ERR_INVALID_ARG;
     if (E > nvq::kMaxExperts) return NV_ERR_UNSUPPORTED;
     if (dt != NV_BF16 || !nvq::tc_gather_mm_supported(K, N > 0 ? N : 1)) return NV_ERR_UNSUPPORTED;
-    if (x_rows * K >= (int64_t(1) << 32)) return NV_ERR_UNSUPPORTED;  // 32-bit offsets into x
+    if (x_rows * K >= (int64_t(1) << 35)) return NV_ERR_UNSUPPORTED;  // 32-bit 16-byte offsets into x
     if (!workspace || !aligned16(workspace)) return NV_ERR_WORKSPACE;
     if (workspace_bytes < nvq::gather_workspace_bytes(R, E)) return NV_ERR_WORKSPACE;
     if (R == 0) return NV_OK;
@@ -232,10 +292,17 @@ nv_status nv_pipeline_error(uint32_t* host_code) {
     const unsigned int b = nvq::tc_error_take();
     const unsigned int c = nvq::tc_gather_error_take();
     const unsigned int d = nvq::tc_gather_mm_error_take();
-    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu || d == 0xFFFFFFFFu)
+    const unsigned int t = nvq::selftest_error_take();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu || d == 0xFFFFFFFFu ||
+        t == 0xFFFFFFFFu)
         return NV_ERR_CUDA;
-    *host_code = a ? a : b ? b : c ? c : d;
+    *host_code = a ? a : b ? b : c ? c : d ? d : t;
     return NV_OK;
+}
+
+nv_status nv_pipeline_selftest(uint32_t limit_us, nv_stream_t stream) {
+    if (limit_us == 0 || limit_us > 2000000u) return NV_ERR_INVALID_ARG;
+    return from_cuda(nvq::launch_pipeline_selftest(static_cast<uint64_t>(limit_us) * 1000u, stream));
 }
 
 }  // extern "C"

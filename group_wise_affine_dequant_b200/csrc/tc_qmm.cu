@@ -20,6 +20,15 @@
 //               swizzle) so the row reads hit distinct banks; scales and biases
 //               arrive by TMA in blocks of 8 groups x BN rows through a 2-slot
 //               ring that the dequant warps release.
+// Split-K (the split-K kernel of "Docs / Quantization", section "Products on
+// the GPU", for outputs too small to fill the GPU with tiles while K is long):
+// the S CTAs of a thread-block cluster share one output tile, CTA r running
+// the same pipeline over k-steps [r * ks / S, (r + 1) * ks / S). Each writes its
+// fp32 partial tile from TMEM into its own shared memory; after a cluster
+// barrier, CTA r sums rows [r * 128 / S, (r + 1) * 128 / S) of the S partials
+// through distributed shared memory in rank order 0, 1, ..., S - 1 and stores
+// bf16 y. The order is fixed, so results are deterministic; no global scratch
+// is needed.
 // The contraction runs on the tensor cores in bf16 with fp32 accumulation; the
 // dequantized weight is rounded once to bf16 (relative error <= 2^-9), and the
 // result once to bf16 on output: together within the product tolerance.
@@ -61,9 +70,34 @@ struct TcParams {
     int sb_tma;               // scales/biases by TMA (rows of 16-byte multiples)
     uint32_t m2, m4, m6;      // shift counts 2, 4, 6
     int lg_gs;                // log2(group size)
+    int splits;               // split-K: CTAs per cluster (1 = no split)
 };
 
-template <int BITS>
+// Cluster helpers (split-K): this CTA's rank, the shared::cluster address of
+// a local shared-memory location in CTA `rank`, a load from it, and a barrier
+// of every thread of the cluster (release / acquire: shared-memory writes
+// before it are visible to the other CTAs' reads after it).
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_map(uint32_t local_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int BITS, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_b,
@@ -119,6 +153,14 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     const int ksteps = static_cast<int>(prm.K / BK);
     const int sgk = 8 * prm.gs / BK;  // k-steps per block of 8 groups
     const int tiles = prm.m_tiles * prm.n_tiles;
+    // Tiles of this CTA: persistent over tiles, or (split-K) the one tile of
+    // its cluster, k-steps [k0, k1) of it.
+    const int S = SPLIT ? prm.splits : 1;
+    const int rank = SPLIT ? static_cast<int>(cluster_rank()) : 0;
+    const int tile0 = SPLIT ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
+    const int tstep = SPLIT ? tiles : static_cast<int>(gridDim.x);
+    const int k0 = SPLIT ? rank * ksteps / S : 0;
+    const int k1 = SPLIT ? (rank + 1) * ksteps / S : ksteps;
     const uint32_t a_bytes = BM * BK * 2;
     const uint32_t c_bytes = static_cast<uint32_t>(BN) * BK * BITS / 8;
 
@@ -130,11 +172,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             uint32_t blk = 0;     // scale/bias blocks issued
             int issued = 0;       // loads issued (bounded by the drain below)
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int tile = tile0; tile < tiles && ok; tile += tstep) {
                 const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
-                int kb = 0;  // k-step within the current scale block
-                for (int ks = 0; ks < ksteps && ok; ++ks) {
-                    if (prm.sb_tma && kb == 0) {
+                int kb = k0 % sgk;  // k-step within the current scale block
+                for (int ks = k0; ks < k1 && ok; ++ks) {
+                    if (prm.sb_tma && (kb == 0 || ks == k0)) {
                         const int slot = blk & 1;
                         const uint32_t u = blk >> 1;
                         if (u > 0 && !(ok = mbar_wait(&sb_empty[slot], (u - 1) & 1, 7))) break;
@@ -171,13 +213,13 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             uint32_t use = 0;
             int local = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+            for (int tile = tile0; tile < tiles && ok; tile += tstep, ++local) {
                 const int a = local & 1;
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
                 if (ause > 0 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, 2))) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
-                for (int ks = 0; ks < ksteps; ++ks) {
+                for (int ks = k0; ks < k1; ++ks) {
                     if (!(ok = mbar_wait(&full_a[s], use & 1, 3))) break;
                     if (!(ok = mbar_wait(&full_b[s], use & 1, 4))) break;
                     tc_fence_after();
@@ -187,7 +229,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         // advance 16 bf16 (32 bytes) along K inside the swizzle atom
                         tc_mma(d_tmem, ad + (kk * UMMA_K * 2 >> 4), bd + (kk * UMMA_K * 2 >> 4), idesc,
-                               (ks > 0 || kk > 0) ? 1u : 0u);
+                               (ks > k0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                     if (++s == NS) { s = 0; ++use; }
@@ -200,11 +242,37 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         const int row_in_tile = q * 32 + lane;
         int local = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+        for (int tile = tile0; tile < tiles; tile += tstep, ++local) {
             const int a = local & 1;
             const uint32_t ause = static_cast<uint32_t>(local >> 1);
             if (!mbar_wait_backoff(&acc_full[a], ause & 1, 5, 2048)) break;
             tc_fence_after();
+            if constexpr (SPLIT) {
+                // the partial tile into this CTA's shared memory, [row][BN + 1]
+                // fp32 (the pipeline's stages are all consumed by now)
+                float* part = reinterpret_cast<float*>(smem) + row_in_tile * (BN + 1);
+                for (int j = 0; j < BN / 32; ++j) {
+                    uint32_t v[32];
+                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                           static_cast<uint32_t>(a * BN + j * 32);
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+                          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+                          "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                        : "r"(taddr));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) part[j * 32 + e] = __uint_as_float(v[e]);
+                }
+                tc_fence_before();
+                continue;
+            }
             const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
             const int64_t row = static_cast<int64_t>(mt) * BM + row_in_tile;
             const int64_t col0 = static_cast<int64_t>(nt) * BN;
@@ -259,20 +327,20 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         uint32_t use = 0;
         uint32_t blk = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        for (int tile = tile0; tile < tiles && ok; tile += tstep) {
             const int nt = tile / prm.m_tiles;
-            int kb = 0;
+            int kb = k0 % sgk;
             const int64_t n = static_cast<int64_t>(nt) * BN + r;
             const bool live = has_row && n < prm.N;
             const uint16_t* srow = prm.scales + (live ? n : 0) * gpr;
             const uint16_t* brow = prm.biases + (live ? n : 0) * gpr;
-            for (int ks = 0; ks < ksteps; ++ks) {
+            for (int ks = k0; ks < k1; ++ks) {
                 // 32 k lie in one group (groups are 32-k aligned multiples of 32)
                 const int g = ((ks * BK + 32 * h) >> prm.lg_gs);
                 float sc = 0.f, bc = 0.f;
                 const int slot = blk & 1;
                 if (prm.sb_tma) {
-                    if (kb == 0 && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
+                    if ((kb == 0 || ks == k0) && !(ok = mbar_wait(&sb_full[slot], (blk >> 1) & 1, 8))) break;
                     if (has_row) {
                         const uint16_t* ss = reinterpret_cast<const uint16_t*>(sb_ring + slot * sb_slot_bytes);
                         const int gi = g & 7;
@@ -320,7 +388,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);
-                if (prm.sb_tma && (kb == sgk - 1 || ks == ksteps - 1)) {
+                if (prm.sb_tma && (kb == sgk - 1 || ks == k1 - 1)) {
                     if (lane == 0) mbar_arrive(&sb_empty[slot]);  // this warp is done with the block
                     ++blk;
                 }
@@ -332,6 +400,27 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (SPLIT) {
+        // Sum the cluster's S partial tiles in rank order: CTA `rank` owns rows
+        // [rank * 128 / S, (rank + 1) * 128 / S); a warp takes a row, its lanes
+        // 32 consecutive columns.
+        cluster_sync();
+        const int mt = tile0 % prm.m_tiles, nt = tile0 / prm.m_tiles;
+        const int r_lo = rank * BM / S, r_hi = (rank + 1) * BM / S;
+        const uint32_t part0 = smem_u32(smem);
+        for (int r = r_lo + warp; r < r_hi; r += kThreads / 32) {
+            const int64_t row = static_cast<int64_t>(mt) * BM + r;
+            if (row >= prm.M) break;
+            for (int c = lane; c < BN; c += 32) {
+                const int64_t col = static_cast<int64_t>(nt) * BN + c;
+                const uint32_t off = static_cast<uint32_t>((r * (BN + 1) + c) * 4);
+                float acc = ld_cluster_f32(cluster_map(part0 + off, 0));
+                for (int src = 1; src < S; ++src) acc += ld_cluster_f32(cluster_map(part0 + off, src));
+                if (col < prm.N) prm.y[row * prm.N + col] = f32_to_bf16_bits(acc);
+            }
+        }
+        cluster_sync();  // no CTA leaves while the others still read its partial
+    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -355,9 +444,43 @@ int pick_bn(int64_t M, int64_t N, int num_sms) {
     return best;
 }
 
+// Split-K plan for an item of m_rows rows: when the unsplit tiles would fill
+// less than half of the SMs and K holds at least 8 k-steps, split K over a
+// cluster of S <= 8 CTAs (at least 4 k-steps each) and pick the tile width
+// that keeps the most SMs busy with the least column padding. A pure function
+// of (rows, N, K, SM count).
+struct TcPlan {
+    int bn, splits;
+};
+
+TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms) {
+    const int bn0 = pick_bn(m_rows, N, num_sms);
+    const int64_t mt = (m_rows + BM - 1) / BM;
+    const int64_t ks = K / BK;
+    if (2 * mt * ((N + bn0 - 1) / bn0) > num_sms || ks < 8) return {bn0, 1};
+    TcPlan best{bn0, 1};
+    double best_eff = -1.0;
+    for (int bn = 256; bn >= 64; bn -= 32) {
+        const int64_t nt = (N + bn - 1) / bn;
+        const int64_t tiles = mt * nt;
+        int64_t sp = num_sms / tiles;
+        if (sp > 8) sp = 8;
+        if (sp > ks / 4) sp = ks / 4;
+        if (sp < 2) continue;
+        const double eff = static_cast<double>(tiles * sp) / num_sms *
+                           (static_cast<double>(N) / static_cast<double>(nt * bn));
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = {bn, static_cast<int>(sp)}; }
+    }
+    return best;
+}
+
 }  // namespace
 
 unsigned int tc_error_take() { return pipeline_error_take(); }
+
+int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms) {
+    return plan_tc(m_rows, N, K, num_sms).splits;
+}
 
 bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
     return M > 0 && N > 0 && K % BK == 0 && K >= BK && (bits == 2 || bits == 4 || bits == 8) &&
@@ -366,10 +489,13 @@ bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
 
 cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                           const void* scales, const void* biases, int gs, int bits, void* y,
-                          cudaStream_t stream, int num_sms) {
+                          cudaStream_t stream, int num_sms, int64_t item_rows) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    const int bn = pick_bn(M, N, num_sms);
+    // the tiling and the split follow one item's rows (all of x for a plain
+    // product): every row's arithmetic is then that of its item's own call
+    const TcPlan plan = plan_tc(item_rows > 0 ? item_rows : M, N, K, num_sms);
+    const int bn = plan.bn;
     CUtensorMap map_x, map_c;
     {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
@@ -450,17 +576,44 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     prm.b_stage_bytes = b_stage;
     prm.c_stage_bytes = c_stage;
     prm.tmem_cols = 2 * bn <= 256 ? 256 : 512;
+    prm.splits = plan.splits;
     const size_t smem = prm.bar_off + (4 * stages + 8) * 8 + 16 + 1024;  // + alignment slack
     const int tiles = prm.m_tiles * prm.n_tiles;
-    const int grid = tiles < num_sms ? tiles : num_sms;
-    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-              const TcParams) =
-        bits == 4 ? tc_qmm_kernel<4> : bits == 8 ? tc_qmm_kernel<8> : tc_qmm_kernel<2>;
+    using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const TcParams);
+    if (plan.splits == 1) {
+        const int grid = tiles < num_sms ? tiles : num_sms;
+        Kern k = bits == 4 ? tc_qmm_kernel<4, false>
+                 : bits == 8 ? tc_qmm_kernel<8, false>
+                             : tc_qmm_kernel<2, false>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        k<<<grid, kThreads, smem, stream>>>(map_x, map_c, map_s, map_b, prm);
+        return cudaGetLastError();
+    }
+    // split-K: one cluster of `splits` CTAs per tile; the partial tile
+    // ([128][bn + 1] fp32) reuses the pipeline's stages in shared memory
+    if (static_cast<size_t>(BM) * (bn + 1) * 4 > prm.sb_off) return cudaErrorInvalidConfiguration;
+    Kern k = bits == 4 ? tc_qmm_kernel<4, true>
+             : bits == 8 ? tc_qmm_kernel<8, true>
+                         : tc_qmm_kernel<2, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, stream>>>(map_x, map_c, map_s, map_b, prm);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * plan.splits), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(plan.splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, map_x, map_c, map_s, map_b, prm);
 }
 
 }  // namespace nvq

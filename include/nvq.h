@@ -109,9 +109,9 @@ nv_status nv_quantize_affine(const void* w, nv_dtype dt, int64_t rows, int64_t c
  *
  * codes   uint32 [rows, cols * bits / 32]; scales, biases `dt` [rows,
  *         cols / group_size] (inputs, the layout nv_quantize_affine writes).
- * w       `dt` [rows, cols] (output): w[r, c] = scale * code + bias, one fp32
- *         fused multiply-add (rounded once), stored in `dt` (bf16 by
- *         round-to-nearest-even). Deterministic and exact up to that rounding.
+ * w       `dt` [rows, cols] (output): w[r, c] = scale * code + bias, the exact
+ *         value rounded once (to nearest, ties to even) to `dt`: one fused
+ *         multiply-add in fp32 or in bf16. Deterministic.
  * dt in {NV_F32, NV_BF16}; group_size in {32, 64, 128}; bits in {1, 2, 4, 8};
  * cols % group_size == 0; rows == 0 is a no-op returning NV_OK. Bits 3, 5, 6
  * return NV_ERR_UNSUPPORTED.
@@ -140,6 +140,36 @@ nv_status nv_dequantize_affine(const uint32_t* codes, const void* scales, const 
 nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
                  const uint32_t* codes, const void* scales, const void* biases, int group_size,
                  int bits, int transpose, int row_exact, void* y, nv_stream_t stream);
+
+/*
+ * Batched quantized product: B items of L rows each, all with the same
+ * weights ("Docs / Quantization", section "Products on the GPU"; nuvec crate
+ * docs, section "Determinism": batch items of quantized products give each
+ * item the bits of its own call, the split-K partitions being counted per
+ * item).
+ *
+ * x      [B, L, K] in `dt`; y [B, L, N] in `dt`; weights as for nv_qmm.
+ * Routing (kernel, tile shape and split-K partition count) is the function of
+ * (L, N, K, dt, group_size, bits, transpose) that nv_qmm applies to an L-row
+ * call, so that item b of the result is bitwise equal to
+ * nv_qmm(x[b], M = L, row_exact = 0). B * L == 0 or N == 0 is a no-op
+ * returning NV_OK; B * L above 2^40 returns NV_ERR_INVALID_ARG.
+ */
+nv_status nv_qmm_batched(const void* x, nv_dtype dt, int64_t B, int64_t L, int64_t K, int64_t N,
+                         const uint32_t* codes, const void* scales, const void* biases,
+                         int group_size, int bits, int transpose, void* y, nv_stream_t stream);
+
+/*
+ * K-partitions (split-K; "Docs / Quantization", section "Products on the
+ * GPU": split-K when the output is small but the inner dimension long) that
+ * nv_qmm uses for an M-row product: 1 when it does not split. Host only, no
+ * launch. Products of more than 8 bf16 rows with transpose = 1 split K over a
+ * cluster of up to 8 CTAs when their 128 x BN output tiles would occupy fewer
+ * than half of the SMs and K holds at least 8 steps of 64; the partial sums
+ * are reduced in a fixed order, so results stay deterministic.
+ */
+int nv_qmm_splits(int64_t M, int64_t K, int64_t N, int bits, int group_size, int transpose,
+                  nv_dtype dt);
 
 /* Bytes of device workspace nv_gather_qmm needs for R pairs and E experts. */
 size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E);
@@ -180,7 +210,7 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
  * w        bf16 [E, N, K]: expert e's weights, row n = output feature n.
  * y[r, n] = sum_k x[lhs[r], k] * w[rhs[r], n, k], fp32 accumulation, stored
  *   in bf16; pairs with an out-of-range id get zero rows and a flag.
- * dt must be NV_BF16, K a multiple of 64 and x_rows * K below 2^32
+ * dt must be NV_BF16, K a multiple of 64 and x_rows * K below 2^35
  * (NV_ERR_UNSUPPORTED otherwise).
  */
 nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
@@ -196,10 +226,24 @@ nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_st
  * Read and clear the sticky error word of the asynchronous (TMA / tensor-core)
  * pipelines into *host_code (a HOST pointer): 0 when every wait inside the
  * kernels completed; otherwise a nonzero code naming the first wait that gave
- * up after its time limit (the kernel then stopped early, and its outputs are
- * not valid). Synchronises the device.
+ * up after its time limit (2 s; the launch that owned it then stopped early,
+ * and its outputs are not valid). A wait that gave up affects only its own
+ * launch: later launches run normally whether or not the word was read.
+ * Synchronises the device. A diagnostic of this library (the pages have no
+ * counterpart): nothing on the device traps or spins without a limit.
  */
 nv_status nv_pipeline_error(uint32_t* host_code);
+
+/*
+ * Self-test of the bounded waits behind nv_pipeline_error (a diagnostic of
+ * this library; the pages have no counterpart). Enqueues on `stream` one
+ * kernel whose single thread waits, through the pipelines' own bounded wait,
+ * on a barrier that nothing completes; after limit_us microseconds the wait
+ * gives up, records code 0x5E in the error word and the kernel returns, so
+ * that nv_pipeline_error then reports 0x5E. limit_us in [1, 2000000], else
+ * NV_ERR_INVALID_ARG. Writes no caller memory.
+ */
+nv_status nv_pipeline_selftest(uint32_t limit_us, nv_stream_t stream);
 
 /*
  * nv_gather_qmm without a workspace argument, for callers that cannot allocate
@@ -211,11 +255,16 @@ nv_status nv_pipeline_error(uint32_t* host_code);
  * (about 200 KB, kept on every GPU that loads the library until exit):
  * R <= 32768 pairs and E <= 256 experts, else NV_ERR_WORKSPACE before any
  * launch. The first call on a device looks the array's address up (with that
- * device current) and should come before any stream capture. Every call
- * shares the array: calls that may overlap on the GPU race and must be
- * serialised by the caller (one stream, or events). Nothing in the array needs
- * to start at zero (each call writes every entry it reads). No device memory
- * is allocated or freed.
+ * device current) and should come before any stream capture; the address is
+ * kept for the life of the process, so a cudaDeviceReset between calls
+ * leaves a stale address behind (do not reset a device this entry point has
+ * been called on). Every call shares the array: calls that may overlap on
+ * the GPU race and must be serialised by the caller (one stream, or events).
+ * Nothing in the array needs to start at zero (each call writes every entry
+ * it reads). The anomaly flags of nv_gather_qmm are written into the array
+ * too and cannot be read back (nv_gather_qmm_flags needs a workspace
+ * pointer); a caller that needs them uses nv_gather_qmm. No device memory is
+ * allocated or freed.
  */
 nv_status nv_gather_qmm_noalloc(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
                                 const uint32_t* lhs_idx, const uint32_t* rhs_idx, int64_t R,

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import group_wise_affine_dequant_b200 as nvq
 from group_wise_affine_dequant_b200 import binding as B
@@ -151,12 +152,14 @@ def test_gather_mm_argument_errors():
     assert call(w=24) == B.NV_ERR_INVALID_ARG        # misaligned
     assert call(lhs=4) == B.NV_ERR_INVALID_ARG
     assert call(R=0, ws_bytes=L.nv_gather_qmm_workspace_size(0, E)) == B.NV_OK
-    assert call(x_rows=1 << 21) == B.NV_ERR_UNSUPPORTED  # x_rows * K = 2^32 elements
+    assert call(x_rows=1 << 24) == B.NV_ERR_UNSUPPORTED  # x_rows * K = 2^35 elements
 
 
 def test_flags_argument_errors():
     L = nvq.lib()
     assert L.nv_pipeline_error(0) == B.NV_ERR_INVALID_ARG
+    assert L.nv_pipeline_selftest(0, None) == B.NV_ERR_INVALID_ARG       # no limit
+    assert L.nv_pipeline_selftest(2000001, None) == B.NV_ERR_INVALID_ARG  # above 2 s
     flags = C.c_uint32(0)
     assert L.nv_gather_qmm_flags(0, C.addressof(flags), None) == B.NV_ERR_INVALID_ARG
     assert L.nv_gather_qmm_flags(16, 0, None) == B.NV_ERR_INVALID_ARG
@@ -169,3 +172,39 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(B._build, "build", lambda *a, **k: None)
     with pytest.raises(RuntimeError, match="libnvq.so missing"):
         B.lib()
+
+
+def test_split_k_routing_is_a_pure_function_of_the_shape():
+    """Split-K only where the output tiles would leave most SMs idle and K is
+    long; the matrix-vector sizes, fp32 and the transposed layout never split."""
+    S = nvq.nv_qmm_splits
+    assert S(64, 14336, 1024) > 1            # small N, long K
+    assert S(20, 2432, 200) > 1
+    assert S(2048, 4096, 14336) == 1         # prefill: tiles fill the GPU
+    assert S(8, 14336, 1024) == 1            # matrix-vector rows
+    assert S(64, 256, 1024) == 1             # K too short to split
+    assert S(64, 14336, 1024, transpose=False) == 1
+    assert S(64, 14336, 1024, dtype=torch.float32) == 1
+    assert S(64, 14336, 1024) == S(64, 14336, 1024)
+    assert 2 <= S(64, 14336, 1024) <= 8
+
+
+def test_batched_argument_errors():
+    L = nvq.lib()
+
+    def call(**kw):
+        a = dict(x=16, dt=1, B=2, L=3, K=128, N=64, c=16, s=16, b=16, gs=64, bits=4, t=1, y=16)
+        a.update(kw)
+        return L.nv_qmm_batched(a["x"], a["dt"], a["B"], a["L"], a["K"], a["N"], a["c"], a["s"],
+                                a["b"], a["gs"], a["bits"], a["t"], a["y"], None)
+
+    assert call(B=-1) == B.NV_ERR_INVALID_ARG
+    assert call(L=-1) == B.NV_ERR_INVALID_ARG
+    assert call(K=100) == B.NV_ERR_INVALID_ARG       # K not a multiple of the group
+    assert call(bits=3) == B.NV_ERR_UNSUPPORTED
+    assert call(dt=5) == B.NV_ERR_UNSUPPORTED
+    assert call(x=0) == B.NV_ERR_INVALID_ARG
+    assert call(y=8) == B.NV_ERR_INVALID_ARG         # misaligned
+    assert call(B=1 << 30, L=1 << 20) == B.NV_ERR_INVALID_ARG
+    assert call(B=0) == B.NV_OK
+    assert call(N=0) == B.NV_OK
