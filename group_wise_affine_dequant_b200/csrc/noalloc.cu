@@ -12,11 +12,14 @@
 // not a device address), so its device address is looked up once per device
 // with cudaGetSymbolAddress, with that device current, on the first call made
 // on the device; that first call should therefore come before any stream
-// capture. All calls share the array: calls that overlap on the GPU (two
-// streams, or two devices' worth of host threads on one device) race on it.
-// Nothing in it needs to start at zero: the routing kernel writes every entry
-// a call reads. Each call leaves its routing tables behind, overwritten by the
-// next call.
+// capture. The looked-up address is kept for the life of the process: after
+// a cudaDeviceReset it would be stale, so a device this entry point has used
+// must not be reset. All calls share the array: calls that overlap on the GPU
+// (two streams, or two devices' worth of host threads on one device) race on
+// it. Nothing in it needs to start at zero: the routing kernel writes every
+// entry a call reads. Each call leaves its routing tables (and its anomaly
+// flags, which no entry point reads back from here) behind, overwritten by
+// the next call.
 #include <mutex>
 
 #include "common.cuh"

@@ -352,7 +352,8 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                 for (int j = 0; j < nr; ++j) {
                     const uint32_t pair = __ldg(prm.perm + first + p0 + r0 + RS * j);
                     const uint32_t row = prm.lhs ? __ldg(prm.lhs + pair) : pair;
-                    s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K) + ch * 8;
+                    // in 16-byte units (K is a multiple of 64): x up to 2^35 elements
+                    s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K / 8) + ch;
                 }
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if (x.use > 0 && !(ok = mbar_wait_backoff(&empty_x[x.s], (x.use - 1) & 1, 31, 256))) break;
@@ -361,7 +362,8 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         const int r = r0 + RS * j;
                         cp_async16(dst + (ch >> 3) * (kMaxPairs * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
                                        (((ch & 7) ^ (r & 7)) << 4),
-                                   prm.x + s_xoff[j * kXThreads + xt] + ks * BK);
+                                   reinterpret_cast<const uint4*>(prm.x) + s_xoff[j * kXThreads + xt] +
+                                       ks * (BK / 8));
                     }
                     cp_async_commit();
                     x.next(DX);
@@ -506,7 +508,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
                              int bits, void* y, cudaStream_t stream, int num_sms) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    if (x_rows * K >= (int64_t(1) << 32)) return cudaErrorInvalidValue;  // 32-bit row offsets
+    if (x_rows * K >= (int64_t(1) << 35)) return cudaErrorInvalidValue;  // 32-bit 16-byte offsets
     CUtensorMap map_c, map_s, map_b;
     const int64_t wpr = K * bits / 32, gpr = K / gs;
     {   // code rows of 128 bytes (several k-steps), 128-byte swizzle

@@ -274,7 +274,8 @@ tc_gather_mm_kernel(const __grid_constant__ CUtensorMap map_w, const MParams prm
                 for (int j = 0; j < nr; ++j) {
                     const uint32_t pair = __ldg(prm.perm + first + p0 + r0 + RS * j);
                     const uint32_t row = prm.lhs ? __ldg(prm.lhs + pair) : pair;
-                    s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K) + ch * 8;
+                    // in 16-byte units (K is a multiple of 64): x up to 2^35 elements
+                    s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K / 8) + ch;
                 }
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if (x.use > 0 && !(ok = mbar_wait_backoff(&empty_x[x.s], (x.use - 1) & 1, 46, 256))) break;
@@ -282,7 +283,8 @@ tc_gather_mm_kernel(const __grid_constant__ CUtensorMap map_w, const MParams prm
                     for (int j = 0; j < nr; ++j) {
                         const int r = r0 + RS * j;
                         cp_async16(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4),
-                                   prm.x + s_xoff[j * kXThreads + xt] + ks * BK);
+                                   reinterpret_cast<const uint4*>(prm.x) + s_xoff[j * kXThreads + xt] +
+                                       ks * (BK / 8));
                     }
                     cp_async_commit();
                     x.next(DX);
@@ -331,7 +333,7 @@ cudaError_t launch_tc_gather_mm(const void* x, int64_t x_rows, int64_t K, const 
                                 const void* w, void* y, cudaStream_t stream, int num_sms) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    if (x_rows * K >= (int64_t(1) << 32)) return cudaErrorInvalidValue;  // 32-bit row offsets
+    if (x_rows * K >= (int64_t(1) << 35)) return cudaErrorInvalidValue;  // 32-bit 16-byte offsets
     CUtensorMap map_w;
     {   // experts [E][N][K] bf16: boxes of 64 k (128 bytes) x 256 rows, 128-byte swizzle
         cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N),

@@ -52,7 +52,25 @@ def test_noalloc_matches_workspace_entry_point(row_exact):
         # within the tolerance of the tests, against the workspace entry point's output
         ok = (y.double() - y_ws.double()).abs() <= O.TOL_REL[torch.bfloat16] * a + O.TOL_ABS
         assert bool(ok.all()), f"call {call}"
+        # the same kernels on the same routing: the same bits
+        assert torch.equal(y.view(torch.int16), y_ws.view(torch.int16)), f"call {call}"
         P.assert_within(y, yr, a, torch.bfloat16, f"noalloc call {call}")
+
+
+def test_noalloc_at_its_capacity():
+    """R = 32768 pairs over E = 256 experts, the largest request the fixed
+    array holds: twice in a row, bitwise equal to the workspace entry point."""
+    E, N, K, tokens, top_k = 256, 128, 512, 8192, 4
+    w = W.normal((E, N, K), 0.02, 7, "bf16")
+    c, s, b = P.to_dev(*O.quantize_affine(w, 64, 4))
+    x = W.normal((tokens, K), 1.0, 8, "bf16").cuda()
+    lhs, rhs = W.flatten_pairs(W.expert_ids(tokens, E, top_k, 9))
+    assert rhs.numel() == 32768
+    dl, dr = lhs.to(torch.int32).cuda(), rhs.to(torch.int32).cuda()
+    y_ws = nvq.nv_gather_qmm(x, c, s, b, dr, dl, 64, 4, True, False, False)
+    for call in range(2):
+        y = _noalloc(x, c, s, b, dr, dl, 64, 4)
+        assert torch.equal(y.view(torch.int16), y_ws.view(torch.int16)), f"call {call}"
 
 
 def test_noalloc_rejects_requests_beyond_its_capacity():
