@@ -5,16 +5,20 @@
 
 One step is one pass of the hot path over one batch of the headline workload:
 a 4-bit, group-64 decode product y = x . w^T with x [1, 4096] bf16 and
-W [14336, 4096] (Llama-8B MLP shape), i.e. one nv_qmm call. The JSON line
+W [14336, 4096] (Llama-8B MLP shape) on each of the weight copies the batch
+holds (as many copies as it takes to touch more than 3x the L2 cache before a
+copy is read again: 13 on B200), i.e. one nv_qmm call per copy. The JSON line
 reports HBM GB/s of algorithmic bytes (codes + scales + biases + x + y); the
 other workloads (8-bit and transposed decode, few rows, prefill, mixture of
 experts with 4-bit and with bf16 weights, dequantization to bf16) are
-measured in the same run and reported under "also".
+measured in the same run, with the same step definition, and reported under
+"also".
 
 Timing: W untimed warm-up steps, then K timed steps captured in CUDA graphs and
 bracketed by a barrier and torch.cuda.synchronize(); device time from CUDA
-events on the launching stream; max over ranks. The weights rotate over enough
-copies that the set touched between two uses of a copy exceeds the L2 cache.
+events on the launching stream; max over ranks. Within a step the calls rotate
+over the weight copies, so the set touched between two uses of a copy exceeds
+the L2 cache.
 Multi-GPU runs are independent replicas (the product does not shard here):
 value = bytes processed by all ranks / max time. After timing, each workload's
 own output is checked against plain torch arithmetic on the GPU
@@ -284,9 +288,13 @@ class Decode:
         self.bytes = wbytes + 2 * M * (K + N)
         self.flops = 2 * M * N * K
 
-    def step(self, i):
-        c, s, b = self.ws[i % self.copies]
+    def call(self, j):
+        c, s, b = self.ws[j]
         self.nvq.nv_qmm(self.x, c, s, b, self.gs, self.bits, self.t, out=self.y)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
 
 
 class DecodeE2E(Decode):
@@ -295,14 +303,15 @@ class DecodeE2E(Decode):
     def __init__(self, dev, **kw):
         super().__init__(dev, **kw)
         self.xh = self.x.cpu().pin_memory()
-        self.yh = torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
-        self.h2d = self.xh.numel() * 2
-        self.d2h = self.yh.numel() * 2
+        self.yh = [torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
+                   for _ in range(self.copies)]
+        self.h2d = self.xh.numel() * 2 * self.copies
+        self.d2h = self.yh[0].numel() * 2 * self.copies
 
-    def step(self, i):
+    def call(self, j):
         self.x.copy_(self.xh, non_blocking=True)
-        super().step(i)
-        self.yh.copy_(self.y, non_blocking=True)
+        super().call(j)
+        self.yh[j].copy_(self.y, non_blocking=True)
 
 
 class Dequant:
@@ -322,9 +331,13 @@ class Dequant:
         self.out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
         self.bytes = wbytes + N * K * 2
 
-    def step(self, i):
-        c, s, b = self.ws[i % self.copies]
+    def call(self, j):
+        c, s, b = self.ws[j]
         self.nvq.nv_dequantize_affine(c, s, b, self.gs, self.bits, out=self.out)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
 
 
 class GatherMM:
@@ -351,9 +364,13 @@ class GatherMM:
                                device=dev)
         self.bytes = wbytes + self.T * self.K * 2 + self.R * self.N * 2 + self.R * 8
 
-    def step(self, i):
-        self.nvq.nv_gather_mm(self.x, self.ws[i % self.copies], self.rhs, self.lhs,
+    def call(self, j):
+        self.nvq.nv_gather_mm(self.x, self.ws[j], self.rhs, self.lhs,
                               workspace=self.wsp, out=self.y)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
 
 
 def check_gather_mm(wl, samples=64):
@@ -396,10 +413,14 @@ class Gather:
                                device=dev)
         self.bytes = wbytes + self.T * self.K * 2 + self.R * self.N * 2 + self.R * 8
 
-    def step(self, i):
-        c, s, b = self.ws[i % self.copies]
+    def call(self, j):
+        c, s, b = self.ws[j]
         self.nvq.nv_gather_qmm(self.x, c, s, b, self.rhs, self.lhs, 64, 4, True, self.sorted,
                                self.row_exact, workspace=self.wsp, out=self.y)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
 
 
 # --------------------------------------------------------------------------- arms
@@ -436,9 +457,10 @@ def run_nvq(args):
     chk = (lambda f, *a, **k: 0.0) if args.no_output_check else (lambda f, *a, **k: f(*a, **k))
     checks = {"decode": round(chk(check_decode, dec), 4)}
     ms = max_ms(ms)
-    per_step_s = ms / 1e3 / K
-    value = replica_rate(ws, dec.bytes, K, ms) / 1e9
-    achieved = dec.bytes / per_step_s / 1e9  # one launch per step on this rank
+    # the timed region holds K * copies launches of the decode kernel, nothing else
+    per_launch_s = ms / 1e3 / (K * dec.copies)
+    value = replica_rate(ws, dec.bytes * dec.copies, K, ms) / 1e9
+    achieved = dec.bytes / per_launch_s / 1e9
     clocks = clk.summary()
 
     # ---- end to end through host buffers
@@ -446,11 +468,11 @@ def run_nvq(args):
     graphs = timed_graph(e2e.step, K, Wm, stream)
     ms_e2e = max_ms(replay_timed(graphs, stream, barrier))
     del graphs
-    e2e_value = replica_rate(ws, e2e.bytes, K, ms_e2e) / 1e9
+    e2e_value = replica_rate(ws, e2e.bytes * e2e.copies, K, ms_e2e) / 1e9
 
     # ---- the other workloads, same rules (fewer steps)
     also = {}
-    ks = max(3, min(K, 400))
+    ks = max(3, min(K, 40))
     for name, mk in (("decode_8bit_gbs", lambda: Decode(dev, bits=8)),
                      ("decode_transposed_gbs", lambda: Decode(dev, N=14336, K=4096, transpose=False)),
                      ("decode_transposed_8bit_gbs", lambda: Decode(dev, transpose=False, bits=8)),
@@ -459,13 +481,26 @@ def run_nvq(args):
         wl = mk()
         g = timed_graph(wl.step, ks, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
-        also[name] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
+        also[name] = round(replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9, 1)
         checks[name.replace("_gbs", "")] = round(chk(check_decode, wl), 4)
         del g, wl
+    # split-K: a small output with a long inner dimension (HBM-bound: 10.2 MB
+    # moved against 1.9 GFLOP)
+    wl = Decode(dev, N=1024, K=14336, M=64)
+    g = timed_graph(wl.step, ks, Wm, stream)
+    t = max_ms(replay_timed(g, stream, barrier))
+    sk = replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9
+    also["splitk_64x1024x14336_b4g64_gbs"] = round(sk, 1)
+    also["splitk_64x1024x14336_b4g64_tflops"] = round(
+        replica_rate(ws, wl.flops * wl.copies, ks, t) / 1e12, 1)
+    also["splitk_frac_of_hbm"] = round(sk / ws / pk["hbm_gbs"], 4)
+    also["splitk_partitions"] = wl.nvq.nv_qmm_splits(64, 14336, 1024, 4, 64)
+    checks["splitk_64x1024x14336"] = round(chk(check_decode, wl), 4)
+    del g, wl
     wl = Dequant(dev)
     g = timed_graph(wl.step, ks, Wm, stream)
     t = max_ms(replay_timed(g, stream, barrier))
-    dq = replica_rate(ws, wl.bytes, ks, t) / 1e9
+    dq = replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9
     also["dequantize_14336x4096_b4g64_bf16_gbs"] = round(dq, 1)
     also["dequantize_frac_of_hbm"] = round(dq / ws / pk["hbm_gbs"], 4)
     checks["dequantize"] = chk(check_dequant, wl)
@@ -475,25 +510,25 @@ def run_nvq(args):
         wl = Gather(dev, srt, rx)
         g = timed_graph(wl.step, ks, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
-        also[name + "_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
-        also[name + "_gbs"] = round(replica_rate(ws, wl.bytes, ks, t) / 1e9, 1)
+        also[name + "_tok_s"] = round(replica_rate(ws, wl.T * wl.copies, ks, t), 1)
+        also[name + "_gbs"] = round(replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9, 1)
         checks[name] = round(chk(check_gather, wl), 4)
         del g, wl
     wl = GatherMM(dev)
     g = timed_graph(wl.step, ks, Wm, stream)
     t = max_ms(replay_timed(g, stream, barrier))
-    also["gather_mm_bf16_tok_s"] = round(replica_rate(ws, wl.T, ks, t), 1)
-    gm = replica_rate(ws, wl.bytes, ks, t) / 1e9
+    also["gather_mm_bf16_tok_s"] = round(replica_rate(ws, wl.T * wl.copies, ks, t), 1)
+    gm = replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9
     also["gather_mm_bf16_gbs"] = round(gm, 1)
     also["gather_mm_frac_of_hbm"] = round(gm / ws / pk["hbm_gbs"], 4)
     checks["gather_mm_bf16"] = round(chk(check_gather_mm, wl), 4)
     del g, wl
     for bits, gs in W.PREFILL_VARIANTS:
         wl = Decode(dev, N=14336, K=4096, M=2048, bits=bits, gs=gs)
-        kp = max(3, min(K, 100))
+        kp = max(3, min(K, 10))
         g = timed_graph(wl.step, kp, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
-        tf = replica_rate(ws, wl.flops, kp, t) / 1e12
+        tf = replica_rate(ws, wl.flops * wl.copies, kp, t) / 1e12
         key = "prefill_tflops" if (bits, gs) == (4, 64) else f"prefill_b{bits}_g{gs}_tflops"
         also[key] = round(tf, 1)
         if (bits, gs) == (4, 64):
@@ -517,15 +552,17 @@ def run_nvq(args):
         "pct_of_8tbs": round(100 * achieved / HBM_NOMINAL_GBS, 2),
         "config": {"workload": "decode x[1,4096] . W[14336,4096]^T, affine 4-bit g64, bf16",
                    "M": 1, "N": 14336, "K": 4096, "bits": 4, "group_size": 64,
-                   "bytes_per_step": dec.bytes, "parallelism": f"replicas x{ws}",
-                   "l2": f"weights rotate over {dec.copies} copies (> 3x L2 between reuses)"},
+                   "products_per_step": dec.copies, "bytes_per_product": dec.bytes,
+                   "bytes_per_step": dec.bytes * dec.copies, "parallelism": f"replicas x{ws}",
+                   "l2": f"a step multiplies by each of {dec.copies} weight copies in turn "
+                         f"(> 3x L2 between reuses of a copy)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                      "peak_kind": pk_kind, "unit": "GB/s",
                      "frac": round(achieved / pk["hbm_gbs"], 4),
                      "traffic": traffic_for("qmv_decode_b4_g64")},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": e2e.h2d,
                 "d2h_bytes_per_step": e2e.d2h},
-        "gpu_launches": K,
+        "gpu_launches": K * dec.copies,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"]},
         "also": also,
@@ -618,17 +655,60 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_WORKLOADS = {
+    "decode": lambda dev: Decode(dev),
+    "decode8": lambda dev: Decode(dev, bits=8),
+    "decode_t0": lambda dev: Decode(dev, transpose=False),
+    "fewrow8": lambda dev: Decode(dev, M=8),
+    "gather": lambda dev: Gather(dev, sorted_pairs=False),
+    "prefill": lambda dev: Decode(dev, N=14336, K=4096, M=2048, bits=4, gs=64),
+    "splitk": lambda dev: Decode(dev, N=1024, K=14336, M=64),
+    "prefill8": lambda dev: Decode(dev, N=14336, K=4096, M=2048, bits=8, gs=64),
+    "dequant": lambda dev: Dequant(dev),
+    "gather_mm": lambda dev: GatherMM(dev),
+}
+
+
+def run_profile(name: str, launches: int):
+    """Plain stream launches of one workload's product (no graphs), so that a
+    profiler sees one kernel per product (the router and the grouped kernel for
+    a gather). Prints the mean time per product from CUDA events: not a bench
+    value when the process runs under a profiler."""
+    if name not in PROFILE_WORKLOADS:
+        raise SystemExit(f"unknown workload {name!r}; one of {sorted(PROFILE_WORKLOADS)}")
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    wl = PROFILE_WORKLOADS[name](dev)
+    for j in range(3):
+        wl.call(j % wl.copies)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for j in range(launches):
+        wl.call(j % wl.copies)
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"{name}: {launches} products, {e0.elapsed_time(e1) / launches * 1e3:.1f} us per product")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="nvq", choices=["nvq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-output-check", action="store_true",
                     help="skip the torch checks of the timed outputs (for profiler launch lists)")
+    ap.add_argument("--profile", metavar="WORKLOAD", default=None,
+                    help="launch one workload's product --launches times for a profiler "
+                         f"(one of {', '.join(PROFILE_WORKLOADS)}) instead of benchmarking")
+    ap.add_argument("--launches", type=int, default=10)
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args.profile, args.launches)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
