@@ -9,30 +9,28 @@
 //    swizzle so the fragment reads below hit distinct banks) plus the slice's
 //    scales and biases into its own ring of shared-memory stages, completing
 //    on a per-warp mbarrier, several tiles ahead of the math.
-//  * Codes become bf16 exactly with one mask each: OR-ing a field worth
-//    c * 2^p <= 127 into the mantissa of 128.0 gives 128 + c * 2^p (bf16 holds
-//    every integer below 256). A 4-bit word takes three shifts and four masks;
-//    an 8-bit code is split into its two nibbles (c = lo + 16 hi), which are
-//    unpacked like two 4-bit codes; a 2-bit word takes two shifts and eight
-//    masks.
+//  * Every weight is dequantized in registers to bf16 w = scale * code + bias,
+//    the exact value rounded once (one bf16 fused multiply-add on the code
+//    held as an exact bf16 number; 8-bit codes through one fp32 fma and a
+//    conversion), exactly as the tiled kernels do. Codes become exact bf16
+//    with one mask each: OR-ing a field worth c * 2^p <= 127 into the mantissa
+//    of 128.0 gives 128 + c * 2^p, then 128 is subtracted; a 2-bit field held
+//    as c * 4^j meets the scale divided by 4^j (exact).
 //  * The multiply-adds run on the tensor cores (mma.sync m16n8k16, bf16 in,
-//    fp32 accumulate): A = 16 weight rows x 16 k of codes, B = the activations
-//    (one column per activation row, up to 8). Which physical k feeds which MMA
-//    k-slot is chosen so that each thread's loaded words feed its own A
-//    fragments; the activations are permuted the same way once, in registers,
-//    and the activation of a slot holding c * 2^p is multiplied by 2^-p (by 2
-//    for the high nibble of an 8-bit code held as 8 hi).
+//    fp32 accumulate): A = 16 weight rows x 16 k of weights, B = the
+//    activations (one column per activation row, up to 8). Which physical k
+//    feeds which MMA k-slot is chosen so that each thread's loaded words feed
+//    its own A fragments; the activations are permuted the same way once, in
+//    registers.
 //  * Activations enter the MMA as bf16, the type they arrive in: bf16 has the
 //    exponent range of fp32, so no value is rounded or flushed on the way in.
 //    Only a slice whose largest magnitude reaches 2^100 is first multiplied by
-//    2^-(e - 100) (e its exponent), which keeps every fp32 sum finite, and its
+//    2^-(e - 100) (e its exponent), which keeps the fp32 sums finite, and its
 //    partial sums are multiplied back by 2^(e - 100); both steps are exact.
-//    Every product x * code is therefore exact for every finite bf16 input
-//    (down to the bf16 subnormals), and only fp32 sums round.
-//  * Scale and bias are applied per group outside the MMA, with the 128s
-//    removed by an MMA over the same activations:
-//        sum_k x_k w_k = s * (D - 128-sum) + b * sum_k x_k,
-//    so only the group sums round.
+//    Every product of an activation and a dequantized weight is exact in
+//    fp32: the only roundings are the weights' (relative 2^-9) and the fp32
+//    sums', so the error is bounded by a small multiple of sum_k |x_k w_k|
+//    for every finite input.
 //  * A warp owns a k-slice of 16 MMA k-steps (256 k at 2/4 bits, 128 at 8) and
 //    keeps its activations in registers while it walks the rows of its CTA.
 //    Each CTA owns a contiguous range of rows (N split evenly over the SMs) and
@@ -56,12 +54,12 @@ namespace {
 constexpr int kSteps = 16;
 constexpr int kMaxWarps = 16;
 
-template <int BITS, int GS, int STEPS = kSteps>
+template <int BITS, int GS, int STEPS = (BITS == 8 ? kSteps / 2 : kSteps)>
 struct Shape {
     static constexpr int PER = 32 / BITS;                // codes per word
     static constexpr int GW = GS * BITS / 32;            // words per group
     static constexpr int LW = GW / 4 < 4 ? GW / 4 : 4;   // words per thread per row per chunk
-    static constexpr int MPW = BITS == 2 ? 4 : 2;       // MMAs per word
+    static constexpr int MPW = BITS == 2 ? 4 : BITS == 4 ? 2 : 1;  // MMAs per word
     static constexpr int NP = 2 * MPW;                   // fp16x2 registers per unpacked word
     static constexpr int CW = 4 * LW;                    // words per chunk (one lane quad)
     static constexpr int CK = CW * PER;                  // k per chunk
@@ -74,59 +72,88 @@ struct Shape {
     static_assert(CK <= GS && GS % CK == 0, "a chunk lies inside one group");
 };
 
-// Word -> NP bf16x2 registers of 128 + (code field); MMA u of the word uses
-// p[2u] (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). For register i:
-//   lo(i), hi(i)  the codes of the word behind its low and high halves;
-//   mul(i)        the factor of the activations in its slots (2^-p, or 2 for
-//                 the high nibble of an 8-bit code, held as 8 hi);
-//   sumw(i)       the A constant of the x-sum MMA: sum over slots of
-//                 sumw * mul * x counts every activation exactly once.
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// A group's scale and bias for one weight row, ready for the dequantizer:
+// (s, s) and (b, b) as bf16 pairs, s / 4 and s / 16 (2-bit fields held as
+// c * 4^j), and s, b as fp32 (8-bit codes).
+struct GroupSB {
+    uint32_t s2, b2, s2q, s2h;
+    float sf, bf;
+};
 template <int BITS>
-struct Unpack;
+__device__ __forceinline__ GroupSB group_sb(float sf, float bf) {
+    GroupSB g;
+    g.sf = sf;
+    g.bf = bf;
+    g.s2 = (__float_as_uint(sf) >> 16) * 0x00010001u;
+    g.b2 = (__float_as_uint(bf) >> 16) * 0x00010001u;
+    if constexpr (BITS == 2) {  // exact: powers of two (bf16 keeps s's 8 bits)
+        g.s2q = (__float_as_uint(sf * 0.25f) >> 16) * 0x00010001u;
+        g.s2h = (__float_as_uint(sf * 0.0625f) >> 16) * 0x00010001u;
+    } else {
+        g.s2q = g.s2h = 0u;
+    }
+    return g;
+}
+
+// Word -> NP bf16x2 registers of dequantized weights; MMA u of the word uses
+// p[2u] (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). lo(i), hi(i):
+// the codes of the word behind register i's low and high halves.
+template <int BITS>
+struct Dequant;
 
 template <>
-struct Unpack<4> {  // (c0,c4) (c1,c5)*8 (c2,c6) (c3,c7)*8
+struct Dequant<4> {  // (c0,c4) (c1,c5) (c2,c6) (c3,c7)
     __host__ __device__ static constexpr int lo(int i) { return i; }
     __host__ __device__ static constexpr int hi(int i) { return i + 4; }
-    __host__ __device__ static constexpr float mul(int i) { return (i & 1) ? 0.125f : 1.f; }
-    __host__ __device__ static constexpr float sumw(int i) { return (i & 1) ? 8.f : 1.f; }
-    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
-        p[0] = codes_to_bf16x2(w, 0x000F000Fu);
-        p[1] = codes_to_bf16x2(w >> 1, 0x00780078u);
-        p[2] = codes_to_bf16x2(w >> 8, 0x000F000Fu);
-        p[3] = codes_to_bf16x2(w >> 9, 0x00780078u);
+    __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            p[i] = bf2_fma(g.s2, bf2_sub(codes_to_bf16x2(w >> (4 * i), 0x000F000Fu), 0x43004300u), g.b2);
     }
 };
 
 template <>
-struct Unpack<8> {  // nibbles: (c0 lo, c2 lo) (c0 hi, c2 hi)*8 (c1 lo, c3 lo) (c1 hi, c3 hi)*8
-    __host__ __device__ static constexpr int lo(int i) { return i >> 1; }
-    __host__ __device__ static constexpr int hi(int i) { return (i >> 1) + 2; }
-    __host__ __device__ static constexpr float mul(int i) { return (i & 1) ? 2.f : 1.f; }
-    __host__ __device__ static constexpr float sumw(int i) { return (i & 1) ? 0.f : 1.f; }
-    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
-        Unpack<4>::run(w, p);  // the same fields: nibble j at bits 4j
-    }
-};
-
-template <>
-struct Unpack<2> {  // (c_i, c_i+8) * (1, 4, 16, 1, 4, 16, 1, 4)
+struct Dequant<2> {  // (c_i, c_i+8), fields held as c * (1, 4, 16, 1, 4, 16, 1, 4)
     __host__ __device__ static constexpr int lo(int i) { return i; }
     __host__ __device__ static constexpr int hi(int i) { return i + 8; }
-    __host__ __device__ static constexpr float sumw(int i) {
-        return static_cast<float>(1 << (2 * (i % 3)));
-    }
-    __host__ __device__ static constexpr float mul(int i) { return 1.f / sumw(i); }
-    __device__ static __forceinline__ void run(uint32_t w, uint32_t* p) {
+    __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
         const uint32_t v = w >> 6, u = w >> 12;
-        p[0] = codes_to_bf16x2(w, 0x00030003u);
-        p[1] = codes_to_bf16x2(w, 0x000C000Cu);
-        p[2] = codes_to_bf16x2(w, 0x00300030u);
-        p[3] = codes_to_bf16x2(v, 0x00030003u);
-        p[4] = codes_to_bf16x2(v, 0x000C000Cu);
-        p[5] = codes_to_bf16x2(v, 0x00300030u);
-        p[6] = codes_to_bf16x2(u, 0x00030003u);
-        p[7] = codes_to_bf16x2(u, 0x000C000Cu);
+        const uint32_t r[8] = {codes_to_bf16x2(w, 0x00030003u), codes_to_bf16x2(w, 0x000C000Cu),
+                               codes_to_bf16x2(w, 0x00300030u), codes_to_bf16x2(v, 0x00030003u),
+                               codes_to_bf16x2(v, 0x000C000Cu), codes_to_bf16x2(v, 0x00300030u),
+                               codes_to_bf16x2(u, 0x00030003u), codes_to_bf16x2(u, 0x000C000Cu)};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t s2 = (i % 3) == 0 ? g.s2 : (i % 3) == 1 ? g.s2q : g.s2h;
+            p[i] = bf2_fma(s2, bf2_sub(r[i], 0x43004300u), g.b2);
+        }
+    }
+};
+
+template <>
+struct Dequant<8> {  // (c0,c1) (c2,c3): fp32 s * c + b, converted once to bf16
+    __host__ __device__ static constexpr int lo(int i) { return 2 * i; }
+    __host__ __device__ static constexpr int hi(int i) { return 2 * i + 1; }
+    __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
+        float f[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // byte k under the mantissa of 2^23, minus 2^23: exact
+            const float c = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7640 | k)) - 8388608.0f;
+            f[k] = fmaf(g.sf, c, g.bf);
+        }
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[0]) : "f"(f[1]), "f"(f[0]));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[1]) : "f"(f[3]), "f"(f[2]));
     }
 };
 
@@ -138,19 +165,16 @@ __device__ __forceinline__ uint32_t f2_to_bf2x(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
-__device__ __forceinline__ uint32_t bf2_const(float v) { return f2_to_bf2x(v, v); }
 
-// The activations matching Unpack: b[u][0..1] for MMA u of a word whose first k
-// is k0, from xv = x[k0 .. k0 + PER) as bf16 pairs, times f (a power of two)
-// and the slot's factor: exact products of powers of two, exact in bf16.
+// The activations matching Dequant: b[u][0..1] for MMA u of a word whose first
+// k is k0, from xv = x[k0 .. k0 + PER) as bf16 pairs, times f (a power of
+// two: exact).
 template <int BITS>
 __device__ __forceinline__ void x_fragments(const uint32_t* xv, float f, uint32_t (*b)[2]) {
-    using U = Unpack<BITS>;
+    using D = Dequant<BITS>;
 #pragma unroll
-    for (int i = 0; i < 2 * (BITS == 2 ? 4 : 2); ++i) {
-        const float m = f * U::mul(i);
-        b[i >> 1][i & 1] = f2_to_bf2x(bf16_elem(xv, U::lo(i)) * m, bf16_elem(xv, U::hi(i)) * m);
-    }
+    for (int i = 0; i < 2 * (BITS == 2 ? 4 : BITS == 4 ? 2 : 1); ++i)
+        b[i >> 1][i & 1] = f2_to_bf2x(bf16_elem(xv, D::lo(i)) * f, bf16_elem(xv, D::hi(i)) * f);
 }
 
 __device__ __forceinline__ float group_value(const uint32_t* v, int i) {
@@ -474,28 +498,10 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         const float ef1 = __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
 
         uint32_t bfr[S::KS][S::MMAS][2];
-        float xoff[S::KS][2], xsum[S::KS][2];  // per chunk and column: 128-sum, sum of x
-        const uint32_t k128 = 0x43004300u;       // bf16x2 (128, 128)
 #pragma unroll
-        for (int q = 0; q < S::KS; ++q) {
+        for (int q = 0; q < S::KS; ++q)
 #pragma unroll
             for (int j = 0; j < S::LW; ++j) x_fragments<BITS>(xall[q][j], f, &bfr[q][j * S::MPW]);
-            float d1[4] = {0.f, 0.f, 0.f, 0.f}, d0[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int j = 0; j < S::LW; ++j)
-#pragma unroll
-                for (int u = 0; u < S::MPW; ++u) {
-                    const uint32_t* b2 = bfr[q][j * S::MPW + u];
-                    mma_bf16_16816(d1, k128, k128, k128, k128, b2[0], b2[1]);
-                    const uint32_t lo = bf2_const(Unpack<BITS>::sumw(2 * u));
-                    const uint32_t hi = bf2_const(Unpack<BITS>::sumw(2 * u + 1));
-                    mma_bf16_16816(d0, lo, lo, hi, hi, b2[0], b2[1]);
-                }
-            xoff[q][0] = d1[0];
-            xoff[q][1] = d1[1];
-            xsum[q][0] = d0[0];
-            xsum[q][1] = d0[1];
-        }
 
         const int oa = (g * RG::SBOX + goff) * 2, ob = ((g + 8) * RG::SBOX + goff) * 2;
         const int sbgmask = (1 << (prm.sbw_log - 1)) - 1;  // group columns per box - 1
@@ -557,32 +563,25 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
                 }
             }
 
+            // acc: rows g, g + 8 x activation rows 2t, 2t + 1 (the MMA's D fragment)
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < S::KS; ++q) {
                 uint32_t wa[S::LW], wb[S::LW];
                 lds_words<S::LW>(cst + offa[q], wa);
                 lds_words<S::LW>(cst + offb[q], wb);
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                const int gi = q / S::CPG;
+                const GroupSB gA = group_sb<BITS>(group_value(sa, gi), group_value(ba, gi));
+                const GroupSB gB = group_sb<BITS>(group_value(sb, gi), group_value(bb, gi));
 #pragma unroll
                 for (int j = 0; j < S::LW; ++j) {
                     uint32_t pa[S::NP], pb[S::NP];
-                    Unpack<BITS>::run(wa[j], pa);
-                    Unpack<BITS>::run(wb[j], pb);
+                    Dequant<BITS>::run(wa[j], gA, pa);
+                    Dequant<BITS>::run(wb[j], gB, pb);
 #pragma unroll
                     for (int u = 0; u < S::MPW; ++u)
-                        mma_bf16_16816(d, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
-                                      bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
-                }
-                const int gi = q / S::CPG;
-                const float s_a = group_value(sa, gi), s_b = group_value(sb, gi);
-                const float b_a = group_value(ba, gi), b_b = group_value(bb, gi);
-                // columns 2t (every call) and 2t + 1 (only when a second row exists)
-                acc[0] = fmaf(b_a, xsum[q][0], fmaf(s_a, d[0] - xoff[q][0], acc[0]));
-                acc[2] = fmaf(b_b, xsum[q][0], fmaf(s_b, d[2] - xoff[q][0], acc[2]));
-                if (!M1) {
-                    acc[1] = fmaf(b_a, xsum[q][1], fmaf(s_a, d[1] - xoff[q][1], acc[1]));
-                    acc[3] = fmaf(b_b, xsum[q][1], fmaf(s_b, d[3] - xoff[q][1], acc[3]));
+                        mma_bf16_16816(acc, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
+                                       bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
                 }
             }
             // every lane has read the stage: refill it with tile + NS
