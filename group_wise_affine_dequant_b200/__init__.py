@@ -14,6 +14,8 @@ from .binding import (  # noqa: F401
     nv_gather_qmm_flags,
     nv_gather_qmm_workspace_size,
     nv_dequantize_affine,
+    nv_moe_swiglu,
+    nv_moe_swiglu_workspace_size,
     nv_pipeline_error,
     nv_pipeline_selftest,
     nv_qmm,

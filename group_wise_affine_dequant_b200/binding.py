@@ -25,7 +25,7 @@ NV_FLAG_TOKEN_OUT_OF_RANGE = 0x4
 
 # Every entry point declared in include/nvq.h.
 EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_dequantize_affine", "nv_qmm",
-           "nv_qmm_batched", "nv_qmm_splits",
+           "nv_qmm_batched", "nv_qmm_splits", "nv_moe_swiglu", "nv_moe_swiglu_workspace_size",
            "nv_gather_qmm_workspace_size", "nv_gather_mm",
            "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_pipeline_selftest",
            "nv_last_cuda_error",
@@ -80,6 +80,11 @@ def lib():
             L.nv_gather_mm.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p, _i, _p,
                                        _sz, _p, _p]
             L.nv_gather_mm.restype = _i
+            L.nv_moe_swiglu_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64]
+            L.nv_moe_swiglu_workspace_size.restype = _sz
+            L.nv_moe_swiglu.argtypes = [_p, _i, _i64, _i64, _p, _p, _i, _i64, _i64, _p, _p, _p,
+                                        _p, _p, _p, _p, _p, _p, _i, _i, _p, _sz, _p, _p]
+            L.nv_moe_swiglu.restype = _i
             L.nv_gather_qmm_flags.argtypes = [_p, _p, _p]
             L.nv_gather_qmm_flags.restype = _i
             L.nv_gather_qmm_noalloc.argtypes = [_p, _i, _i64, _i64, _p, _p, _i64, _i64, _i64, _p,
@@ -316,6 +321,46 @@ def nv_gather_mm(x: torch.Tensor, w: torch.Tensor, rhs: torch.Tensor,
                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                             y.data_ptr(), _stream(stream))
     _check("nv_gather_mm", st)
+    return y
+
+
+def nv_moe_swiglu_workspace_size(T: int, topk: int, E: int, I: int, K: int) -> int:
+    return int(lib().nv_moe_swiglu_workspace_size(T, topk, E, I, K))
+
+
+def nv_moe_swiglu(x: torch.Tensor, gate, up, down, ids: torch.Tensor, rw: torch.Tensor,
+                  group_size: int = 64, bits: int = 4, workspace: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The routed SwiGLU block: y[t] = sum_j rw[t, j] down_e(silu(gate_e x[t]) *
+    up_e x[t]). gate, up: (codes, scales, biases) of [E, I, K] weights; down:
+    of [E, K, I]; ids int32 [T, topk]; rw fp32 [T, topk]. Returns y [T, K]."""
+    (gc, gsc, gb), (uc, usc, ub), (dc, dsc, db) = gate, up, down
+    for t, n in ((x, "x"), (gc, "gate codes"), (gsc, "gate scales"), (gb, "gate biases"),
+                 (uc, "up codes"), (usc, "up scales"), (ub, "up biases"), (dc, "down codes"),
+                 (dsc, "down scales"), (db, "down biases"), (ids, "ids"), (rw, "rw")):
+        _dev(t, n)
+    T, K = x.shape
+    E, I = gc.shape[0], gc.shape[1]
+    if tuple(gc.shape) != (E, I, K * bits // 32) or tuple(uc.shape) != tuple(gc.shape) or \
+            tuple(dc.shape) != (E, K, I * bits // 32):
+        raise ValueError("gate/up must be [E, I, K] and down [E, K, I] quantized weights")
+    if ids.dim() != 2 or ids.shape[0] != T or tuple(rw.shape) != tuple(ids.shape) or \
+            rw.dtype != torch.float32:
+        raise ValueError("ids [T, topk] and fp32 rw [T, topk] expected")
+    topk = ids.shape[1]
+    need = nv_moe_swiglu_workspace_size(T, topk, E, I, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    y = out if out is not None else torch.empty(T, K, dtype=x.dtype, device=x.device)
+    if y.numel() != T * K or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
+    st = lib().nv_moe_swiglu(x.data_ptr(), _DT.get(x.dtype, -1), T, K, ids.data_ptr(),
+                             rw.data_ptr(), topk, E, I, gc.data_ptr(), gsc.data_ptr(),
+                             gb.data_ptr(), uc.data_ptr(), usc.data_ptr(), ub.data_ptr(),
+                             dc.data_ptr(), dsc.data_ptr(), db.data_ptr(), group_size, bits,
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             y.data_ptr(), _stream(stream))
+    _check("nv_moe_swiglu", st)
     return y
 
 

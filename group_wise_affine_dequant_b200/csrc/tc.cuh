@@ -22,10 +22,13 @@ unsigned int tc_error_take();
 // 128-row operand, each expert's gathered activation rows as N). perm/offsets
 // come from the gather router.
 bool tc_gather_supported(int64_t K, int64_t N, int bits, int gs);
+// act_gate (nullable, bf16 [R, N]): store silu(act_gate) * product instead of
+// the product, over act_gate in place when y == act_gate.
 cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
                              const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
                              const uint32_t* codes, const void* scales, const void* biases, int gs,
-                             int bits, void* y, cudaStream_t stream, int num_sms);
+                             int bits, void* y, cudaStream_t stream, int num_sms,
+                             const void* act_gate = nullptr);
 unsigned int tc_gather_error_take();
 
 // The same grouped product with full-precision (bf16) experts [E, N, K].

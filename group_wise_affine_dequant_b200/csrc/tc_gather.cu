@@ -74,6 +74,10 @@ static_assert(2 * kAccCols + kDA * kACols <= static_cast<int>(kTmemCols), "TMEM 
 
 struct GParams {
     uint16_t* y;                // [R, N]
+    // nullable: gate values g [R, N] (bf16); the stored result is then
+    // silu(g) * (the product), the SwiGLU activation of a mixture-of-experts
+    // block, written over g in place
+    const uint16_t* act;
     const uint16_t* x;          // [x_rows, K]
     const uint32_t* lhs;        // nullable
     const uint32_t* perm;       // [R] pairs in expert order
@@ -314,9 +318,15 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
-                        if (c0 + j < cn && n < prm.N)
-                            prm.y[static_cast<int64_t>(pair) * prm.N + n] =
-                                f32_to_bf16_bits(__uint_as_float(v[j]));
+                        if (c0 + j < cn && n < prm.N) {
+                            const int64_t o = static_cast<int64_t>(pair) * prm.N + n;
+                            float val = __uint_as_float(v[j]);
+                            if (prm.act) {  // silu(g) * u = g / (1 + e^-g) * u
+                                const float gv = bf16_bits_to_f32(prm.act[o]);
+                                val = gv / (1.0f + expf(-gv)) * val;
+                            }
+                            prm.y[o] = f32_to_bf16_bits(val);
+                        }
                     }
                 }
                 tc_fence_before();
@@ -505,7 +515,8 @@ unsigned int tc_gather_error_take() { return pipeline_error_take(); }
 cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
                              const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
                              const uint32_t* codes, const void* scales, const void* biases, int gs,
-                             int bits, void* y, cudaStream_t stream, int num_sms) {
+                             int bits, void* y, cudaStream_t stream, int num_sms,
+                             const void* act_gate) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     if (x_rows * K >= (int64_t(1) << 35)) return cudaErrorInvalidValue;  // 32-bit 16-byte offsets
@@ -545,6 +556,7 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     }
     GParams prm{};
     prm.y = static_cast<uint16_t*>(y);
+    prm.act = static_cast<const uint16_t*>(act_gate);
     prm.x = static_cast<const uint16_t*>(x);
     prm.lhs = lhs;
     prm.perm = perm;

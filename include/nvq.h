@@ -218,6 +218,47 @@ nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
                        int64_t N, const void* w, int sorted, void* workspace,
                        size_t workspace_bytes, void* y, nv_stream_t stream);
 
+/* Bytes of device workspace nv_moe_swiglu needs for T tokens with topk
+ * experts each, E experts, hidden size I and model size K (0 for invalid
+ * sizes). */
+size_t nv_moe_swiglu_workspace_size(int64_t T, int64_t topk, int64_t E, int64_t I, int64_t K);
+
+/*
+ * The routed SwiGLU mixture-of-experts block over quantized experts
+ * ("Docs / Quantization", section "Mixture of experts": gather_qmm multiplies
+ * every row by its own expert's quantized weights without gathering them; the
+ * block around it is the gate and up products, silu(gate) * up, the down
+ * product, and the sum over each token's experts):
+ *   y[t] = sum_j rw[t, j] * down_e( silu(gate_e(x[t])) * up_e(x[t]) ),
+ *   e = ids[t, j], silu(z) = z / (1 + e^-z),
+ * in one routed pass: the pairs (t, j) are sorted by expert once, the gate
+ * and up products run on the grouped tensor-core kernel (the up product's
+ * epilogue applies silu(gate) * up), the down product runs on the pairs'
+ * hidden rows, and the combine sums each token's experts in j order (fp32,
+ * rounded once to bf16).
+ *
+ * x       bf16 [T, K]; ids uint32 [T, topk]; rw fp32 [T, topk] (routing weights).
+ * gate_*, up_*: quantized [E, I, K] (codes [E, I, K*bits/32], scales/biases
+ *   [E, I, K/group_size], grouped along K); down_*: quantized [E, K, I].
+ * y       bf16 [T, K] (output).
+ * workspace: >= nv_moe_swiglu_workspace_size(T, topk, E, I, K) bytes, 16-byte
+ *   aligned, caller-owned; it holds the routing tables and flags (the flags
+ *   first: nv_gather_qmm_flags(workspace, ...) reads them), the hidden rows
+ *   and the down products. Calls sharing a workspace must not overlap.
+ * An expert id >= E contributes nothing to y and sets NV_FLAG_EXPERT_OUT_OF_RANGE.
+ * dt must be NV_BF16, K and I multiples of 128 with (K / group_size) and
+ * (I / group_size) multiples of 8, 1 <= topk <= 64, E <= 1023
+ * (NV_ERR_UNSUPPORTED otherwise); bits in {2, 4, 8}. T == 0 is a no-op.
+ */
+nv_status nv_moe_swiglu(const void* x, nv_dtype dt, int64_t T, int64_t K, const uint32_t* ids,
+                        const float* rw, int topk, int64_t E, int64_t I,
+                        const uint32_t* gate_codes, const void* gate_scales,
+                        const void* gate_biases, const uint32_t* up_codes, const void* up_scales,
+                        const void* up_biases, const uint32_t* down_codes,
+                        const void* down_scales, const void* down_biases, int group_size,
+                        int bits, void* workspace, size_t workspace_bytes, void* y,
+                        nv_stream_t stream);
+
 /* Copy the anomaly flags of the last nv_gather_qmm (or nv_gather_mm) that used
  * `workspace` into *host_flags (a HOST pointer). Synchronises `stream`. */
 nv_status nv_gather_qmm_flags(const void* workspace, uint32_t* host_flags, nv_stream_t stream);

@@ -421,8 +421,16 @@ int orc_gather_mm(const void* x, int xdtype, int64_t x_rows, int64_t K, const ui
 //     y[t, n] += rw[t, j] * sum_i h_i * wd_hat[e, n, i]
 // Gate and up weights are [E, I, K] grouped along K, down weights [E, K, I]
 // grouped along I; all share one group size, width and scale dtype. fp64
-// throughout, sums in index order; a[t, n] = sum_j |rw| sum_i |h_i * wd_hat|.
-// Returns -1 on an out-of-range expert id or a bad quantization.
+// throughout, sums in index order. Out-of-range expert ids are skipped (they
+// contribute nothing), so a caller can state them.
+// a[t, n] is the scale of the block's tolerance: the product tolerance
+// carried to first order through h = silu(g) * u, each term doubled for the
+// rounding of the intermediate g and h to the activations' dtype:
+//   a[t, n] = sum_j |rw| sum_i |wd_hat[e, n, i]| *
+//             2 (|h_i| + |silu'(g_i) u_i| a_g,i + |silu(g_i)| a_u,i),
+// with a_g,i = sum_k |x_k wg_hat[e, i, k]|, a_u,i likewise, and
+// silu'(z) = s(z) (1 + z (1 - s(z))), s(z) = 1 / (1 + exp(-z)).
+// Returns -1 on a bad quantization.
 int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32_t* ids,
                    const float* rw, int topk, int64_t E, int64_t I,
                    const uint32_t* g_codes, const void* g_scales, const void* g_biases,
@@ -430,8 +438,6 @@ int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32
                    const uint32_t* d_codes, const void* d_scales, const void* d_biases,
                    int sdtype, int gs, int bits, double* y, double* a) {
     if (!valid_quant(K, gs, bits) || !valid_quant(I, gs, bits) || topk < 1) return -1;
-    for (int64_t i = 0; i < T * topk; ++i)
-        if ((int64_t)ids[i] >= E) return -1;
     const size_t sz = sdtype == DT_F32 ? 4 : 2;
     const int64_t gu_words = I * K * bits / 32, gu_groups = I * K / gs;   // per expert
     const int64_t d_words = K * I * bits / 32, d_groups = K * I / gs;
@@ -441,8 +447,10 @@ int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32
         double* at = a + t * K;
         for (int64_t n = 0; n < K; ++n) { yt[n] = 0.0; at[n] = 0.0; }
         double* h = new double[I];
+        double* eh = new double[I];  // error scale of h_i
         for (int j = 0; j < topk; ++j) {
             const int64_t e = (int64_t)ids[t * topk + j];
+            if (e >= E) continue;
             const double w = (double)rw[t * topk + j];
             const uint32_t* gc = g_codes + e * gu_words;
             const uint32_t* uc = u_codes + e * gu_words;
@@ -451,13 +459,20 @@ int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32
             const char* usc = (const char*)u_scales + (size_t)(e * gu_groups) * sz;
             const char* ubi = (const char*)u_biases + (size_t)(e * gu_groups) * sz;
             for (int64_t i = 0; i < I; ++i) {
-                double g = 0.0, u = 0.0;
+                double g = 0.0, u = 0.0, ag = 0.0, au = 0.0;
                 for (int64_t k = 0; k < K; ++k) {
                     const double xv = load_value(x, xdtype, t * K + k);
-                    g += xv * dequant_at(gc, gsc, gbi, sdtype, i, k, K, gs, bits);
-                    u += xv * dequant_at(uc, usc, ubi, sdtype, i, k, K, gs, bits);
+                    const double pg = xv * dequant_at(gc, gsc, gbi, sdtype, i, k, K, gs, bits);
+                    const double pu = xv * dequant_at(uc, usc, ubi, sdtype, i, k, K, gs, bits);
+                    g += pg;
+                    u += pu;
+                    ag += std::fabs(pg);
+                    au += std::fabs(pu);
                 }
                 h[i] = g / (1.0 + std::exp(-g)) * u;
+                const double sg = 1.0 / (1.0 + std::exp(-g));
+                const double dsilu = sg * (1.0 + g * (1.0 - sg));
+                eh[i] = 2.0 * (std::fabs(h[i]) + std::fabs(dsilu * u) * ag + std::fabs(g * sg) * au);
             }
             const uint32_t* dc = d_codes + e * d_words;
             const char* dsc = (const char*)d_scales + (size_t)(e * d_groups) * sz;
@@ -465,15 +480,16 @@ int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32
             for (int64_t n = 0; n < K; ++n) {
                 double acc = 0.0, mag = 0.0;
                 for (int64_t i = 0; i < I; ++i) {
-                    const double p = h[i] * dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits);
-                    acc += p;
-                    mag += std::fabs(p);
+                    const double wd = dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits);
+                    acc += h[i] * wd;
+                    mag += std::fabs(wd) * eh[i];
                 }
                 yt[n] += w * acc;
                 at[n] += std::fabs(w) * mag;
             }
         }
         delete[] h;
+        delete[] eh;
     }
     return 0;
 }

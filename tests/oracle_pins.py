@@ -478,12 +478,64 @@ def pin_moe_swiglu(lib):
     assert torch.equal(y2, 2 * yp), "routing weights scale the output"
     ys, _ = O.moe_swiglu(x, G, U, D, ids.flip(1), rw.flip(1), gs, bits, lib=lib)
     assert (ys - yp).abs().le(tol).all(), "top-k order"
-    try:
-        O.moe_swiglu(x, G, U, D, torch.full((T, top), E), rw, gs, bits, lib=lib)
-    except ValueError:
-        pass
-    else:
-        raise AssertionError("expert id E accepted")
+    # an expert id out of range contributes nothing (as a zero routing weight)
+    bad = ids.clone()
+    bad[:, 1] = E
+    rw0 = rw.clone()
+    rw0[:, 1] = 0
+    yb, _ = O.moe_swiglu(x, G, U, D, bad, rw, gs, bits, lib=lib)
+    y0w, _ = O.moe_swiglu(x, G, U, D, ids, rw0, gs, bits, lib=lib)
+    assert (yb - y0w).abs().le(tol).all(), "out-of-range expert"
+
+
+def pin_moe_swiglu_tolerance_scale(lib):
+    """The block's tolerance scale carries each product's sum |x w_hat| through
+    h = silu(g) * u: a = sum_j |rw| sum_i |wd| 2 (|h| + |silu'(g) u| a_g +
+    |silu(g)| a_u). Two cases where h = 0 exactly but the products do not
+    vanish term by term (x = (1, 1, 0, ...); weights +1 and -1 as codes 2 and 0
+    with scale 1, bias -1):
+    * gate rows (1, -1, ...): g = 0, a_g = 2, silu'(0) = 1/2, so
+      a[n] = 2 |rw| sum_i |wd_ni| |u_i| (an exact integer) and y = 0;
+    * up rows (1, -1, ...) and gate rows (2, 0, ...) (codes 3, 1 with bias -1):
+      u = 0, a_u = 2, g = 2, so a[n] = 2 |rw| sum_i |wd_ni| silu(2) 2 with
+      silu(2) = 2 / (1 + e^-2)."""
+    g = torch.Generator().manual_seed(54)
+    E, I, K, T, top, gs, bits = 2, 32, 32, 1, 1, 32, 4
+    x = torch.zeros(T, K, dtype=torch.bfloat16)
+    x[0, 0] = 1.0
+    x[0, 1] = 1.0
+    pm = torch.zeros(E, I, K, dtype=torch.int64)
+    pm[:, :, 0], pm[:, :, 1] = 2, 0                 # w_hat = code - 1: +1, -1, then -1 ...
+    Uc = torch.randint(1, 16, (E, I, K), generator=g)
+    Dc = torch.randint(0, 16, (E, K, I), generator=g)
+    ids = torch.tensor([[1]])
+    rw = torch.tensor([[-3.0]])
+    one = lambda shape, v: torch.full(shape, float(v), dtype=torch.bfloat16)  # noqa: E731
+    q = lambda c, b: (_pack_codes(c, bits), one((*c.shape[:-1], c.shape[-1] // gs), 1),  # noqa: E731
+                      one((*c.shape[:-1], c.shape[-1] // gs), b))
+    y, a = O.moe_swiglu(x, q(pm, -1), q(Uc, 0), q(Dc, 0), ids, rw, gs, bits, lib=lib)
+    u = Uc[1, :, 0] + Uc[1, :, 1]                    # x . w_up, exact integers
+    want = 2 * 3 * (Dc[1] @ u)
+    assert (y == 0).all(), "zero gate gives zero"
+    assert torch.equal(a[0], want.to(torch.float64)), (a[0], want)
+    gc = pm.clone()
+    gc[:, :, 0], gc[:, :, 1] = 3, 1                  # w_hat = code - 1: 2, 0, so g = 2
+    y2, a2 = O.moe_swiglu(x, q(gc, -1), q(pm, -1), q(Dc, 0), ids, rw, gs, bits, lib=lib)
+    silu2 = 2.0 / (1.0 + math.exp(-2.0))
+    want2 = 2 * 3 * Dc[1].sum(1).to(torch.float64) * silu2 * 2
+    assert (y2 == 0).all(), "zero up gives zero"
+    assert (a2[0] - want2).abs().le(1e-12 * want2).all(), (a2[0], want2)
+    # g = 2 and u = 2 (up weights +1, +1): every term counts, the slope
+    # silu'(2) = s(2) (1 + 2 (1 - s(2))) with s(2) = 1 / (1 + e^-2)
+    uc = torch.zeros(E, I, K, dtype=torch.int64)
+    uc[:, :, 0], uc[:, :, 1] = 1, 1
+    y3, a3 = O.moe_swiglu(x, q(gc, -1), q(uc, 0), q(Dc, 0), ids, rw, gs, bits, lib=lib)
+    s2 = 1.0 / (1.0 + math.exp(-2.0))
+    slope2 = s2 * (1.0 + 2.0 * (1.0 - s2))
+    h = silu2 * 2.0
+    want3 = 2 * 3 * Dc[1].sum(1).to(torch.float64) * (h + slope2 * 2.0 * 2.0 + silu2 * 2.0)
+    assert (y3[0] - (-3.0) * Dc[1].sum(1).to(torch.float64) * h).abs().le(1e-9).all()
+    assert (a3[0] - want3).abs().le(1e-12 * want3).all(), (a3[0], want3)
 
 
 def pin_sampled_match_full(lib):

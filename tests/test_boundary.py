@@ -208,3 +208,32 @@ def test_batched_argument_errors():
     assert call(B=1 << 30, L=1 << 20) == B.NV_ERR_INVALID_ARG
     assert call(B=0) == B.NV_OK
     assert call(N=0) == B.NV_OK
+
+
+def test_moe_swiglu_argument_errors():
+    L = nvq.lib()
+    T, topk, E, I, K = 8, 2, 4, 512, 512
+    need = L.nv_moe_swiglu_workspace_size(T, topk, E, I, K)
+    assert need > 0 and L.nv_moe_swiglu_workspace_size(T, 0, E, I, K) == 0
+
+    def call(ws=16, ws_bytes=need, **kw):
+        a = dict(x=16, dt=1, T=T, K=K, ids=16, rw=16, topk=topk, E=E, I=I, gs=64, bits=4, y=16)
+        a.update(kw)
+        p = 16
+        return L.nv_moe_swiglu(a["x"], a["dt"], a["T"], a["K"], a["ids"], a["rw"], a["topk"],
+                               a["E"], a["I"], p, p, p, p, p, p, p, p, p, a["gs"], a["bits"],
+                               ws, ws_bytes, a["y"], None)
+
+    assert call(ws_bytes=need - 1) == B.NV_ERR_WORKSPACE
+    assert call(ws=0) == B.NV_ERR_WORKSPACE
+    assert call(dt=0) == B.NV_ERR_UNSUPPORTED        # fp32 activations: not implemented
+    assert call(bits=3) == B.NV_ERR_UNSUPPORTED
+    assert call(bits=7) == B.NV_ERR_INVALID_ARG
+    assert call(K=320) == B.NV_ERR_UNSUPPORTED       # K not a multiple of 128
+    assert call(I=96) == B.NV_ERR_INVALID_ARG        # I not a multiple of the group size
+    assert call(I=256) == B.NV_ERR_UNSUPPORTED       # I / group_size not a multiple of 8
+    assert call(topk=0) == B.NV_ERR_INVALID_ARG
+    assert call(E=5000) == B.NV_ERR_UNSUPPORTED
+    assert call(x=0) == B.NV_ERR_INVALID_ARG
+    assert call(rw=8) == B.NV_ERR_INVALID_ARG        # misaligned
+    assert call(T=0) == B.NV_OK

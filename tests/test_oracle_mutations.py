@@ -62,6 +62,12 @@ MUTANTS = [
      "const double v = (double)(float)(p + load_value(biases, sdtype, g));"),
     ("stored value rounded through fp64", "if (err == 0.0 || !std::isfinite(sum)) return sum;",
      "return sum;"),
+    ("tolerance drops the gate term", "std::fabs(dsilu * u) * ag", "0.0 * ag"),
+    ("tolerance drops the up term", "std::fabs(g * sg) * au", "0.0 * au"),
+    ("tolerance silu slope", "const double dsilu = sg * (1.0 + g * (1.0 - sg));",
+     "const double dsilu = sg;"),
+    ("out-of-range expert kept", "const int64_t e = (int64_t)ids[t * topk + j];",
+     "const int64_t e = (int64_t)ids[t * topk + j] % E;"),
     ("down transposed", "dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits)",
      "dequant_at(dc, dsc, dbi, sdtype, i, n, K, gs, bits)"),
 ]
