@@ -423,6 +423,74 @@ class Gather:
             self.call(j)
 
 
+class MoeBlock:
+    """The routed SwiGLU block: 64 experts, gate/up [1536, 2048] and down
+    [2048, 1536] 4-bit g64, 512 tokens x top-4 (uniform without replacement),
+    normalized uniform routing weights."""
+
+    def __init__(self, dev):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        m = W.MOE
+        self.E, self.I, self.K, self.T, self.top = m["E"], m["N"], m["K"], m["tokens"], m["top_k"]
+        qs = []
+        for seed, shape in ((0, (self.E, self.I, self.K)), (3, (self.E, self.I, self.K)),
+                            (4, (self.E, self.K, self.I))):
+            w = W.normal(shape, 0.02, seed, "bf16").to(dev)
+            qs.append(nvq.nv_quantize_affine(w, 64, 4))
+            del w
+        wbytes = 3 * qbytes(self.E * self.I, self.K, 4, 64)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))
+        self.ws = [tuple(tuple(t.clone() for t in q) for q in qs) for _ in range(self.copies)]
+        self.ids = W.expert_ids(self.T, self.E, self.top, 2).to(torch.int32).to(dev)
+        g = torch.Generator().manual_seed(6)
+        rw = torch.rand(self.T, self.top, generator=g)
+        self.rw = (rw / rw.sum(1, keepdim=True)).to(torch.float32).to(dev)
+        self.x = W.normal((self.T, self.K), 1.0, 1, "bf16").to(dev)
+        self.y = torch.empty(self.T, self.K, dtype=torch.bfloat16, device=dev)
+        self.wsp = torch.empty(nvq.nv_moe_swiglu_workspace_size(self.T, self.top, self.E, self.I,
+                                                                self.K),
+                               dtype=torch.uint8, device=dev)
+        self.bytes = wbytes + 2 * self.T * self.K * 2 + self.T * self.top * 8
+
+    def call(self, j):
+        gate, up, down = self.ws[j]
+        self.nvq.nv_moe_swiglu(self.x, gate, up, down, self.ids, self.rw, 64, 4,
+                               workspace=self.wsp, out=self.y)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
+
+
+def check_moe(wl, tokens=8):
+    """A few tokens' outputs against the block in plain torch arithmetic (fp32,
+    codes unpacked by shifts and masks)."""
+    gate, up, down = wl.ws[0]
+    worst = 0.0
+    for t in range(tokens):
+        x = wl.x[t:t + 1].float()
+        acc = torch.zeros(1, wl.K, device=x.device)
+        mag = torch.zeros(1, wl.K, device=x.device)
+        for j in range(wl.top):
+            e = int(wl.ids[t, j])
+            wg = unpack_dequant(gate[0][e], gate[1][e], gate[2][e], 64, 4)
+            wu = unpack_dequant(up[0][e], up[1][e], up[2][e], 64, 4)
+            wd = unpack_dequant(down[0][e], down[1][e], down[2][e], 64, 4)
+            g, u = x @ wg.T, x @ wu.T
+            ag, au = x.abs() @ wg.abs().T, x.abs() @ wu.abs().T
+            sg = torch.sigmoid(g)
+            h = g * sg * u
+            # the product tolerance carried through silu(g) * u (as the oracle's)
+            eh = 2 * (h.abs() + (sg * (1 + g * (1 - sg)) * u).abs() * ag + (g * sg).abs() * au)
+            acc += float(wl.rw[t, j]) * (h @ wd.T)
+            mag += abs(float(wl.rw[t, j])) * (eh @ wd.abs().T)
+        tol = 4e-3 * mag + 1e-5
+        worst = max(worst, float(((wl.y[t:t + 1].float() - acc).abs() / tol).max()))
+    return worst
+
+
 # --------------------------------------------------------------------------- arms
 def run_nvq(args):
     import torch.distributed as dist
@@ -514,6 +582,15 @@ def run_nvq(args):
         also[name + "_gbs"] = round(replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9, 1)
         checks[name] = round(chk(check_gather, wl), 4)
         del g, wl
+    wl = MoeBlock(dev)
+    g = timed_graph(wl.step, ks, Wm, stream)
+    t = max_ms(replay_timed(g, stream, barrier))
+    also["moe_swiglu_tok_s"] = round(replica_rate(ws, wl.T * wl.copies, ks, t), 1)
+    mb = replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9
+    also["moe_swiglu_gbs"] = round(mb, 1)
+    also["moe_swiglu_frac_of_hbm"] = round(mb / ws / pk["hbm_gbs"], 4)
+    checks["moe_swiglu"] = round(chk(check_moe, wl), 4)
+    del g, wl
     wl = GatherMM(dev)
     g = timed_graph(wl.step, ks, Wm, stream)
     t = max_ms(replay_timed(g, stream, barrier))
@@ -666,6 +743,7 @@ PROFILE_WORKLOADS = {
     "prefill8": lambda dev: Decode(dev, N=14336, K=4096, M=2048, bits=8, gs=64),
     "dequant": lambda dev: Dequant(dev),
     "gather_mm": lambda dev: GatherMM(dev),
+    "moe": lambda dev: MoeBlock(dev),
 }
 
 

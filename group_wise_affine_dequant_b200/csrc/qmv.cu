@@ -146,14 +146,21 @@ struct Dequant<8> {  // (c0,c1) (c2,c3): fp32 s * c + b, converted once to bf16
     __host__ __device__ static constexpr int lo(int i) { return 2 * i; }
     __host__ __device__ static constexpr int hi(int i) { return 2 * i + 1; }
     __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
-        float f[4];
+        // packed fp32 pairs: byte k under the mantissa of 2^23 is 2^23 + c_k;
+        // one fma removes the 2^23 (exact), one applies scale and bias
+        const uint64_t one = 0x3F8000003F800000ull, off = 0xCB000000CB000000ull;
+        const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(g.sf)) << 32) | __float_as_uint(g.sf);
+        const uint64_t b2 = (static_cast<uint64_t>(__float_as_uint(g.bf)) << 32) | __float_as_uint(g.bf);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {  // byte k under the mantissa of 2^23, minus 2^23: exact
-            const float c = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7640 | k)) - 8388608.0f;
-            f[k] = fmaf(g.sf, c, g.bf);
+        for (int i = 0; i < 2; ++i) {
+            const uint64_t r = (static_cast<uint64_t>(__byte_perm(w, 0x4B000000u, 0x7640 | (2 * i + 1))) << 32) |
+                               __byte_perm(w, 0x4B000000u, 0x7640 | (2 * i));
+            uint64_t c, f;
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(c) : "l"(r), "l"(one), "l"(off));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f) : "l"(s2), "l"(c), "l"(b2));
+            asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+                : "=r"(p[i]) : "l"(f));
         }
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[0]) : "f"(f[1]), "f"(f[0]));
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[1]) : "f"(f[3]), "f"(f[2]));
     }
 };
 
@@ -285,6 +292,22 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     const int64_t N = prm.N, K = prm.K;
     const int64_t gpr = K / GS;  // groups per row
 
+    // shared memory: [warps][NS] code stages | scale+bias block (mode 2) or
+    // [warps][NS] scale+bias stages (mode 1) | [warps][NS] + 1 mbarriers |
+    // slice partials
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.off_bar);
+    uint64_t* full = bars + warp * NS;
+    uint64_t* sb_full = bars + nwarps * NS;
+    // The barriers live in this CTA's shared memory only, so they are set up
+    // before the wait for the previous kernel (made visible by the barrier
+    // below, before any use).
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+        if (warp == 0) mbar_init(sb_full, 1);
+        mbar_init_fence();
+    }
+
     int M;
     const uint16_t* scales = prm.scales;
     const uint16_t* biases = prm.biases;
@@ -367,25 +390,12 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         return;
     }
 
-    // shared memory: [warps][NS] code stages | scale+bias block (mode 2) or
-    // [warps][NS] scale+bias stages (mode 1) | [warps][NS] + 1 mbarriers |
-    // slice partials
-    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const int sb_mode = prm.sb_mode;
     uint8_t* code_ring = smem + static_cast<size_t>(warp) * NS * RG::CODE_STAGE;
     uint8_t* sb_base = smem + prm.off_sb;
     uint8_t* sb_ring = sb_base + static_cast<size_t>(warp) * NS * 2 * RG::SB_STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.off_bar);
-    uint64_t* full = bars + warp * NS;
-    uint64_t* sb_full = bars + nwarps * NS;
     float* red = reinterpret_cast<float*>(smem + prm.off_red);
 
-    if (lane == 0) {
-        for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
-        if (warp == 0) mbar_init(sb_full, 1);
-        mbar_init_fence();
-    }
-    __syncthreads();
     if (sb_mode == 2 && warp == 0 && elect_one()) {
         // the CTA's scales and biases: rows [n0, n0 + rows_max), all groups
         const uint32_t box = static_cast<uint32_t>(prm.rows_max) << prm.sbw_log;
@@ -424,6 +434,37 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         const int goff = g0 - gbox;                 // slice's first group in the box
         const int cword = kslice0 * BITS / 32;
 
+        // ---- activations of this slice, loaded before the weight copies are
+        // issued (so that these few loads do not queue behind the stream) ----
+        uint32_t xall[S::KS][S::LW][S::PER / 2];
+#pragma unroll
+        for (int q = 0; q < S::KS; ++q) {
+            const int64_t kq = static_cast<int64_t>(kslice0) + q * S::CK;
+            const bool valid = kq < K && g < M;
+#pragma unroll
+            for (int j = 0; j < S::LW; ++j) {
+                const int64_t k0 = kq + (t * S::LW + j) * S::PER;
+                uint32_t* xv = xall[q][j];
+                if (valid) {
+                    const uint16_t* xp = prm.x + s_xrow[g] * K + k0;
+                    if constexpr (S::PER == 4) {
+                        uint2 v = __ldg(reinterpret_cast<const uint2*>(xp));
+                        xv[0] = v.x; xv[1] = v.y;
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < S::PER / 8; ++h) {
+                            uint4 v = __ldg(reinterpret_cast<const uint4*>(xp) + h);
+                            xv[4 * h] = v.x; xv[4 * h + 1] = v.y;
+                            xv[4 * h + 2] = v.z; xv[4 * h + 3] = v.w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < S::PER / 2; ++h) xv[h] = 0u;
+                }
+            }
+        }
+
         // one lane: copy tile `tile` of this slice into ring stage `s`
         auto issue = [&](int tile, int s) {
             uint64_t* bar = &full[s];
@@ -450,41 +491,16 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
             }
         }
 
-        // ---- activations of this slice: B fragments and per-chunk sums ----
-        uint32_t xall[S::KS][S::LW][S::PER / 2];
         float xmax = 0.f;  // largest |x| of this lane's part of the slice
 #pragma unroll
-        for (int q = 0; q < S::KS; ++q) {
-            const int64_t kq = static_cast<int64_t>(kslice0) + q * S::CK;
-            const bool valid = kq < K && g < M;
+        for (int q = 0; q < S::KS; ++q)
 #pragma unroll
-            for (int j = 0; j < S::LW; ++j) {
-                const int64_t k0 = kq + (t * S::LW + j) * S::PER;
-                uint32_t* xv = xall[q][j];
-                if (valid) {
-                    const uint16_t* xp = prm.x + s_xrow[g] * K + k0;
-                    if constexpr (S::PER == 4) {
-                        uint2 v = __ldg(reinterpret_cast<const uint2*>(xp));
-                        xv[0] = v.x; xv[1] = v.y;
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < S::PER / 8; ++h) {
-                            uint4 v = __ldg(reinterpret_cast<const uint4*>(xp) + h);
-                            xv[4 * h] = v.x; xv[4 * h + 1] = v.y;
-                            xv[4 * h + 2] = v.z; xv[4 * h + 3] = v.w;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < S::PER / 2; ++h) xv[h] = 0u;
-                }
+            for (int j = 0; j < S::LW; ++j)
 #pragma unroll
                 for (int h = 0; h < S::PER / 2; ++h) {
-                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xv[h] << 16)));
-                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xv[h] & 0xFFFF0000u)));
+                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xall[q][j][h] << 16)));
+                    xmax = fmaxf(xmax, fabsf(__uint_as_float(xall[q][j][h] & 0xFFFF0000u)));
                 }
-            }
-        }
         // per activation row (lane quad g): a slice whose largest |x| reaches
         // 2^100 is brought below 2^101 by 2^-es (exact); the rest keep es = 0
         xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 1));

@@ -168,17 +168,39 @@ struct Dequant<2> {  // word: 16 codes -> 8 pairs
     }
 };
 
+// Packed fp32 pairs (sm_100a): d = a * b + c on both halves, one rounding each.
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+// (lo, hi) fp32 pair -> bf16x2, round to nearest even.
+__device__ __forceinline__ uint32_t f2_to_bf2_packed(uint64_t v) {
+    uint32_t d;
+    asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(d) : "l"(v));
+    return d;
+}
+
 template <>
-struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes
+struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes in packed pairs
     static constexpr int PAIRS = 2;
     __device__ static __forceinline__ void run(uint32_t w, uint32_t, uint32_t, float s, float b,
                                                uint32_t, uint32_t, uint32_t, uint32_t* out) {
-        const uint32_t magic = 0x4B000000u;  // 2^23: byte i -> 2^23 + c_i
+        const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);   // (1, 1)
+        const uint64_t off = f2_pack(0xCB000000u, 0xCB000000u);     // (-2^23, -2^23)
+        const uint64_t s2 = f2_pack(__float_as_uint(s), __float_as_uint(s));
+        const uint64_t b2 = f2_pack(__float_as_uint(b), __float_as_uint(b));
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            const float c0 = __uint_as_float(prmt(w, magic, (2 * i) | 0x7440)) - 8388608.0f;
-            const float c1 = __uint_as_float(prmt(w, magic, (2 * i + 1) | 0x7440)) - 8388608.0f;
-            out[i] = f2_to_bf2(fmaf(s, c0, b), fmaf(s, c1, b));
+            // bytes 2i, 2i + 1 under the mantissa of 2^23: 2^23 + c, exact
+            const uint64_t r = f2_pack(prmt(w, 0x4B000000u, (2 * i) | 0x7440),
+                                       prmt(w, 0x4B000000u, (2 * i + 1) | 0x7440));
+            const uint64_t c = f2_fma(r, one_m, off);                  // c, exact
+            out[i] = f2_to_bf2_packed(f2_fma(s2, c, b2));              // s * c + b
         }
     }
 };

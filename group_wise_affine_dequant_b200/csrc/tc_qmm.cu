@@ -87,10 +87,19 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t local_addr, uint32_t ra
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
     return v;
+}
+// Byte offset of columns [4 c, 4 c + 4) of row r in a [128][bn] fp32 partial
+// tile whose 16-byte chunks are XOR-swizzled by (row mod 8): the epilogue's
+// stores (one row per lane) and the reduction's loads hit distinct banks.
+__device__ __forceinline__ uint32_t part_off(int r, int c, int bn) {
+    return static_cast<uint32_t>(r * bn * 4 + ((c ^ (r & 7)) << 4));
 }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -248,9 +257,9 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             if (!mbar_wait_backoff(&acc_full[a], ause & 1, 5, 2048)) break;
             tc_fence_after();
             if constexpr (SPLIT) {
-                // the partial tile into this CTA's shared memory, [row][BN + 1]
-                // fp32 (the pipeline's stages are all consumed by now)
-                float* part = reinterpret_cast<float*>(smem) + row_in_tile * (BN + 1);
+                // the partial tile into this CTA's shared memory, [row][BN] fp32
+                // with swizzled 16-byte chunks (the pipeline's stages are all
+                // consumed by now)
                 for (int j = 0; j < BN / 32; ++j) {
                     uint32_t v[32];
                     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -268,7 +277,9 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                         : "r"(taddr));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) part[j * 32 + e] = __uint_as_float(v[e]);
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(smem + part_off(row_in_tile, j * 8 + c, BN)) =
+                            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                 }
                 tc_fence_before();
                 continue;
@@ -402,21 +413,35 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     __syncthreads();
     if constexpr (SPLIT) {
         // Sum the cluster's S partial tiles in rank order: CTA `rank` owns rows
-        // [rank * 128 / S, (rank + 1) * 128 / S); a warp takes a row, its lanes
-        // 32 consecutive columns.
+        // [rank * 128 / S, (rank + 1) * 128 / S); a thread takes 4 columns of a
+        // row, loads them from all S partials (16-byte loads, all in flight)
+        // and adds them in order 0, 1, ..., S - 1.
         cluster_sync();
         const int mt = tile0 % prm.m_tiles, nt = tile0 / prm.m_tiles;
         const int r_lo = rank * BM / S, r_hi = (rank + 1) * BM / S;
         const uint32_t part0 = smem_u32(smem);
-        for (int r = r_lo + warp; r < r_hi; r += kThreads / 32) {
+        const int chunks = BN / 4;
+        for (int i = threadIdx.x; i < (r_hi - r_lo) * chunks; i += kThreads) {
+            const int r = r_lo + i / chunks, c = i % chunks;
             const int64_t row = static_cast<int64_t>(mt) * BM + r;
-            if (row >= prm.M) break;
-            for (int c = lane; c < BN; c += 32) {
-                const int64_t col = static_cast<int64_t>(nt) * BN + c;
-                const uint32_t off = static_cast<uint32_t>((r * (BN + 1) + c) * 4);
-                float acc = ld_cluster_f32(cluster_map(part0 + off, 0));
-                for (int src = 1; src < S; ++src) acc += ld_cluster_f32(cluster_map(part0 + off, src));
-                if (col < prm.N) prm.y[row * prm.N + col] = f32_to_bf16_bits(acc);
+            if (row >= prm.M) continue;
+            const uint32_t off = part0 + part_off(r, c, BN);
+            float4 v[8];
+#pragma unroll
+            for (int src = 0; src < 8; ++src)
+                if (src < S) v[src] = ld_cluster_f32x4(cluster_map(off, src));
+            float4 acc = v[0];
+#pragma unroll
+            for (int src = 1; src < 8; ++src)
+                if (src < S) { acc.x += v[src].x; acc.y += v[src].y; acc.z += v[src].z; acc.w += v[src].w; }
+            const int64_t col = static_cast<int64_t>(nt) * BN + 4 * c;
+            uint16_t* yp = prm.y + row * prm.N + col;
+            const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+            if (col + 4 <= prm.N && (prm.N % 4) == 0) {
+                *reinterpret_cast<uint2*>(yp) = make_uint2(f2_to_bf2(a4[0], a4[1]), f2_to_bf2(a4[2], a4[3]));
+            } else {
+                for (int e = 0; e < 4; ++e)
+                    if (col + e < prm.N) yp[e] = f32_to_bf16_bits(a4[e]);
             }
         }
         cluster_sync();  // no CTA leaves while the others still read its partial
@@ -453,23 +478,67 @@ struct TcPlan {
     int bn, splits;
 };
 
+// Clusters of `size` CTAs (one CTA per SM) that the device runs at once: a
+// property of the device's GPC layout (e.g. 74, 33 and 15 clusters of 2, 4
+// and 8 on a 148-SM B200), queried once per device and size.
+int max_clusters(int size) {
+    static int cache[64][4] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int slot = size == 2 ? 0 : size == 4 ? 1 : size == 8 ? 2 : 3;
+    if (cache[dev][slot] > 0) return cache[dev][slot];
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(size), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 160 * 1024;  // > half an SM: one CTA per SM, as every plan here
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(size);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+              const TcParams) = tc_qmm_kernel<4, true>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(cfg.dynamicSmemBytes)) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(k), &cfg) != cudaSuccess ||
+        n <= 0) {
+        cudaGetLastError();  // clear a failed query; assume one cluster per 8 SMs
+        n = 148 / (size * 2);
+    }
+    cache[dev][slot] = n;
+    return n;
+}
+
+// The tiling and split-K plan for an item of m_rows rows: with the unsplit
+// tiles filling at least half the SMs (or fewer than 8 k-steps), no split;
+// otherwise the (tile width bn, cluster size S in {2, 4, 8}) of least
+// estimated time, counting waves of co-resident clusters, k-steps per CTA and
+// a per-step time that grows with bn (measured on B200: about 0.5 us per
+// 64-k step at bn 64, 0.8 at bn 256, plus about 8 us of fixed cost per CTA).
+// A pure function of (rows, N, K) and the device.
+double tc_cost(int64_t waves, int64_t steps, int bn) {
+    return static_cast<double>(waves) * (static_cast<double>(steps) * (0.45 + 0.0013 * bn) + 8.0);
+}
+
 TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms) {
     const int bn0 = pick_bn(m_rows, N, num_sms);
     const int64_t mt = (m_rows + BM - 1) / BM;
     const int64_t ks = K / BK;
-    if (2 * mt * ((N + bn0 - 1) / bn0) > num_sms || ks < 8) return {bn0, 1};
+    const int64_t tiles0 = mt * ((N + bn0 - 1) / bn0);
+    if (2 * tiles0 > num_sms || ks < 8) return {bn0, 1};
     TcPlan best{bn0, 1};
-    double best_eff = -1.0;
-    for (int bn = 256; bn >= 64; bn -= 32) {
-        const int64_t nt = (N + bn - 1) / bn;
-        const int64_t tiles = mt * nt;
-        int64_t sp = num_sms / tiles;
-        if (sp > 8) sp = 8;
-        if (sp > ks / 4) sp = ks / 4;
-        if (sp < 2) continue;
-        const double eff = static_cast<double>(tiles * sp) / num_sms *
-                           (static_cast<double>(N) / static_cast<double>(nt * bn));
-        if (eff > best_eff + 1e-9) { best_eff = eff; best = {bn, static_cast<int>(sp)}; }
+    double best_cost = tc_cost((tiles0 + num_sms - 1) / num_sms, ks, bn0);
+    for (int sp = 2; sp <= 8; sp *= 2) {
+        if (ks / sp < 4) break;
+        const int64_t mc = max_clusters(sp);
+        for (int bn = 64; bn <= 256; bn += 32) {
+            const int64_t tiles = mt * ((N + bn - 1) / bn);
+            const double cost = tc_cost((tiles + mc - 1) / mc, (ks + sp - 1) / sp, bn);
+            if (cost < best_cost - 1e-9) { best_cost = cost; best = {bn, sp}; }
+        }
     }
     return best;
 }
@@ -593,8 +662,8 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
         return cudaGetLastError();
     }
     // split-K: one cluster of `splits` CTAs per tile; the partial tile
-    // ([128][bn + 1] fp32) reuses the pipeline's stages in shared memory
-    if (static_cast<size_t>(BM) * (bn + 1) * 4 > prm.sb_off) return cudaErrorInvalidConfiguration;
+    // ([128][bn] fp32) reuses the pipeline's stages in shared memory
+    if (static_cast<size_t>(BM) * bn * 4 > prm.sb_off) return cudaErrorInvalidConfiguration;
     Kern k = bits == 4 ? tc_qmm_kernel<4, true>
              : bits == 8 ? tc_qmm_kernel<8, true>
                          : tc_qmm_kernel<2, true>;
