@@ -133,6 +133,9 @@ nv_status nv_qmm(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N,
                 }
                 return NV_OK;
             }
+            if (M > NV_ROW_INDEPENDENT_ROWS && nvq::tc_supported_t0(M, K, N, bits, group_size))
+                return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases, group_size,
+                                                    bits, y, s, sms, 0, 0));
         }
     }
     return from_cuda(nvq::launch_qmm_simt(x, dt, M, K, N, codes, scales, biases, group_size, bits,
@@ -175,6 +178,9 @@ nv_status nv_qmm_batched(const void* x, nv_dtype dt, int64_t B, int64_t L, int64
             if (L > NV_ROW_INDEPENDENT_ROWS && nvq::tc_supported(M, K, N, bits, group_size))
                 return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases, group_size,
                                                     bits, y, s, sms, L));
+        } else if (L > NV_ROW_INDEPENDENT_ROWS && nvq::tc_supported_t0(M, K, N, bits, group_size)) {
+            return from_cuda(nvq::launch_tc_qmm(x, M, K, N, codes, scales, biases, group_size, bits,
+                                                y, s, sms, L, 0));
         } else if (L <= NV_ROW_INDEPENDENT_ROWS && nvq::qmvt_supported_m(bits, group_size, 1)) {
             int64_t chunk = NV_ROW_INDEPENDENT_ROWS;
             while (chunk > 1 && !nvq::qmvt_supported_m(bits, group_size, chunk)) --chunk;
@@ -194,9 +200,11 @@ nv_status nv_qmm_batched(const void* x, nv_dtype dt, int64_t B, int64_t L, int64
 
 int nv_qmm_splits(int64_t M, int64_t K, int64_t N, int bits, int group_size, int transpose,
                   nv_dtype dt) {
-    if (dt != NV_BF16 || !transpose || M <= NV_ROW_INDEPENDENT_ROWS) return 1;
-    if (!nvq::tc_supported(M, K, N, bits, group_size)) return 1;
-    return nvq::tc_splits(M, K, N, sm_count());
+    if (dt != NV_BF16 || M <= NV_ROW_INDEPENDENT_ROWS) return 1;
+    if (transpose ? !nvq::tc_supported(M, K, N, bits, group_size)
+                  : !nvq::tc_supported_t0(M, K, N, bits, group_size))
+        return 1;
+    return nvq::tc_splits(M, K, N, sm_count(), bits, transpose);
 }
 
 size_t nv_gather_qmm_workspace_size(int64_t R, int64_t E) {

@@ -4,20 +4,25 @@
 // GatherQmm and quantized_matmul take a transpose flag, nuvec crate docs).
 //
 // Here the scale varies along the contraction (one per k-row and group of
-// columns), so it cannot be pulled out of a k-sum: each k-row contributes
-//     y[n] += (x_k * s[k, g(n)]) * code[k, n]  +  x_k * b[k, g(n)],
-// and the second term is shared by a group's columns. Design (sm_100a):
+// columns): every weight is dequantized first, w = s[k, g(n)] * code[k, n] +
+// b[k, g(n)] (one fp32 fused multiply-add on the exact code), and then
+// y[n] += x_k * w. Keeping scale * code and bias in one term matters: summed
+// apart they can cancel (a weight that dequantizes to exactly 0 under a huge
+// activation). Design (sm_100a):
 //  * A thread owns TW consecutive code words of a k-row (one group) and walks
 //    k-rows; a warp reads consecutive columns of one k-row (coalesced).
 //  * Codes become exact fp32 values without int->float conversions: a field
 //    masked into the mantissa of 2^23 gives 2^23 + c * 2^e exactly, and one
 //    packed fma.rn.f32x2 per two codes rescales and removes the 2^23.
-//  * Multiply-adds use packed fma.rn.f32x2 (two columns per instruction).
-//  * K is split between the two CTAs of a cluster and over 64 thread-rows of a
-//    CTA; the partial sums are reduced in a fixed order (thread-rows through
-//    shared memory, then the cluster's two halves through distributed shared
-//    memory), so results are deterministic and every output is computed by the
-//    same operations whatever M is (row exactness).
+//  * Dequantization and multiply-adds use packed fma.rn.f32x2 (two columns
+//    per instruction).
+//  * K is split between the two CTAs of a cluster and over kp thread-rows of a
+//    CTA (64, or 32 / 16 where a CTA spans many columns, so that one CTA per
+//    SM covers the whole output in one wave); the partial sums are reduced in
+//    a fixed order (thread-rows through shared memory, then the cluster's two
+//    halves through distributed shared memory), so results are deterministic.
+//    kp follows N, bits and the group size only, so every output is computed
+//    by the same operations whatever M is (row exactness).
 #include <algorithm>
 #include <cooperative_groups.h>
 
@@ -29,8 +34,8 @@ namespace cg = cooperative_groups;
 namespace nvq {
 namespace {
 
-constexpr int KP = 64;          // thread-rows (k-parts) per CTA
-constexpr int KP_ROUND = 16;    // thread-rows reduced per shared-memory round
+constexpr int KP = 64;          // most thread-rows (k-parts) per CTA
+constexpr int KP_ROUND = 16;    // thread-rows reduced per shared-memory round (kp >= 16)
 constexpr int kClusterK = 2;    // CTAs per cluster, splitting K
 
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
@@ -124,12 +129,13 @@ struct QmvtParams {
     int64_t ncols;           // column units (TW words each)
     int ranges;              // CTAs along the columns
     int ctm;                 // max column units per CTA
+    int kp;                  // thread-rows (k-parts) per CTA: 64, 32 or 16
 };
 
-constexpr int kMaxColUnits = 8;  // column units per CTA: at most 8 * KP = 512 threads
+constexpr int kMaxThreads = 512;  // column units per CTA x thread-rows
 
 template <int BITS, int TW, int MT>
-__global__ void __cluster_dims__(1, kClusterK, 1) __launch_bounds__(kMaxColUnits * KP)
+__global__ void __cluster_dims__(1, kClusterK, 1) __launch_bounds__(kMaxThreads)
 qmvt_kernel(const QmvtParams prm) {
     using C = Codes<BITS>;
     constexpr int COLS_T = TW * C::PER;   // columns a thread owns
@@ -148,18 +154,16 @@ qmvt_kernel(const QmvtParams prm) {
     const int64_t wpr = N * BITS / 32;  // words per k-row
     const int64_t gpr = N / prm.gs;     // groups per k-row
     const int M = prm.M;
-    const bool active = ct < ncol && p < KP;
+    const int kp = prm.kp;
+    const bool active = ct < ncol && p < kp;
 
     uint64_t acc[MT][TW][C::PAIRS];
-    float bacc[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        bacc[m] = 0.f;
+    for (int m = 0; m < MT; ++m)
 #pragma unroll
         for (int w = 0; w < TW; ++w)
 #pragma unroll
             for (int j = 0; j < C::PAIRS; ++j) acc[m][w][j] = 0ull;
-    }
 
     if (active) {
         const int64_t word0 = (c0 + ct) * TW;
@@ -170,12 +174,12 @@ qmvt_kernel(const QmvtParams prm) {
         // Loads in flight per thread; halved where 64 accumulators fill the registers.
         constexpr int U = MT * COLS_T >= 64 ? 2 : MT * COLS_T > 32 ? 4 : 8;
         int64_t k = kr0 + p;
-        for (; k + (U - 1) * KP < kr1; k += U * KP) {
+        for (; k + (U - 1) * kp < kr1; k += U * kp) {
             uint32_t wv[U][TW];
             float sv[U], bv[U], xv[U][MT];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int64_t kk = k + u * KP;
+                const int64_t kk = k + u * kp;
                 load_tw<TW>(cp + kk * wpr, wv[u]);
                 sv[u] = bf16_bits_to_f32(__ldg(sp + kk * gpr));
                 bv[u] = bf16_bits_to_f32(__ldg(bp + kk * gpr));
@@ -185,23 +189,23 @@ qmvt_kernel(const QmvtParams prm) {
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
+                const uint64_t s2 = pack2(sv[u], sv[u]), b2 = pack2(bv[u], bv[u]);
 #pragma unroll
                 for (int w = 0; w < TW; ++w) {
                     uint64_t cv[C::PAIRS];
                     C::to_f32(wv[u][w], cv);
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const float xs = xv[u][m] * sv[u];
-                        const uint64_t xs2 = pack2(xs, xs);
+                    for (int j = 0; j < C::PAIRS; ++j) cv[j] = fma2(s2, cv[j], b2);  // the weights
 #pragma unroll
-                        for (int j = 0; j < C::PAIRS; ++j) acc[m][w][j] = fma2(xs2, cv[j], acc[m][w][j]);
+                    for (int m = 0; m < MT; ++m) {
+                        const uint64_t x2 = pack2(xv[u][m], xv[u][m]);
+#pragma unroll
+                        for (int j = 0; j < C::PAIRS; ++j) acc[m][w][j] = fma2(x2, cv[j], acc[m][w][j]);
                     }
                 }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) bacc[m] = fmaf(xv[u][m], bv[u], bacc[m]);
             }
         }
-        for (; k < kr1; k += KP) {
+        for (; k < kr1; k += kp) {
             uint32_t wv[TW];
             load_tw<TW>(cp + k * wpr, wv);
             const float s = bf16_bits_to_f32(__ldg(sp + k * gpr));
@@ -209,24 +213,24 @@ qmvt_kernel(const QmvtParams prm) {
             float xv[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m) xv[m] = m < M ? bf16_bits_to_f32(__ldg(prm.x + m * K + k)) : 0.f;
+            const uint64_t s2 = pack2(s, s), b2 = pack2(b, b);
 #pragma unroll
             for (int w = 0; w < TW; ++w) {
                 uint64_t cv[C::PAIRS];
                 C::to_f32(wv[w], cv);
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const float xs = xv[m] * s;
-                    const uint64_t xs2 = pack2(xs, xs);
+                for (int j = 0; j < C::PAIRS; ++j) cv[j] = fma2(s2, cv[j], b2);
 #pragma unroll
-                    for (int j = 0; j < C::PAIRS; ++j) acc[m][w][j] = fma2(xs2, cv[j], acc[m][w][j]);
+                for (int m = 0; m < MT; ++m) {
+                    const uint64_t x2 = pack2(xv[m], xv[m]);
+#pragma unroll
+                    for (int j = 0; j < C::PAIRS; ++j) acc[m][w][j] = fma2(x2, cv[j], acc[m][w][j]);
                 }
             }
-#pragma unroll
-            for (int m = 0; m < MT; ++m) bacc[m] = fmaf(xv[m], b, bacc[m]);
         }
     }
 
-    // ---- fixed-order reduction over the 64 thread-rows, 16 per round ----
+    // ---- fixed-order reduction over the kp thread-rows, 16 per round ----
     const int cols_cta = ctm * COLS_T;            // columns of the CTA's buffer
     const int entries = MT * cols_cta;
     float* buf = smem;                            // [KP_ROUND][MT][cols_cta]
@@ -237,7 +241,7 @@ qmvt_kernel(const QmvtParams prm) {
     float run[kMaxOwn];
 #pragma unroll
     for (int i = 0; i < kMaxOwn; ++i) run[i] = 0.f;
-    for (int r0 = 0; r0 < KP; r0 += KP_ROUND) {
+    for (int r0 = 0; r0 < kp; r0 += KP_ROUND) {
         if (p >= r0 && p < r0 + KP_ROUND && ct < ctm) {
             float* dst = buf + (p - r0) * entries;
 #pragma unroll
@@ -249,8 +253,8 @@ qmvt_kernel(const QmvtParams prm) {
                         float lo, hi;
                         unpack2(acc[m][w][j], lo, hi);
                         const int cb = ct * COLS_T + w * C::PER;
-                        dst[m * cols_cta + cb + C::col(j, 0)] = lo + bacc[m];
-                        dst[m * cols_cta + cb + C::col(j, 1)] = hi + bacc[m];
+                        dst[m * cols_cta + cb + C::col(j, 0)] = lo;
+                        dst[m * cols_cta + cb + C::col(j, 1)] = hi;
                     }
         }
         __syncthreads();
@@ -288,14 +292,15 @@ cudaError_t launch_one(const QmvtParams& prm0, int num_sms, cudaStream_t stream)
     QmvtParams prm = prm0;
     using C = Codes<BITS>;
     const int cols_t = TW * C::PER;
-    // Column ranges: enough CTAs for every SM (two per cluster), each at most
-    // kMaxColUnits column units wide.
+    // Column ranges: one cluster (two CTAs) per two SMs, each CTA at most
+    // kMaxThreads / kp column units wide; wider outputs take more ranges.
     int64_t ranges = std::max<int64_t>(1, num_sms / kClusterK);
     ranges = std::min<int64_t>(ranges, prm.ncols);
-    while ((prm.ncols + ranges - 1) / ranges > kMaxColUnits) ranges *= 2;
+    const int64_t max_units = kMaxThreads / prm.kp;
+    while ((prm.ncols + ranges - 1) / ranges > max_units) ranges *= 2;
     prm.ranges = static_cast<int>(ranges);
     prm.ctm = static_cast<int>((prm.ncols + ranges - 1) / ranges);
-    const int threads = prm.ctm * KP;
+    const int threads = prm.ctm * prm.kp;
     const size_t entries = static_cast<size_t>(MT) * prm.ctm * cols_t;
     if ((entries + threads - 1) / threads > 4) return cudaErrorInvalidConfiguration;
     const size_t smem = (KP_ROUND + 1) * entries * sizeof(float);
@@ -348,6 +353,19 @@ cudaError_t dispatch_m(int mt, int tw, const QmvtParams& prm, int num_sms, cudaS
 
 int mt_for(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
+// Thread-rows per CTA: 64 unless the one-row plan's CTAs would span more
+// column units than 512 threads hold at 64 rows each. A function of N, bits
+// and the group size only, so every M sums each output in the same order.
+int kp_for(int64_t N, int bits, int gs, int num_sms) {
+    const int tw = tw_for(bits, gs, 1);
+    const int64_t ncols = N * bits / 32 / tw;
+    const int64_t ranges = std::max<int64_t>(1, std::min<int64_t>(num_sms / kClusterK, ncols));
+    const int64_t ctm = (ncols + ranges - 1) / ranges;
+    int kp = KP;
+    while (kp > KP_ROUND && ctm * kp > kMaxThreads) kp /= 2;
+    return kp;
+}
+
 }  // namespace
 
 bool qmvt_supported(int bits, int gs) {
@@ -375,6 +393,7 @@ cudaError_t launch_qmvt(const void* x, int64_t M, int64_t K, int64_t N, const ui
     prm.M = static_cast<int>(M);
     prm.gs = gs;
     prm.ncols = N * bits / 32 / tw;
+    prm.kp = kp_for(N, bits, gs, num_sms);
     switch (bits) {
         case 2: return dispatch_m<2>(mt, tw, prm, num_sms, stream);
         case 4: return dispatch_m<4>(mt, tw, prm, num_sms, stream);

@@ -9,11 +9,14 @@ namespace nvq {
 bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs);
 // item_rows: rows of one item of a batch (0: all M rows are one item); the
 // tiling and the split-K partition count follow it.
+// transpose = 0: weights stored [K, N] grouped along N (tc_supported_t0).
 cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                           const void* scales, const void* biases, int gs, int bits, void* y,
-                          cudaStream_t stream, int num_sms, int64_t item_rows = 0);
+                          cudaStream_t stream, int num_sms, int64_t item_rows = 0,
+                          int transpose = 1);
+bool tc_supported_t0(int64_t M, int64_t K, int64_t N, int bits, int gs);
 // K-partitions the tiled kernel uses for an item of m_rows rows (1: no split).
-int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms);
+int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms, int bits, int transpose);
 
 // Read and clear the error word of the tensor-core kernels (synchronous).
 unsigned int tc_error_take();

@@ -106,7 +106,7 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int BITS, bool SPLIT>
+template <int BITS, bool SPLIT, bool TR0>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_b,
@@ -201,8 +201,12 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     mbar_expect_tx(&full_a[s], a_bytes);
                     tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], ks * BK, mt * BM);
                     mbar_expect_tx(&full_c[s], c_bytes);
-                    tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
-                                ks * BK * BITS / 32, nt * BN);
+                    if constexpr (TR0)  // weights [K, N]: 64 k-rows x BN columns
+                        tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
+                                    nt * BN * BITS / 32, ks * BK);
+                    else
+                        tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
+                                    ks * BK * BITS / 32, nt * BN);
                     ++issued;
                     if (++s == NS) { s = 0; ++use; }
                 }
@@ -328,6 +332,81 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ dequantize
+        if constexpr (TR0) {
+            // Weights stored [K, N], grouped along N: the stage holds 64 k-rows of
+            // BN * BITS / 32 code words. A task is (4 consecutive k-rows, one code
+            // word): PER columns x 4 k, dequantized into (k, k + 1) pairs and
+            // written transposed into the K-major B tile (row = column n).
+            constexpr int PER = 32 / BITS;
+            const int wpr = BN * BITS / 32;
+            const int tasks = (BK / 4) * wpr;
+            const int dt = threadIdx.x - kDequantWarp0 * 32;
+            const int64_t gpr = prm.N / prm.gs;  // groups per k-row of W
+            int s = 0;
+            uint32_t use = 0;
+            bool ok = true;
+            for (int tile = tile0; tile < tiles && ok; tile += tstep) {
+                const int nt = tile / prm.m_tiles;
+                for (int ks = k0; ks < k1; ++ks) {
+                    if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
+                    const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
+                    uint8_t* bst = b_ring + s * prm.b_stage_bytes;
+                    for (int task = dt; task < tasks; task += kDequantThreads) {
+                        const int kq = task % (BK / 4), j = task / (BK / 4);
+                        const int nl = j * PER;                                  // first column in the tile
+                        const int64_t ng = static_cast<int64_t>(nt) * BN + nl;   // and in W
+                        const int64_t kg = static_cast<int64_t>(ks) * BK + 4 * kq;
+                        uint32_t w[4], sraw[4], braw[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            w[i] = *reinterpret_cast<const uint32_t*>(cst + (4 * kq + i) * (wpr * 4) + 4 * j);
+                            const int64_t gi = (kg + i) * gpr + (ng < prm.N ? ng / prm.gs : 0);
+                            sraw[i] = ng < prm.N ? __ldg(prm.scales + gi) : 0u;
+                            braw[i] = ng < prm.N ? __ldg(prm.biases + gi) : 0u;
+                        }
+                        // (k, k + 1) pairs of scales and biases as bf16x2
+                        const uint32_t s01 = sraw[0] | (sraw[1] << 16), s23 = sraw[2] | (sraw[3] << 16);
+                        const uint32_t b01 = braw[0] | (braw[1] << 16), b23 = braw[2] | (braw[3] << 16);
+#pragma unroll
+                        for (int f = 0; f < PER; ++f) {
+                            uint32_t v[2];
+                            if constexpr (BITS == 8) {
+                                // packed fp32: 2^23 + c exactly, minus 2^23, then s c + b
+                                const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);
+                                const uint64_t off = f2_pack(0xCB000000u, 0xCB000000u);
+#pragma unroll
+                                for (int p = 0; p < 2; ++p) {
+                                    const uint64_t r = f2_pack(prmt(w[2 * p], 0x4B000000u, f | 0x7440),
+                                                               prmt(w[2 * p + 1], 0x4B000000u, f | 0x7440));
+                                    const uint64_t c = f2_fma(r, one_m, off);
+                                    const uint64_t sc = f2_pack(sraw[2 * p] << 16, sraw[2 * p + 1] << 16);
+                                    const uint64_t bc = f2_pack(braw[2 * p] << 16, braw[2 * p + 1] << 16);
+                                    v[p] = f2_to_bf2_packed(f2_fma(sc, c, bc));
+                                }
+                            } else {
+                                // field f of k-rows (k, k + 1) into the two halves: 128 + c
+                                const int byte = (f * BITS) >> 3, sh = (f * BITS) & 7;
+                                const uint32_t sel = static_cast<uint32_t>(byte | ((4 + byte) << 8));
+                                constexpr uint32_t MSK = ((1u << BITS) - 1u) * 0x00010001u;
+                                const uint32_t r0 = codes_to_bf16x2(prmt(w[0], w[1], sel) >> sh, MSK);
+                                const uint32_t r1 = codes_to_bf16x2(prmt(w[2], w[3], sel) >> sh, MSK);
+                                v[0] = bf2_fma(s01, bf2_sub(r0, 0x43004300u), b01);
+                                v[1] = bf2_fma(s23, bf2_sub(r1, 0x43004300u), b23);
+                            }
+                            // row n = nl + f of the B tile: k-chunk kq / 2 (8 k), half (kq & 1)
+                            const int n = nl + f;
+                            *reinterpret_cast<uint2*>(bst + (n >> 3) * 1024 + (n & 7) * 128 +
+                                                      ((((kq >> 1) ^ (n & 7))) << 4) + (kq & 1) * 8) =
+                                make_uint2(v[0], v[1]);
+                        }
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_b[s]);
+                    if (++s == NS) { s = 0; ++use; }
+                }
+            }
+        } else {
         const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 511
         const int r = dt >> 1;                            // weight row within the tile
         const int h = dt & 1;                             // k 32 h .. 32 h + 31 of the k-step
@@ -407,6 +486,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 if (++s == NS) { s = 0; ++use; }
             }
         }
+        }  // TR0
     }
 
     tc_fence_before();
@@ -454,11 +534,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
 }
 
 // ---------------------------------------------------------------- host side
-int pick_bn(int64_t M, int64_t N, int num_sms) {
+int pick_bn(int64_t M, int64_t N, int num_sms, int step = 32) {
     const int64_t mt = (M + BM - 1) / BM;
     int best = 256;
     double best_eff = -1.0;
-    for (int bn = 256; bn >= 128; bn -= 32) {
+    for (int bn = 256; bn >= 128; bn -= step) {
         const int64_t tiles = mt * ((N + bn - 1) / bn);
         const int64_t waves = (tiles + num_sms - 1) / num_sms;
         // useful work over the work of the waves, counting padded columns
@@ -500,7 +580,7 @@ int max_clusters(int size) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-              const TcParams) = tc_qmm_kernel<4, true>;
+              const TcParams) = tc_qmm_kernel<4, true, false>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(cfg.dynamicSmemBytes)) != cudaSuccess ||
         cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(k), &cfg) != cudaSuccess ||
@@ -523,8 +603,8 @@ double tc_cost(int64_t waves, int64_t steps, int bn) {
     return static_cast<double>(waves) * (static_cast<double>(steps) * (0.45 + 0.0013 * bn) + 8.0);
 }
 
-TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms) {
-    const int bn0 = pick_bn(m_rows, N, num_sms);
+TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms, int step = 32) {
+    const int bn0 = pick_bn(m_rows, N, num_sms, step);
     const int64_t mt = (m_rows + BM - 1) / BM;
     const int64_t ks = K / BK;
     const int64_t tiles0 = mt * ((N + bn0 - 1) / bn0);
@@ -534,7 +614,7 @@ TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms) {
     for (int sp = 2; sp <= 8; sp *= 2) {
         if (ks / sp < 4) break;
         const int64_t mc = max_clusters(sp);
-        for (int bn = 64; bn <= 256; bn += 32) {
+        for (int bn = step < 64 ? 64 : step; bn <= 256; bn += step) {
             const int64_t tiles = mt * ((N + bn - 1) / bn);
             const double cost = tc_cost((tiles + mc - 1) / mc, (ks + sp - 1) / sp, bn);
             if (cost < best_cost - 1e-9) { best_cost = cost; best = {bn, sp}; }
@@ -547,8 +627,17 @@ TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms) {
 
 unsigned int tc_error_take() { return pipeline_error_take(); }
 
-int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms) {
-    return plan_tc(m_rows, N, K, num_sms).splits;
+// Tile widths the transposed layout can take: the code rows of a tile
+// (bn * bits / 8 bytes) must be 16-byte multiples for its TMA box.
+static int bn_step(int bits, int transpose) { return (!transpose && bits == 2) ? 64 : 32; }
+
+int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms, int bits, int transpose) {
+    return plan_tc(m_rows, N, K, num_sms, bn_step(bits, transpose)).splits;
+}
+
+bool tc_supported_t0(int64_t M, int64_t K, int64_t N, int bits, int gs) {
+    // weights [K, N] grouped along N: rows of codes are 16-byte multiples
+    return tc_supported(M, K, N, bits, gs) && (N * bits / 8) % 16 == 0 && N % gs == 0;
 }
 
 bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
@@ -558,12 +647,12 @@ bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
 
 cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                           const void* scales, const void* biases, int gs, int bits, void* y,
-                          cudaStream_t stream, int num_sms, int64_t item_rows) {
+                          cudaStream_t stream, int num_sms, int64_t item_rows, int transpose) {
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     // the tiling and the split follow one item's rows (all of x for a plain
     // product): every row's arithmetic is then that of its item's own call
-    const TcPlan plan = plan_tc(item_rows > 0 ? item_rows : M, N, K, num_sms);
+    const TcPlan plan = plan_tc(item_rows > 0 ? item_rows : M, N, K, num_sms, bn_step(bits, transpose));
     const int bn = plan.bn;
     CUtensorMap map_x, map_c;
     {
@@ -576,7 +665,18 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {
+    if (!transpose) {
+        // weights [K, N]: boxes of 64 k-rows x bn columns (bn * bits / 32 words)
+        const int64_t wpr = N * bits / 32;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(K)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(bn * bits / 32), static_cast<cuuint32_t>(BK)};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&map_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    } else {
         const int64_t wpr = K * bits / 32;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(N)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
@@ -595,7 +695,7 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     // scales and biases: blocks of 8 groups x bn rows, when rows are 16-byte multiples
     CUtensorMap map_s, map_b;
     const int64_t gpr = K / gs;
-    const bool sb_tma = (gpr * 2) % 16 == 0;
+    const bool sb_tma = transpose && (gpr * 2) % 16 == 0;  // transpose = 0 loads them directly
     if (sb_tma) {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(gpr) * 2};
@@ -652,9 +752,12 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
                           const TcParams);
     if (plan.splits == 1) {
         const int grid = tiles < num_sms ? tiles : num_sms;
-        Kern k = bits == 4 ? tc_qmm_kernel<4, false>
-                 : bits == 8 ? tc_qmm_kernel<8, false>
-                             : tc_qmm_kernel<2, false>;
+        Kern k = transpose ? (bits == 4 ? tc_qmm_kernel<4, false, false>
+                              : bits == 8 ? tc_qmm_kernel<8, false, false>
+                                          : tc_qmm_kernel<2, false, false>)
+                           : (bits == 4 ? tc_qmm_kernel<4, false, true>
+                              : bits == 8 ? tc_qmm_kernel<8, false, true>
+                                          : tc_qmm_kernel<2, false, true>);
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
@@ -664,9 +767,12 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     // split-K: one cluster of `splits` CTAs per tile; the partial tile
     // ([128][bn] fp32) reuses the pipeline's stages in shared memory
     if (static_cast<size_t>(BM) * bn * 4 > prm.sb_off) return cudaErrorInvalidConfiguration;
-    Kern k = bits == 4 ? tc_qmm_kernel<4, true>
-             : bits == 8 ? tc_qmm_kernel<8, true>
-                         : tc_qmm_kernel<2, true>;
+    Kern k = transpose ? (bits == 4 ? tc_qmm_kernel<4, true, false>
+                          : bits == 8 ? tc_qmm_kernel<8, true, false>
+                                      : tc_qmm_kernel<2, true, false>)
+                       : (bits == 4 ? tc_qmm_kernel<4, true, true>
+                          : bits == 8 ? tc_qmm_kernel<8, true, true>
+                                      : tc_qmm_kernel<2, true, true>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;

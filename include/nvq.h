@@ -163,7 +163,7 @@ nv_status nv_qmm_batched(const void* x, nv_dtype dt, int64_t B, int64_t L, int64
  * K-partitions (split-K; "Docs / Quantization", section "Products on the
  * GPU": split-K when the output is small but the inner dimension long) that
  * nv_qmm uses for an M-row product: 1 when it does not split. Host only, no
- * launch. Products of more than 8 bf16 rows with transpose = 1 split K over a
+ * launch. Products of more than 8 bf16 rows (either layout) split K over a
  * cluster of up to 8 CTAs when their 128 x BN output tiles would occupy fewer
  * than half of the SMs and K holds at least 8 steps of 64; the partial sums
  * are reduced in a fixed order, so results stay deterministic.

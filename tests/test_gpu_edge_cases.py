@@ -4,7 +4,7 @@ Routes (a pure function of the call's shape, dtype and flags):
   * nv_qmm transpose=1, M <= 8, bf16   -> matrix-vector kernel (tensor cores, exact codes)
   * nv_qmm transpose=0, M <= 8, bf16   -> transposed matrix-vector kernel
   * nv_qmm transpose=1, M > 8, bf16    -> tcgen05 tiled kernel
-  * nv_qmm transpose=0, M > 8, bf16    -> plain per-output kernel
+  * nv_qmm transpose=0, M > 8, bf16    -> tcgen05 tiled kernel (transposing dequantizer)
   * nv_qmm fp32, either layout         -> plain per-output kernel
   * nv_gather_qmm transpose=1, bf16    -> grouped tensor-core kernel (row_exact: per-row kernel)
   * nv_gather_qmm transpose=0          -> plain per-output kernel
@@ -39,7 +39,7 @@ QMM_ROUTES = [
     ("matvec_t0", False, 3, BF16),
     ("matvec_t0_m1", False, 1, BF16),
     ("tiled", True, 40, BF16),
-    ("simt_t0_bf16", False, 20, BF16),
+    ("tiled_t0", False, 20, BF16),
     ("simt_fp32_t1", True, 5, F32),
     ("simt_fp32_t0", False, 5, F32),
 ]
@@ -233,3 +233,42 @@ def test_gather_with_more_than_2_32_activation_elements():
     torch.cuda.empty_cache()
     yr, a = O.gather_qmm(xs, c, s, b, pick, rhs, 64, 4)
     P.assert_within(y, yr, a, BF16, "gather beyond 2^32 elements of x")
+
+
+def _cancelling_case(t, M, bits, gs, big):
+    """Integer weights in [-(2^bits - 1), 0] with both ends in every group, so
+    scale 1 and bias -(2^bits - 1): code 2^bits - 1 dequantizes to exactly 0
+    while scale * code and bias are each large. Activations +-big where the
+    weight is 0, N(0, 1) elsewhere. A route that sums scale * code * x and
+    bias * x separately cancels 2^60-sized terms and loses the rest."""
+    N, K = _shape(t, M, gs)
+    hi = 2 ** bits - 1
+    g = torch.Generator().manual_seed(90 + bits)
+    S = torch.arange(3, K, 64)  # never a group's first column
+    if t:  # W [N, K] grouped along K: column k in S is 0 (the groups' maximum)
+        w = -torch.randint(0, hi + 1, (N, K), generator=g).to(torch.float32)
+        w[:, ::gs] = -hi
+        w[:, 1::gs] = 0.0
+        w[:, S] = 0.0
+    else:  # W [K, N] grouped along N: rows k in S are 0 except one -max per group
+        w = -torch.randint(0, hi + 1, (K, N), generator=g).to(torch.float32)
+        w[:, ::gs] = -hi
+        w[:, 1::gs] = 0.0
+        w[S, :] = 0.0
+        w[S.unsqueeze(1), torch.arange(0, N, gs).unsqueeze(0)] = -hi
+    x = torch.randn(M, K, generator=g)
+    x[:, S] = big * torch.where(torch.rand(len(S), generator=g) < 0.5, -1.0, 1.0)
+    return w, x
+
+
+@pytest.mark.parametrize("bits,gs", [(4, 64), (8, 64), (2, 32), (4, 128)])
+@pytest.mark.parametrize("name,t,M,dt", [r for r in QMM_ROUTES if r[3] == BF16])
+def test_zero_weights_with_nonzero_bias_under_huge_activations(name, t, M, dt, bits, gs):
+    w, x = _cancelling_case(t, M, bits, gs, 2.0 ** 60)
+    w, x = w.to(dt), x.to(dt)
+    c, s, b = O.quantize_affine(w, gs, bits)
+    assert (s.float() == 1).all() and (b.float() == -(2 ** bits - 1)).all()
+    y = _run(x, c, s, b, gs, bits, t)
+    yr, a = O.qmm(x, c, s, b, gs, bits, t)
+    assert torch.isfinite(y).all(), name
+    P.assert_within(y, yr, a, dt, f"{name} cancelling bias b{bits} g{gs}")

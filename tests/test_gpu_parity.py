@@ -113,6 +113,33 @@ def test_qmm_no_transpose_small(bits, gs, M):
     _check_product(640, 1000, M, bits, gs, False)
 
 
+@pytest.mark.parametrize("bits,gs", QUANTS)
+@pytest.mark.parametrize("M", [9, 300])
+def test_qmm_no_transpose_tiled(bits, gs, M):
+    """Weights stored [K, N] grouped along N with more than 8 rows: the tiled
+    tensor-core kernel with its transposing dequantizer (ragged rows, several
+    column tiles; N is a multiple of the group size but not of 256)."""
+    _check_product(704 if gs < 128 else 896, 1024, M, bits, gs, False)
+
+
+@pytest.mark.parametrize("bits,gs", [(4, 64), (8, 64), (2, 128)])
+def test_qmm_no_transpose_tiled_2048_rows(bits, gs):
+    """x [2048, 4096] . W with W stored [4096, 14336] (grouped along N):
+    sampled outputs and whole rows against the oracle."""
+    w = W.normal((4096, 14336), 0.02, 0, "bf16")
+    x = W.activations(2048, 4096)
+    c, s, b = O.quantize_affine(w, gs, bits)
+    y = _run(x, c, s, b, gs, bits, False)
+    g = torch.Generator().manual_seed(bits * 10 + gs)
+    mi = torch.randint(0, 2048, (2000,), generator=g)
+    ni = torch.randint(0, 14336, (2000,), generator=g)
+    yr, a = O.qmm_sampled(x, c, s, b, gs, bits, False, mi, ni)
+    P.assert_within(y[mi, ni], yr, a, BF16, f"transpose=0 2048 rows b{bits} g{gs} sampled")
+    for m in (0, 2047):
+        yr, a = O.qmm(x[m:m + 1], c, s, b, gs, bits, False)
+        P.assert_within(y[m:m + 1], yr, a, BF16, f"transpose=0 2048 rows b{bits} g{gs} row {m}")
+
+
 @pytest.mark.parametrize("transpose", [True, False])
 @pytest.mark.parametrize("M", [1, 3, 8, 20])
 def test_qmm_fp32_small(transpose, M):
