@@ -40,6 +40,7 @@
 //    to a call with that row alone (row exactness, nuvec crate docs,
 //    "Determinism").
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -83,32 +84,38 @@ __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
     return d;
 }
 
-// A group's scale and bias for one weight row, ready for the dequantizer:
-// (s, s) and (b, b) as bf16 pairs, s / 4 and s / 16 (2-bit fields held as
-// c * 4^j), and s, b as fp32 (8-bit codes).
+// A group's scale and bias for one weight row, ready for the dequantizers:
+// (s, s) and (b, b) as bf16 pairs, taken from a word holding two groups'
+// values (half i & 1), and whether the fast dequantizer applies.
 struct GroupSB {
-    uint32_t s2, b2, s2q, s2h;
-    float sf, bf;
+    uint32_t s2, b2;
+    bool fast;
 };
-template <int BITS>
-__device__ __forceinline__ GroupSB group_sb(float sf, float bf) {
+__device__ __forceinline__ GroupSB group_sb(uint32_t sv, uint32_t bv, int i) {
     GroupSB g;
-    g.sf = sf;
-    g.bf = bf;
-    g.s2 = (__float_as_uint(sf) >> 16) * 0x00010001u;
-    g.b2 = (__float_as_uint(bf) >> 16) * 0x00010001u;
-    if constexpr (BITS == 2) {  // exact: powers of two (bf16 keeps s's 8 bits)
-        g.s2q = (__float_as_uint(sf * 0.25f) >> 16) * 0x00010001u;
-        g.s2h = (__float_as_uint(sf * 0.0625f) >> 16) * 0x00010001u;
-    } else {
-        g.s2q = g.s2h = 0u;
-    }
+    const uint32_t sel = (i & 1) ? 0x3232u : 0x1010u;
+    g.s2 = __byte_perm(sv, 0u, sel);
+    g.b2 = __byte_perm(bv, 0u, sel);
+    // s normal and below 2^-5: biased exponent 1 .. 121
+    g.fast = ((g.s2 >> 7) & 0xFFu) - 1u < 121u;
     return g;
 }
 
 // Word -> NP bf16x2 registers of dequantized weights; MMA u of the word uses
 // p[2u] (k-slots 2t, 2t+1) and p[2u+1] (k-slots 2t+8, 2t+9). lo(i), hi(i):
 // the codes of the word behind register i's low and high halves.
+//
+// Two exact forms of w = s * c + b, rounded once to bf16 (one bf16 fma):
+//  * run: OR-ing a field worth c * 2^p <= 127 into the mantissa of 128.0
+//    gives 128 + c * 2^p; 128 is subtracted (exact) and the fma takes s (or
+//    s / 2^p, exact for these powers of two).
+//  * run_fast (s a normal number below 2^-5): a 16-bit pattern below 0x100
+//    read as a bf16 is exactly pattern * 2^-133 (subnormals and the lowest
+//    binade are one linear scale), so a field masked in place is
+//    c * 2^(p - 133) with no subtraction, and the fma takes s * 2^(133 - p),
+//    formed by adding 133 - p to s's exponent (exact, and finite because s
+//    is below 2^-5). The product is the same real number s * c, so both
+//    forms round to the same bf16.
 template <int BITS>
 struct Dequant;
 
@@ -121,6 +128,15 @@ struct Dequant<4> {  // (c0,c4) (c1,c5) (c2,c6) (c3,c7)
         for (int i = 0; i < 4; ++i)
             p[i] = bf2_fma(g.s2, bf2_sub(codes_to_bf16x2(w >> (4 * i), 0x000F000Fu), 0x43004300u), g.b2);
     }
+    __device__ static __forceinline__ void run_fast(uint32_t w, const GroupSB& g, uint32_t* p) {
+        const uint32_t s0 = g.s2 + 0x42804280u;  // s * 2^133: fields at bits 0-3
+        const uint32_t s1 = g.s2 + 0x40804080u;  // s * 2^129: fields at bits 4-7
+        const uint32_t v = w >> 8;
+        p[0] = bf2_fma(s0, w & 0x000F000Fu, g.b2);
+        p[1] = bf2_fma(s1, w & 0x00F000F0u, g.b2);
+        p[2] = bf2_fma(s0, v & 0x000F000Fu, g.b2);
+        p[3] = bf2_fma(s1, v & 0x00F000F0u, g.b2);
+    }
 };
 
 template <>
@@ -128,6 +144,10 @@ struct Dequant<2> {  // (c_i, c_i+8), fields held as c * (1, 4, 16, 1, 4, 16, 1,
     __host__ __device__ static constexpr int lo(int i) { return i; }
     __host__ __device__ static constexpr int hi(int i) { return i + 8; }
     __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
+        // s / 4 and s / 16 for fields held as c * 4 and c * 16 (exact)
+        const float sf = __uint_as_float(g.s2 << 16);
+        const uint32_t s2q = (__float_as_uint(sf * 0.25f) >> 16) * 0x00010001u;
+        const uint32_t s2h = (__float_as_uint(sf * 0.0625f) >> 16) * 0x00010001u;
         const uint32_t v = w >> 6, u = w >> 12;
         const uint32_t r[8] = {codes_to_bf16x2(w, 0x00030003u), codes_to_bf16x2(w, 0x000C000Cu),
                                codes_to_bf16x2(w, 0x00300030u), codes_to_bf16x2(v, 0x00030003u),
@@ -135,32 +155,50 @@ struct Dequant<2> {  // (c_i, c_i+8), fields held as c * (1, 4, 16, 1, 4, 16, 1,
                                codes_to_bf16x2(u, 0x00030003u), codes_to_bf16x2(u, 0x000C000Cu)};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t s2 = (i % 3) == 0 ? g.s2 : (i % 3) == 1 ? g.s2q : g.s2h;
+            const uint32_t s2 = (i % 3) == 0 ? g.s2 : (i % 3) == 1 ? s2q : s2h;
             p[i] = bf2_fma(s2, bf2_sub(r[i], 0x43004300u), g.b2);
+        }
+    }
+    __device__ static __forceinline__ void run_fast(uint32_t w, const GroupSB& g, uint32_t* p) {
+        // fields at bits 0-1, 2-3, 4-5, 6-7 of each half: s * 2^133, 2^131, 2^129, 2^127
+        const uint32_t m[4] = {g.s2 + 0x42804280u, g.s2 + 0x41804180u, g.s2 + 0x40804080u,
+                               g.s2 + 0x3F803F80u};
+        const uint32_t v = w >> 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            p[i] = bf2_fma(m[i], w & (0x00030003u << (2 * i)), g.b2);
+            p[i + 4] = bf2_fma(m[i], v & (0x00030003u << (2 * i)), g.b2);
         }
     }
 };
 
 template <>
-struct Dequant<8> {  // (c0,c1) (c2,c3): fp32 s * c + b, converted once to bf16
-    __host__ __device__ static constexpr int lo(int i) { return 2 * i; }
-    __host__ __device__ static constexpr int hi(int i) { return 2 * i + 1; }
+struct Dequant<8> {  // (c0,c2) (c1,c3)
+    __host__ __device__ static constexpr int lo(int i) { return i; }
+    __host__ __device__ static constexpr int hi(int i) { return i + 2; }
     __device__ static __forceinline__ void run(uint32_t w, const GroupSB& g, uint32_t* p) {
         // packed fp32 pairs: byte k under the mantissa of 2^23 is 2^23 + c_k;
-        // one fma removes the 2^23 (exact), one applies scale and bias
+        // one fma removes the 2^23 (exact), one applies scale and bias, and
+        // the sum is converted once to bf16
         const uint64_t one = 0x3F8000003F800000ull, off = 0xCB000000CB000000ull;
-        const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(g.sf)) << 32) | __float_as_uint(g.sf);
-        const uint64_t b2 = (static_cast<uint64_t>(__float_as_uint(g.bf)) << 32) | __float_as_uint(g.bf);
+        const uint32_t sf = g.s2 << 16, bf = g.b2 << 16;
+        const uint64_t s2 = (static_cast<uint64_t>(sf) << 32) | sf;
+        const uint64_t b2 = (static_cast<uint64_t>(bf) << 32) | bf;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            const uint64_t r = (static_cast<uint64_t>(__byte_perm(w, 0x4B000000u, 0x7640 | (2 * i + 1))) << 32) |
-                               __byte_perm(w, 0x4B000000u, 0x7640 | (2 * i));
+            const uint64_t r = (static_cast<uint64_t>(__byte_perm(w, 0x4B000000u, 0x7640 | hi(i))) << 32) |
+                               __byte_perm(w, 0x4B000000u, 0x7640 | lo(i));
             uint64_t c, f;
             asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(c) : "l"(r), "l"(one), "l"(off));
             asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f) : "l"(s2), "l"(c), "l"(b2));
             asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
                 : "=r"(p[i]) : "l"(f));
         }
+    }
+    __device__ static __forceinline__ void run_fast(uint32_t w, const GroupSB& g, uint32_t* p) {
+        const uint32_t s0 = g.s2 + 0x42804280u;  // s * 2^133: bytes at bits 0-7
+        p[0] = bf2_fma(s0, w & 0x00FF00FFu, g.b2);
+        p[1] = bf2_fma(s0, (w >> 8) & 0x00FF00FFu, g.b2);
     }
 };
 
@@ -184,9 +222,6 @@ __device__ __forceinline__ void x_fragments(const uint32_t* xv, float f, uint32_
         b[i >> 1][i & 1] = f2_to_bf2x(bf16_elem(xv, D::lo(i)) * f, bf16_elem(xv, D::hi(i)) * f);
 }
 
-__device__ __forceinline__ float group_value(const uint32_t* v, int i) {
-    return __uint_as_float((i & 1) ? (v[i >> 1] & 0xFFFF0000u) : (v[i >> 1] << 16));
-}
 
 struct QmvParams {
     const uint16_t* x;       // bf16 [x_rows, K]
@@ -581,25 +616,44 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
 
             // acc: rows g, g + 8 x activation rows 2t, 2t + 1 (the MMA's D fragment)
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // One dequantizer for the whole tile and warp: the fast form when
+            // every group this warp meets in the tile allows it (the usual
+            // case), else the general form (same results either way).
+            bool lane_fast = true;
 #pragma unroll
-            for (int q = 0; q < S::KS; ++q) {
-                uint32_t wa[S::LW], wb[S::LW];
-                lds_words<S::LW>(cst + offa[q], wa);
-                lds_words<S::LW>(cst + offb[q], wb);
+            for (int q = 0; q < S::KS; q += S::CPG) {
                 const int gi = q / S::CPG;
-                const GroupSB gA = group_sb<BITS>(group_value(sa, gi), group_value(ba, gi));
-                const GroupSB gB = group_sb<BITS>(group_value(sb, gi), group_value(bb, gi));
-#pragma unroll
-                for (int j = 0; j < S::LW; ++j) {
-                    uint32_t pa[S::NP], pb[S::NP];
-                    Dequant<BITS>::run(wa[j], gA, pa);
-                    Dequant<BITS>::run(wb[j], gB, pb);
-#pragma unroll
-                    for (int u = 0; u < S::MPW; ++u)
-                        mma_bf16_16816(acc, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
-                                       bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
-                }
+                lane_fast = lane_fast && group_sb(sa[gi >> 1], ba[gi >> 1], gi).fast &&
+                            group_sb(sb[gi >> 1], bb[gi >> 1], gi).fast;
             }
+            auto tile_products = [&](auto fast_tag) {
+#pragma unroll
+                for (int q = 0; q < S::KS; ++q) {
+                    uint32_t wa[S::LW], wb[S::LW];
+                    lds_words<S::LW>(cst + offa[q], wa);
+                    lds_words<S::LW>(cst + offb[q], wb);
+                    const int gi = q / S::CPG;
+                    const GroupSB gA = group_sb(sa[gi >> 1], ba[gi >> 1], gi);
+                    const GroupSB gB = group_sb(sb[gi >> 1], bb[gi >> 1], gi);
+#pragma unroll
+                    for (int j = 0; j < S::LW; ++j) {
+                        uint32_t pa[S::NP], pb[S::NP];
+                        if constexpr (decltype(fast_tag)::value) {
+                            Dequant<BITS>::run_fast(wa[j], gA, pa);
+                            Dequant<BITS>::run_fast(wb[j], gB, pb);
+                        } else {
+                            Dequant<BITS>::run(wa[j], gA, pa);
+                            Dequant<BITS>::run(wb[j], gB, pb);
+                        }
+#pragma unroll
+                        for (int u = 0; u < S::MPW; ++u)
+                            mma_bf16_16816(acc, pa[2 * u], pb[2 * u], pa[2 * u + 1], pb[2 * u + 1],
+                                           bfr[q][j * S::MPW + u][0], bfr[q][j * S::MPW + u][1]);
+                    }
+                }
+            };
+            if (__all_sync(__activemask(), lane_fast)) tile_products(std::true_type{});
+            else tile_products(std::false_type{});
             // every lane has read the stage: refill it with tile + NS
             __syncwarp();
             if (tile + NS < tiles && elect_one()) issue(tile + NS, st);

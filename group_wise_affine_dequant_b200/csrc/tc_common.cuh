@@ -133,9 +133,29 @@ __device__ __forceinline__ uint32_t shr(uint32_t w, uint32_t bits) { return w >>
 template <int BITS>
 struct Dequant;
 
+// run_fast (s a normal number below 2^-5, see dq_fast_ok): a 16-bit pattern
+// below 0x100 read as a bf16 is exactly pattern * 2^-133 (subnormals and the
+// lowest binade form one linear scale), so a code field masked in place at
+// bits p .. p + bits - 1 of a half is c * 2^(p - 133), and the bf16 fma takes
+// s * 2^(133 - p) for that half, formed by adding 133 - p to s's exponent
+// (exact, finite since s < 2^-5). The product is the same real number s * c
+// as in run, so both round to the same bf16 w = s * c + b.
+__device__ __forceinline__ bool dq_fast_ok(uint32_t s2) {
+    return ((s2 >> 7) & 0xFFu) - 1u < 121u;  // biased exponent 1 .. 121
+}
+
 template <>
 struct Dequant<4> {  // word: 8 codes -> 4 pairs
     static constexpr int PAIRS = 4;
+    __device__ static __forceinline__ void run_fast(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* out) {
+        const uint32_t m = s2 + 0x40804280u;  // (s * 2^133, s * 2^129)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // byte i into bytes 0 and 2: code 2i at bits 0-3, code 2i+1 at bits 20-23
+            const uint32_t r = prmt(w, w, i | (i << 8)) & 0x00F0000Fu;
+            out[i] = bf2_fma(m, r, b2);
+        }
+    }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
                                                float, uint32_t, uint32_t m4, uint32_t,
                                                uint32_t* out) {
@@ -153,6 +173,16 @@ struct Dequant<4> {  // word: 8 codes -> 4 pairs
 template <>
 struct Dequant<2> {  // word: 16 codes -> 8 pairs
     static constexpr int PAIRS = 8;
+    __device__ static __forceinline__ void run_fast(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* out) {
+        const uint32_t m01 = s2 + 0x41804280u;  // fields at bits 0-1 / 2-3: (s * 2^133, s * 2^131)
+        const uint32_t m23 = s2 + 0x3F804080u;  // fields at bits 4-5 / 6-7: (s * 2^129, s * 2^127)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t r = prmt(w, w, i | (i << 8));  // byte i in both halves
+            out[2 * i] = bf2_fma(m01, r & 0x000C0003u, b2);      // codes 4i, 4i+1
+            out[2 * i + 1] = bf2_fma(m23, r & 0x00C00030u, b2);  // codes 4i+2, 4i+3
+        }
+    }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t s2, uint32_t b2, float,
                                                float, uint32_t m2, uint32_t m4, uint32_t m6,
                                                uint32_t* out) {
@@ -188,6 +218,12 @@ __device__ __forceinline__ uint32_t f2_to_bf2_packed(uint64_t v) {
 template <>
 struct Dequant<8> {  // word: 4 codes -> 2 pairs, through exact fp32 codes in packed pairs
     static constexpr int PAIRS = 2;
+    __device__ static __forceinline__ void run_fast(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* out) {
+        const uint32_t m = s2 + 0x42804280u;  // (s * 2^133, s * 2^133)
+#pragma unroll
+        for (int i = 0; i < 2; ++i)  // bytes 2i, 2i + 1 into bytes 0 and 2, zeros elsewhere
+            out[i] = bf2_fma(m, prmt(w, 0u, (2 * i) | (4 << 4) | ((2 * i + 1) << 8) | (4 << 12)), b2);
+    }
     __device__ static __forceinline__ void run(uint32_t w, uint32_t, uint32_t, float s, float b,
                                                uint32_t, uint32_t, uint32_t, uint32_t* out) {
         const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);   // (1, 1)

@@ -457,14 +457,24 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (++kc == spk) kc = 0;
                     if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
+                    // one dequantizer for the warp's step: the fast form when every
+                    // lane's groups allow it (same results either way)
+                    const bool fast = __all_sync(__activemask(),
+                                                 dq_fast_ok((__float_as_uint(sc[0]) >> 16) * 0x00010001u) &&
+                                                 dq_fast_ok((__float_as_uint(sc[1]) >> 16) * 0x00010001u));
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const uint32_t s2 = (__float_as_uint(sc[h2]) >> 16) * 0x00010001u;
                         const uint32_t b2 = (__float_as_uint(bc[h2]) >> 16) * 0x00010001u;
                         uint32_t out[16];
+                        if (fast) {
 #pragma unroll
-                        for (int i = 0; i < NW; ++i)
-                            DQ::run(w[h2][i], s2, b2, sc[h2], bc[h2], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                            for (int i = 0; i < NW; ++i) DQ::run_fast(w[h2][i], s2, b2, out + i * DQ::PAIRS);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < NW; ++i)
+                                DQ::run(w[h2][i], s2, b2, sc[h2], bc[h2], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                        }
                         tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + (BK / 2) * tt +
                                         32 * hf + 16 * h2,
                                     out);

@@ -442,6 +442,10 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     bc = bf16_bits_to_f32(__ldg(brow + g));
                 }
                 if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
+                // one dequantizer for the warp's step: the fast form when every
+                // live row's group allows it (same results either way)
+                const bool fast = __all_sync(__activemask(),
+                                             !live || dq_fast_ok((__float_as_uint(sc) >> 16) * 0x00010001u));
                 if (has_row) {
                     const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
                     constexpr int NW = BITS;  // code words per 32 k
@@ -464,9 +468,14 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
                     uint32_t out[16];
+                    if (fast) {
 #pragma unroll
-                    for (int i = 0; i < NW; ++i)
-                        DQ::run(w[i], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + i * DQ::PAIRS);
+                        for (int i = 0; i < NW; ++i) DQ::run_fast(w[i], s2, b2, out + i * DQ::PAIRS);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i)
+                            DQ::run(w[i], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + i * DQ::PAIRS);
+                    }
                     // chunks 4 h .. 4 h + 3 (8 k each) of the row, under the 128-byte swizzle
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {

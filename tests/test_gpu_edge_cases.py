@@ -272,3 +272,39 @@ def test_zero_weights_with_nonzero_bias_under_huge_activations(name, t, M, dt, b
     yr, a = O.qmm(x, c, s, b, gs, bits, t)
     assert torch.isfinite(y).all(), name
     P.assert_within(y, yr, a, dt, f"{name} cancelling bias b{bits} g{gs}")
+
+
+def _wide_magnitude_weights(rows, cols, gs, dtype, seed):
+    """Rows of N(0, 1) weights scaled by 10^u, u uniform in [-5, 2], plus a
+    share of constant groups: group scales from ~1e-7 to ~1e1, on both sides
+    of every power-of-two threshold a kernel might special-case."""
+    g = torch.Generator().manual_seed(seed)
+    w = torch.randn(rows, cols, generator=g) * (10.0 ** (torch.rand(rows, 1, generator=g) * 7 - 5))
+    blocks = w.view(rows, cols // gs, gs)
+    pick = torch.rand(rows, cols // gs, generator=g) < 0.1
+    blocks[pick] = blocks[pick][:, :1].expand(-1, gs).clone()
+    return w.to(dtype)
+
+
+@pytest.mark.parametrize("bits,gs", QUANTS)
+@pytest.mark.parametrize("name,t,M,dt", QMM_ROUTES)
+def test_unit_activations_read_out_the_weights(name, t, M, dt, bits, gs):
+    """x rows that are unit vectors e_k: every output is one exact product
+    1 * w_hat plus exact zeros, so y[m, n] must equal the dequantized weight
+    (scale * code + bias rounded once to the scales' type) bit for bit, for
+    groups of every magnitude."""
+    N, K = _shape(t, M, gs)
+    w = _wide_magnitude_weights(N, K, gs, dt, 50 + bits) if t else \
+        _wide_magnitude_weights(K, N, gs, dt, 50 + bits)
+    c, s, b = O.quantize_affine(w, gs, bits)
+    assert (s.float() < 2.0 ** -5).any() and (s.float() >= 2.0 ** -5).any()
+    wh = O.dequantize_stored(c, s, b, gs, bits)          # [N, K] or [K, N]
+    ks = torch.randperm(K, generator=torch.Generator().manual_seed(bits + gs))[:M]
+    x = torch.zeros(M, K, dtype=dt)
+    x[torch.arange(M), ks] = 1.0
+    y = _run(x, c, s, b, gs, bits, t)
+    want = wh[:, ks].t() if t else wh[ks, :]
+    bad = (y.view(torch.int16 if dt == BF16 else torch.int32) !=
+           want.to(dt).view(torch.int16 if dt == BF16 else torch.int32))
+    assert not bad.any(), (f"{name} b{bits} g{gs}: {int(bad.sum())} outputs differ from the "
+                           f"dequantized weight, first at {bad.nonzero()[0].tolist()}")
