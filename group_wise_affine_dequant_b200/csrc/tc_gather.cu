@@ -107,17 +107,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Byte offset of group column gc of row r in a scale/bias box with rows of
-// 2^lg bytes, under the TMA swizzle of that row width.
-__device__ __forceinline__ uint32_t sb_swz(int r, int gc, int lg) {
-    const uint32_t o = static_cast<uint32_t>(gc) * 2;
-    uint32_t c = o >> 4;
-    if (lg == 7) c ^= r & 7;
-    else if (lg == 6) c ^= (r >> 1) & 3;
-    else if (lg == 5) c ^= (r >> 2) & 1;
-    return (static_cast<uint32_t>(r) << lg) + (c << 4) + (o & 15);
-}
-
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_s,
@@ -405,6 +394,18 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
         uint32_t blk = 0;
         bool ok = true;
         const uint32_t half = static_cast<uint32_t>(prm.sb_slot) / 2;
+        // this thread's fixed parts of the scale/bias box offsets (row rr, the
+        // box's swizzle by row width) and of its code row (128-byte swizzle)
+        const int lg = prm.lg_sbw;
+        const uint32_t sb_row = static_cast<uint32_t>(rr) << lg;
+        const uint32_t sb_x = lg == 7 ? (rr & 7) : lg == 6 ? ((rr >> 1) & 3) : lg == 5 ? ((rr >> 2) & 1) : 0;
+        const uint32_t c_row = static_cast<uint32_t>(rr) * 128;
+        const uint32_t r7 = static_cast<uint32_t>(r & 7);
+        const bool two_groups = prm.lg_gs == 5;  // the two 32-k runs lie in different groups
+        auto sb_off = [&](int gc) {
+            const uint32_t o = static_cast<uint32_t>(gc) * 2;
+            return sb_row + (((o >> 4) ^ sb_x) << 4) + (o & 15);
+        };
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int e, wt, first, count;
             unit_pairs(u, e, wt, first, count);
@@ -422,29 +423,37 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     // runs of 32 k, each inside one group (groups are multiples of 32)
                     constexpr int NW = BITS;  // code words per 32 k
                     uint32_t w[2][NW];
-                    float sc[2], bc[2];
+                    uint32_t sv[2], bv[2];  // bf16 bits of the runs' scales and biases
+                    {
+                        const uint32_t so = sb_off(((ks * BK + 64 * hf) >> prm.lg_gs) - gb);
+                        sv[0] = sv[1] = *reinterpret_cast<const uint16_t*>(ss + so);
+                        bv[0] = bv[1] = *reinterpret_cast<const uint16_t*>(ss + half + so);
+                        if (two_groups) {
+                            const uint32_t so1 = sb_off(((ks * BK + 64 * hf) >> prm.lg_gs) + 1 - gb);
+                            sv[1] = *reinterpret_cast<const uint16_t*>(ss + so1);
+                            bv[1] = *reinterpret_cast<const uint16_t*>(ss + half + so1);
+                        }
+                    }
+                    const uint8_t* crow = c_ring + c.s * kCStage + c_row;
+                    // 16-byte chunk of run 0 in the row: o = kc * (BK BITS / 8) + 64 hf BITS / 8
+                    const uint32_t o0 = static_cast<uint32_t>(kc * (BK * BITS / 8) + 64 * hf * BITS / 8);
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
-                        const int gc = ((ks * BK + 64 * hf + 32 * h2) >> prm.lg_gs) - gb;
-                        const uint32_t so = sb_swz(rr, gc, prm.lg_sbw);
-                        sc[h2] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + so));
-                        bc[h2] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + half + so));
-                        const uint8_t* crow = c_ring + c.s * kCStage + rr * 128;
-                        const int o = kc * (BK * BITS / 8) + (64 * hf + 32 * h2) * BITS / 8;
+                        const uint32_t o = o0 + 32 * h2 * BITS / 8;
                         if constexpr (BITS == 4) {
-                            const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ (r & 7)) << 4));
+                            const uint4 v4 = *reinterpret_cast<const uint4*>(crow + (((o >> 4) ^ r7) << 4));
                             w[h2][0] = v4.x; w[h2][1] = v4.y; w[h2][2] = v4.z; w[h2][3] = v4.w;
                         } else if constexpr (BITS == 8) {
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
                                 const uint4 v4 = *reinterpret_cast<const uint4*>(
-                                    crow + ((((o >> 4) + h) ^ (r & 7)) << 4));
+                                    crow + ((((o >> 4) + h) ^ r7) << 4));
                                 w[h2][4 * h] = v4.x; w[h2][4 * h + 1] = v4.y;
                                 w[h2][4 * h + 2] = v4.z; w[h2][4 * h + 3] = v4.w;
                             }
                         } else {
                             const uint2 v2 = *reinterpret_cast<const uint2*>(
-                                crow + (((o >> 4) ^ (r & 7)) << 4) + (o & 15));
+                                crow + (((o >> 4) ^ r7) << 4) + (o & 15));
                             w[h2][0] = v2.x; w[h2][1] = v2.y;
                         }
                     }
@@ -457,28 +466,27 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     if (++kc == spk) kc = 0;
                     if (a.use > 0 && !(ok = mbar_wait_backoff(&empty_a[a.s], (a.use - 1) & 1, 32, 128))) break;
                     tc_fence_after();
+                    const uint32_t s2[2] = {sv[0] * 0x00010001u, sv[1] * 0x00010001u};
+                    const uint32_t b2[2] = {bv[0] * 0x00010001u, bv[1] * 0x00010001u};
                     // one dequantizer for the warp's step: the fast form when every
                     // lane's groups allow it (same results either way)
-                    const bool fast = __all_sync(__activemask(),
-                                                 dq_fast_ok((__float_as_uint(sc[0]) >> 16) * 0x00010001u) &&
-                                                 dq_fast_ok((__float_as_uint(sc[1]) >> 16) * 0x00010001u));
+                    const bool fast = __all_sync(__activemask(), dq_fast_ok(s2[0]) && dq_fast_ok(s2[1]));
+                    const uint32_t ta = tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + (BK / 2) * tt + 32 * hf;
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
-                        const uint32_t s2 = (__float_as_uint(sc[h2]) >> 16) * 0x00010001u;
-                        const uint32_t b2 = (__float_as_uint(bc[h2]) >> 16) * 0x00010001u;
                         uint32_t out[16];
                         if (fast) {
 #pragma unroll
-                            for (int i = 0; i < NW; ++i) DQ::run_fast(w[h2][i], s2, b2, out + i * DQ::PAIRS);
+                            for (int i = 0; i < NW; ++i) DQ::run_fast(w[h2][i], s2[h2], b2[h2], out + i * DQ::PAIRS);
                         } else {
+                            const float sc = __uint_as_float(sv[h2] << 16), bc = __uint_as_float(bv[h2] << 16);
 #pragma unroll
                             for (int i = 0; i < NW; ++i)
-                                DQ::run(w[h2][i], s2, b2, sc[h2], bc[h2], 2u, 4u, 6u, out + i * DQ::PAIRS);
+                                DQ::run(w[h2][i], s2[h2], b2[h2], sc, bc, 2u, 4u, 6u, out + i * DQ::PAIRS);
                         }
-                        tmem_st_x16(tmem_base + lane_addr + 2 * kAccCols + kACols * a.s + (BK / 2) * tt +
-                                        32 * hf + 16 * h2,
-                                    out);
+                        tmem_st_x16_async(ta + 16 * h2, out);
                     }
+                    tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_a[a.s]);
