@@ -106,7 +106,7 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int BITS, bool SPLIT, bool TR0>
+template <int BITS, bool SPLIT, bool TR0, int MS = 1>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_b,
@@ -170,7 +170,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     const int tstep = SPLIT ? tiles : static_cast<int>(gridDim.x);
     const int k0 = SPLIT ? rank * ksteps / S : 0;
     const int k1 = SPLIT ? (rank + 1) * ksteps / S : ksteps;
-    const uint32_t a_bytes = BM * BK * 2;
+    const uint32_t a_bytes = MS * BM * BK * 2;  // MS row subtiles of 128 x 64
     const uint32_t c_bytes = static_cast<uint32_t>(BN) * BK * BITS / 8;
 
     if (warp == 0) {
@@ -199,7 +199,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     if (++kb == sgk) kb = 0;
                     if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, 1))) break;
                     mbar_expect_tx(&full_a[s], a_bytes);
-                    tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], ks * BK, mt * BM);
+                    tma_load_2d(a_ring + s * a_bytes, &map_x, &full_a[s], ks * BK, mt * BM * MS);
                     mbar_expect_tx(&full_c[s], c_bytes);
                     if constexpr (TR0)  // weights [K, N]: 64 k-rows x BN columns
                         tma_load_2d(c_ring + s * prm.c_stage_bytes, &map_c, &full_c[s],
@@ -231,7 +231,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 const uint32_t ause = static_cast<uint32_t>(local >> 1);
                 if (ause > 0 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, 2))) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * MS * BN);
                 for (int ks = k0; ks < k1; ++ks) {
                     if (!(ok = mbar_wait(&full_a[s], use & 1, 3))) break;
                     if (!(ok = mbar_wait(&full_b[s], use & 1, 4))) break;
@@ -239,11 +239,13 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     const uint64_t ad = sw128_desc(a_ring + s * a_bytes);
                     const uint64_t bd = sw128_desc(b_ring + s * prm.b_stage_bytes);
 #pragma unroll
-                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        // advance 16 bf16 (32 bytes) along K inside the swizzle atom
-                        tc_mma(d_tmem, ad + (kk * UMMA_K * 2 >> 4), bd + (kk * UMMA_K * 2 >> 4), idesc,
-                               (ks > k0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int m = 0; m < MS; ++m)  // every row subtile against the same weights
+#pragma unroll
+                        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                            // advance 16 bf16 (32 bytes) along K inside the swizzle atom
+                            tc_mma(d_tmem + m * BN, ad + (m * (BM * BK * 2) >> 4) + (kk * UMMA_K * 2 >> 4),
+                                   bd + (kk * UMMA_K * 2 >> 4), idesc, (ks > k0 || kk > 0) ? 1u : 0u);
+                        }
                     tc_commit(&empty[s]);
                     if (++s == NS) { s = 0; ++use; }
                 }
@@ -289,12 +291,13 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 continue;
             }
             const int mt = tile % prm.m_tiles, nt = tile / prm.m_tiles;
-            const int64_t row = static_cast<int64_t>(mt) * BM + row_in_tile;
             const int64_t col0 = static_cast<int64_t>(nt) * BN;
+            for (int m = 0; m < MS; ++m)
             for (int j = 0; j < BN / 32; ++j) {
+                const int64_t row = (static_cast<int64_t>(mt) * MS + m) * BM + row_in_tile;
                 uint32_t v[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(a * BN + j * 32);
+                                       static_cast<uint32_t>((a * MS + m) * BN + j * 32);
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
                     "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -323,6 +326,40 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     } else {
                         for (int e = 0; e < 32; ++e)
                             if (c + e < prm.N) yp[e] = f32_to_bf16_bits(__uint_as_float(v[e]));
+                    }
+                }
+            }
+            if (BN & 16) {  // tiles 16 columns past a multiple of 32
+                for (int m = 0; m < MS; ++m) {
+                    const int64_t row = (static_cast<int64_t>(mt) * MS + m) * BM + row_in_tile;
+                    uint32_t v[16];
+                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                           static_cast<uint32_t>((a * MS + m) * BN + (BN & ~31));
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                        : "r"(taddr));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    const int64_t c = col0 + (BN & ~31);
+                    if (row < prm.M) {
+                        uint16_t* yp = prm.y + row * prm.N + c;
+                        if (c + 16 <= prm.N && (prm.N % 8) == 0) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                uint4 o;
+                                o.x = f2_to_bf2(__uint_as_float(v[8 * h + 0]), __uint_as_float(v[8 * h + 1]));
+                                o.y = f2_to_bf2(__uint_as_float(v[8 * h + 2]), __uint_as_float(v[8 * h + 3]));
+                                o.z = f2_to_bf2(__uint_as_float(v[8 * h + 4]), __uint_as_float(v[8 * h + 5]));
+                                o.w = f2_to_bf2(__uint_as_float(v[8 * h + 6]), __uint_as_float(v[8 * h + 7]));
+                                *reinterpret_cast<uint4*>(yp + 8 * h) = o;
+                            }
+                        } else {
+                            for (int e = 0; e < 16; ++e)
+                                if (c + e < prm.N) yp[e] = f32_to_bf16_bits(__uint_as_float(v[e]));
+                        }
                     }
                 }
             }
@@ -408,8 +445,12 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             }
         } else {
         const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0 .. 511
-        const int r = dt >> 1;                            // weight row within the tile
-        const int h = dt & 1;                             // k 32 h .. 32 h + 31 of the k-step
+        // tiles of up to 128 columns: four threads per weight row (16 k each);
+        // wider tiles: two (32 k each)
+        const bool quad = BN <= 128;
+        const int r = quad ? dt >> 2 : dt >> 1;           // weight row within the tile
+        const int h = quad ? dt & 3 : dt & 1;             // k part of the k-step
+        const int kpart = quad ? 16 : 32;                 // k per thread and step
         const bool has_row = r < BN;
         const int64_t gpr = prm.K / prm.gs;
         using DQ = Dequant<BITS>;
@@ -425,8 +466,8 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
             const uint16_t* srow = prm.scales + (live ? n : 0) * gpr;
             const uint16_t* brow = prm.biases + (live ? n : 0) * gpr;
             for (int ks = k0; ks < k1; ++ks) {
-                // 32 k lie in one group (groups are 32-k aligned multiples of 32)
-                const int g = ((ks * BK + 32 * h) >> prm.lg_gs);
+                // a thread's k part lies in one group (groups are 32-k aligned multiples of 32)
+                const int g = ((ks * BK + kpart * h) >> prm.lg_gs);
                 float sc = 0.f, bc = 0.f;
                 const int slot = blk & 1;
                 if (prm.sb_tma) {
@@ -446,7 +487,7 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                 // live row's group allows it (same results either way)
                 const bool fast = __all_sync(__activemask(),
                                              !live || dq_fast_ok((__float_as_uint(sc) >> 16) * 0x00010001u));
-                if (has_row) {
+                if (has_row && !quad) {
                     const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
                     constexpr int NW = BITS;  // code words per 32 k
                     uint32_t w[NW];
@@ -482,6 +523,41 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                         uint4 o;
                         o.x = out[4 * c]; o.y = out[4 * c + 1]; o.z = out[4 * c + 2]; o.w = out[4 * c + 3];
                         *reinterpret_cast<uint4*>(brow_s + (((4 * h + c) ^ (r & 7)) << 4)) = o;
+                    }
+                    fence_proxy_async();
+                } else if (has_row) {
+                    // 16 k of the row: k 16 h .. 16 h + 15 of the k-step
+                    const uint8_t* cst = c_ring + s * prm.c_stage_bytes;
+                    constexpr int NW = BITS / 2;  // code words per 16 k
+                    uint32_t w[NW];
+                    if constexpr (BITS == 4) {  // 32-byte rows, 32-byte swizzle: 8 bytes
+                        const uint2 v2 = *reinterpret_cast<const uint2*>(
+                            cst + r * 32 + (((h >> 1) ^ ((r >> 2) & 1)) << 4) + (h & 1) * 8);
+                        w[0] = v2.x; w[1] = v2.y;
+                    } else if constexpr (BITS == 8) {  // 64-byte rows, 64-byte swizzle: 16 bytes
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(cst + r * 64 + ((h ^ ((r >> 1) & 3)) << 4));
+                        w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+                    } else {  // 16-byte rows, unswizzled: one word
+                        w[0] = *reinterpret_cast<const uint32_t*>(cst + r * 16 + h * 4);
+                    }
+                    uint8_t* brow_s = b_ring + s * prm.b_stage_bytes + (r >> 3) * 1024 + (r & 7) * 128;
+                    const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
+                    const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
+                    uint32_t out[8];
+                    if (fast) {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) DQ::run_fast(w[i], s2, b2, out + i * DQ::PAIRS);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i)
+                            DQ::run(w[i], s2, b2, sc, bc, prm.m2, prm.m4, prm.m6, out + i * DQ::PAIRS);
+                    }
+                    // chunks 2 h, 2 h + 1 (8 k each) of the row, under the 128-byte swizzle
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint4 o;
+                        o.x = out[4 * c]; o.y = out[4 * c + 1]; o.z = out[4 * c + 2]; o.w = out[4 * c + 3];
+                        *reinterpret_cast<uint4*>(brow_s + (((2 * h + c) ^ (r & 7)) << 4)) = o;
                     }
                     fence_proxy_async();
                 }
@@ -543,16 +619,19 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
 }
 
 // ---------------------------------------------------------------- host side
-int pick_bn(int64_t M, int64_t N, int num_sms, int step = 32) {
-    const int64_t mt = (M + BM - 1) / BM;
-    int best = 256;
+// Tile width of least padded work over whole waves, for tiles of bm rows and
+// bn in [bn_lo, bn_hi] (steps of `step`).
+int pick_bn(int64_t M, int64_t N, int num_sms, int step = 32, int bm = BM, int bn_hi = 256,
+            int bn_lo = 128) {
+    const int64_t mt = (M + bm - 1) / bm;
+    int best = bn_hi;
     double best_eff = -1.0;
-    for (int bn = 256; bn >= 128; bn -= step) {
+    for (int bn = bn_hi; bn >= bn_lo; bn -= step) {
         const int64_t tiles = mt * ((N + bn - 1) / bn);
         const int64_t waves = (tiles + num_sms - 1) / num_sms;
-        // useful work over the work of the waves, counting padded columns
+        // useful work over the work of the waves, counting padded rows and columns
         const double eff = static_cast<double>(M * N) /
-                           (static_cast<double>(waves * num_sms) * BM * bn);
+                           (static_cast<double>(waves * num_sms) * bm * bn);
         if (eff > best_eff + 1e-9) { best_eff = eff; best = bn; }
     }
     return best;
@@ -565,6 +644,7 @@ int pick_bn(int64_t M, int64_t N, int num_sms, int step = 32) {
 // of (rows, N, K, SM count).
 struct TcPlan {
     int bn, splits;
+    int ms = 1;  // 128-row subtiles per tile: 2 pairs every dequantized weight tile with 256 rows
 };
 
 // Clusters of `size` CTAs (one CTA per SM) that the device runs at once: a
@@ -612,12 +692,22 @@ double tc_cost(int64_t waves, int64_t steps, int bn) {
     return static_cast<double>(waves) * (static_cast<double>(steps) * (0.45 + 0.0013 * bn) + 8.0);
 }
 
-TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms, int step = 32) {
+TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms, int step = 32, int step2 = 16) {
     const int bn0 = pick_bn(m_rows, N, num_sms, step);
     const int64_t mt = (m_rows + BM - 1) / BM;
     const int64_t ks = K / BK;
     const int64_t tiles0 = mt * ((N + bn0 - 1) / bn0);
-    if (2 * tiles0 > num_sms || ks < 8) return {bn0, 1};
+    if (2 * tiles0 > num_sms || ks < 8) {
+        // Enough tiles without a split. From 256 rows on, tiles of 256 rows x
+        // bn <= 128 columns (four accumulators fill TMEM's 512 columns) use
+        // every dequantized weight tile for twice the rows; widths step by 16.
+        if (m_rows >= 2 * BM) {
+            const int bn2 = pick_bn(m_rows, N, num_sms, step2, 2 * BM, 128, 64);
+            const int64_t tiles2 = ((m_rows + 2 * BM - 1) / (2 * BM)) * ((N + bn2 - 1) / bn2);
+            if (2 * tiles2 > num_sms) return {bn2, 1, 2};
+        }
+        return {bn0, 1};
+    }
     TcPlan best{bn0, 1};
     double best_cost = tc_cost((tiles0 + num_sms - 1) / num_sms, ks, bn0);
     for (int sp = 2; sp <= 8; sp *= 2) {
@@ -637,11 +727,16 @@ TcPlan plan_tc(int64_t m_rows, int64_t N, int64_t K, int num_sms, int step = 32)
 unsigned int tc_error_take() { return pipeline_error_take(); }
 
 // Tile widths the transposed layout can take: the code rows of a tile
-// (bn * bits / 8 bytes) must be 16-byte multiples for its TMA box.
+// (bn * bits / 8 bytes) must be 16-byte multiples for its TMA box. bn_step:
+// 128-row tiles (multiples of 32 for the split-K partial tiles); bn_step2:
+// 256-row tiles (multiples of 16, the MMA's N granularity).
 static int bn_step(int bits, int transpose) { return (!transpose && bits == 2) ? 64 : 32; }
+static int bn_step2(int bits, int transpose) {
+    return transpose ? 16 : bits == 2 ? 64 : bits == 4 ? 32 : 16;
+}
 
 int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms, int bits, int transpose) {
-    return plan_tc(m_rows, N, K, num_sms, bn_step(bits, transpose)).splits;
+    return plan_tc(m_rows, N, K, num_sms, bn_step(bits, transpose), bn_step2(bits, transpose)).splits;
 }
 
 bool tc_supported_t0(int64_t M, int64_t K, int64_t N, int bits, int gs) {
@@ -661,13 +756,15 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     if (!enc) return cudaErrorNotSupported;
     // the tiling and the split follow one item's rows (all of x for a plain
     // product): every row's arithmetic is then that of its item's own call
-    const TcPlan plan = plan_tc(item_rows > 0 ? item_rows : M, N, K, num_sms, bn_step(bits, transpose));
+    const TcPlan plan = plan_tc(item_rows > 0 ? item_rows : M, N, K, num_sms, bn_step(bits, transpose),
+                                bn_step2(bits, transpose));
     const int bn = plan.bn;
+    const int ms = plan.ms;
     CUtensorMap map_x, map_c;
     {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-        cuuint32_t box[2] = {BK, BM};
+        cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(BM * ms)};
         cuuint32_t es[2] = {1, 1};
         if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -734,9 +831,9 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     prm.K = K;
     prm.gs = gs;
     prm.bn = bn;
-    prm.m_tiles = static_cast<int>((M + BM - 1) / BM);
+    prm.m_tiles = static_cast<int>((M + BM * ms - 1) / (BM * ms));
     prm.n_tiles = static_cast<int>((N + bn - 1) / bn);
-    const uint32_t a_stage = BM * BK * 2;                         // 16 KB, 1024-aligned
+    const uint32_t a_stage = BM * BK * 2 * ms;                    // 16 KB per row subtile, 1024-aligned
     const uint32_t b_stage = static_cast<uint32_t>(bn) * BK * 2;  // bn * 128
     const uint32_t c_stage = (static_cast<uint32_t>(bn) * BK * bits / 8 + 1023) / 1024 * 1024;
     const uint32_t per_stage = a_stage + b_stage + c_stage;
@@ -753,7 +850,7 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     prm.bar_off = prm.sb_off + sb_ring;
     prm.b_stage_bytes = b_stage;
     prm.c_stage_bytes = c_stage;
-    prm.tmem_cols = 2 * bn <= 256 ? 256 : 512;
+    prm.tmem_cols = 2 * ms * bn <= 256 ? 256 : 512;
     prm.splits = plan.splits;
     const size_t smem = prm.bar_off + (4 * stages + 8) * 8 + 16 + 1024;  // + alignment slack
     const int tiles = prm.m_tiles * prm.n_tiles;
@@ -761,12 +858,21 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
                           const TcParams);
     if (plan.splits == 1) {
         const int grid = tiles < num_sms ? tiles : num_sms;
-        Kern k = transpose ? (bits == 4 ? tc_qmm_kernel<4, false, false>
-                              : bits == 8 ? tc_qmm_kernel<8, false, false>
-                                          : tc_qmm_kernel<2, false, false>)
-                           : (bits == 4 ? tc_qmm_kernel<4, false, true>
-                              : bits == 8 ? tc_qmm_kernel<8, false, true>
-                                          : tc_qmm_kernel<2, false, true>);
+        Kern k;
+        if (ms == 2)
+            k = transpose ? (bits == 4 ? tc_qmm_kernel<4, false, false, 2>
+                             : bits == 8 ? tc_qmm_kernel<8, false, false, 2>
+                                         : tc_qmm_kernel<2, false, false, 2>)
+                          : (bits == 4 ? tc_qmm_kernel<4, false, true, 2>
+                             : bits == 8 ? tc_qmm_kernel<8, false, true, 2>
+                                         : tc_qmm_kernel<2, false, true, 2>);
+        else
+            k = transpose ? (bits == 4 ? tc_qmm_kernel<4, false, false>
+                             : bits == 8 ? tc_qmm_kernel<8, false, false>
+                                         : tc_qmm_kernel<2, false, false>)
+                          : (bits == 4 ? tc_qmm_kernel<4, false, true>
+                             : bits == 8 ? tc_qmm_kernel<8, false, true>
+                                         : tc_qmm_kernel<2, false, true>);
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
