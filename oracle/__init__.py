@@ -70,6 +70,16 @@ def _bind(lib):
     lib.orc_moe_swiglu.argtypes = [_p, _i, _i64, _i64, _p, _p, _i, _i64, _i64,
                                    _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p]
     lib.orc_moe_swiglu.restype = _i
+    lib.orc_quantize_fp.argtypes = [_p, _i, _i64, _i64, _i, _p, _p]
+    lib.orc_quantize_fp.restype = _i
+    lib.orc_dequantize_fp.argtypes = [_p, _p, _i64, _i64, _i, _p]
+    lib.orc_dequantize_fp.restype = _i
+    lib.orc_qmm_fp.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _i, _p, _p]
+    lib.orc_qmm_fp.restype = _i
+    lib.orc_fp_value.argtypes = [_i, C.c_uint32]
+    lib.orc_fp_value.restype = C.c_double
+    lib.orc_fp_nearest.argtypes = [_i, C.c_double]
+    lib.orc_fp_nearest.restype = C.c_uint32
     return lib
 
 
@@ -316,3 +326,68 @@ def within_tolerance(y, y_ref, a, dtype) -> torch.Tensor:
     """Element-wise acceptance mask of the product tolerance."""
     err = (y.to(torch.float64) - y_ref).abs()
     return err <= TOL_REL[dtype] * a + TOL_ABS
+
+
+# ---- floating-point modes ("Docs / Quantization", section "Floating-point
+# formats"): MXFP4 = E2M1 values with an E8M0 scale per 32, MXFP8 = E4M3
+# values with an E8M0 scale per 32, NVFP4 = E2M1 values with an E4M3 scale per
+# 16 (the published definitions of the names; the pages' own table of the
+# formats did not survive extraction). Parity with MLX's quantizer is unpinned.
+FP_MODES = {"mxfp4": 1, "mxfp8": 2, "nvfp4": 3}
+FP_GROUP = {"mxfp4": 32, "mxfp8": 32, "nvfp4": 16}
+FP_BITS = {"mxfp4": 4, "mxfp8": 8, "nvfp4": 4}
+
+
+def quantize_fp(w: torch.Tensor, mode: str, lib=None):
+    """Codes [rows, cols*bits/32] (uint32 as int32) and uint8 scale codes
+    [rows, cols/group] of w [rows, cols] (fp32 or bf16) in a floating-point mode."""
+    lib = lib or load()
+    w = _cpu(w)
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    codes = torch.zeros(*w.shape[:-1], cols * FP_BITS[mode] // 32, dtype=torch.int32)
+    scales = torch.empty(*w.shape[:-1], cols // FP_GROUP[mode], dtype=torch.uint8)
+    rc = lib.orc_quantize_fp(w.data_ptr(), _DT[w.dtype], rows, cols, FP_MODES[mode],
+                             codes.data_ptr(), scales.data_ptr())
+    _check(rc, "quantize_fp")
+    return codes, scales
+
+
+def dequantize_fp(codes, scales, mode: str, lib=None) -> torch.Tensor:
+    """element value x scale value, as bf16 [rows, cols]."""
+    lib = lib or load()
+    codes, scales = _cpu(codes), _cpu(scales)
+    cols = codes.shape[-1] * 32 // FP_BITS[mode]
+    rows = codes.numel() // codes.shape[-1]
+    out = torch.empty(*codes.shape[:-1], cols, dtype=torch.int16)
+    rc = lib.orc_dequantize_fp(codes.data_ptr(), scales.data_ptr(), rows, cols, FP_MODES[mode],
+                               out.data_ptr())
+    _check(rc, "dequantize_fp")
+    return out.view(torch.bfloat16)
+
+
+def qmm_fp(x, codes, scales, mode: str, lib=None):
+    """(y, a): y = x . w_hat^T in fp64 with weights [N, K] in a floating-point
+    mode, and a = sum_k |x w_hat| (the tolerance's scale)."""
+    lib = lib or load()
+    x, codes, scales = _cpu(x), _cpu(codes), _cpu(scales)
+    M, K = x.shape
+    N = codes.shape[0]
+    y = torch.empty(M, N, dtype=torch.float64)
+    a = torch.empty(M, N, dtype=torch.float64)
+    rc = lib.orc_qmm_fp(x.data_ptr(), _DT[x.dtype], M, K, N, codes.data_ptr(), scales.data_ptr(),
+                        FP_MODES[mode], y.data_ptr(), a.data_ptr())
+    _check(rc, "qmm_fp")
+    return y, a
+
+
+def fp_value(kind: str, code: int, lib=None) -> float:
+    """Value of one code: kind 'e2m1', 'e4m3' (elements) or 'e8m0' (scales)."""
+    lib = lib or load()
+    return lib.orc_fp_value({"e2m1": 0, "e4m3": 1, "e8m0": 2}[kind], code)
+
+
+def fp_nearest(kind: str, v: float, lib=None) -> int:
+    """Nearest code of v in 'e2m1' or 'e4m3' (ties to even, saturating)."""
+    lib = lib or load()
+    return lib.orc_fp_nearest({"e2m1": 0, "e4m3": 1}[kind], v)

@@ -187,6 +187,69 @@ const void* row_ptr(const void* base, int dtype, int64_t row, int64_t len) {
     return (const char*)base + (size_t)row * (size_t)len * esz;
 }
 
+// ---- floating-point modes ["Docs / Quantization", section "Floating-point
+// formats": every value a small float, one shared scale per group stored as
+// a uint8 code, no biases; dequantized to bfloat16]. The pages' table of the
+// formats did not survive extraction, so the formats are the published
+// definitions of the three names:
+//   MXFP4: E2M1 values, one E8M0 scale per 32 values;
+//   MXFP8: E4M3 values (no infinities), one E8M0 scale per 32 values;
+//   NVFP4: E2M1 values, one E4M3 scale per 16 values.
+// Codes pack like the affine codes (code j of a word at bits [j*b, (j+1)*b)).
+enum { FP_MXFP4 = 1, FP_MXFP8 = 2, FP_NVFP4 = 3 };
+
+int fp_group(int mode) { return mode == FP_NVFP4 ? 16 : 32; }
+int fp_bits(int mode) { return mode == FP_MXFP8 ? 8 : 4; }
+
+// E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0; exponent 0
+// is subnormal (0.5 * mantissa).
+double e2m1_value(uint32_t c) {
+    const int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    const double mag = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+// E4M3 without infinities: sign bit 7, exponent bits 6..3 (bias 7), mantissa
+// bits 2..0; exponent 0 is subnormal (mantissa / 8 * 2^-6); S.1111.111 is NaN.
+double e4m3_value(uint32_t c) {
+    const int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return std::nan("");
+    const double mag = e == 0 ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+// E8M0: 2^(code - 127); code 255 is NaN.
+double e8m0_value(uint32_t c) { return c == 255 ? std::nan("") : std::ldexp(1.0, (int)c - 127); }
+
+// The code of a finite value in E2M1 (elem = 0) or E4M3 (elem = 1): the sign
+// of v, and the magnitude of the grid nearest to |v|, ties to the code whose
+// mantissa field is even, magnitudes past the largest finite one saturated to
+// it. Brute force over the grid.
+uint32_t nearest_code(double v, int elem) {
+    const uint32_t sign_bit = elem == 0 ? 8u : 128u;
+    const uint32_t top = elem == 0 ? 7u : 126u;  // largest finite magnitude code
+    const double a = std::fabs(v);
+    uint32_t best = 0;
+    double best_d = a;  // distance to code 0 (zero)
+    for (uint32_t c = 1; c <= top; ++c) {
+        const double g = elem == 0 ? e2m1_value(c) : e4m3_value(c);
+        const double d = std::fabs(a - g);
+        if (d < best_d || (d == best_d && (c & 1u) == 0u)) { best = c; best_d = d; }
+    }
+    const double gmax = elem == 0 ? e2m1_value(top) : e4m3_value(top);
+    if (a >= gmax) best = top;
+    return std::signbit(v) ? (best | sign_bit) : best;
+}
+
+// Value of element code c and scale code s of a mode.
+double fp_element(int mode, uint32_t c) { return mode == FP_MXFP8 ? e4m3_value(c) : e2m1_value(c); }
+double fp_scale(int mode, uint32_t s) { return mode == FP_NVFP4 ? e4m3_value(s) : e8m0_value(s); }
+
+double fp_dequant_at(const uint32_t* codes, const uint8_t* scales, int mode, int64_t row, int64_t col,
+                     int64_t cols) {
+    const int gs = fp_group(mode), bits = fp_bits(mode);
+    const uint32_t c = code_at(codes, row, col, cols, bits);
+    return fp_element(mode, c) * fp_scale(mode, scales[row * (cols / gs) + col / gs]);
+}
+
 }  // namespace
 
 extern "C" {
@@ -493,5 +556,113 @@ int orc_moe_swiglu(const void* x, int xdtype, int64_t T, int64_t K, const uint32
     }
     return 0;
 }
+
+
+// Quantizer of the floating-point modes ["Docs / Quantization", section
+// "Floating-point formats"; the scale rule is the shared-exponent rule of the
+// published microscaling formats, written out step by step]. w [rows, cols]
+// in `dtype` (fp32 or bf16), groups along cols. Writes codes [rows,
+// cols*bits/32] and scale codes [rows, cols/gs] (uint8). Returns 0, or -1 on
+// bad arguments.
+//   MXFP4 / MXFP8: amax = max |w| of the group; X = 2^(floor(log2 amax) -
+//   emax), emax = 2 (E2M1) or 8 (E4M3), the scale code clamped to 0..254 (an
+//   all-zero group gets code 0); each code is the nearest element of w / X
+//   (exact: X is a power of two).
+//   NVFP4: the scale is fl32(amax / 6) rounded to E4M3; each code is the
+//   nearest element of fl32(w / S), S the stored scale (code 0 when S is 0).
+int orc_quantize_fp(const void* w, int dtype, int64_t rows, int64_t cols, int mode,
+                    uint32_t* codes, uint8_t* scales) {
+    if (mode != FP_MXFP4 && mode != FP_MXFP8 && mode != FP_NVFP4) return -1;
+    const int gs = fp_group(mode), bits = fp_bits(mode);
+    if (rows < 0 || cols <= 0 || cols % gs != 0) return -1;
+    if (std::fegetround() != FE_TONEAREST) return -1;
+    const int64_t groups = cols / gs;
+    const int per_word = 32 / bits;
+    const int elem = mode == FP_MXFP8 ? 1 : 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const int64_t c0 = g * gs;
+            // Step 1: the group's largest magnitude.
+            float amax = 0.0f;
+            for (int i = 0; i < gs; ++i) amax = std::fmax(amax, std::fabs(load_f32(w, dtype, r * cols + c0 + i)));
+            // Step 2: the shared scale.
+            uint32_t scode = 0;
+            if (mode == FP_NVFP4) {
+                const float sv = amax / 6.0f;
+                scode = nearest_code((double)sv, 1) & 127u;
+            } else if (amax > 0.0f) {
+                int ex = 0;
+                std::frexp((double)amax, &ex);            // amax = f * 2^ex, f in [0.5, 1)
+                const int e = (ex - 1) - (elem == 0 ? 2 : 8);  // floor(log2 amax) - emax
+                int sc = e + 127;
+                if (sc < 0) sc = 0;
+                if (sc > 254) sc = 254;
+                scode = (uint32_t)sc;
+            }
+            scales[r * groups + g] = (uint8_t)scode;
+            const double sval = fp_scale(mode, scode);
+            // Step 3: one element code per value, then pack.
+            for (int i = 0; i < gs; ++i) {
+                const float v = load_f32(w, dtype, r * cols + c0 + i);
+                uint32_t q = 0;
+                if (mode == FP_NVFP4) {
+                    if (sval != 0.0) q = nearest_code((double)(v / (float)sval), 0);
+                } else {
+                    q = nearest_code((double)v / sval, elem);
+                }
+                const int64_t col = c0 + i;
+                const int64_t wi = r * words_per_row(cols, bits) + col / per_word;
+                const int j = (int)(col % per_word);
+                if (j == 0) codes[wi] = 0u;
+                codes[wi] |= q << (j * bits);
+            }
+        }
+    }
+    return 0;
+}
+
+// Dequantized weights of a floating-point mode, element value times scale
+// value, as bf16 bit patterns (rounded once to nearest even; exact whenever
+// the product is a bf16 number, which it is outside extreme underflow).
+int orc_dequantize_fp(const uint32_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                      int mode, uint16_t* out) {
+    if (mode != FP_MXFP4 && mode != FP_MXFP8 && mode != FP_NVFP4) return -1;
+    if (cols <= 0 || cols % fp_group(mode) != 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = f64_to_bf16(fp_dequant_at(codes, scales, mode, r, c, cols));
+    return 0;
+}
+
+// Product with floating-point-mode weights [N, K] ("Floating-point formats":
+// quantized_matmul(q, transpose = true) in x's dtype): y[m, n] = sum_k
+// x[m, k] * w_hat(n, k) in fp64, k in order, and a[m, n] = sum_k |x w_hat|.
+int orc_qmm_fp(const void* x, int xdtype, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+               const uint8_t* scales, int mode, double* y, double* a) {
+    if (mode != FP_MXFP4 && mode != FP_MXFP8 && mode != FP_NVFP4) return -1;
+    if (K <= 0 || K % fp_group(mode) != 0 || M < 0 || N < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M * N; ++i) {
+        const int64_t m = i / N, n = i % N;
+        double acc = 0.0, mag = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double p = load_value(x, xdtype, m * K + k) * fp_dequant_at(codes, scales, mode, n, k, K);
+            acc += p;
+            mag += std::fabs(p);
+        }
+        y[i] = acc;
+        a[i] = mag;
+    }
+    return 0;
+}
+
+// Single values of the formats, for the pins: element (elem 0 = E2M1, 1 =
+// E4M3) or scale (2 = E8M0) code -> value, and value -> nearest element code.
+double orc_fp_value(int kind, uint32_t code) {
+    return kind == 0 ? e2m1_value(code) : kind == 1 ? e4m3_value(code) : e8m0_value(code);
+}
+uint32_t orc_fp_nearest(int elem, double v) { return nearest_code(v, elem); }
 
 }  // extern "C"

@@ -558,4 +558,147 @@ def pin_sampled_match_full(lib):
     assert torch.equal(ys, y[ri, ni]) and torch.equal(as_, a[ri, ni])
 
 
+# ---- floating-point modes ("Docs / Quantization", section "Floating-point
+# formats"; the formats are the published definitions of MXFP4 / MXFP8 / NVFP4)
+
+# E2M1 magnitudes listed in the microscaling format definition, codes 0..7.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def pin_fp_element_and_scale_values(lib):
+    """Codes -> values from the format definitions: the E2M1 list with its
+    sign bit, E4M3 (bias 7, no infinities, S.1111.111 NaN) and E8M0 (2^(s-127),
+    255 NaN) at their edges."""
+    for c in range(16):
+        want = E2M1_TABLE[c & 7] * (-1.0 if c & 8 else 1.0)
+        got = O.fp_value("e2m1", c, lib=lib)
+        assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), (c, got)
+    e4m3 = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+            0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0}
+    for c, want in e4m3.items():
+        assert O.fp_value("e4m3", c, lib=lib) == want, (hex(c), want)
+    assert math.isnan(O.fp_value("e4m3", 0x7F, lib=lib)) and math.isnan(O.fp_value("e4m3", 0xFF, lib=lib))
+    assert O.fp_value("e4m3", 0x77, lib=lib) == 240.0  # 2^7 * (1 + 7/8)
+    for c, want in {127: 1.0, 0: 2.0 ** -127, 254: 2.0 ** 127, 128: 2.0, 120: 2.0 ** -7}.items():
+        assert O.fp_value("e8m0", c, lib=lib) == want, (c, want)
+    assert math.isnan(O.fp_value("e8m0", 255, lib=lib))
+
+
+def pin_fp_nearest_ties_and_saturation(lib):
+    """Round to nearest, ties to the even mantissa field, saturate at the
+    largest finite value (E2M1 6, E4M3 448); the sign follows the value."""
+    e2m1 = {0.25: 0.0, 0.26: 0.5, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0,
+            5.01: 6.0, 6.0: 6.0, 7.0: 6.0, 1e30: 6.0, -2.5: -2.0, -0.2: -0.0, -5.5: -6.0}
+    for v, want in e2m1.items():
+        got = O.fp_value("e2m1", O.fp_nearest("e2m1", v, lib=lib), lib=lib)
+        assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), (v, got, want)
+    e4m3 = {1.0 + 1 / 16: 1.0, 1.0 + 3 / 16: 1.25, 2.0 ** -10: 0.0, 3 * 2.0 ** -10: 2.0 ** -8,
+            464.0: 448.0, 1e9: 448.0, -(1.0 + 1 / 16): -1.0, 240.0: 240.0, 248.0: 256.0}
+    for v, want in e4m3.items():
+        assert O.fp_value("e4m3", O.fp_nearest("e4m3", v, lib=lib), lib=lib) == want, (v, want)
+
+
+def _fp_group_row(vals, gs):
+    return torch.tensor([(vals * ((gs + len(vals) - 1) // len(vals)))[:gs]], dtype=torch.float32)
+
+
+def pin_fp_mx_scale_rule(lib):
+    """MXFP4 / MXFP8: X = 2^(floor(log2 amax) - emax), emax 2 (E2M1) or 8 (E4M3):
+    amax in [4, 8) * 2^k gives scale code 127 + k at 4 bits, amax in [256, 512)
+    * 2^k gives 127 + k at 8 bits; a zero group gets scale code 0 and zero codes."""
+    for k in (-20, -3, 0, 5, 40):
+        for amax, want in ((4.0, 127), (6.0, 127), (7.99, 127), (8.0, 128), (3.99, 126)):
+            w = _fp_group_row([0.5, -1.0, amax * 2.0 ** k / 2 ** k], 32) * 2.0 ** k
+            w[0, 0] = amax * 2.0 ** k
+            _, s = O.quantize_fp(w, "mxfp4", lib=lib)
+            assert int(s[0, 0]) == want + k, (k, amax, int(s[0, 0]))
+        for amax, want in ((256.0, 127), (448.0, 127), (511.0, 127), (512.0, 128)):
+            w = torch.zeros(1, 32)
+            w[0, 5] = amax * 2.0 ** k
+            w[0, 6] = -1.0 * 2.0 ** k
+            _, s = O.quantize_fp(w, "mxfp8", lib=lib)
+            assert int(s[0, 0]) == want + k, (k, amax, int(s[0, 0]))
+    c, s = O.quantize_fp(torch.zeros(2, 64), "mxfp4", lib=lib)
+    assert (s == 0).all() and (c == 0).all()
+    # the saturating step: a 7.5 * 2^k value in a group whose scale is 2^k
+    w = torch.tensor([[7.5, 1.0] + [0.0] * 30])
+    c, s = O.quantize_fp(w, "mxfp4", lib=lib)
+    wh = O.dequantize_fp(c, s, "mxfp4", lib=lib).float()
+    assert int(s[0, 0]) == 127 and wh[0, 0] == 6.0 and wh[0, 1] == 1.0
+
+
+def pin_fp_grid_round_trip(lib):
+    """Values already on a mode's grid come back exactly: E2M1 values (both
+    signs) times 2^k for MXFP4, E4M3 values for MXFP8, E2M1 values times an
+    E4M3 scale S = amax / 6 for NVFP4; dequantized to bf16 exactly."""
+    g = torch.Generator().manual_seed(7)
+    for k in (-9, 0, 3):
+        vals = torch.tensor(E2M1_TABLE + [-v for v in E2M1_TABLE[1:]] + [6.0] * 17)[:32] * 2.0 ** k
+        vals = vals[torch.randperm(32, generator=g)].view(1, 32)
+        c, s = O.quantize_fp(vals, "mxfp4", lib=lib)
+        assert int(s[0, 0]) == 127 + k
+        assert torch.equal(O.dequantize_fp(c, s, "mxfp4", lib=lib).float(), vals)
+    e4m3_vals = torch.tensor([O.fp_value("e4m3", c, lib=lib) for c in range(0, 127, 4)])
+    vals = e4m3_vals.clone()
+    vals[0] = 448.0  # amax 448: scale 2^0
+    vals = vals.view(1, 32)
+    c, s = O.quantize_fp(vals, "mxfp8", lib=lib)
+    assert int(s[0, 0]) == 127
+    assert torch.equal(O.dequantize_fp(c, s, "mxfp8", lib=lib).float(), vals)
+    for S in (1.0, 1.25, 0.09375, 3.5):  # E4M3 numbers
+        base = torch.tensor(E2M1_TABLE + [-v for v in E2M1_TABLE])[:16]
+        base[3] = 6.0
+        vals = (base * S).view(1, 16)
+        c, s = O.quantize_fp(vals, "nvfp4", lib=lib)
+        assert O.fp_value("e4m3", int(s[0, 0]), lib=lib) == S, (S, int(s[0, 0]))
+        assert torch.equal(O.dequantize_fp(c, s, "nvfp4", lib=lib).float(), vals), S
+
+
+def pin_fp_round_trip_bound(lib):
+    """Random groups: every MXFP4 value is within half the E2M1 grid step of
+    w / X (times X), or saturated at 6X; NVFP4 the same with the stored scale;
+    the codes pack 8 to a word and unpack by division and remainder."""
+    g = torch.Generator().manual_seed(11)
+    w = torch.randn(8, 256, generator=g) * (10.0 ** (torch.rand(8, 1, generator=g) * 4 - 2))
+    for mode, gs in (("mxfp4", 32), ("nvfp4", 16)):
+        c, s = O.quantize_fp(w, mode, lib=lib)
+        codes = _unpack_div_mod(c, 4)
+        kind = "e8m0" if mode == "mxfp4" else "e4m3"
+        X = torch.tensor([[O.fp_value(kind, int(v), lib=lib) for v in row] for row in s.tolist()],
+                         dtype=torch.float64).repeat_interleave(gs, dim=1)
+        elem = torch.tensor([[E2M1_TABLE[q & 7] * (-1.0 if q & 8 else 1.0) for q in row]
+                             for row in codes.tolist()], dtype=torch.float64)
+        t = w.double() / X
+        step = torch.where(t.abs() < 2, 0.5, torch.where(t.abs() < 4, 1.0, 2.0))
+        ok = ((elem - t).abs() <= step / 2 + 1e-6) | ((t.abs() >= 6) & (elem.abs() == 6))
+        assert ok.all(), (mode, int((~ok).sum()))
+        wh = O.dequantize_fp(c, s, mode, lib=lib).double()
+        assert torch.equal(wh, (elem * X).to(torch.bfloat16).double())
+
+
+def pin_fp_products(lib):
+    """qmm_fp against a brute force over unpacked codes: on-grid weights with
+    scale 1 and integer x give exact results (8 x 8 outputs), and a random case
+    agrees with fp64 sums of the dequantized weights."""
+    g = torch.Generator().manual_seed(13)
+    idx = torch.randint(0, 16, (8, 64), generator=g)
+    w = torch.tensor([[E2M1_TABLE[q & 7] * (-1.0 if q & 8 else 1.0) for q in row] for row in idx.tolist()])
+    w[:, 0] = 6.0
+    w[:, 32] = -6.0
+    x = torch.randint(-2, 3, (8, 64), generator=g).float()
+    c, s = O.quantize_fp(w, "mxfp4", lib=lib)
+    y, a = O.qmm_fp(x, c, s, "mxfp4", lib=lib)
+    brute = [[sum(x[m, k].item() * w[n, k].item() for k in range(64)) for n in range(8)] for m in range(8)]
+    assert torch.equal(y, torch.tensor(brute, dtype=torch.float64))
+    assert torch.equal(a, (x.double().abs() @ w.double().abs().t()))
+    w = torch.randn(16, 96, generator=g)
+    x = torch.randn(3, 96, generator=g).to(torch.bfloat16)
+    for mode in ("mxfp4", "mxfp8", "nvfp4"):
+        c, s = O.quantize_fp(w, mode, lib=lib)
+        wh = O.dequantize_fp(c, s, mode, lib=lib).double()
+        y, a = O.qmm_fp(x, c, s, mode, lib=lib)
+        ref = x.double() @ wh.t()
+        assert torch.allclose(y, ref, rtol=0, atol=1e-12), mode
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -70,6 +70,16 @@ MUTANTS = [
      "const int64_t e = (int64_t)ids[t * topk + j] % E;"),
     ("down transposed", "dequant_at(dc, dsc, dbi, sdtype, n, i, I, gs, bits)",
      "dequant_at(dc, dsc, dbi, sdtype, i, n, K, gs, bits)"),
+    ("e2m1 exponent bias", "std::ldexp(1.0 + 0.5 * m, e - 1)", "std::ldexp(1.0 + 0.5 * m, e - 2)"),
+    ("e4m3 exponent bias", "std::ldexp(1.0 + m / 8.0, e - 7)", "std::ldexp(1.0 + m / 8.0, e - 8)"),
+    ("e8m0 bias", "std::ldexp(1.0, (int)c - 127)", "std::ldexp(1.0, (int)c - 128)"),
+    ("fp ties to larger", "(d == best_d && (c & 1u) == 0u)", "(d == best_d)"),
+    ("fp no saturation", "if (a >= gmax) best = top;", "(void)gmax;"),
+    ("fp sign dropped", "return std::signbit(v) ? (best | sign_bit) : best;", "return best;"),
+    ("mx scale rounds up", "const int e = (ex - 1) - (elem == 0 ? 2 : 8);",
+     "const int e = ex - (elem == 0 ? 2 : 8);"),
+    ("nvfp4 scale over 4", "const float sv = amax / 6.0f;", "const float sv = amax / 4.0f;"),
+    ("fp scale index", "scales[row * (cols / gs) + col / gs]", "scales[row * (cols / gs) + col / (2 * gs)]"),
 ]
 
 RUNNER = r"""
