@@ -14,13 +14,16 @@ from .binding import (  # noqa: F401
     nv_gather_qmm_flags,
     nv_gather_qmm_workspace_size,
     nv_dequantize_affine,
+    nv_dequantize_fp,
     nv_moe_swiglu,
     nv_moe_swiglu_workspace_size,
     nv_pipeline_error,
     nv_pipeline_selftest,
     nv_qmm,
     nv_qmm_batched,
+    nv_qmm_fp,
     nv_qmm_splits,
     nv_quantize_affine,
+    nv_quantize_fp,
     nv_status_string,
 )

@@ -29,7 +29,10 @@ EXPORTS = ("nv_status_string", "nv_quantize_affine", "nv_dequantize_affine", "nv
            "nv_gather_qmm_workspace_size", "nv_gather_mm",
            "nv_gather_qmm", "nv_gather_qmm_flags", "nv_pipeline_error", "nv_pipeline_selftest",
            "nv_last_cuda_error",
-           "nv_gather_qmm_noalloc")
+           "nv_gather_qmm_noalloc", "nv_quantize_fp", "nv_dequantize_fp", "nv_qmm_fp")
+NV_FP_MODES = {"mxfp4": 1, "mxfp8": 2, "nvfp4": 3}
+_FP_GROUP = {"mxfp4": 32, "mxfp8": 32, "nvfp4": 16}
+_FP_BITS = {"mxfp4": 4, "mxfp8": 8, "nvfp4": 4}
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16}
 _LOCK = threading.Lock()
@@ -96,6 +99,12 @@ def lib():
             L.nv_pipeline_error.restype = _i
             L.nv_pipeline_selftest.argtypes = [C.c_uint32, _p]
             L.nv_pipeline_selftest.restype = _i
+            L.nv_quantize_fp.argtypes = [_p, _i, _i64, _i64, _i, _p, _p, _p]
+            L.nv_quantize_fp.restype = _i
+            L.nv_dequantize_fp.argtypes = [_p, _p, _i64, _i64, _i, _p, _p]
+            L.nv_dequantize_fp.restype = _i
+            L.nv_qmm_fp.argtypes = [_p, _i, _i64, _i64, _i64, _p, _p, _i, _p, _p]
+            L.nv_qmm_fp.restype = _i
             _LIB = L
         return _LIB
 
@@ -384,3 +393,69 @@ def nv_pipeline_selftest(limit_us: int = 1000, stream=None) -> None:
     limit_us and records code 0x5E (read it with nv_pipeline_error)."""
     st = lib().nv_pipeline_selftest(int(limit_us), _stream(stream))
     _check("nv_pipeline_selftest", st)
+
+
+def _fp_mode(mode: str) -> int:
+    if mode not in NV_FP_MODES:
+        raise ValueError(f"mode must be one of {sorted(NV_FP_MODES)}")
+    return NV_FP_MODES[mode]
+
+
+def nv_quantize_fp(w: torch.Tensor, mode: str = "mxfp4", stream=None):
+    """Codes [..., rows, cols * b / 32] (uint32 as int32) and uint8 scale codes
+    [..., rows, cols / group] of w [..., rows, cols] in a floating-point mode
+    ('mxfp4', 'mxfp8', 'nvfp4')."""
+    m = _fp_mode(mode)
+    _dev(w, "w")
+    cols = w.shape[-1]
+    rows = w.numel() // cols if cols else 0
+    codes = torch.empty(*w.shape[:-1], cols * _FP_BITS[mode] // 32, dtype=torch.int32, device=w.device)
+    scales = torch.empty(*w.shape[:-1], cols // _FP_GROUP[mode], dtype=torch.uint8, device=w.device)
+    st = lib().nv_quantize_fp(w.data_ptr(), _DT.get(w.dtype, -1), rows, cols, m, codes.data_ptr(),
+                              scales.data_ptr(), _stream(stream))
+    _check("nv_quantize_fp", st)
+    return codes, scales
+
+
+def nv_dequantize_fp(codes: torch.Tensor, scales: torch.Tensor, mode: str = "mxfp4",
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16 [..., rows, cols]: element value times scale value."""
+    m = _fp_mode(mode)
+    _dev(codes, "codes")
+    _dev(scales, "scales")
+    cols = codes.shape[-1] * 32 // _FP_BITS[mode]
+    rows = codes.numel() // codes.shape[-1] if codes.shape[-1] else 0
+    if scales.dtype != torch.uint8 or tuple(scales.shape) != (*codes.shape[:-1], cols // _FP_GROUP[mode]):
+        raise ValueError("scales must be uint8 [..., rows, cols / group]")
+    w = out if out is not None else torch.empty(*codes.shape[:-1], cols, dtype=torch.bfloat16,
+                                                device=codes.device)
+    if w.numel() != rows * cols or w.dtype != torch.bfloat16:
+        raise ValueError("out has the wrong size or dtype")
+    _dev(w, "out")
+    st = lib().nv_dequantize_fp(codes.data_ptr(), scales.data_ptr(), rows, cols, m, w.data_ptr(),
+                                _stream(stream))
+    _check("nv_dequantize_fp", st)
+    return w
+
+
+def nv_qmm_fp(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, mode: str = "mxfp4",
+              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x . w^T with floating-point-mode weights [N, K]; bf16 x and y."""
+    m = _fp_mode(mode)
+    for t, n in ((x, "x"), (codes, "codes"), (scales, "scales")):
+        _dev(t, n)
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    if codes.dim() != 2 or scales.dim() != 2 or scales.dtype != torch.uint8:
+        raise ValueError("codes and uint8 scales must be 2-D")
+    N = codes.shape[0]
+    if tuple(codes.shape) != (N, K * _FP_BITS[mode] // 32) or tuple(scales.shape) != (N, K // _FP_GROUP[mode]):
+        raise ValueError(f"weights do not match x: codes {tuple(codes.shape)}, scales {tuple(scales.shape)}")
+    y = out if out is not None else torch.empty(*x.shape[:-1], N, dtype=x.dtype, device=x.device)
+    if y.numel() != M * N or y.dtype != x.dtype:
+        raise ValueError("out has the wrong size or dtype")
+    _dev(y, "out")
+    st = lib().nv_qmm_fp(x.data_ptr(), _DT.get(x.dtype, -1), M, K, N, codes.data_ptr(), scales.data_ptr(), m,
+                         y.data_ptr(), _stream(stream))
+    _check("nv_qmm_fp", st)
+    return y

@@ -13,7 +13,7 @@ bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs);
 cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                           const void* scales, const void* biases, int gs, int bits, void* y,
                           cudaStream_t stream, int num_sms, int64_t item_rows = 0,
-                          int transpose = 1);
+                          int transpose = 1, int fmt = 0);
 bool tc_supported_t0(int64_t M, int64_t K, int64_t N, int bits, int gs);
 // K-partitions the tiled kernel uses for an item of m_rows rows (1: no split).
 int tc_splits(int64_t m_rows, int64_t K, int64_t N, int num_sms, int bits, int transpose);

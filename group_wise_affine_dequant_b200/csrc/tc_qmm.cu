@@ -35,6 +35,7 @@
 // Every wait on an mbarrier is bounded by a timer; on expiry the kernel records
 // an error code, stops issuing work and exits after draining its copies.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -106,7 +107,38 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int BITS, bool SPLIT, bool TR0, int MS = 1>
+// Floating-point modes (FMT 1 = MXFP4, 2 = MXFP8, 3 = NVFP4): codes decode
+// exactly to f16 pairs by the hardware conversion, widen to fp32, take the
+// group's scale (E8M0 or E4M3 code, one uint8 per group) and round once to
+// bf16 pairs: the products of small floats and their scales are bf16 numbers,
+// so the B tile holds the exact dequantized weights.
+__device__ __forceinline__ float fp_scale(int fmt, uint32_t code) {
+    if (fmt == 3) {
+        uint32_t h;
+        asm("{\n\t.reg .b16 s;\n\tcvt.u16.u32 s, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, s;\n\t}" : "=r"(h) : "r"(code & 255u));
+        return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+    }
+    return code == 0 ? __uint_as_float(0x00400000u) : code == 255 ? __uint_as_float(0x7FC00000u)
+                                                                  : __uint_as_float(code << 23);
+}
+template <int FMT>
+__device__ __forceinline__ void fp_dequant_word(uint32_t w, float S, uint32_t* out) {
+    constexpr int PAIRS = FMT == 2 ? 2 : 4;
+#pragma unroll
+    for (int i = 0; i < PAIRS; ++i) {
+        uint32_t h;
+        if constexpr (FMT == 2)
+            asm("{\n\t.reg .b16 s;\n\tcvt.u16.u32 s, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, s;\n\t}" : "=r"(h) : "r"((w >> (16 * i)) & 0xFFFFu));
+        else
+            asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h) : "r"((w >> (8 * i)) & 255u));
+        float lo, hi;
+        asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+            : "=f"(lo), "=f"(hi) : "r"(h));
+        out[i] = f2_to_bf2(lo * S, hi * S);
+    }
+}
+
+template <int BITS, bool SPLIT, bool TR0, int MS = 1, int FMT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_b,
@@ -479,8 +511,14 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                         bc = bf16_bits_to_f32(ss[BN * 8 + r * 8 + gi]);
                     }
                 } else if (live) {
-                    sc = bf16_bits_to_f32(__ldg(srow + g));
-                    bc = bf16_bits_to_f32(__ldg(brow + g));
+                    if constexpr (FMT != 0) {  // uint8 scale codes; NVFP4: a second group for k 16..31
+                        const uint8_t* s8 = reinterpret_cast<const uint8_t*>(prm.scales) + n * gpr;
+                        sc = fp_scale(FMT, __ldg(s8 + g));
+                        bc = (FMT == 3 && kpart == 32) ? fp_scale(FMT, __ldg(s8 + g + 1)) : sc;
+                    } else {
+                        sc = bf16_bits_to_f32(__ldg(srow + g));
+                        bc = bf16_bits_to_f32(__ldg(brow + g));
+                    }
                 }
                 if (!(ok = mbar_wait(&full_c[s], use & 1, 6))) break;
                 // one dequantizer for the warp's step: the fast form when every
@@ -509,7 +547,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
                     uint32_t out[16];
-                    if (fast) {
+                    if constexpr (FMT != 0) {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i)  // NVFP4: words 2, 3 hold k 16..31 (second group)
+                            fp_dequant_word<FMT>(w[i], (FMT == 3 && i >= 2) ? bc : sc, out + i * DQ::PAIRS);
+                    } else if (fast) {
 #pragma unroll
                         for (int i = 0; i < NW; ++i) DQ::run_fast(w[i], s2, b2, out + i * DQ::PAIRS);
                     } else {
@@ -544,7 +586,10 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
                     const uint32_t s2 = (__float_as_uint(sc) >> 16) * 0x00010001u;
                     const uint32_t b2 = (__float_as_uint(bc) >> 16) * 0x00010001u;
                     uint32_t out[8];
-                    if (fast) {
+                    if constexpr (FMT != 0) {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) fp_dequant_word<FMT>(w[i], sc, out + i * DQ::PAIRS);
+                    } else if (fast) {
 #pragma unroll
                         for (int i = 0; i < NW; ++i) DQ::run_fast(w[i], s2, b2, out + i * DQ::PAIRS);
                     } else {
@@ -751,7 +796,11 @@ bool tc_supported(int64_t M, int64_t K, int64_t N, int bits, int gs) {
 
 cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
                           const void* scales, const void* biases, int gs, int bits, void* y,
-                          cudaStream_t stream, int num_sms, int64_t item_rows, int transpose) {
+                          cudaStream_t stream, int num_sms, int64_t item_rows, int transpose, int fmt) {
+    if (fmt != 0) {  // floating-point modes: weights [N, K], uint8 scale codes, no biases
+        transpose = 1;
+        biases = scales;
+    }
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     // the tiling and the split follow one item's rows (all of x for a plain
@@ -801,7 +850,7 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     // scales and biases: blocks of 8 groups x bn rows, when rows are 16-byte multiples
     CUtensorMap map_s, map_b;
     const int64_t gpr = K / gs;
-    const bool sb_tma = transpose && (gpr * 2) % 16 == 0;  // transpose = 0 loads them directly
+    const bool sb_tma = fmt == 0 && transpose && (gpr * 2) % 16 == 0;  // else loaded directly
     if (sb_tma) {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(N)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(gpr) * 2};
@@ -822,7 +871,7 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     prm.m2 = 2;
     prm.m4 = 4;
     prm.m6 = 6;
-    prm.lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
+    prm.lg_gs = gs == 16 ? 4 : gs == 32 ? 5 : gs == 64 ? 6 : 7;
     prm.y = static_cast<uint16_t*>(y);
     prm.scales = static_cast<const uint16_t*>(scales);
     prm.biases = static_cast<const uint16_t*>(biases);
@@ -859,7 +908,14 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     if (plan.splits == 1) {
         const int grid = tiles < num_sms ? tiles : num_sms;
         Kern k;
-        if (ms == 2)
+        if (fmt != 0)
+            k = ms == 2 ? (fmt == 1 ? tc_qmm_kernel<4, false, false, 2, 1>
+                           : fmt == 2 ? tc_qmm_kernel<8, false, false, 2, 2>
+                                      : tc_qmm_kernel<4, false, false, 2, 3>)
+                        : (fmt == 1 ? tc_qmm_kernel<4, false, false, 1, 1>
+                           : fmt == 2 ? tc_qmm_kernel<8, false, false, 1, 2>
+                                      : tc_qmm_kernel<4, false, false, 1, 3>);
+        else if (ms == 2)
             k = transpose ? (bits == 4 ? tc_qmm_kernel<4, false, false, 2>
                              : bits == 8 ? tc_qmm_kernel<8, false, false, 2>
                                          : tc_qmm_kernel<2, false, false, 2>)
@@ -882,12 +938,15 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     // split-K: one cluster of `splits` CTAs per tile; the partial tile
     // ([128][bn] fp32) reuses the pipeline's stages in shared memory
     if (static_cast<size_t>(BM) * bn * 4 > prm.sb_off) return cudaErrorInvalidConfiguration;
-    Kern k = transpose ? (bits == 4 ? tc_qmm_kernel<4, true, false>
-                          : bits == 8 ? tc_qmm_kernel<8, true, false>
-                                      : tc_qmm_kernel<2, true, false>)
-                       : (bits == 4 ? tc_qmm_kernel<4, true, true>
-                          : bits == 8 ? tc_qmm_kernel<8, true, true>
-                                      : tc_qmm_kernel<2, true, true>);
+    Kern k = fmt == 1   ? tc_qmm_kernel<4, true, false, 1, 1>
+             : fmt == 2 ? tc_qmm_kernel<8, true, false, 1, 2>
+             : fmt == 3 ? tc_qmm_kernel<4, true, false, 1, 3>
+             : transpose ? (bits == 4 ? tc_qmm_kernel<4, true, false>
+                            : bits == 8 ? tc_qmm_kernel<8, true, false>
+                                        : tc_qmm_kernel<2, true, false>)
+                         : (bits == 4 ? tc_qmm_kernel<4, true, true>
+                            : bits == 8 ? tc_qmm_kernel<8, true, true>
+                                        : tc_qmm_kernel<2, true, true>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -904,6 +963,18 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k, map_x, map_c, map_s, map_b, prm);
+}
+
+// Floating-point modes on the tiled kernel (weights [N, K]; mode 1 = MXFP4,
+// 2 = MXFP8, 3 = NVFP4).
+bool qmm_fp_tiled_supported(int64_t K, int mode) {
+    return K % BK == 0 && K >= BK && mode >= 1 && mode <= 3;
+}
+
+cudaError_t launch_tc_qmm_fp(const void* x, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+                             const uint8_t* scales, int mode, void* y, cudaStream_t stream, int num_sms) {
+    const int bits = mode == 2 ? 8 : 4, gs = mode == 3 ? 16 : 32;
+    return launch_tc_qmm(x, M, K, N, codes, scales, nullptr, gs, bits, y, stream, num_sms, 0, 1, mode);
 }
 
 }  // namespace nvq

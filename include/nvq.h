@@ -121,6 +121,64 @@ nv_status nv_dequantize_affine(const uint32_t* codes, const void* scales, const 
                                int bits, void* w, nv_stream_t stream);
 
 /*
+ * Floating-point quantization modes ("Docs / Quantization", section
+ * "Floating-point formats": every value stored as a small float with one
+ * shared scale per group, scales stored as uint8 codes, no biases; the
+ * dequantized weights are bfloat16; quantized_matmul(q, true) returns x's
+ * dtype). The pages' table of the formats did not survive; the modes are the
+ * published definitions of their names:
+ *   NV_MXFP4  E2M1 codes (4 bits), one E8M0 scale (2^(s - 127)) per 32 values;
+ *   NV_MXFP8  E4M3 codes (8 bits, no infinities), one E8M0 scale per 32;
+ *   NV_NVFP4  E2M1 codes, one E4M3 scale per 16 values.
+ * Codes pack like the affine codes (code j of a uint32 at bits [j*b, (j+1)*b)).
+ * Parity with MLX's own quantizer (which the pages say these equal) is not
+ * established: the scale rule used here is written out at nv_quantize_fp.
+ */
+typedef enum nv_fp_mode {
+    NV_MXFP4 = 1,
+    NV_MXFP8 = 2,
+    NV_NVFP4 = 3
+} nv_fp_mode;
+
+/*
+ * Quantizer of the floating-point modes.
+ * w       [rows, cols] in dt (NV_F32 or NV_BF16), grouped along cols
+ *         (input); cols a multiple of 32.
+ * codes   uint32 [rows, cols * b / 32] (b = 4, or 8 for NV_MXFP8), output.
+ * scales  uint8 [rows, cols / group] (group 32, or 16 for NV_NVFP4), output.
+ * Per group: amax = max |w|. MX modes: scale 2^(floor(log2 amax) - emax),
+ * emax = 2 (E2M1) or 8 (E4M3), code clamped to 0..254 (0 for an all-zero
+ * group); each code is w / scale rounded to the nearest element (ties to the
+ * even mantissa, saturated at the largest finite one: 6 or 448). NVFP4: scale
+ * = fl32(amax / 6) rounded to E4M3 the same way; codes from fl32(w / scale),
+ * all 0 when the scale is 0. Bit-exact with the oracle. Deterministic.
+ * Errors: NV_ERR_INVALID_ARG (mode, shape, null or unaligned pointers;
+ * 16-byte alignment of w and codes), NV_ERR_UNSUPPORTED (dtype).
+ */
+nv_status nv_quantize_fp(const void* w, nv_dtype dt, int64_t rows, int64_t cols, nv_fp_mode mode,
+                         uint32_t* codes, uint8_t* scales, nv_stream_t stream);
+
+/*
+ * Dequantizer of the floating-point modes: out bf16 [rows, cols] (16-byte
+ * aligned), element value times scale value, rounded once to bf16 (exact
+ * unless the product underflows bf16). Errors as nv_quantize_fp.
+ */
+nv_status nv_dequantize_fp(const uint32_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                           nv_fp_mode mode, void* out, nv_stream_t stream);
+
+/*
+ * Product with floating-point-mode weights stored [N, K] (codes and scales
+ * as nv_quantize_fp writes them for rows = N, cols = K): y [M, N] = x [M, K]
+ * . w^T, bf16 x and y (dt must be NV_BF16, else NV_ERR_UNSUPPORTED); K a
+ * multiple of 32. M <= 8: a matrix-vector kernel (every row computed as in a
+ * one-row call: row-exact); M > 8 with K a multiple of 64: the tiled
+ * tcgen05 kernel with the weights dequantized exactly into its bf16 tiles.
+ * Tolerance as nv_qmm. Errors as nv_quantize_fp; M == 0 or N == 0 is a no-op.
+ */
+nv_status nv_qmm_fp(const void* x, nv_dtype dt, int64_t M, int64_t K, int64_t N, const uint32_t* codes,
+                    const uint8_t* scales, nv_fp_mode mode, void* y, nv_stream_t stream);
+
+/*
  * Quantized product ("Docs / Quantization", sections "Affine" (example
  * x.quantized_matmul(&q, true)) and "Products on the GPU").
  *
