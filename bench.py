@@ -110,6 +110,39 @@ def worst_ratio(y, x, w):
     return float(((y.float() - ref).abs() / tol).max())
 
 
+def _fp_tables(dev):
+    """Values of every E2M1 code (16) and E4M3 code (256), from the bit fields."""
+    e2 = []
+    for c in range(16):
+        e, m = (c >> 1) & 3, c & 1
+        v = 0.5 * m if e == 0 else (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+        e2.append(-v if c & 8 else v)
+    e4 = []
+    for c in range(256):
+        e, m = (c >> 3) & 15, c & 7
+        v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        if e == 15 and m == 7:
+            v = float("nan")
+        e4.append(-v if c & 128 else v)
+    return torch.tensor(e2, device=dev), torch.tensor(e4, device=dev)
+
+
+def unpack_fp(codes, scales, mode):
+    """Dequantized floating-point-mode weights in fp32 with torch ops (codes by
+    shifts and masks, values by table lookup, times the scale)."""
+    e2, e4 = _fp_tables(codes.device)
+    bits = 8 if mode == "mxfp8" else 4
+    gs = 16 if mode == "nvfp4" else 32
+    per = 32 // bits
+    c = codes.to(torch.int64) & 0xFFFFFFFF
+    sh = torch.arange(per, device=codes.device, dtype=torch.int64) * bits
+    q = ((c.unsqueeze(-1) >> sh) & ((1 << bits) - 1)).flatten(-2)
+    v = (e4 if bits == 8 else e2)[q]
+    sc = scales.to(torch.int64)
+    sv = e4[sc] if mode == "nvfp4" else torch.exp2(sc.to(torch.float32) - 127)
+    return v * sv.repeat_interleave(gs, -1)
+
+
 def check_decode(wl, rows=None):
     c, s, b = wl.ws[0]
     w = unpack_dequant(c, s, b, wl.gs, wl.bits)
@@ -312,6 +345,44 @@ class DecodeE2E(Decode):
         self.x.copy_(self.xh, non_blocking=True)
         super().call(j)
         self.yh[j].copy_(self.y, non_blocking=True)
+
+
+class DecodeFp:
+    """x [M, K] . W[N, K]^T with W in a floating-point mode (MXFP4, MXFP8, NVFP4)."""
+
+    def __init__(self, dev, N=14336, K=4096, M=1, mode="mxfp4"):
+        import group_wise_affine_dequant_b200 as nvq
+        self.nvq = nvq
+        self.N, self.K, self.M, self.mode = N, K, M, mode
+        w = W.normal((N, K), 0.02, 0, "bf16").to(dev)
+        c, s = nvq.nv_quantize_fp(w, mode)
+        del w
+        bits, gs = (8, 32) if mode == "mxfp8" else (4, 16 if mode == "nvfp4" else 32)
+        wbytes = N * K * bits // 8 + N * (K // gs)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.copies = max(2, -(-3 * l2 // wbytes))
+        self.ws = [(c.clone(), s.clone()) for _ in range(self.copies)]
+        self.x = W.activations(M, K).to(dev)
+        self.y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.bytes = wbytes + 2 * M * (K + N)
+        self.flops = 2 * M * N * K
+
+    def call(self, j):
+        c, s = self.ws[j]
+        self.nvq.nv_qmm_fp(self.x, c, s, self.mode, out=self.y)
+
+    def step(self, i):
+        for j in range(self.copies):
+            self.call(j)
+
+
+def check_decode_fp(wl, rows=None):
+    c, s = wl.ws[0]
+    w = unpack_fp(c, s, wl.mode)
+    x, y = wl.x, wl.y
+    if rows is not None:
+        x, y = x[rows], y[rows]
+    return worst_ratio(y, x, w)
 
 
 class Dequant:
@@ -612,6 +683,23 @@ def run_nvq(args):
             also["prefill_frac_of_bf16_peak"] = round(tf / pk["bf16_tflops"], 4)
         checks[key.replace("_tflops", "")] = round(chk(check_decode, wl, rows=torch.arange(0, 2048, 128)), 4)
         del g, wl
+    # floating-point modes: decode (GB/s) at 14336 x 4096, and MXFP4 prefill (TFLOP/s)
+    for mode in ("mxfp4", "nvfp4", "mxfp8"):
+        wl = DecodeFp(dev, mode=mode)
+        g = timed_graph(wl.step, ks, Wm, stream)
+        t = max_ms(replay_timed(g, stream, barrier))
+        gb = replica_rate(ws, wl.bytes * wl.copies, ks, t) / 1e9
+        also[f"decode_{mode}_gbs"] = round(gb, 1)
+        also[f"decode_{mode}_frac_of_hbm"] = round(gb / ws / pk["hbm_gbs"], 4)
+        checks[f"decode_{mode}"] = round(chk(check_decode_fp, wl), 4)
+        del g, wl
+    wl = DecodeFp(dev, M=2048, mode="mxfp4")
+    kp = max(3, min(K, 10))
+    g = timed_graph(wl.step, kp, Wm, stream)
+    t = max_ms(replay_timed(g, stream, barrier))
+    also["prefill_mxfp4_tflops"] = round(replica_rate(ws, wl.flops * wl.copies, kp, t) / 1e12, 1)
+    checks["prefill_mxfp4"] = round(chk(check_decode_fp, wl, rows=torch.arange(0, 2048, 128)), 4)
+    del g, wl
 
     line = {
         "metric": METRIC,
@@ -744,6 +832,8 @@ PROFILE_WORKLOADS = {
     "dequant": lambda dev: Dequant(dev),
     "gather_mm": lambda dev: GatherMM(dev),
     "moe": lambda dev: MoeBlock(dev),
+    "decode_mxfp4": lambda dev: DecodeFp(dev, mode="mxfp4"),
+    "prefill_mxfp4": lambda dev: DecodeFp(dev, M=2048, mode="mxfp4"),
 }
 
 

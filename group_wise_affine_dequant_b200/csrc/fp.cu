@@ -206,6 +206,17 @@ qmv_fp_kernel(const uint16_t* __restrict__ x, int M, int64_t K, int64_t N, const
         const uint4 q4 = ldg_stream(crow + c);
         const uint32_t q[4] = {q4.x, q4.y, q4.z, q4.w};
         const int64_t k0 = c * F::CPC;
+        // the chunk's activations, 16 bytes at a time: xr[m][i] = x[m, k0 + 2i .. 2i + 1]
+        uint32_t xr[MT][F::CPC / 2];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+#pragma unroll
+            for (int v = 0; v < F::CPC / 8; ++v) {
+                uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+                if (m < M) xv = __ldg(reinterpret_cast<const uint4*>(x + m * K + k0) + v);
+                xr[m][4 * v] = xv.x; xr[m][4 * v + 1] = xv.y; xr[m][4 * v + 2] = xv.z; xr[m][4 * v + 3] = xv.w;
+            }
+        }
 #pragma unroll
         for (int part = 0; part < PARTS; ++part) {
             const float S = scale_f32<MODE>(__ldg(scales + n * groups + (k0 + part * CODES_PART) / F::GS));
@@ -224,11 +235,9 @@ qmv_fp_kernel(const uint16_t* __restrict__ x, int M, int64_t K, int64_t N, const
                 f16x2_f32(h, e0, e1);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    if (m < M) {
-                        const uint32_t xv = __ldg(reinterpret_cast<const uint32_t*>(x + m * K + k0 + ci));
-                        partial[m] = fmaf(__uint_as_float(xv << 16), e0, partial[m]);
-                        partial[m] = fmaf(__uint_as_float(xv & 0xFFFF0000u), e1, partial[m]);
-                    }
+                    const uint32_t xv = xr[m][ci / 2];
+                    partial[m] = fmaf(__uint_as_float(xv << 16), e0, partial[m]);
+                    partial[m] = fmaf(__uint_as_float(xv & 0xFFFF0000u), e1, partial[m]);
                 }
             }
 #pragma unroll

@@ -28,3 +28,14 @@ def test_worst_ratio_passes_the_oracle_product_and_fails_a_wrong_one():
     bad = y.clone()
     bad[1, 7] += 0.5
     assert bench.worst_ratio(bad.to(torch.bfloat16), x, wh) > 1.0
+
+
+def test_unpack_fp_equals_the_oracle_dequantization():
+    """The bench's torch decode of the floating-point modes (table lookup of
+    every code, times the scale) equals the oracle's dequantization."""
+    g = torch.Generator().manual_seed(4)
+    w = torch.randn(24, 256, generator=g) * (10.0 ** (torch.rand(24, 1, generator=g) * 6 - 4))
+    for mode in ("mxfp4", "mxfp8", "nvfp4"):
+        c, s = O.quantize_fp(w, mode)
+        got = bench.unpack_fp(c, s, mode)
+        assert torch.equal(got.to(torch.bfloat16), O.dequantize_fp(c, s, mode)), mode
