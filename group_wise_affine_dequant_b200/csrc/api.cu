@@ -244,6 +244,10 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
         x_rows * K < (int64_t(1) << 35))
         return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
                                                codes, scales, biases, group_size, bits, y, s, sms));
+    if (dt == NV_BF16 && !transpose && !row_exact && nvq::tc_gather_t0_supported(K, N, bits, group_size) &&
+        x_rows * K < (int64_t(1) << 35))
+        return from_cuda(nvq::launch_tc_gather_t0(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
+                                                  codes, scales, biases, group_size, bits, y, s, sms));
     // Matrix-vector route (row_exact): every pair's output is bitwise equal to
     // nv_qmm(M = 1) of that row with its expert's weights.
     if (dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size))
@@ -300,11 +304,12 @@ nv_status nv_pipeline_error(uint32_t* host_code) {
     const unsigned int b = nvq::tc_error_take();
     const unsigned int c = nvq::tc_gather_error_take();
     const unsigned int d = nvq::tc_gather_mm_error_take();
+    const unsigned int g = nvq::tc_gather_t0_error_take();
     const unsigned int t = nvq::selftest_error_take();
     if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu || d == 0xFFFFFFFFu ||
-        t == 0xFFFFFFFFu)
+        g == 0xFFFFFFFFu || t == 0xFFFFFFFFu)
         return NV_ERR_CUDA;
-    *host_code = a ? a : b ? b : c ? c : d ? d : t;
+    *host_code = a ? a : b ? b : c ? c : d ? d : g ? g : t;
     return NV_OK;
 }
 

@@ -41,4 +41,13 @@ cudaError_t launch_tc_gather_mm(const void* x, int64_t x_rows, int64_t K, const 
                                 const void* w, void* y, cudaStream_t stream, int num_sms);
 unsigned int tc_gather_mm_error_take();
 
+// The quantized grouped product with experts stored [E][K, N] (transpose = 0),
+// grouped along N; N * bits a multiple of 128 and K of 64.
+bool tc_gather_t0_supported(int64_t K, int64_t N, int bits, int gs);
+cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                                const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
+                                const uint32_t* codes, const void* scales, const void* biases, int gs,
+                                int bits, void* y, cudaStream_t stream, int num_sms);
+unsigned int tc_gather_t0_error_take();
+
 }  // namespace nvq

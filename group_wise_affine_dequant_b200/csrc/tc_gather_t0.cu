@@ -1,0 +1,516 @@
+// Tensor-core mixture-of-experts product with quantized experts stored [K, N]
+// (gather_qmm with transpose = 0: "Docs / Quantization", section "Mixture of
+// experts", each row meets its own expert's weights; the product's transpose
+// flag, section "Affine", and the crate docs' GatherQmm take either layout).
+// The experts are [E][K, N], grouped along N, so the scale varies along the
+// contraction. The same grouped, transposed form as the other grouped kernels:
+// D^T = W_e . X_e^T with 256 weight columns n (two 128-row tiles) as the MMA's
+// M side and the expert's gathered activation rows (<= 64 per pass) as N, so
+// each expert's weights cross HBM once for all its rows. Roles, per CTA
+// (persistent):
+//   warp 0      one lane streams code boxes of 64 k-rows x 256 columns by TMA
+//               into a ring released by the dequantizing warps.
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma (M = 128,
+//               N = pairs rounded up to 16, K = 16) with both operands in
+//               shared memory, two tiles per k-step, into a double-buffered
+//               accumulator (64 columns per tile).
+//   warps 2-5   epilogue: TMEM lane = weight column, column = pair; each pair's
+//               value is stored to its output row.
+//   warps 6-9   copy the pairs' activation rows with cp.async into the
+//               128-byte-swizzled B layout.
+//   warps 10-25 dequantize and transpose: a task is 4 k-rows x one code word
+//               (PER columns); each column's 4 values w = s[k, g(n)] * code +
+//               b[k, g(n)] (one bf16 fma on the exact code, rounded once) go to
+//               the column's row of the K-major A tile as one 8-byte piece.
+// The kernel is the programmatic dependent of the routing kernel. Pairs with
+// an out-of-range id get zero rows. Waits are bounded by a timer.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc.cuh"
+#include "tc_common.cuh"
+#include "tma.cuh"
+
+namespace nvq {
+namespace {
+
+using namespace tc;
+
+constexpr int WM = 128;          // weight rows per tile (TMEM lanes)
+constexpr int kTiles = 2;        // tiles per unit, sharing every activation stage
+constexpr int UW = WM * kTiles;  // weight rows per unit
+constexpr int BK = 64;           // k per stage: one 128-byte swizzle atom of bf16
+constexpr int UMMA_K = 16;
+constexpr int kMaxPairs = 64;    // pairs per pass (accumulator columns per tile)
+static_assert(kMaxPairs == 64, "the epilogue keeps two pair ids per lane");
+constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-9
+constexpr int kXThreads = 128;
+constexpr int kDequantWarp0 = 10; // warps 10-25: dequantize into the A tiles
+constexpr int kDequantThreads = 512;
+constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;  // 832
+constexpr int kWStage = UW * BK * 2;                  // 32 KB of dequantized weights per stage
+constexpr int kXStage = kMaxPairs * BK * 2;           // 8 KB of activations per stage
+constexpr int kAccCols = kTiles * kMaxPairs;          // 128 columns per accumulator
+constexpr uint32_t kTmemCols = 2 * kAccCols;          // double-buffered: 256
+
+struct TParams {
+    uint16_t* y;                // [R, N]
+    const uint16_t* scales;     // [E][K, N / gs]
+    const uint16_t* biases;
+    int gs;
+    int dc;                     // code ring depth
+    uint32_t c_off;
+    uint32_t c_stage;           // bytes of one code stage (64 k-rows x 256 columns)
+    const uint16_t* x;          // [x_rows, K]
+    const uint32_t* lhs;        // nullable
+    const uint32_t* perm;       // [R] pairs in expert order
+    const uint32_t* offsets;    // [E + 2]
+    int64_t N, K, E;
+    int wunits;                 // ceil(N / UW)
+    int dw, dx;                 // ring depths: weights, activations
+    uint32_t x_off, w_off, row_off, bar_off;
+};
+
+struct RingPos {
+    int s = 0;
+    uint32_t use = 0;
+    __device__ __forceinline__ void next(int depth) {
+        if (++s == depth) { s = 0; ++use; }
+    }
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Row of the A tiles that holds column n of a unit, and (being an involution)
+// the column that TMEM lane (tile * 128 + lane) holds: the low three bits are
+// XORed with three bits above them, those of the code word index for 2- and
+// 4-bit codes.
+template <int BITS>
+__device__ __forceinline__ int a_row(int n) {
+    constexpr int S = BITS == 2 ? 4 : 3;
+    return n ^ ((n >> S) & 7);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int DW = prm.dw, DX = prm.dx, DC = prm.dc;
+    uint8_t* x_ring = smem + prm.x_off;
+    uint8_t* w_ring = smem + prm.w_off;
+    uint8_t* c_ring = smem + prm.c_off;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.bar_off);
+    uint64_t* full_w = bars;
+    uint64_t* empty_w = full_w + DW;
+    uint64_t* full_x = empty_w + DW;
+    uint64_t* empty_x = full_x + DX;
+    uint64_t* full_c = empty_x + DX;
+    uint64_t* empty_c = full_c + DC;
+    uint64_t* acc_full = empty_c + DC;
+    uint64_t* acc_empty = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    // [kMaxPairs / (kXThreads / 8)][kXThreads]: x element offsets of each loader thread's rows
+    uint32_t* s_xoff = reinterpret_cast<uint32_t*>(smem + prm.row_off);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < DW; ++i) { mbar_init(&full_w[i], kDequantThreads / 32); mbar_init(&empty_w[i], 1); }
+        for (int i = 0; i < DC; ++i) { mbar_init(&full_c[i], 1); mbar_init(&empty_c[i], kDequantThreads / 32); }
+        for (int i = 0; i < DX; ++i) { mbar_init(&full_x[i], kXThreads); mbar_init(&empty_x[i], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4); }
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    const int ksteps = static_cast<int>(prm.K / BK);
+    const int units = static_cast<int>(prm.E) * prm.wunits;
+
+    // Before the routing tables exist: L2 prefetch of the first unit's first
+    // code stages (the weights do not depend on the routing).
+    if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < units) {
+        const int e = static_cast<int>(blockIdx.x) / prm.wunits;
+        const int col = (static_cast<int>(blockIdx.x) - e * prm.wunits) * UW;
+        for (int i = 0; i < DC && i < ksteps; ++i) tma_prefetch_3d(&map_c, col * BITS / 32, i * BK, e);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // the routing tables (offsets, perm) come from the previous kernel
+
+    auto unit_pairs = [&](int u, int& e, int& wt, int& first, int& count) {
+        e = u / prm.wunits;
+        wt = u - e * prm.wunits;
+        first = static_cast<int>(__ldg(prm.offsets + e));
+        count = static_cast<int>(__ldg(prm.offsets + e + 1)) - first;
+    };
+
+    if (warp == 0) {
+        // --------------------------------------------------- producer: codes
+        if (lane == 0) {
+            RingPos c;
+            int issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int e, wt, first, count;
+                unit_pairs(u, e, wt, first, count);
+                for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
+                    for (int ks = 0; ks < ksteps; ++ks) {
+                        if (c.use > 0 && !(ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 61, 512))) break;
+                        mbar_expect_tx(&full_c[c.s], prm.c_stage);
+                        tma_load_3d(c_ring + c.s * prm.c_stage, &map_c, &full_c[c.s], wt * UW * BITS / 32, ks * BK, e);
+                        ++issued;
+                        c.next(DC);
+                    }
+                }
+            }
+            for (int j = 0; j < DC && j < issued; ++j) {  // drain the last copies
+                if (--c.s < 0) { c.s = DC - 1; --c.use; }
+                mbar_wait(&full_c[c.s], c.use & 1, 69);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            RingPos w, x;
+            int local = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int e, wt, first, count;
+                unit_pairs(u, e, wt, first, count);
+                for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs, ++local) {
+                    const int cn = min(kMaxPairs, count - p0);
+                    const int npad = (cn + 15) / 16 * 16;
+                    const uint32_t idesc = idesc_bf16(WM, npad);
+                    const int acc = local & 1;
+                    const uint32_t ause = static_cast<uint32_t>(local >> 1);
+                    if (ause > 0 && !(ok = mbar_wait_backoff(&acc_empty[acc], (ause - 1) & 1, 42, 256))) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+                    for (int ks = 0; ks < ksteps; ++ks) {
+                        if (!(ok = mbar_wait(&full_w[w.s], w.use & 1, 43))) break;
+                        if (!(ok = mbar_wait(&full_x[x.s], x.use & 1, 44))) break;
+                        tc_fence_after();
+                        const uint64_t bd = sw128_desc(x_ring + x.s * kXStage);
+#pragma unroll
+                        for (int tt = 0; tt < kTiles; ++tt) {  // both tiles against the same activations
+                            const uint64_t ad = sw128_desc(w_ring + w.s * kWStage + tt * (WM * BK * 2));
+#pragma unroll
+                            for (int kk = 0; kk < BK / UMMA_K; ++kk)  // 16 k = 32 bytes of each row
+                                tc_mma(d_tmem + tt * kMaxPairs, ad + (kk * UMMA_K * 2 >> 4),
+                                       bd + (kk * UMMA_K * 2 >> 4), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&empty_w[w.s]);
+                        tc_commit(&empty_x[x.s]);
+                        w.next(DW);
+                        x.next(DX);
+                    }
+                    if (ok) tc_commit(&acc_full[acc]);
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        int local = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int e, wt, first, count;
+            unit_pairs(u, e, wt, first, count);
+            for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs, ++local) {
+                const int cn = min(kMaxPairs, count - p0);
+                const int acc = local & 1;
+                const uint32_t ause = static_cast<uint32_t>(local >> 1);
+                // output rows of the pass's pairs: lane l holds columns l and l + 32
+                uint32_t prow[kMaxPairs / 32];
+#pragma unroll
+                for (int h = 0; h < kMaxPairs / 32; ++h) {
+                    const int c = h * 32 + lane;
+                    prow[h] = c < cn ? __ldg(prm.perm + first + p0 + c) : 0u;
+                }
+                if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 45, 2048))) break;
+                tc_fence_after();
+                for (int tt = 0; tt < kTiles; ++tt)
+                for (int c0 = 0; c0 < cn; c0 += 16) {
+                    // column of W held by TMEM lane (tile * 128 + lane)
+                    const int64_t n = static_cast<int64_t>(wt) * UW + a_row<BITS>(tt * WM + q * 32 + lane);
+                    uint32_t v[16];
+                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                           static_cast<uint32_t>(acc * kAccCols + tt * kMaxPairs + c0);
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                        : "r"(taddr));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    const uint32_t rows = (c0 >> 5) ? prow[1] : prow[0];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
+                        if (c0 + j < cn && n < prm.N)
+                            prm.y[static_cast<int64_t>(pair) * prm.N + n] =
+                                f32_to_bf16_bits(__uint_as_float(v[j]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            }
+        }
+    } else if (warp < kDequantWarp0) {
+        // ------------------------------------------- activation rows (cp.async)
+        // Thread i copies 16-byte chunk (i & 7) of rows (i >> 3) + 16 j of every
+        // k-step. Stages are completed in order, LAG k-steps behind the copies.
+        const int xt = threadIdx.x - kXWarp0 * 32;  // 0 .. kXThreads - 1
+        constexpr int RS = kXThreads / 8;            // row stride between a thread's rows
+        const int ch = xt & 7, r0 = xt >> 3;
+        const int lag = DX - 1 < 4 ? DX - 1 : 4;
+        RingPos x, done;  // next stage to fill, next stage to complete
+        int pending = 0;
+        bool ok = true;
+        auto complete_one = [&]() {
+            fence_proxy_async();
+            mbar_arrive(&full_x[done.s]);
+            done.next(DX);
+            --pending;
+        };
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int e, wt, first, count;
+            unit_pairs(u, e, wt, first, count);
+            for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
+                const int cn = min(kMaxPairs, count - p0);
+                const int nr = cn > r0 ? (cn - r0 + RS - 1) / RS : 0;  // rows of this thread
+                for (int j = 0; j < nr; ++j) {
+                    const uint32_t pair = __ldg(prm.perm + first + p0 + r0 + RS * j);
+                    const uint32_t row = prm.lhs ? __ldg(prm.lhs + pair) : pair;
+                    // in 16-byte units (K is a multiple of 64): x up to 2^35 elements
+                    s_xoff[j * kXThreads + xt] = row * static_cast<uint32_t>(prm.K / 8) + ch;
+                }
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (x.use > 0 && !(ok = mbar_wait_backoff(&empty_x[x.s], (x.use - 1) & 1, 46, 256))) break;
+                    uint8_t* dst = x_ring + x.s * kXStage;
+                    for (int j = 0; j < nr; ++j) {
+                        const int r = r0 + RS * j;
+                        cp_async16(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4),
+                                   reinterpret_cast<const uint4*>(prm.x) + s_xoff[j * kXThreads + xt] +
+                                       ks * (BK / 8));
+                    }
+                    cp_async_commit();
+                    x.next(DX);
+                    if (++pending > lag) {
+                        // the oldest of the lag + 1 outstanding groups has landed
+                        if (lag == 4) cp_async_wait<4>();
+                        else if (lag == 3) cp_async_wait<3>();
+                        else if (lag == 2) cp_async_wait<2>();
+                        else cp_async_wait<0>();
+                        complete_one();
+                    }
+                }
+            }
+        }
+        cp_async_wait<0>();
+        while (pending > 0) complete_one();
+    } else {
+        // ------------------------------------------ dequantize and transpose
+        // A warp task is 16 code words x 8 k-rows: lane (l & 15) takes word
+        // j = 16 jh + (l & 15), lane bit 4 picks k-rows 4 kq .. 4 kq + 3 with
+        // kq = 2 kh + (l >> 4). Column n of the unit goes to A-row a_row(n)
+        // (an involution on the low three bits), which spreads a warp's
+        // 8-byte stores over all 32 banks; the code reads are two-way.
+        constexpr int PER = 32 / BITS;
+        constexpr int WPR = UW * BITS / 32;          // code words per k-row of a stage
+        constexpr int WTASKS = (WPR / 16) * (BK / 8);
+        const int dw = warp - kDequantWarp0;          // 0 .. 15
+        const int jl = lane & 15, kl = lane >> 4;
+        const int64_t gpr = prm.N / prm.gs;           // groups per k-row of W
+        RingPos c, w;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int e, wt, first, count;
+            unit_pairs(u, e, wt, first, count);
+            const uint16_t* se = prm.scales + static_cast<int64_t>(e) * prm.K * gpr;
+            const uint16_t* be = prm.biases + static_cast<int64_t>(e) * prm.K * gpr;
+            for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (!(ok = mbar_wait(&full_c[c.s], c.use & 1, 62))) break;
+                    if (w.use > 0 && !(ok = mbar_wait_backoff(&empty_w[w.s], (w.use - 1) & 1, 63, 128))) break;
+                    const uint8_t* cst = c_ring + c.s * prm.c_stage;
+                    uint8_t* wst = w_ring + w.s * kWStage;
+                    for (int wtask = dw; wtask < WTASKS; wtask += kDequantThreads / 32) {
+                        const int j = (wtask / (BK / 8)) * 16 + jl;
+                        const int kq = (wtask % (BK / 8)) * 2 + kl;
+                        const int nl = j * PER;                                   // first column in the unit
+                        const int64_t ng = static_cast<int64_t>(wt) * UW + nl;    // and in W
+                        const int64_t kg = static_cast<int64_t>(ks) * BK + 4 * kq;
+                        const bool live = ng < prm.N;
+                        uint32_t cw[4], sraw[4], braw[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            cw[i] = *reinterpret_cast<const uint32_t*>(cst + (4 * kq + i) * (WPR * 4) + 4 * j);
+                            const int64_t gi = (kg + i) * gpr + (live ? ng / prm.gs : 0);
+                            sraw[i] = live ? __ldg(se + gi) : 0u;
+                            braw[i] = live ? __ldg(be + gi) : 0u;
+                        }
+                        // (k, k + 1) pairs of scales and biases as bf16x2
+                        const uint32_t s01 = sraw[0] | (sraw[1] << 16), s23 = sraw[2] | (sraw[3] << 16);
+                        const uint32_t b01 = braw[0] | (braw[1] << 16), b23 = braw[2] | (braw[3] << 16);
+#pragma unroll
+                        for (int f = 0; f < PER; ++f) {
+                            uint32_t v[2];
+                            if constexpr (BITS == 8) {
+                                // packed fp32: 2^23 + c exactly, minus 2^23, then s c + b
+                                const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);
+                                const uint64_t off = f2_pack(0xCB000000u, 0xCB000000u);
+#pragma unroll
+                                for (int p = 0; p < 2; ++p) {
+                                    const uint64_t r = f2_pack(prmt(cw[2 * p], 0x4B000000u, f | 0x7440),
+                                                               prmt(cw[2 * p + 1], 0x4B000000u, f | 0x7440));
+                                    const uint64_t cc = f2_fma(r, one_m, off);
+                                    const uint64_t sc = f2_pack(sraw[2 * p] << 16, sraw[2 * p + 1] << 16);
+                                    const uint64_t bc = f2_pack(braw[2 * p] << 16, braw[2 * p + 1] << 16);
+                                    v[p] = f2_to_bf2_packed(f2_fma(sc, cc, bc));
+                                }
+                            } else {
+                                // field f of k-rows (k, k + 1) into the two halves: 128 + c
+                                const int byte = (f * BITS) >> 3, sh = (f * BITS) & 7;
+                                const uint32_t sel = static_cast<uint32_t>(byte | ((4 + byte) << 8));
+                                constexpr uint32_t MSK = ((1u << BITS) - 1u) * 0x00010001u;
+                                const uint32_t r0 = codes_to_bf16x2(prmt(cw[0], cw[1], sel) >> sh, MSK);
+                                const uint32_t r1 = codes_to_bf16x2(prmt(cw[2], cw[3], sel) >> sh, MSK);
+                                v[0] = bf2_fma(s01, bf2_sub(r0, 0x43004300u), b01);
+                                v[1] = bf2_fma(s23, bf2_sub(r1, 0x43004300u), b23);
+                            }
+                            // A-row of column nl + f: 8-row atom, k-chunk kq / 2 (8 k), half kq & 1
+                            const int ar = a_row<BITS>(nl + f);
+                            *reinterpret_cast<uint2*>(wst + (ar >> 3) * 1024 + (ar & 7) * 128 +
+                                                      (((kq >> 1) ^ (ar & 7)) << 4) + (kq & 1) * 8) =
+                                make_uint2(v[0], v[1]);
+                        }
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) { mbar_arrive(&empty_c[c.s]); mbar_arrive(&full_w[w.s]); }
+                    c.next(DC);
+                    w.next(DW);
+                }
+            }
+        }
+    }
+
+    // pairs whose expert or token id is out of range (the router's last
+    // bucket) get zero rows
+    {
+        const int64_t first = __ldg(prm.offsets + prm.E), last = __ldg(prm.offsets + prm.E + 1);
+        for (int64_t i = first + blockIdx.x; i < last; i += gridDim.x) {
+            uint16_t* row = prm.y + static_cast<int64_t>(__ldg(prm.perm + i)) * prm.N;
+            for (int64_t n = threadIdx.x; n < prm.N; n += blockDim.x) row[n] = 0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols));
+    }
+}
+
+}  // namespace
+
+bool tc_gather_t0_supported(int64_t K, int64_t N, int bits, int gs) {
+    // code rows of 16-byte multiples (TMA), 64-k steps
+    return K % BK == 0 && K >= BK && N > 0 && (bits == 2 || bits == 4 || bits == 8) &&
+           (gs == 32 || gs == 64 || gs == 128) && N % gs == 0 && (N * bits) % 128 == 0;
+}
+
+unsigned int tc_gather_t0_error_take() { return pipeline_error_take(); }
+
+cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const uint32_t* lhs,
+                                const uint32_t* perm, const uint32_t* offsets, int64_t E, int64_t N,
+                                const uint32_t* codes, const void* scales, const void* biases, int gs,
+                                int bits, void* y, cudaStream_t stream, int num_sms) {
+    EncodeTiled enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    if (x_rows * K >= (int64_t(1) << 35)) return cudaErrorInvalidValue;  // 32-bit 16-byte offsets
+    CUtensorMap map_c;
+    const int64_t wpr = N * bits / 32;
+    {   // codes [E][K][N * bits / 32]: boxes of 256 columns x 64 k-rows, unswizzled
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(K),
+                              static_cast<cuuint64_t>(E)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(wpr) * 4, static_cast<cuuint64_t>(wpr * K) * 4};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(UW * bits / 32), BK, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&map_c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(codes), dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    TParams prm{};
+    prm.y = static_cast<uint16_t*>(y);
+    prm.x = static_cast<const uint16_t*>(x);
+    prm.scales = static_cast<const uint16_t*>(scales);
+    prm.biases = static_cast<const uint16_t*>(biases);
+    prm.gs = gs;
+    prm.lhs = lhs;
+    prm.perm = perm;
+    prm.offsets = offsets;
+    prm.N = N;
+    prm.K = K;
+    prm.E = E;
+    prm.wunits = static_cast<int>((N + UW - 1) / UW);
+    prm.c_stage = static_cast<uint32_t>(BK * UW * bits / 8);
+    int dw = 3, dx = 8, dc = 4;
+    auto bytes = [&]() {
+        return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kWStage) * dw +
+               static_cast<size_t>(prm.c_stage) * dc + kMaxPairs * 8 * 4 +
+               static_cast<size_t>(2 * (dw + dx + dc) + 4) * 8 + 16;
+    };
+    const size_t budget = 227 * 1024 - 2048 - 1024;
+    while (bytes() > budget && dx > 4) --dx;
+    while (bytes() > budget && dc > 2) --dc;
+    if (bytes() > budget) return cudaErrorInvalidConfiguration;
+    prm.dw = dw;
+    prm.dx = dx;
+    prm.dc = dc;
+    prm.x_off = 0;
+    prm.w_off = kXStage * dx;
+    prm.c_off = prm.w_off + kWStage * dw;
+    prm.row_off = prm.c_off + prm.c_stage * dc;
+    prm.bar_off = prm.row_off + kMaxPairs * 8 * 4;
+    const size_t smem = bytes() + 1024;
+    const int units = static_cast<int>(E) * prm.wunits;
+    const int grid = units < num_sms ? units : num_sms;
+    void (*k)(const CUtensorMap, const TParams) =
+        bits == 4 ? tc_gather_t0_kernel<4> : bits == 8 ? tc_gather_t0_kernel<8> : tc_gather_t0_kernel<2>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    // programmatic dependent launch on the routing kernel (see the kernel)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, map_c, prm);
+}
+
+}  // namespace nvq

@@ -1,0 +1,145 @@
+"""The grouped tensor-core route of gather_qmm with experts stored [E, K, N]
+(transpose = 0, grouped along N; "Docs / Quantization", section "Mixture of
+experts", and the product's transpose flag, section "Affine") against the
+oracle: ragged experts, a unit of weight columns that ends inside the tile,
+experts with more pairs than one pass holds, invalid ids, unit activations that
+read out every dequantized weight exactly, and the mixture-of-experts shapes on
+sampled outputs. Tolerance as in the other parity tests."""
+import pytest
+import torch
+
+import group_wise_affine_dequant_b200 as nvq
+import oracle as O
+from group_wise_affine_dequant_b200 import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+BF16 = torch.bfloat16
+QUANTS = [(4, 32), (4, 64), (4, 128), (8, 32), (8, 64), (8, 128), (2, 32), (2, 64), (2, 128)]
+
+
+def _gather(x, c, s, b, rhs, lhs, gs, bits, sorted_=False, ws=None):
+    if ws is None:
+        ws = torch.empty(max(nvq.nv_gather_qmm_workspace_size(rhs.numel(), c.shape[0]), 16),
+                         dtype=torch.uint8, device="cuda")
+    y = nvq.nv_gather_qmm(x.cuda(), c.cuda(), s.cuda(), b.cuda(), rhs.to(torch.int32).cuda(),
+                          None if lhs is None else lhs.to(torch.int32).cuda(), gs, bits, False,
+                          sorted_, False, workspace=ws)
+    flags = nvq.nv_gather_qmm_flags(ws)
+    assert nvq.nv_pipeline_error() == 0
+    return y.cpu(), flags
+
+
+@pytest.mark.parametrize("bits,gs", QUANTS)
+def test_ragged_experts(bits, gs):
+    """37 pairs over 5 experts (one empty, one with 17 pairs); N = 384 is one
+    full unit of 256 columns and one that ends half way."""
+    g = torch.Generator().manual_seed(70 + bits + gs)
+    E, K, N, T = 5, 512, 384, 23
+    w = W.normal((E, K, N), 0.02, 71, "bf16")
+    x = W.normal((T, K), 1.0, 72, "bf16")
+    c, s, b = O.quantize_affine(w, gs, bits)
+    rhs = torch.tensor([0] * 9 + [2] * 17 + [3] * 4 + [4] * 7)[torch.randperm(37, generator=g)]
+    lhs = torch.randint(0, T, (37,), generator=g)
+    y, flags = _gather(x, c, s, b, rhs, lhs, gs, bits)
+    assert flags == 0
+    yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, gs, bits, False)
+    P.assert_within(y, yr, a, BF16, f"transpose=0 ragged b{bits} g{gs}")
+
+
+@pytest.mark.parametrize("bits", [4, 8, 2])
+def test_unit_activations_read_out_the_weights(bits):
+    """x rows are unit vectors e_k: every output is one dequantized weight
+    w_hat[k, n] times 1 plus exact zeros, so it must equal the oracle's stored
+    (once-rounded) weight bit for bit. Covers every column of two units, the
+    A-tile row order and the epilogue's column map."""
+    E, K, N, gs = 3, 256, 512, 64
+    w = W.normal((E, K, N), 0.02, 73, "bf16")
+    c, s, b = O.quantize_affine(w, gs, bits)
+    wh = O.dequantize_stored(c, s, b, gs, bits)  # [E, K, N] bf16
+    g = torch.Generator().manual_seed(74)
+    R = 96
+    ks = torch.randint(0, K, (R,), generator=g)
+    rhs = torch.randint(0, E, (R,), generator=g)
+    x = torch.zeros(R, K, dtype=BF16)
+    x[torch.arange(R), ks] = 1.0
+    y, flags = _gather(x, c, s, b, rhs, None, gs, bits)
+    assert flags == 0
+    want = wh[rhs, ks]  # [R, N]
+    bad = y.float() != want.float()
+    assert not bad.any(), f"b{bits}: {int(bad.sum())} differ, first {bad.nonzero()[0].tolist()}"
+
+
+def test_many_pairs_per_expert_and_deterministic():
+    """One expert with 600 pairs (ten passes of 64), and a second call that
+    must give the same bits."""
+    E, K, N = 3, 256, 768
+    w = W.normal((E, K, N), 0.02, 75, "bf16")
+    x = W.normal((700, K), 1.0, 76, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    g = torch.Generator().manual_seed(77)
+    rhs = torch.cat([torch.full((600,), 1), torch.full((40,), 2), torch.full((5,), 0)])
+    rhs = rhs[torch.randperm(645, generator=g)]
+    lhs = torch.randint(0, 700, (645,), generator=g)
+    y, flags = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    y2, _ = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    assert flags == 0
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, 64, 4, False)
+    P.assert_within(y, yr, a, BF16, "transpose=0 many pairs")
+
+
+def test_invalid_ids_get_zero_rows():
+    E, K, N = 4, 128, 256
+    w = W.normal((E, K, N), 0.02, 78, "bf16")
+    x = W.normal((6, K), 1.0, 79, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    rhs = torch.tensor([0, 1, 9, 2, 1])
+    lhs = torch.tensor([0, 1, 2, 7, 5])
+    y, flags = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    assert flags & nvq.binding.NV_FLAG_EXPERT_OUT_OF_RANGE
+    assert flags & nvq.binding.NV_FLAG_TOKEN_OUT_OF_RANGE
+    assert (y[2] == 0).all() and (y[3] == 0).all()
+    ok = torch.tensor([0, 1, 4])
+    yr, a = O.gather_qmm(x, c, s, b, lhs[ok], rhs[ok], 64, 4, False)
+    P.assert_within(y[ok], yr, a, BF16, "transpose=0 valid rows")
+
+
+def test_shapes_outside_the_tiles_take_the_general_route():
+    """N * bits not a multiple of 128 (N = 96, 2-bit) and K not a multiple of
+    64 (K = 96) still give the right products (the general kernel)."""
+    g = torch.Generator().manual_seed(80)
+    for K, N, bits in ((512, 96, 2), (96, 256, 4)):
+        w = W.normal((3, K, N), 0.02, 81, "bf16")
+        x = W.normal((9, K), 1.0, 82, "bf16")
+        c, s, b = O.quantize_affine(w, 32, bits)
+        rhs = torch.randint(0, 3, (20,), generator=g)
+        lhs = torch.randint(0, 9, (20,), generator=g)
+        y, flags = _gather(x, c, s, b, rhs, lhs, 32, bits)
+        assert flags == 0
+        yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, 32, bits, False)
+        P.assert_within(y, yr, a, BF16, f"transpose=0 general K={K} N={N} b{bits}")
+
+
+def test_moe_shapes_sampled():
+    """The mixture-of-experts workload's shapes with the experts stored
+    [E, K, N]: 2048 pairs over 64 experts, K = 2048, N = 1536; sorted and
+    unsorted pair orders give the same bits, sampled outputs match the oracle."""
+    m = W.MOE
+    w = W.normal((m["E"], m["K"], m["N"]), 0.02, 83, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    x = W.normal((m["tokens"], m["K"]), 1.0, 84, "bf16")
+    ids = W.expert_ids(m["tokens"], m["E"], m["top_k"], 2)
+    lhs, rhs = W.flatten_pairs(ids)
+    lhs_s, rhs_s, order = W.stable_sort_pairs(lhs, rhs)
+    y_u, f_u = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    y_s, f_s = _gather(x, c, s, b, rhs_s, lhs_s, 64, 4, sorted_=True)
+    assert f_u == 0 and f_s == 0
+    assert torch.equal(y_s.view(torch.int16), y_u[order].view(torch.int16))
+    g = torch.Generator().manual_seed(85)
+    R, N = rhs.numel(), m["N"]
+    r_idx = torch.randint(0, R, (4096,), generator=g)
+    n_idx = torch.randint(0, N, (4096,), generator=g)
+    yr, a = O.gather_qmm_sampled(x, c, s, b, lhs, rhs, 64, 4, False, r_idx, n_idx)
+    P.assert_within(y_u[r_idx, n_idx], yr, a, BF16, "transpose=0 moe sampled")
