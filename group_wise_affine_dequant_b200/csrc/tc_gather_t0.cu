@@ -49,6 +49,8 @@ constexpr int kXWarp0 = 6;       // activation-row loaders: warps 6-9
 constexpr int kXThreads = 128;
 constexpr int kDequantWarp0 = 10; // warps 10-25: dequantize into the A tiles
 constexpr int kDequantThreads = 512;
+constexpr int kDequantGroups = 2; // groups of dequantizing warps on alternate stages
+constexpr int kL2Ahead = 8;       // stages prefetched into L2 ahead of the code copies
 constexpr int kThreads = kDequantWarp0 * 32 + kDequantThreads;  // 832
 constexpr int kWStage = UW * BK * 2;                  // 32 KB of dequantized weights per stage
 constexpr int kXStage = kMaxPairs * BK * 2;           // 8 KB of activations per stage
@@ -59,7 +61,7 @@ struct TParams {
     uint16_t* y;                // [R, N]
     const uint16_t* scales;     // [E][K, N / gs]
     const uint16_t* biases;
-    int gs;
+    int gs, lg_gs;
     int dc;                     // code ring depth
     uint32_t c_off;
     uint32_t c_stage;           // bytes of one code stage (64 k-rows x 256 columns)
@@ -81,12 +83,26 @@ struct RingPos {
     }
 };
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 // Row of the A tiles that holds column n of a unit, and (being an involution)
 // the column that TMEM lane (tile * 128 + lane) holds: the low three bits are
@@ -122,8 +138,9 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
     uint32_t* s_xoff = reinterpret_cast<uint32_t*>(smem + prm.row_off);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < DW; ++i) { mbar_init(&full_w[i], kDequantThreads / 32); mbar_init(&empty_w[i], 1); }
-        for (int i = 0; i < DC; ++i) { mbar_init(&full_c[i], 1); mbar_init(&empty_c[i], kDequantThreads / 32); }
+        // a stage is dequantized by one group of warps
+        for (int i = 0; i < DW; ++i) { mbar_init(&full_w[i], kDequantThreads / 32 / kDequantGroups); mbar_init(&empty_w[i], 1); }
+        for (int i = 0; i < DC; ++i) { mbar_init(&full_c[i], 1); mbar_init(&empty_c[i], kDequantThreads / 32 / kDequantGroups); }
         for (int i = 0; i < DX; ++i) { mbar_init(&full_x[i], kXThreads); mbar_init(&empty_x[i], 1); }
         for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4); }
         mbar_init_fence();
@@ -142,7 +159,7 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
     if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < units) {
         const int e = static_cast<int>(blockIdx.x) / prm.wunits;
         const int col = (static_cast<int>(blockIdx.x) - e * prm.wunits) * UW;
-        for (int i = 0; i < DC && i < ksteps; ++i) tma_prefetch_3d(&map_c, col * BITS / 32, i * BK, e);
+        for (int i = 0; i < kL2Ahead && i < ksteps; ++i) tma_prefetch_3d(&map_c, col * BITS / 32, i * BK, e);
     }
     tc_fence_before();
     __syncthreads();
@@ -159,23 +176,58 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
 
     if (warp == 0) {
         // --------------------------------------------------- producer: codes
-        if (lane == 0) {
-            RingPos c;
-            int issued = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                int e, wt, first, count;
-                unit_pairs(u, e, wt, first, count);
-                for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
-                    for (int ks = 0; ks < ksteps; ++ks) {
-                        if (c.use > 0 && !(ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 61, 512))) break;
-                        mbar_expect_tx(&full_c[c.s], prm.c_stage);
-                        tma_load_3d(c_ring + c.s * prm.c_stage, &map_c, &full_c[c.s], wt * UW * BITS / 32, ks * BK, e);
-                        ++issued;
-                        c.next(DC);
+        // Lane 0 copies the code box of each stage. The warp also prefetches
+        // into L2, kL2Ahead stages ahead of the copies (into the next unit at
+        // the end of one), the code box and the 64 rows of the unit's scales
+        // and biases (first and last element of each row), so the copies and
+        // the dequantizers' loads meet L2 rather than HBM: the ring alone
+        // holds too few bytes in flight to cover HBM's latency.
+        const int64_t gpr = prm.N >> prm.lg_gs;
+        const int gu = UW >> prm.lg_gs;  // groups of a unit
+        auto prefetch_stage = [&](int u2, int ks2) {
+            const int e2 = u2 / prm.wunits, wt2 = u2 - e2 * prm.wunits;
+            if (lane == 0) tma_prefetch_3d(&map_c, wt2 * UW * BITS / 32, ks2 * BK, e2);
+            const int64_t g0 = static_cast<int64_t>(wt2) * gu;
+            const int64_t g1 = min(g0 + gu, gpr) - 1;
+#pragma unroll
+            for (int h = 0; h < BK / 32; ++h) {
+                const int64_t row = (static_cast<int64_t>(e2) * prm.K + ks2 * BK + h * 32 + lane) * gpr;
+                prefetch_l2(prm.scales + row + g0);
+                prefetch_l2(prm.scales + row + g1);
+                prefetch_l2(prm.biases + row + g0);
+                prefetch_l2(prm.biases + row + g1);
+            }
+        };
+        if (static_cast<int>(blockIdx.x) < units)
+            for (int i = 0; i < kL2Ahead && i < ksteps; ++i) prefetch_stage(blockIdx.x, i);
+        RingPos c;
+        int issued = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int e, wt, first, count;
+            unit_pairs(u, e, wt, first, count);
+            for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (lane == 0) {
+                        if (c.use > 0) ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 61, 512);
+                        if (ok) {
+                            mbar_expect_tx(&full_c[c.s], prm.c_stage);
+                            tma_load_3d(c_ring + c.s * prm.c_stage, &map_c, &full_c[c.s],
+                                        wt * UW * BITS / 32, ks * BK, e);
+                            ++issued;
+                        }
                     }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    if (ks + kL2Ahead < ksteps) prefetch_stage(u, ks + kL2Ahead);
+                    else if (p0 + kMaxPairs >= count && u + static_cast<int>(gridDim.x) < units &&
+                             ks + kL2Ahead - ksteps < ksteps)
+                        prefetch_stage(u + gridDim.x, ks + kL2Ahead - ksteps);
+                    c.next(DC);
                 }
             }
+        }
+        if (lane == 0) {
             for (int j = 0; j < DC && j < issued; ++j) {  // drain the last copies
                 if (--c.s < 0) { c.s = DC - 1; --c.use; }
                 mbar_wait(&full_c[c.s], c.use & 1, 69);
@@ -326,86 +378,136 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
         while (pending > 0) complete_one();
     } else {
         // ------------------------------------------ dequantize and transpose
-        // A warp task is 16 code words x 8 k-rows: lane (l & 15) takes word
-        // j = 16 jh + (l & 15), lane bit 4 picks k-rows 4 kq .. 4 kq + 3 with
-        // kq = 2 kh + (l >> 4). Column n of the unit goes to A-row a_row(n)
-        // (an involution on the low three bits), which spreads a warp's
-        // 8-byte stores over all 32 banks; the code reads are two-way.
+        // Two groups of 8 warps take alternate stages, so one group's loads of
+        // scales and biases overlap the other's arithmetic. A warp task is 16
+        // code words x 8 k-rows: lane l takes word j = 16 jh + (l >> 1) and
+        // k-rows 4 kq .. 4 kq + 3 with kq = 2 kh + (l & 1). Column n of the unit
+        // goes to A-row a_row(n) (an involution on the low three bits), so each
+        // half-warp's 8-byte stores cover the 32 banks once; the code reads are
+        // two-way.
         constexpr int PER = 32 / BITS;
         constexpr int WPR = UW * BITS / 32;          // code words per k-row of a stage
         constexpr int WTASKS = (WPR / 16) * (BK / 8);
+        constexpr int GW = kDequantThreads / 32 / kDequantGroups;  // warps per group
         const int dw = warp - kDequantWarp0;          // 0 .. 15
-        const int jl = lane & 15, kl = lane >> 4;
-        const int64_t gpr = prm.N / prm.gs;           // groups per k-row of W
+        const int grp = dw / GW, wig = dw % GW;
+        const int jl = lane >> 1, kl = lane & 1;
+        const int64_t gpr = prm.N >> prm.lg_gs;       // groups per k-row of W
         RingPos c, w;
         bool ok = true;
+        int st = 0;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int e, wt, first, count;
             unit_pairs(u, e, wt, first, count);
             const uint16_t* se = prm.scales + static_cast<int64_t>(e) * prm.K * gpr;
             const uint16_t* be = prm.biases + static_cast<int64_t>(e) * prm.K * gpr;
             for (int p0 = 0; p0 < count && ok; p0 += kMaxPairs) {
-                for (int ks = 0; ks < ksteps; ++ks) {
+                for (int ks = 0; ks < ksteps; ++ks, c.next(DC), w.next(DW)) {
+                    if (st++ % kDequantGroups != grp) continue;
                     if (!(ok = mbar_wait(&full_c[c.s], c.use & 1, 62))) break;
                     if (w.use > 0 && !(ok = mbar_wait_backoff(&empty_w[w.s], (w.use - 1) & 1, 63, 128))) break;
                     const uint8_t* cst = c_ring + c.s * prm.c_stage;
-                    uint8_t* wst = w_ring + w.s * kWStage;
-                    for (int wtask = dw; wtask < WTASKS; wtask += kDequantThreads / 32) {
+                    const uint32_t wst = smem_u32(w_ring + w.s * kWStage);
+#pragma unroll
+                    for (int mt = 0; mt < WTASKS / GW; ++mt) {
+                        const int wtask = wig + mt * GW;
                         const int j = (wtask / (BK / 8)) * 16 + jl;
                         const int kq = (wtask % (BK / 8)) * 2 + kl;
-                        const int nl = j * PER;                                   // first column in the unit
-                        const int64_t ng = static_cast<int64_t>(wt) * UW + nl;    // and in W
-                        const int64_t kg = static_cast<int64_t>(ks) * BK + 4 * kq;
-                        const bool live = ng < prm.N;
+                        const int64_t ng = static_cast<int64_t>(wt) * UW + j * PER;  // first column in W
+                        // scales and biases of k-rows kg .. kg + 3 in the words' group
+                        // (a word past N reads column N - 1's: its outputs are dropped)
+                        const uint32_t kg = static_cast<uint32_t>(ks * BK + 4 * kq);
+                        const uint32_t o = kg * static_cast<uint32_t>(gpr) +
+                                           static_cast<uint32_t>((ng < prm.N ? ng : prm.N - 1) >> prm.lg_gs);
                         uint32_t cw[4], sraw[4], braw[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             cw[i] = *reinterpret_cast<const uint32_t*>(cst + (4 * kq + i) * (WPR * 4) + 4 * j);
-                            const int64_t gi = (kg + i) * gpr + (live ? ng / prm.gs : 0);
-                            sraw[i] = live ? __ldg(se + gi) : 0u;
-                            braw[i] = live ? __ldg(be + gi) : 0u;
+                            sraw[i] = __ldg(se + o + i * static_cast<uint32_t>(gpr));
+                            braw[i] = __ldg(be + o + i * static_cast<uint32_t>(gpr));
                         }
                         // (k, k + 1) pairs of scales and biases as bf16x2
-                        const uint32_t s01 = sraw[0] | (sraw[1] << 16), s23 = sraw[2] | (sraw[3] << 16);
-                        const uint32_t b01 = braw[0] | (braw[1] << 16), b23 = braw[2] | (braw[3] << 16);
+                        const uint32_t s01 = prmt(sraw[0], sraw[1], 0x5410), s23 = prmt(sraw[2], sraw[3], 0x5410);
+                        const uint32_t b01 = prmt(braw[0], braw[1], 0x5410), b23 = prmt(braw[2], braw[3], 0x5410);
+                        // Shared address of column (j * PER + f), k-rows 4 kq .. 4 kq + 3: its A-row
+                        // ar = a_row(n) has ar & 7 = (f & 7) ^ t and ar >> 3 = r8 + (f >> 3), so
+                        // the address is A ^ ((f & 7) * 0x90) + (f >> 3) * 1024 (the XOR only
+                        // touches bits 4 - 9, which A holds as (t << 7) | ((q ^ t) << 4)).
+                        const int r8 = PER >= 8 ? j * (PER / 8) : j >> 1;
+                        const int t = PER >= 8 ? (j & 7) : ((4 * (j & 1)) ^ ((j >> 1) & 7));
+                        const int q = kq >> 1;
+                        const uint32_t A = wst + static_cast<uint32_t>(r8 * 1024 + (kq & 1) * 8 +
+                                                                      ((t << 7) | ((q ^ t) << 4)));
+                        auto put = [&](int f, uint32_t v0, uint32_t v1) {
+                            const uint32_t a = (A ^ static_cast<uint32_t>((f & 7) * 0x90)) + (f >> 3) * 1024;
+                            // no memory clobber: the stage is published by the fence and
+                            // arrive below, and no load here reads the A tiles
+                            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a), "r"(v0), "r"(v1));
+                        };
+                        // fast form (every scale of the warp task normal and below 2^-5): a
+                        // code field masked in place at bit p of a half is c * 2^(p - 133)
+                        // as a bf16, and the fma takes s * 2^(133 - p): the same exact
+                        // product s * c, rounded once with the bias.
+                        // (magnitudes of the four scales in [2^-126, 2^-5): bf16 patterns
+                        // 0x0080 .. 0x3CFF without the sign)
+                        const uint32_t mn = vmin_u16x2(s01 & 0x7FFF7FFFu, s23 & 0x7FFF7FFFu);
+                        const uint32_t mx = vmax_u16x2(s01 & 0x7FFF7FFFu, s23 & 0x7FFF7FFFu);
+                        const bool fast = vmin_u16x2(mn, mn >> 16) >= 0x0080u &&
+                                          (vmax_u16x2(mx, mx >> 16) & 0xFFFFu) < 0x3D00u;
+                        if (__all_sync(0xffffffffu, fast)) {
+                            constexpr int FPB = 8 / BITS;  // fields per byte
+                            constexpr uint32_t FM = ((1u << BITS) - 1u) * 0x00010001u;
+                            uint32_t m01[FPB], m23[FPB];
 #pragma unroll
-                        for (int f = 0; f < PER; ++f) {
-                            uint32_t v[2];
-                            if constexpr (BITS == 8) {
-                                // packed fp32: 2^23 + c exactly, minus 2^23, then s c + b
-                                const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);
-                                const uint64_t off = f2_pack(0xCB000000u, 0xCB000000u);
-#pragma unroll
-                                for (int p = 0; p < 2; ++p) {
-                                    const uint64_t r = f2_pack(prmt(cw[2 * p], 0x4B000000u, f | 0x7440),
-                                                               prmt(cw[2 * p + 1], 0x4B000000u, f | 0x7440));
-                                    const uint64_t cc = f2_fma(r, one_m, off);
-                                    const uint64_t sc = f2_pack(sraw[2 * p] << 16, sraw[2 * p + 1] << 16);
-                                    const uint64_t bc = f2_pack(braw[2 * p] << 16, braw[2 * p + 1] << 16);
-                                    v[p] = f2_to_bf2_packed(f2_fma(sc, cc, bc));
-                                }
-                            } else {
-                                // field f of k-rows (k, k + 1) into the two halves: 128 + c
-                                const int byte = (f * BITS) >> 3, sh = (f * BITS) & 7;
-                                const uint32_t sel = static_cast<uint32_t>(byte | ((4 + byte) << 8));
-                                constexpr uint32_t MSK = ((1u << BITS) - 1u) * 0x00010001u;
-                                const uint32_t r0 = codes_to_bf16x2(prmt(cw[0], cw[1], sel) >> sh, MSK);
-                                const uint32_t r1 = codes_to_bf16x2(prmt(cw[2], cw[3], sel) >> sh, MSK);
-                                v[0] = bf2_fma(s01, bf2_sub(r0, 0x43004300u), b01);
-                                v[1] = bf2_fma(s23, bf2_sub(r1, 0x43004300u), b23);
+                            for (int p = 0; p < FPB; ++p) {
+                                const uint32_t ex = static_cast<uint32_t>(133 - p * BITS) * 0x00800080u;
+                                m01[p] = s01 + ex;
+                                m23[p] = s23 + ex;
                             }
-                            // A-row of column nl + f: 8-row atom, k-chunk kq / 2 (8 k), half kq & 1
-                            const int ar = a_row<BITS>(nl + f);
-                            *reinterpret_cast<uint2*>(wst + (ar >> 3) * 1024 + (ar & 7) * 128 +
-                                                      (((kq >> 1) ^ (ar & 7)) << 4) + (kq & 1) * 8) =
-                                make_uint2(v[0], v[1]);
+#pragma unroll
+                            for (int by = 0; by < 4; ++by) {
+                                // byte by of k-rows (k, k + 1) into the low bytes of the halves
+                                const uint32_t sel = static_cast<uint32_t>(by | ((4 + by) << 8));
+                                const uint32_t x01 = prmt(cw[0], cw[1], sel), x23 = prmt(cw[2], cw[3], sel);
+#pragma unroll
+                                for (int p = 0; p < FPB; ++p)
+                                    put(by * FPB + p, bf2_fma(m01[p], x01 & (FM << (p * BITS)), b01),
+                                        bf2_fma(m23[p], x23 & (FM << (p * BITS)), b23));
+                            }
+                        } else {
+#pragma unroll
+                            for (int f = 0; f < PER; ++f) {
+                                uint32_t v[2];
+                                if constexpr (BITS == 8) {
+                                    // packed fp32: 2^23 + c exactly, minus 2^23, then s c + b
+                                    const uint64_t one_m = f2_pack(0x3F800000u, 0x3F800000u);
+                                    const uint64_t off = f2_pack(0xCB000000u, 0xCB000000u);
+#pragma unroll
+                                    for (int pp = 0; pp < 2; ++pp) {
+                                        const uint64_t r = f2_pack(prmt(cw[2 * pp], 0x4B000000u, f | 0x7440),
+                                                                   prmt(cw[2 * pp + 1], 0x4B000000u, f | 0x7440));
+                                        const uint64_t cc = f2_fma(r, one_m, off);
+                                        const uint64_t sc = f2_pack(sraw[2 * pp] << 16, sraw[2 * pp + 1] << 16);
+                                        const uint64_t bc = f2_pack(braw[2 * pp] << 16, braw[2 * pp + 1] << 16);
+                                        v[pp] = f2_to_bf2_packed(f2_fma(sc, cc, bc));
+                                    }
+                                } else {
+                                    // field f of k-rows (k, k + 1) into the two halves: 128 + c
+                                    const int byte = (f * BITS) >> 3, sh = (f * BITS) & 7;
+                                    const uint32_t sel = static_cast<uint32_t>(byte | ((4 + byte) << 8));
+                                    constexpr uint32_t MSK = ((1u << BITS) - 1u) * 0x00010001u;
+                                    const uint32_t r0 = codes_to_bf16x2(prmt(cw[0], cw[1], sel) >> sh, MSK);
+                                    const uint32_t r1 = codes_to_bf16x2(prmt(cw[2], cw[3], sel) >> sh, MSK);
+                                    v[0] = bf2_fma(s01, bf2_sub(r0, 0x43004300u), b01);
+                                    v[1] = bf2_fma(s23, bf2_sub(r1, 0x43004300u), b23);
+                                }
+                                put(f, v[0], v[1]);
+                            }
                         }
                     }
                     fence_proxy_async();
                     __syncwarp();
                     if (lane == 0) { mbar_arrive(&empty_c[c.s]); mbar_arrive(&full_w[w.s]); }
-                    c.next(DC);
-                    w.next(DW);
                 }
             }
         }
@@ -433,9 +535,11 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
 }  // namespace
 
 bool tc_gather_t0_supported(int64_t K, int64_t N, int bits, int gs) {
-    // code rows of 16-byte multiples (TMA), 64-k steps
+    // code rows of 16-byte multiples (TMA), 64-k steps, 32-bit offsets into
+    // one expert's scales
     return K % BK == 0 && K >= BK && N > 0 && (bits == 2 || bits == 4 || bits == 8) &&
-           (gs == 32 || gs == 64 || gs == 128) && N % gs == 0 && (N * bits) % 128 == 0;
+           (gs == 32 || gs == 64 || gs == 128) && N % gs == 0 && (N * bits) % 128 == 0 &&
+           K * (N / gs) < (int64_t(1) << 32);
 }
 
 unsigned int tc_gather_t0_error_take() { return pipeline_error_take(); }
@@ -466,6 +570,7 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     prm.scales = static_cast<const uint16_t*>(scales);
     prm.biases = static_cast<const uint16_t*>(biases);
     prm.gs = gs;
+    prm.lg_gs = gs == 32 ? 5 : gs == 64 ? 6 : 7;
     prm.lhs = lhs;
     prm.perm = perm;
     prm.offsets = offsets;
@@ -474,7 +579,7 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     prm.E = E;
     prm.wunits = static_cast<int>((N + UW - 1) / UW);
     prm.c_stage = static_cast<uint32_t>(BK * UW * bits / 8);
-    int dw = 3, dx = 8, dc = 4;
+    int dw = 4, dx = 8, dc = 4;
     auto bytes = [&]() {
         return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kWStage) * dw +
                static_cast<size_t>(prm.c_stage) * dc + kMaxPairs * 8 * 4 +
@@ -482,7 +587,8 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
     while (bytes() > budget && dx > 4) --dx;
-    while (bytes() > budget && dc > 2) --dc;
+    while (bytes() > budget && dc > 3) --dc;
+    while (bytes() > budget && dw > 3) --dw;
     if (bytes() > budget) return cudaErrorInvalidConfiguration;
     prm.dw = dw;
     prm.dx = dx;

@@ -48,14 +48,22 @@ def test_ragged_experts(bits, gs):
     P.assert_within(y, yr, a, BF16, f"transpose=0 ragged b{bits} g{gs}")
 
 
+@pytest.mark.parametrize("spread", ["small", "wide"])
 @pytest.mark.parametrize("bits", [4, 8, 2])
-def test_unit_activations_read_out_the_weights(bits):
+def test_unit_activations_read_out_the_weights(bits, spread):
     """x rows are unit vectors e_k: every output is one dequantized weight
     w_hat[k, n] times 1 plus exact zeros, so it must equal the oracle's stored
     (once-rounded) weight bit for bit. Covers every column of two units, the
-    A-tile row order and the epilogue's column map."""
+    A-tile row order and the epilogue's column map. "small": N(0, 0.02)
+    weights (scales below 2^-5); "wide": k-rows scaled by 10^u, u in [-5, 3],
+    and a constant row (scale 0), so scales on both sides of 2^-5 and zero
+    meet in the same stages."""
     E, K, N, gs = 3, 256, 512, 64
     w = W.normal((E, K, N), 0.02, 73, "bf16")
+    if spread == "wide":
+        g = torch.Generator().manual_seed(86)
+        w = (w.float() * 10.0 ** (torch.rand(E, K, 1, generator=g) * 8 - 5)).to(BF16)
+        w[:, 5, :] = 0.75
     c, s, b = O.quantize_affine(w, gs, bits)
     wh = O.dequantize_stored(c, s, b, gs, bits)  # [E, K, N] bf16
     g = torch.Generator().manual_seed(74)
