@@ -65,6 +65,7 @@ struct TParams {
     int dc;                     // code ring depth
     uint32_t c_off;
     uint32_t c_stage;           // bytes of one code stage (64 k-rows x 256 columns)
+    uint32_t sb_off;            // staged scales and biases (STAGED): 2 KB per code stage
     const uint16_t* x;          // [x_rows, K]
     const uint32_t* lhs;        // nullable
     const uint32_t* perm;       // [R] pairs in expert order
@@ -114,9 +115,13 @@ __device__ __forceinline__ int a_row(int n) {
     return n ^ ((n >> S) & 7);
 }
 
-template <int BITS>
+// STAGED (N / gs a multiple of 8): each stage's scales and biases arrive by
+// TMA with its codes, as [64 k-rows][8 groups] boxes that cover the unit's
+// groups; otherwise the dequantizers read them from global memory.
+template <int BITS, bool STAGED>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm) {
+tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_s,
+                    const __grid_constant__ CUtensorMap map_b, const TParams prm) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -124,6 +129,7 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
     uint8_t* x_ring = smem + prm.x_off;
     uint8_t* w_ring = smem + prm.w_off;
     uint8_t* c_ring = smem + prm.c_off;
+    uint8_t* sb_ring = smem + prm.sb_off;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prm.bar_off);
     uint64_t* full_w = bars;
     uint64_t* empty_w = full_w + DW;
@@ -187,6 +193,13 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
         auto prefetch_stage = [&](int u2, int ks2) {
             const int e2 = u2 / prm.wunits, wt2 = u2 - e2 * prm.wunits;
             if (lane == 0) tma_prefetch_3d(&map_c, wt2 * UW * BITS / 32, ks2 * BK, e2);
+            if constexpr (STAGED) {
+                if (lane == 0) {
+                    tma_prefetch_3d(&map_s, (wt2 * gu) & ~7, ks2 * BK, e2);
+                    tma_prefetch_3d(&map_b, (wt2 * gu) & ~7, ks2 * BK, e2);
+                }
+                return;
+            }
             const int64_t g0 = static_cast<int64_t>(wt2) * gu;
             const int64_t g1 = min(g0 + gu, gpr) - 1;
 #pragma unroll
@@ -211,9 +224,14 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
                     if (lane == 0) {
                         if (c.use > 0) ok = mbar_wait_backoff(&empty_c[c.s], (c.use - 1) & 1, 61, 512);
                         if (ok) {
-                            mbar_expect_tx(&full_c[c.s], prm.c_stage);
+                            mbar_expect_tx(&full_c[c.s], prm.c_stage + (STAGED ? 2048u : 0u));
                             tma_load_3d(c_ring + c.s * prm.c_stage, &map_c, &full_c[c.s],
                                         wt * UW * BITS / 32, ks * BK, e);
+                            if constexpr (STAGED) {
+                                uint8_t* sbs = sb_ring + c.s * 2048;
+                                tma_load_3d(sbs, &map_s, &full_c[c.s], (wt * gu) & ~7, ks * BK, e);
+                                tma_load_3d(sbs + 1024, &map_b, &full_c[c.s], (wt * gu) & ~7, ks * BK, e);
+                            }
                             ++issued;
                         }
                     }
@@ -417,14 +435,23 @@ tc_gather_t0_kernel(const __grid_constant__ CUtensorMap map_c, const TParams prm
                         // scales and biases of k-rows kg .. kg + 3 in the words' group
                         // (a word past N reads column N - 1's: its outputs are dropped)
                         const uint32_t kg = static_cast<uint32_t>(ks * BK + 4 * kq);
-                        const uint32_t o = kg * static_cast<uint32_t>(gpr) +
-                                           static_cast<uint32_t>((ng < prm.N ? ng : prm.N - 1) >> prm.lg_gs);
+                        const uint32_t gc = static_cast<uint32_t>((ng < prm.N ? ng : prm.N - 1) >> prm.lg_gs);
+                        const uint32_t o = kg * static_cast<uint32_t>(gpr) + gc;
                         uint32_t cw[4], sraw[4], braw[4];
+                        // staged: [64 k-rows][8 groups] from group (wt * gu) & ~7 on, scales
+                        // then biases
+                        const uint16_t* sbs = reinterpret_cast<const uint16_t*>(sb_ring + c.s * 2048) + 4 * kq * 8 +
+                                              (gc & 7);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             cw[i] = *reinterpret_cast<const uint32_t*>(cst + (4 * kq + i) * (WPR * 4) + 4 * j);
-                            sraw[i] = __ldg(se + o + i * static_cast<uint32_t>(gpr));
-                            braw[i] = __ldg(be + o + i * static_cast<uint32_t>(gpr));
+                            if constexpr (STAGED) {
+                                sraw[i] = sbs[i * 8];
+                                braw[i] = sbs[512 + i * 8];
+                            } else {
+                                sraw[i] = __ldg(se + o + i * static_cast<uint32_t>(gpr));
+                                braw[i] = __ldg(be + o + i * static_cast<uint32_t>(gpr));
+                            }
                         }
                         // (k, k + 1) pairs of scales and biases as bf16x2
                         const uint32_t s01 = prmt(sraw[0], sraw[1], 0x5410), s23 = prmt(sraw[2], sraw[3], 0x5410);
@@ -564,6 +591,22 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    // scales and biases [E][K][N / gs] as boxes of 8 groups x 64 k-rows, when
+    // their rows are whole multiples of 16 bytes
+    const int64_t gpr = N / gs;
+    const bool staged = gpr % 8 == 0;
+    CUtensorMap map_s = map_c, map_b = map_c;
+    if (staged) {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(gpr), static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(E)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(gpr) * 2, static_cast<cuuint64_t>(gpr * K) * 2};
+        cuuint32_t box[3] = {8, BK, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        for (int i = 0; i < 2; ++i)
+            if (enc(i ? &map_b : &map_s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(i ? biases : scales),
+                    dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+    }
     TParams prm{};
     prm.y = static_cast<uint16_t*>(y);
     prm.x = static_cast<const uint16_t*>(x);
@@ -582,7 +625,7 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     int dw = 4, dx = 8, dc = 4;
     auto bytes = [&]() {
         return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kWStage) * dw +
-               static_cast<size_t>(prm.c_stage) * dc + kMaxPairs * 8 * 4 +
+               static_cast<size_t>(prm.c_stage + (staged ? 2048 : 0)) * dc + kMaxPairs * 8 * 4 +
                static_cast<size_t>(2 * (dw + dx + dc) + 4) * 8 + 16;
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
@@ -596,13 +639,17 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     prm.x_off = 0;
     prm.w_off = kXStage * dx;
     prm.c_off = prm.w_off + kWStage * dw;
-    prm.row_off = prm.c_off + prm.c_stage * dc;
+    prm.sb_off = prm.c_off + prm.c_stage * dc;
+    prm.row_off = prm.sb_off + (staged ? 2048 : 0) * dc;
     prm.bar_off = prm.row_off + kMaxPairs * 8 * 4;
     const size_t smem = bytes() + 1024;
     const int units = static_cast<int>(E) * prm.wunits;
     const int grid = units < num_sms ? units : num_sms;
-    void (*k)(const CUtensorMap, const TParams) =
-        bits == 4 ? tc_gather_t0_kernel<4> : bits == 8 ? tc_gather_t0_kernel<8> : tc_gather_t0_kernel<2>;
+    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TParams) =
+        staged ? (bits == 4 ? tc_gather_t0_kernel<4, true> : bits == 8 ? tc_gather_t0_kernel<8, true>
+                                                                      : tc_gather_t0_kernel<2, true>)
+               : (bits == 4 ? tc_gather_t0_kernel<4, false> : bits == 8 ? tc_gather_t0_kernel<8, false>
+                                                                       : tc_gather_t0_kernel<2, false>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     // programmatic dependent launch on the routing kernel (see the kernel)
@@ -616,7 +663,7 @@ cudaError_t launch_tc_gather_t0(const void* x, int64_t x_rows, int64_t K, const 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k, map_c, prm);
+    return cudaLaunchKernelEx(&cfg, k, map_c, map_s, map_b, prm);
 }
 
 }  // namespace nvq

@@ -31,12 +31,15 @@ def _gather(x, c, s, b, rhs, lhs, gs, bits, sorted_=False, ws=None):
     return y.cpu(), flags
 
 
+@pytest.mark.parametrize("N", [384, 1024])
 @pytest.mark.parametrize("bits,gs", QUANTS)
-def test_ragged_experts(bits, gs):
+def test_ragged_experts(bits, gs, N):
     """37 pairs over 5 experts (one empty, one with 17 pairs); N = 384 is one
-    full unit of 256 columns and one that ends half way."""
+    full unit of 256 columns and one that ends half way, and its scale rows
+    are read from global memory; N = 1024 has N / gs a multiple of 8, so the
+    scales and biases come with the codes by TMA."""
     g = torch.Generator().manual_seed(70 + bits + gs)
-    E, K, N, T = 5, 512, 384, 23
+    E, K, T = 5, 512, 23
     w = W.normal((E, K, N), 0.02, 71, "bf16")
     x = W.normal((T, K), 1.0, 72, "bf16")
     c, s, b = O.quantize_affine(w, gs, bits)
