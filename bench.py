@@ -162,6 +162,8 @@ def check_gather(wl, samples=64):
     for r in pick:
         e, t = int(wl.rhs[r]), int(wl.lhs[r])
         w = unpack_dequant(c[e], s[e], b[e], 64, 4)
+        if not getattr(wl, "transpose", True):
+            w = w.t()
         worst = max(worst, worst_ratio(wl.y[r:r + 1], wl.x[t:t + 1], w))
     return worst
 
@@ -455,15 +457,18 @@ def check_gather_mm(wl, samples=64):
 
 
 class Gather:
-    """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4."""
+    """Mixture of experts: 64 experts [1536, 2048] 4-bit g64, 512 tokens x top-4
+    (transpose False: the experts stored [2048, 1536], grouped along N)."""
 
-    def __init__(self, dev, sorted_pairs: bool, row_exact: bool = False):
+    def __init__(self, dev, sorted_pairs: bool, row_exact: bool = False, transpose: bool = True):
         import group_wise_affine_dequant_b200 as nvq
         self.row_exact = row_exact
+        self.transpose = transpose
         self.nvq = nvq
         m = W.MOE
         self.E, self.N, self.K, self.T = m["E"], m["N"], m["K"], m["tokens"]
-        w = W.normal((self.E, self.N, self.K), 0.02, 0, "bf16").to(dev)
+        shape = (self.E, self.N, self.K) if transpose else (self.E, self.K, self.N)
+        w = W.normal(shape, 0.02, 0, "bf16").to(dev)
         c, s, b = nvq.nv_quantize_affine(w, 64, 4)
         del w
         wbytes = qbytes(self.E * self.N, self.K, 4, 64)
@@ -486,7 +491,7 @@ class Gather:
 
     def call(self, j):
         c, s, b = self.ws[j]
-        self.nvq.nv_gather_qmm(self.x, c, s, b, self.rhs, self.lhs, 64, 4, True, self.sorted,
+        self.nvq.nv_gather_qmm(self.x, c, s, b, self.rhs, self.lhs, 64, 4, self.transpose, self.sorted,
                                self.row_exact, workspace=self.wsp, out=self.y)
 
     def step(self, i):
@@ -644,9 +649,10 @@ def run_nvq(args):
     also["dequantize_frac_of_hbm"] = round(dq / ws / pk["hbm_gbs"], 4)
     checks["dequantize"] = chk(check_dequant, wl)
     del g, wl
-    for name, srt, rx in (("gather_sorted", True, False), ("gather_unsorted", False, False),
-                          ("gather_row_exact", False, True)):
-        wl = Gather(dev, srt, rx)
+    for name, srt, rx, tr in (("gather_sorted", True, False, True), ("gather_unsorted", False, False, True),
+                              ("gather_row_exact", False, True, True),
+                              ("gather_kn_sorted", True, False, False)):
+        wl = Gather(dev, srt, rx, tr)
         g = timed_graph(wl.step, ks, Wm, stream)
         t = max_ms(replay_timed(g, stream, barrier))
         also[name + "_tok_s"] = round(replica_rate(ws, wl.T * wl.copies, ks, t), 1)

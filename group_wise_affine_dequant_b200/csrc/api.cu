@@ -234,23 +234,25 @@ nv_status nv_gather_qmm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
 
     cudaStream_t s = stream;
     const int sms = sm_count();
-    nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
-    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
-    if (e != cudaSuccess) return from_cuda(e);
-    if (N == 0) return NV_OK;
-    // Tensor-core route: each expert's weights are read once for all its rows.
-    // (the tensor-core kernel keeps 32-bit offsets into x in 16-byte units)
-    if (dt == NV_BF16 && transpose && !row_exact && nvq::tc_gather_supported(K, N, bits, group_size) &&
-        x_rows * K < (int64_t(1) << 35))
-        return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
-                                               codes, scales, biases, group_size, bits, y, s, sms));
-    if (dt == NV_BF16 && !transpose && !row_exact && nvq::tc_gather_t0_supported(K, N, bits, group_size) &&
-        x_rows * K < (int64_t(1) << 35))
-        return from_cuda(nvq::launch_tc_gather_t0(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
-                                                  codes, scales, biases, group_size, bits, y, s, sms));
+    // Tensor-core routes: each expert's weights are read once for all its rows
+    // (the kernels keep 32-bit offsets into x in 16-byte units).
+    const bool tc = dt == NV_BF16 && !row_exact && x_rows * K < (int64_t(1) << 35) &&
+                    (transpose ? nvq::tc_gather_supported(K, N, bits, group_size)
+                               : nvq::tc_gather_t0_supported(K, N, bits, group_size));
     // Matrix-vector route (row_exact): every pair's output is bitwise equal to
     // nv_qmm(M = 1) of that row with its expert's weights.
-    if (dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size))
+    const bool mv = !tc && dt == NV_BF16 && transpose && nvq::qmv_supported(bits, group_size);
+    nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
+    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s, mv);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (N == 0) return NV_OK;
+    if (tc && transpose)
+        return from_cuda(nvq::launch_tc_gather(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
+                                               codes, scales, biases, group_size, bits, y, s, sms));
+    if (tc)
+        return from_cuda(nvq::launch_tc_gather_t0(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N,
+                                                  codes, scales, biases, group_size, bits, y, s, sms));
+    if (mv)
         return from_cuda(nvq::launch_qmv_gather(x, K, N, codes, scales, biases, group_size, bits,
                                                 lhs_idx, ws.perm, ws.problems, ws.num_problems,
                                                 ws.max_problems, E, y, s, sms));
@@ -277,7 +279,7 @@ nv_status nv_gather_mm(const void* x, nv_dtype dt, int64_t x_rows, int64_t K,
         return NV_ERR_INVALID_ARG;
     cudaStream_t s = stream;
     nvq::GatherWorkspace ws = nvq::gather_workspace_carve(workspace, R, E);
-    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s);
+    cudaError_t e = nvq::launch_gather_route(lhs_idx, rhs_idx, R, E, x_rows, sorted, ws, s, false);
     if (e != cudaSuccess) return from_cuda(e);
     if (N == 0) return NV_OK;
     return from_cuda(nvq::launch_tc_gather_mm(x, x_rows, K, lhs_idx, ws.perm, ws.offsets, E, N, w,

@@ -56,12 +56,17 @@ __device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32
     return r;
 }
 
+// Pairs per lane whose keys stay in registers between the histogram and the
+// scatter (a warp's segment of up to 32 * kKeyRegs pairs is read once; longer
+// segments read the rest again in the scatter).
+constexpr int kKeyRegs = 4;
+
 __global__ void __launch_bounds__(kRouteThreads, 1) gather_route_kernel(
     const uint32_t* __restrict__ lhs, const uint32_t* __restrict__ rhs, int64_t R, int E,
-    int64_t x_rows, int sorted, uint32_t* __restrict__ flags_out,
+    int64_t x_rows, int sorted, int want_problems, uint32_t* __restrict__ flags_out,
     uint32_t* __restrict__ num_problems, uint32_t* __restrict__ offsets_out,
     uint32_t* __restrict__ perm, uint32_t* __restrict__ problems) {
-    extern __shared__ uint32_t hist[];  // [kRouteWarps][E + 1]
+    extern __shared__ uint32_t hist[];  // [kRouteWarps][E + 1], then bucket offsets [E + 1]
     __shared__ uint32_t warp_sums[33];
     __shared__ uint32_t s_flags;
     const int NB = E + 1;  // buckets: experts, then "invalid"
@@ -72,7 +77,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1) gather_route_kernel(
 
     for (int i = threadIdx.x; i < kRouteWarps * NB; i += kRouteThreads) hist[i] = 0;
     if (threadIdx.x == 0) s_flags = 0;
-    __syncthreads();
 
     const int64_t seg0 = warp * R / kRouteWarps, seg1 = (warp + 1) * R / kRouteWarps;
     uint32_t my_flags = 0;
@@ -86,66 +90,86 @@ __global__ void __launch_bounds__(kRouteThreads, 1) gather_route_kernel(
         }
         return (e < static_cast<uint32_t>(E) && t < x_rows) ? static_cast<int>(e) : E;
     };
+    // the first kKeyRegs chunks of the segment: all loads issued before any use
+    int key[kKeyRegs];
+#pragma unroll
+    for (int i = 0; i < kKeyRegs; ++i) {
+        const int64_t r = seg0 + 32 * i + lane;
+        key[i] = r < seg1 ? key_of(r, true) : NB;
+    }
+    __syncthreads();  // histograms zeroed
 
     // Phase 1: per-warp histograms.
-    for (int64_t c = seg0; c < seg1; c += 32) {
-        const int64_t r = c + lane;
-        const bool valid = r < seg1;
-        const int key = valid ? key_of(r, true) : NB;
-        const uint32_t mask = __match_any_sync(0xffffffffu, key);
-        if (valid && lane == __ffs(mask) - 1) hist[warp * NB + key] += __popc(mask);
+    auto count_key = [&](int k) {
+        const uint32_t mask = __match_any_sync(0xffffffffu, k);
+        if (k < NB && lane == __ffs(mask) - 1) hist[warp * NB + k] += __popc(mask);
         __syncwarp();
+    };
+#pragma unroll
+    for (int i = 0; i < kKeyRegs; ++i) count_key(key[i]);
+    for (int64_t c = seg0 + 32 * kKeyRegs; c < seg1; c += 32) {
+        const int64_t r = c + lane;
+        count_key(r < seg1 ? key_of(r, true) : NB);
     }
     if (my_flags) atomicOr(&s_flags, my_flags);
     __syncthreads();
 
-    // Phase 2: per-bucket totals, per-warp bases within a bucket, bucket offsets.
+    // Phase 2: per-bucket totals and per-warp bases within a bucket (warp w
+    // scans buckets w, w + 32, ...: lane l holds warp l's count), then the
+    // bucket offsets.
+    uint32_t* cnt = hist + kRouteWarps * NB;  // bucket totals, then offsets
+    for (int bk = warp; bk < NB; bk += kRouteWarps) {
+        const uint32_t h = hist[lane * NB + bk];
+        uint32_t inc = h;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += n;
+        }
+        hist[lane * NB + bk] = inc - h;
+        if (lane == 31) cnt[bk] = inc;
+    }
+    __syncthreads();
     const int b = threadIdx.x;  // NB <= kRouteThreads
-    uint32_t count = 0;
-    if (b < NB) {
-        for (int w = 0; w < kRouteWarps; ++w) {
-            const uint32_t h = hist[w * NB + b];
-            hist[w * NB + b] = count;
-            count += h;
-        }
-    }
+    const uint32_t count = b < NB ? cnt[b] : 0u;
     uint32_t total;
-    const uint32_t off = block_exclusive_scan(b < NB ? count : 0u, warp_sums, total);
-    if (b < NB) offsets_out[b] = off;
-    if (b == 0) offsets_out[NB] = total;
-    // Problems: ceil(count / 8) per bucket, bucket by bucket.
-    const uint32_t np = (count + 7) / 8;
-    uint32_t np_total;
-    const uint32_t poff = block_exclusive_scan(b < NB ? np : 0u, warp_sums, np_total);
+    const uint32_t off = block_exclusive_scan(count, warp_sums, total);
     if (b < NB) {
-        for (uint32_t i = 0; i < np; ++i) {
-            uint32_t* pr = problems + 4 * (poff + i);
-            pr[0] = static_cast<uint32_t>(b);
-            pr[1] = off + 8 * i;
-            pr[2] = min(8u, count - 8 * i);
-            pr[3] = 0;
-        }
-        hist[kRouteWarps * NB + b] = off;  // scratch row: bucket offsets for phase 3
+        offsets_out[b] = off;
+        cnt[b] = off;  // bucket offsets for phase 3 (each thread rewrites its own entry)
     }
-    if (b == 0) {
-        *num_problems = np_total;
+    if (b == 0) offsets_out[NB] = total;
+    if (want_problems) {
+        // Problems: ceil(count / 8) per bucket, bucket by bucket.
+        const uint32_t np = (count + 7) / 8;
+        uint32_t np_total;
+        const uint32_t poff = block_exclusive_scan(b < NB ? np : 0u, warp_sums, np_total);
+        if (b < NB) {
+            for (uint32_t i = 0; i < np; ++i) {
+                uint32_t* pr = problems + 4 * (poff + i);
+                pr[0] = static_cast<uint32_t>(b);
+                pr[1] = off + 8 * i;
+                pr[2] = min(8u, count - 8 * i);
+                pr[3] = 0;
+            }
+        }
+        if (b == 0) *num_problems = np_total;
     }
     __syncthreads();
 
     // Phase 3: stable scatter into expert order.
-    const uint32_t* boff = hist + kRouteWarps * NB;
-    for (int64_t c = seg0; c < seg1; c += 32) {
+    auto place = [&](int64_t r, int k) {
+        const uint32_t mask = __match_any_sync(0xffffffffu, k);
+        if (k < NB) perm[cnt[k] + hist[warp * NB + k] + __popc(mask & lanemask_lt())] = static_cast<uint32_t>(r);
+        __syncwarp();
+        if (k < NB && lane == __ffs(mask) - 1) hist[warp * NB + k] += __popc(mask);
+        __syncwarp();
+    };
+#pragma unroll
+    for (int i = 0; i < kKeyRegs; ++i) place(seg0 + 32 * i + lane, key[i]);
+    for (int64_t c = seg0 + 32 * kKeyRegs; c < seg1; c += 32) {
         const int64_t r = c + lane;
-        const bool valid = r < seg1;
-        const int key = valid ? key_of(r, false) : NB;
-        const uint32_t mask = __match_any_sync(0xffffffffu, key);
-        if (valid) {
-            const uint32_t pos = boff[key] + hist[warp * NB + key] + __popc(mask & lanemask_lt());
-            perm[pos] = static_cast<uint32_t>(r);
-        }
-        __syncwarp();
-        if (valid && lane == __ffs(mask) - 1) hist[warp * NB + key] += __popc(mask);
-        __syncwarp();
+        place(r, r < seg1 ? key_of(r, false) : NB);
     }
     if (threadIdx.x == 0) *flags_out = s_flags;
 }
@@ -176,7 +200,7 @@ GatherWorkspace gather_workspace_carve(void* base, int64_t R, int64_t E) {
 
 cudaError_t launch_gather_route(const uint32_t* lhs, const uint32_t* rhs, int64_t R, int64_t E,
                                 int64_t x_rows, int sorted, const GatherWorkspace& ws,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool want_problems) {
     const int NB = static_cast<int>(E) + 1;
     // per-warp histograms plus one row of bucket offsets
     const size_t smem = static_cast<size_t>(kRouteWarps + 1) * NB * sizeof(uint32_t);
@@ -187,8 +211,8 @@ cudaError_t launch_gather_route(const uint32_t* lhs, const uint32_t* rhs, int64_
         if (e != cudaSuccess) return e;
     }
     gather_route_kernel<<<1, kRouteThreads, smem, stream>>>(
-        lhs, rhs, R, static_cast<int>(E), x_rows, sorted, ws.flags, ws.num_problems, ws.offsets,
-        ws.perm, ws.problems);
+        lhs, rhs, R, static_cast<int>(E), x_rows, sorted, want_problems ? 1 : 0, ws.flags, ws.num_problems,
+        ws.offsets, ws.perm, ws.problems);
     return cudaGetLastError();
 }
 

@@ -73,8 +73,10 @@ struct GatherWorkspace {
 };
 size_t gather_workspace_bytes(int64_t R, int64_t E);
 GatherWorkspace gather_workspace_carve(void* base, int64_t R, int64_t E);
+// want_problems: also write the (expert, first, count <= 8) work items of the
+// matrix-vector route (the tensor-core routes read only offsets and perm).
 cudaError_t launch_gather_route(const uint32_t* lhs, const uint32_t* rhs, int64_t R, int64_t E,
                                 int64_t x_rows, int sorted, const GatherWorkspace& ws,
-                                cudaStream_t stream);
+                                cudaStream_t stream, bool want_problems);
 
 }  // namespace nvq

@@ -145,7 +145,7 @@ nv_status nv_moe_swiglu(const void* x, nv_dtype dt, int64_t T, int64_t K, const 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return NV_ERR_CUDA;
     const nvq::GatherWorkspace rt = nvq::gather_workspace_carve(w.route, R, E);
-    e = nvq::launch_gather_route(w.lhs, ids, R, E, T, 0, rt, s);
+    e = nvq::launch_gather_route(w.lhs, ids, R, E, T, 0, rt, s, false);
     if (e != cudaSuccess) return NV_ERR_CUDA;
     // gate, then up with silu(gate) * up over the gate values, then down
     e = nvq::launch_tc_gather(x, T, K, w.lhs, rt.perm, rt.offsets, E, I, gate_codes, gate_scales,
