@@ -832,6 +832,7 @@ PROFILE_WORKLOADS = {
     "decode_t0": lambda dev: Decode(dev, transpose=False),
     "fewrow8": lambda dev: Decode(dev, M=8),
     "gather": lambda dev: Gather(dev, sorted_pairs=False),
+    "gather_kn": lambda dev: Gather(dev, sorted_pairs=True, transpose=False),
     "prefill": lambda dev: Decode(dev, N=14336, K=4096, M=2048, bits=4, gs=64),
     "splitk": lambda dev: Decode(dev, N=1024, K=14336, M=64),
     "prefill8": lambda dev: Decode(dev, N=14336, K=4096, M=2048, bits=8, gs=64),
