@@ -333,20 +333,24 @@ class Decode:
 
 
 class DecodeE2E(Decode):
-    """The same product from host buffers: pinned x in, y out, every step."""
+    """The same step from host buffers: each step copies its input x from pinned
+    host memory, runs the product with every weight copy (one output row block
+    per copy) and reads all the step's outputs back into pinned host memory."""
 
     def __init__(self, dev, **kw):
         super().__init__(dev, **kw)
         self.xh = self.x.cpu().pin_memory()
-        self.yh = [torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
-                   for _ in range(self.copies)]
-        self.h2d = self.xh.numel() * 2 * self.copies
-        self.d2h = self.yh[0].numel() * 2 * self.copies
+        self.yall = torch.empty(self.copies, self.M, self.N, dtype=torch.bfloat16, device=dev)
+        self.yh = torch.empty(self.copies, self.M, self.N, dtype=torch.bfloat16).pin_memory()
+        self.h2d = self.xh.numel() * 2
+        self.d2h = self.yh.numel() * 2
 
-    def call(self, j):
+    def step(self, i):
         self.x.copy_(self.xh, non_blocking=True)
-        super().call(j)
-        self.yh[j].copy_(self.y, non_blocking=True)
+        for j in range(self.copies):
+            c, s, b = self.ws[j]
+            self.nvq.nv_qmm(self.x, c, s, b, self.gs, self.bits, self.t, out=self.yall[j])
+        self.yh.copy_(self.yall, non_blocking=True)
 
 
 class DecodeFp:
