@@ -9,19 +9,23 @@
 // each expert's weights cross HBM once for all its rows. Roles, per CTA
 // (persistent):
 //   warp 0      one lane streams code boxes of 64 k-rows x 256 columns by TMA
-//               into a ring released by the dequantizing warps.
+//               (with the boxes of scales and biases that cover the unit,
+//               when N / gs is a multiple of 8) into a ring released by the
+//               dequantizing warps; the warp prefetches later stages into L2.
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (M = 128,
 //               N = pairs rounded up to 16, K = 16) with both operands in
 //               shared memory, two tiles per k-step, into a double-buffered
 //               accumulator (64 columns per tile).
-//   warps 2-5   epilogue: TMEM lane = weight column, column = pair; each pair's
-//               value is stored to its output row.
+//   warps 2-5   epilogue: TMEM lane = A-tile row (a permutation of the unit's
+//               columns), column = pair; each pair's value is stored to its
+//               output row.
 //   warps 6-9   copy the pairs' activation rows with cp.async into the
 //               128-byte-swizzled B layout.
-//   warps 10-25 dequantize and transpose: a task is 4 k-rows x one code word
-//               (PER columns); each column's 4 values w = s[k, g(n)] * code +
-//               b[k, g(n)] (one bf16 fma on the exact code, rounded once) go to
-//               the column's row of the K-major A tile as one 8-byte piece.
+//   warps 10-25 dequantize and transpose, as two groups of eight warps on
+//               alternate stages: each column's 4 consecutive k-values
+//               w = s[k, g(n)] * code + b[k, g(n)] (one bf16 fma on the exact
+//               code, rounded once) go to the column's row of the K-major A
+//               tile as one 8-byte piece.
 // The kernel is the programmatic dependent of the routing kernel. Pairs with
 // an out-of-range id get zero rows. Waits are bounded by a timer.
 #include <cuda.h>
