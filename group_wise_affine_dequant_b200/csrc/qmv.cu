@@ -231,8 +231,8 @@ struct QmvParams {
     uint16_t* y;             // bf16 [*, N]
     int64_t N, K;
     int M;                   // rows (plain product)
-    int ctas_per_problem;    // G: CTAs along N; CTA c takes rows_q + (c < rows_r) rows
-    int rows_q, rows_r;      // N / G and N % G
+    int ctas_per_problem;    // G: CTAs along N; CTA c takes tiles_q + (c < tiles_r) 16-row tiles
+    int tiles_q, tiles_r;    // T / G and T % G, T = ceil(N / 16)
     int rows_cap;            // max rows of one CTA, multiple of 16
     int rows_max;            // max rows of one CTA (height of the scale/bias block)
     // Scales and biases: 2 = the CTA's whole block by TMA once (nbox boxes of
@@ -373,8 +373,8 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
         // only L2 prefetches (coherent) touch memory before the wait.
         {
             const int cta = static_cast<int>(blockIdx.x);
-            const int r0 = cta * prm.rows_q + min(cta, prm.rows_r);
-            const int nrows = prm.rows_q + (cta < prm.rows_r ? 1 : 0);
+            const int r0 = 16 * (cta * prm.tiles_q + min(cta, prm.tiles_r));
+            const int nrows = min(16 * (prm.tiles_q + (cta < prm.tiles_r ? 1 : 0)), static_cast<int>(N) - r0);
             const int nsl = static_cast<int>((K + S::KSLICE - 1) / S::KSLICE);
             // the first ring's worth of tiles of the warp's first slice
             // (prefetching everything floods HBM while the previous kernel
@@ -412,8 +412,10 @@ qmv_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CU
     __syncthreads();
 
     const int cta = static_cast<int>(blockIdx.x);
-    const int64_t n0 = static_cast<int64_t>(cta) * prm.rows_q + min(cta, prm.rows_r);
-    const int rows = prm.rows_q + (cta < prm.rows_r ? 1 : 0);
+    // whole 16-row tiles per CTA (the last CTA's last tile may be partial)
+    const int64_t n0 = 16 * (static_cast<int64_t>(cta) * prm.tiles_q + min(cta, prm.tiles_r));
+    const int rows = static_cast<int>(
+        min(static_cast<int64_t>(16 * (prm.tiles_q + (cta < prm.tiles_r ? 1 : 0))), N - n0));
     const int64_t n1 = n0 + rows;
     if (rows <= 0) return;
 
@@ -768,9 +770,11 @@ Plan plan(int64_t N, int64_t K, int M, int gs, int kslice, int code_stage, int s
     int64_t ctas = gather ? (N + 127) / 128
                           : std::max<int64_t>(std::min<int64_t>(num_sms, (N + 15) / 16),
                                               (N + 127) / 128);
+    const int64_t tiles = (N + 15) / 16;
     for (;;) {
-        const int64_t rows = (N + ctas - 1) / ctas;
-        const int64_t cap = (rows + 15) / 16 * 16;
+        // whole 16-row tiles per CTA: a CTA's last tile is never nearly empty
+        const int64_t cap = (tiles + ctas - 1) / ctas * 16;
+        const int64_t rows = std::min<int64_t>(cap, N);
         const size_t red = static_cast<size_t>(nslices * cap * M) * sizeof(float);
         Plan p{};
         p.ctas = static_cast<int>(ctas);
@@ -868,8 +872,8 @@ bool encode_maps(const Variant<GATHER>& v, const Plan& p, const uint32_t* codes,
 
 static void set_plan(QmvParams& prm, const Plan& p, int64_t N) {
     prm.ctas_per_problem = p.ctas;
-    prm.rows_q = static_cast<int>(N / p.ctas);
-    prm.rows_r = static_cast<int>(N % p.ctas);
+    prm.tiles_q = static_cast<int>((N + 15) / 16 / p.ctas);
+    prm.tiles_r = static_cast<int>((N + 15) / 16 % p.ctas);
     prm.rows_cap = p.rows_cap;
     prm.rows_max = p.rows_max;
     prm.sb_mode = p.sb_mode;
