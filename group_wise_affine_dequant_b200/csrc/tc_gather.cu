@@ -46,6 +46,10 @@
 namespace nvq {
 namespace {
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 using namespace tc;
 
 constexpr int WM = 128;          // weight rows per tile (TMEM lanes)
@@ -286,12 +290,37 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     const int c = h * 32 + lane;
                     prow[h] = c < cn ? __ldg(prm.perm + first + p0 + c) : 0u;
                 }
+                if (prm.act) {
+                    // SwiGLU: bring the pass's gate values into L2 while the
+                    // products run (each is read once, below, then overwritten)
+                    for (int tt = 0; tt < kTiles; ++tt) {
+                        const int64_t n = static_cast<int64_t>(wt) * UW + tt * WM + q * 32 + lane;
+                        for (int c = 0; c < cn; ++c) {
+                            const uint32_t pair = __shfl_sync(0xffffffffu, (c >> 5) ? prow[1] : prow[0], c & 31);
+                            if (n < prm.N) prefetch_l2(prm.act + static_cast<int64_t>(pair) * prm.N + n);
+                        }
+                    }
+                }
                 if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
                 for (int tt = 0; tt < kTiles; ++tt)
                 for (int c0 = 0; c0 < cn; c0 += 16) {
                     // weight row of the unit = tile * 128 + TMEM lane
                     const int64_t n = static_cast<int64_t>(wt) * UW + tt * WM + q * 32 + lane;
+                    const uint32_t rows = (c0 >> 5) ? prow[1] : prow[0];
+                    // SwiGLU: the chunk's 16 gate values are read before any of its
+                    // outputs is written (over them, in place), all loads in flight
+                    // together and under the accumulator load
+                    float gv[16];
+                    if (prm.act) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
+                            gv[j] = (c0 + j < cn && n < prm.N)
+                                        ? bf16_bits_to_f32(prm.act[static_cast<int64_t>(pair) * prm.N + n])
+                                        : 0.f;
+                        }
+                    }
                     uint32_t v[16];
                     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                            static_cast<uint32_t>(acc * kAccCols + tt * kMaxPairs + c0);
@@ -303,19 +332,19 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                           "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
                         : "r"(taddr));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    const uint32_t rows = (c0 >> 5) ? prow[1] : prow[0];
+                    if (prm.act) {
+                        // silu(g) * u = g / (1 + e^-g) * u, for all 16 columns at once
+                        // (no branch between them); fast exponential and division,
+                        // within a few ulp in fp32
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            v[j] = __float_as_uint(__fdividef(gv[j], 1.0f + __expf(-gv[j])) * __uint_as_float(v[j]));
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
-                        if (c0 + j < cn && n < prm.N) {
-                            const int64_t o = static_cast<int64_t>(pair) * prm.N + n;
-                            float val = __uint_as_float(v[j]);
-                            if (prm.act) {  // silu(g) * u = g / (1 + e^-g) * u
-                                const float gv = bf16_bits_to_f32(prm.act[o]);
-                                val = gv / (1.0f + expf(-gv)) * val;
-                            }
-                            prm.y[o] = f32_to_bf16_bits(val);
-                        }
+                        if (c0 + j < cn && n < prm.N)
+                            prm.y[static_cast<int64_t>(pair) * prm.N + n] = f32_to_bf16_bits(__uint_as_float(v[j]));
                     }
                 }
                 tc_fence_before();
