@@ -301,6 +301,18 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         }
                     }
                 }
+                // the first chunk's gate values while the products run
+                float gv[16];
+                if (prm.act) {
+                    const int64_t n = static_cast<int64_t>(wt) * UW + q * 32 + lane;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t pair = __shfl_sync(0xffffffffu, prow[0], j);
+                        gv[j] = (j < cn && n < prm.N)
+                                    ? bf16_bits_to_f32(prm.act[static_cast<int64_t>(pair) * prm.N + n])
+                                    : 0.f;
+                    }
+                }
                 if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
                 for (int tt = 0; tt < kTiles; ++tt)
@@ -311,8 +323,7 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                     // SwiGLU: the chunk's 16 gate values are read before any of its
                     // outputs is written (over them, in place), all loads in flight
                     // together and under the accumulator load
-                    float gv[16];
-                    if (prm.act) {
+                    if (prm.act && (tt > 0 || c0 > 0)) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
