@@ -157,7 +157,7 @@ def _gather(x, c, s, b, rhs, lhs, gs, bits, t, row_exact=False):
 
 
 GATHER_ROUTES = [("grouped", True, False, BF16), ("per_row", True, True, BF16),
-                 ("simt_t0_bf16", False, False, BF16), ("simt_t0_fp32", False, False, F32),
+                 ("grouped_t0_bf16", False, False, BF16), ("simt_t0_fp32", False, False, F32),
                  ("simt_t1_fp32", True, False, F32)]
 
 
