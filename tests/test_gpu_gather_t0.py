@@ -154,3 +154,55 @@ def test_moe_shapes_sampled():
     n_idx = torch.randint(0, N, (4096,), generator=g)
     yr, a = O.gather_qmm_sampled(x, c, s, b, lhs, rhs, 64, 4, False, r_idx, n_idx)
     P.assert_within(y_u[r_idx, n_idx], yr, a, BF16, "transpose=0 moe sampled")
+
+
+@pytest.mark.parametrize("bits,gs", [(4, 64), (8, 64), (2, 32), (4, 128)])
+def test_zero_weights_with_nonzero_bias_under_huge_activations(bits, gs):
+    """Integer experts in [-(2^bits - 1), 0] with both ends in every group:
+    scale 1 and bias -(2^bits - 1), so code 2^bits - 1 dequantizes to exactly
+    0 while scale * code and bias are each large. k-rows S hold only such
+    zeros (and each group's -max) and meet activations of +-2^60: a product
+    that summed scale * code * x and bias * x apart would cancel 2^60-sized
+    terms. The grouped kernel dequantizes first (the general form here, since
+    the scales are 1)."""
+    E, K, N, T = 3, 512, 512, 12
+    hi = 2 ** bits - 1
+    g = torch.Generator().manual_seed(95 + bits)
+    S = torch.arange(3, K, 64)
+    ws = []
+    for _ in range(E):
+        w = -torch.randint(0, hi + 1, (K, N), generator=g).to(torch.float32)
+        w[:, ::gs] = -hi
+        w[:, 1::gs] = 0.0
+        w[S, :] = 0.0
+        w[S.unsqueeze(1), torch.arange(0, N, gs).unsqueeze(0)] = -hi
+        ws.append(w)
+    w = torch.stack(ws).to(BF16)
+    c, s, b = O.quantize_affine(w, gs, bits)
+    assert (s.float() == 1).all() and (b.float() == -hi).all()
+    x = torch.randn(T, K, generator=g)
+    x[:, S] = 2.0 ** 60 * torch.where(torch.rand(len(S), generator=g) < 0.5, -1.0, 1.0)
+    x = x.to(BF16)
+    R = 40
+    rhs = torch.randint(0, E, (R,), generator=g)
+    lhs = torch.randint(0, T, (R,), generator=g)
+    y, flags = _gather(x, c, s, b, rhs, lhs, gs, bits)
+    assert flags == 0 and torch.isfinite(y.float()).all()
+    yr, a = O.gather_qmm(x, c, s, b, lhs, rhs, gs, bits, False)
+    P.assert_within(y, yr, a, BF16, f"transpose=0 cancelling bias b{bits} g{gs}")
+
+
+@pytest.mark.parametrize("j", [-40, -7, 9, 50])
+def test_power_of_two_scalings_are_exact(j):
+    """y(2^j x) == 2^j y(x) bit for bit: every product and sum scales exactly
+    (no value leaves the fp32 range) and so does the bf16 rounding."""
+    E, K, N, T = 3, 256, 512, 10
+    w = W.normal((E, K, N), 0.02, 96, "bf16")
+    c, s, b = O.quantize_affine(w, 64, 4)
+    x = W.normal((T, K), 1.0, 97, "bf16")
+    g = torch.Generator().manual_seed(98)
+    rhs = torch.randint(0, E, (24,), generator=g)
+    lhs = torch.randint(0, T, (24,), generator=g)
+    y1, _ = _gather(x, c, s, b, rhs, lhs, 64, 4)
+    y2, _ = _gather((x.float() * 2.0 ** j).to(BF16), c, s, b, rhs, lhs, 64, 4)
+    assert torch.equal((y1.float() * 2.0 ** j).to(BF16).view(torch.int16), y2.view(torch.int16)), j
