@@ -46,6 +46,9 @@
 namespace nvq {
 namespace {
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -94,6 +97,7 @@ struct GParams {
     int sb_slot;                // bytes of one slot (scales + biases)
     int dx, dc, da;             // depths: activations, codes, dequantized weights
     uint32_t x_off, c_off, a_off, sb_off, bar_off, row_off;
+    uint32_t g_off;             // act: gate staging, [4 warps][2 tiles][64 pairs][32 columns] bf16
 };
 
 struct RingPos {
@@ -301,35 +305,57 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
                         }
                     }
                 }
-                // the first chunk's gate values while the products run
-                float gv[16];
+                // SwiGLU: the pass's gate values (this warp's 32 columns of both
+                // tiles, every pair) are copied into the warp's staging area while
+                // the products run, 4 bytes a lane (lanes 0-15 one pair, 16-31 the
+                // next), before any output of the pass is written over them
+                const uint32_t gst = smem_u32(smem + prm.g_off) + static_cast<uint32_t>(q) * (kTiles * kMaxPairs * 64);
                 if (prm.act) {
-                    const int64_t n = static_cast<int64_t>(wt) * UW + q * 32 + lane;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const uint32_t pair = __shfl_sync(0xffffffffu, prow[0], j);
-                        gv[j] = (j < cn && n < prm.N)
-                                    ? bf16_bits_to_f32(prm.act[static_cast<int64_t>(pair) * prm.N + n])
-                                    : 0.f;
+                    for (int tt = 0; tt < kTiles; ++tt) {
+                        const int64_t n0 = static_cast<int64_t>(wt) * UW + tt * WM + q * 32;
+                        if (n0 < prm.N) {
+                            for (int c = 0; c < cn; c += 2) {
+                                const int ci = c + (lane >> 4);
+                                const uint32_t pair = __shfl_sync(0xffffffffu, (ci >> 5) ? prow[1] : prow[0], ci & 31);
+                                const int64_t col = n0 + (lane & 15) * 2;  // columns col, col + 1
+                                const uint16_t* src = prm.act + static_cast<int64_t>(pair) * prm.N + col;
+                                const uint32_t dst = gst + (tt * kMaxPairs + ci) * 64 + (lane & 15) * 4;
+                                if (ci < cn) {
+                                    if ((prm.N & 1) == 0 && col + 1 < prm.N) {
+                                        cp_async4(dst, src);  // 4-byte aligned: N and col even
+                                    } else {                  // odd N or the last column
+                                        for (int h = 0; h < 2; ++h)
+                                            if (col + h < prm.N)
+                                                asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + 2 * h),
+                                                             "h"(src[h]) : "memory");
+                                    }
+                                }
+                            }
+                        }
                     }
+                    cp_async_commit();
                 }
                 if (!(ok = mbar_wait_backoff(&acc_full[acc], ause & 1, 25, 2048))) break;
                 tc_fence_after();
+                if (prm.act) {
+                    cp_async_wait<0>();
+                    __syncwarp();
+                }
+                float gv[16];
                 for (int tt = 0; tt < kTiles; ++tt)
                 for (int c0 = 0; c0 < cn; c0 += 16) {
                     // weight row of the unit = tile * 128 + TMEM lane
                     const int64_t n = static_cast<int64_t>(wt) * UW + tt * WM + q * 32 + lane;
                     const uint32_t rows = (c0 >> 5) ? prow[1] : prow[0];
-                    // SwiGLU: the chunk's 16 gate values are read before any of its
-                    // outputs is written (over them, in place), all loads in flight
-                    // together and under the accumulator load
-                    if (prm.act && (tt > 0 || c0 > 0)) {
+                    if (prm.act) {  // the chunk's 16 gate values from the staging area
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const uint32_t pair = __shfl_sync(0xffffffffu, rows, (c0 + j) & 31);
-                            gv[j] = (c0 + j < cn && n < prm.N)
-                                        ? bf16_bits_to_f32(prm.act[static_cast<int64_t>(pair) * prm.N + n])
-                                        : 0.f;
+                            uint16_t gb;
+                            asm volatile("ld.shared.u16 %0, [%1];"
+                                         : "=h"(gb)
+                                         : "r"(gst + (tt * kMaxPairs + c0 + j) * 64 + lane * 2));
+                            gv[j] = bf16_bits_to_f32(gb);
                         }
                     }
                     uint32_t v[16];
@@ -630,9 +656,11 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.sb_slot = 2 * UW * sbw;
     const size_t sb_ring = 2u * static_cast<size_t>(prm.sb_slot);
     int dx = 7, dc = 2;
+    // SwiGLU: the epilogue warps' gate staging, 4 x 2 x 64 pairs x 64 bytes
+    const size_t g_bytes = act_gate ? static_cast<size_t>(4 * kTiles * kMaxPairs * 64) : 0;
     auto bytes = [&]() {
         return static_cast<size_t>(kXStage) * dx + static_cast<size_t>(kCStage) * dc + sb_ring +
-               kXoffBytes +
+               kXoffBytes + g_bytes +
                static_cast<size_t>(2 * (dx + dc + kDA) + 8) * 8 + 16;
     };
     const size_t budget = 227 * 1024 - 2048 - 1024;
@@ -646,7 +674,8 @@ cudaError_t launch_tc_gather(const void* x, int64_t x_rows, int64_t K, const uin
     prm.a_off = 0;  // A stages live in TMEM
     prm.sb_off = prm.c_off + kCStage * dc;
     prm.row_off = prm.sb_off + static_cast<uint32_t>(sb_ring);
-    prm.bar_off = prm.row_off + kXoffBytes;
+    prm.g_off = prm.row_off + kXoffBytes;
+    prm.bar_off = prm.g_off + static_cast<uint32_t>(g_bytes);
     const size_t smem = bytes() + 1024;
     const int units = static_cast<int>(E) * prm.wunits;
     const int grid = units < num_sms ? units : num_sms;
