@@ -182,6 +182,10 @@ tc_gather_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constan
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();  // the routing tables (offsets, perm) come from the previous kernel
+    // A following grouped product (the next one of a SwiGLU block) may launch
+    // now: it sets up and prefetches its own weights as SMs free up, and waits
+    // for this grid before it reads anything this one writes.
+    pdl_launch_dependents();
 
     auto unit_pairs = [&](int u, int& e, int& wt, int& first, int& count) {
         e = u / prm.wunits;
