@@ -190,6 +190,11 @@ __global__ void __launch_bounds__(kFpRowsPerBlock * 32)
 qmv_fp_kernel(const uint16_t* __restrict__ x, int M, int64_t K, int64_t N, const uint32_t* __restrict__ codes,
               const uint8_t* __restrict__ scales, uint16_t* __restrict__ y) {
     using F = FpFormat<MODE>;
+    // launched as the programmatic dependent of the previous kernel: the next
+    // product may launch at once; this one waits for the previous grid (which
+    // may have written x or the weights) before its first read
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31;
     const int64_t n = static_cast<int64_t>(blockIdx.x) * kFpRowsPerBlock + (threadIdx.x >> 5);
     if (n >= N) return;
@@ -263,11 +268,20 @@ cudaError_t launch_qmv_fp(const void* x, int64_t M, int64_t K, int64_t N, const 
     const auto* xp = static_cast<const uint16_t*>(x);
     auto* yp = static_cast<uint16_t*>(y);
     const int m = static_cast<int>(M);
-    if (M <= 1) qmv_fp_kernel<MODE, 1><<<blocks, kFpRowsPerBlock * 32, 0, s>>>(xp, m, K, N, codes, scales, yp);
-    else if (M <= 2) qmv_fp_kernel<MODE, 2><<<blocks, kFpRowsPerBlock * 32, 0, s>>>(xp, m, K, N, codes, scales, yp);
-    else if (M <= 4) qmv_fp_kernel<MODE, 4><<<blocks, kFpRowsPerBlock * 32, 0, s>>>(xp, m, K, N, codes, scales, yp);
-    else qmv_fp_kernel<MODE, 8><<<blocks, kFpRowsPerBlock * 32, 0, s>>>(xp, m, K, N, codes, scales, yp);
-    return cudaGetLastError();
+    void (*k)(const uint16_t*, int, int64_t, int64_t, const uint32_t*, const uint8_t*, uint16_t*) =
+        M <= 1 ? qmv_fp_kernel<MODE, 1> : M <= 2 ? qmv_fp_kernel<MODE, 2> : M <= 4 ? qmv_fp_kernel<MODE, 4>
+                                                                              : qmv_fp_kernel<MODE, 8>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(kFpRowsPerBlock * 32, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, xp, m, K, N, codes, scales, yp);
 }
 
 int fp_group(int mode) { return mode == kNv4 ? 16 : 32; }
