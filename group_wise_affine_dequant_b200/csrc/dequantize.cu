@@ -89,6 +89,11 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restr
                                                          const void* __restrict__ biases,
                                                          int64_t words, int lg_gs,
                                                          void* __restrict__ out) {
+    // launched as the programmatic dependent of the previous kernel: the next
+    // call may launch at once; this one waits for the previous grid before its
+    // first read or write
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int PER = 32 / BITS;
     constexpr int ESZ = DT == NV_F32 ? 4 : 2;
     char* o = static_cast<char*>(out);
@@ -129,15 +134,25 @@ cudaError_t launch_dt(const uint32_t* codes, const void* scales, const void* bia
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    const dim3 grid(static_cast<unsigned>(blocks));
+    void (*k)(const uint32_t*, const void*, const void*, int64_t, int, void*);
     switch (bits) {
-        case 1: dequantize_kernel<DT, 1><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
-        case 2: dequantize_kernel<DT, 2><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
-        case 4: dequantize_kernel<DT, 4><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
-        case 8: dequantize_kernel<DT, 8><<<grid, threads, 0, stream>>>(codes, scales, biases, words, lg_gs, out); break;
+        case 1: k = dequantize_kernel<DT, 1>; break;
+        case 2: k = dequantize_kernel<DT, 2>; break;
+        case 4: k = dequantize_kernel<DT, 4>; break;
+        case 8: k = dequantize_kernel<DT, 8>; break;
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, codes, scales, biases, words, lg_gs, out);
 }
 
 }  // namespace

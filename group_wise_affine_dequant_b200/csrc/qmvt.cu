@@ -137,6 +137,11 @@ constexpr int kMaxThreads = 512;  // column units per CTA x thread-rows
 template <int BITS, int TW, int MT>
 __global__ void __cluster_dims__(1, kClusterK, 1) __launch_bounds__(kMaxThreads)
 qmvt_kernel(const QmvtParams prm) {
+    // launched as the programmatic dependent of the previous kernel: the next
+    // product may launch at once; this one waits for the previous grid before
+    // its first read (x or the weights may come from it)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     using C = Codes<BITS>;
     constexpr int COLS_T = TW * C::PER;   // columns a thread owns
     extern __shared__ float smem[];       // [KP_ROUND][MT][ctm * COLS_T], then [MT][ctm * COLS_T]
@@ -310,8 +315,17 @@ cudaError_t launch_one(const QmvtParams& prm0, int num_sms, cudaStream_t stream)
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    k<<<dim3(static_cast<unsigned>(ranges), kClusterK, 1), threads, smem, stream>>>(prm);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ranges), kClusterK, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, prm);
 }
 
 // Words per thread: as many as fit 64 accumulators per thread, within a group.
