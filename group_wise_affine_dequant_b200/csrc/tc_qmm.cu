@@ -190,6 +190,11 @@ tc_qmm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // launched as the programmatic dependent of the previous kernel: set up
+    // above, then let the next product launch and wait for the previous grid
+    // (x, the weights or y may be its) before the first global access
+    pdl_launch_dependents();
+    pdl_wait();
 
     const int ksteps = static_cast<int>(prm.K / BK);
     const int sgk = 8 * prm.gs / BK;  // k-steps per block of 8 groups
@@ -955,13 +960,15 @@ cudaError_t launch_tc_qmm(const void* x, int64_t M, int64_t K, int64_t N, const 
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(plan.splits);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k, map_x, map_c, map_s, map_b, prm);
 }
 
