@@ -27,6 +27,9 @@ namespace nvq {
 namespace {
 
 __global__ void pair_tokens_kernel(uint32_t* __restrict__ lhs, int64_t R, int topk) {
+    // a programmatic dependent: waits for the previous grid before writing
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < R;
          r += static_cast<int64_t>(gridDim.x) * blockDim.x)
         lhs[r] = static_cast<uint32_t>(r / topk);
@@ -36,6 +39,9 @@ __global__ void pair_tokens_kernel(uint32_t* __restrict__ lhs, int64_t R, int to
 // (16-byte loads and stores), j in order.
 __global__ void combine_kernel(const uint16_t* __restrict__ d, const float* __restrict__ rw,
                                int64_t T, int64_t K, int topk, uint16_t* __restrict__ y) {
+    // a programmatic dependent of the down product: waits for it before reading d
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t chunks = K / 8;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < T * chunks;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -140,9 +146,16 @@ nv_status nv_moe_swiglu(const void* x, nv_dtype dt, int64_t T, int64_t K, const 
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    nvq::pair_tokens_kernel<<<static_cast<unsigned>((R + 255) / 256 < 4 * sms ? (R + 255) / 256 : 4 * sms),
-                              256, 0, s>>>(w.lhs, R, topk);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((R + 255) / 256 < 4 * sms ? (R + 255) / 256 : 4 * sms), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, nvq::pair_tokens_kernel, w.lhs, R, topk);
     if (e != cudaSuccess) return NV_ERR_CUDA;
     const nvq::GatherWorkspace rt = nvq::gather_workspace_carve(w.route, R, E);
     e = nvq::launch_gather_route(w.lhs, ids, R, E, T, 0, rt, s, false);
@@ -159,9 +172,10 @@ nv_status nv_moe_swiglu(const void* x, nv_dtype dt, int64_t T, int64_t K, const 
     if (e != cudaSuccess) return NV_ERR_CUDA;
     const int64_t items = T * (K / 8);
     const int64_t blocks = (items + 255) / 256 < 8 * sms ? (items + 255) / 256 : 8 * sms;
-    nvq::combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        w.d, rw, T, K, topk, static_cast<uint16_t*>(y));
-    return cudaGetLastError() == cudaSuccess ? NV_OK : NV_ERR_CUDA;
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, nvq::combine_kernel, static_cast<const uint16_t*>(w.d), rw, T, K, topk,
+                           static_cast<uint16_t*>(y));
+    return e == cudaSuccess ? NV_OK : NV_ERR_CUDA;
 }
 
 }  // extern "C"
