@@ -74,6 +74,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1) gather_route_kernel(
     // the grouped product may launch now; it waits for this grid to finish
     // before it reads the tables
     pdl_launch_dependents();
+    // launched as a programmatic dependent itself: the previous kernel (the
+    // last call's grouped product, which may still read tables of a shared
+    // workspace, or the kernel that wrote the ids) ends before any access here
+    pdl_wait();
 
     for (int i = threadIdx.x; i < kRouteWarps * NB; i += kRouteThreads) hist[i] = 0;
     if (threadIdx.x == 0) s_flags = 0;
@@ -210,10 +214,19 @@ cudaError_t launch_gather_route(const uint32_t* lhs, const uint32_t* rhs, int64_
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    gather_route_kernel<<<1, kRouteThreads, smem, stream>>>(
-        lhs, rhs, R, static_cast<int>(E), x_rows, sorted, want_problems ? 1 : 0, ws.flags, ws.num_problems,
-        ws.offsets, ws.perm, ws.problems);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(kRouteThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gather_route_kernel, lhs, rhs, R, static_cast<int>(E), x_rows, sorted,
+                              want_problems ? 1 : 0, ws.flags, ws.num_problems, ws.offsets, ws.perm,
+                              ws.problems);
 }
 
 }  // namespace nvq
