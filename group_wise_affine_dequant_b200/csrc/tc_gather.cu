@@ -11,7 +11,9 @@
 // in steps of 128 (every pipeline handshake moves a 128-k slab: 16 MMAs, 16 KB
 // of codes at 4 bits, 16 KB of activations per k-step). The
 // kernel is the programmatic dependent of the routing kernel: it sets up and
-// prefetches its first weights into L2 before waiting for the routing tables.
+// prefetches its first weights into L2 before waiting for the routing tables,
+// then lets the next kernel launch (the next product of a SwiGLU block, or the
+// next call's router, each of which waits for this grid before any access).
 // Roles, per CTA (persistent):
 //   warp 0      one lane streams the code tiles by TMA, 256 rows x 128 bytes
 //               (several k-steps) per copy, into a ring released by the
@@ -22,6 +24,9 @@
 //               double-buffered TMEM accumulator (64 columns per tile).
 //   warps 2-5   epilogue: TMEM lane = weight row, column = pair; each column is
 //               stored to its pair's output row (32 lanes -> 64 contiguous bytes).
+//               With a gate buffer (the SwiGLU block) each warp first copies the
+//               pass's gate values into its shared-memory staging area by
+//               cp.async while the MMAs run, then stores silu(g) * product.
 //   warps 6-9   copy the pairs' activation rows with cp.async (16 bytes per
 //               thread per row and k-step) into the 128-byte-swizzled B layout;
 //               each thread fences its completed copies into the async proxy
